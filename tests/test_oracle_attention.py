@@ -1,0 +1,210 @@
+"""Pins for the oracle's attention forward and metadata (CPU only).
+
+Closed forms, a brute-force pure-Python softmax, scipy's logsumexp and
+invariances tie the oracle to the mathematics rather than to itself.
+"""
+import math
+
+import numpy as np
+import pytest
+from scipy.special import logsumexp
+
+from oracle import attention as oatt
+from oracle import meta as ometa
+from oracle import mxfp8 as omx
+
+SCALE = 1.0 / math.sqrt(128.0)
+
+
+def test_meta_prefix_sums_by_hand():
+    m = ometa.from_lengths([5, 128, 129, 300])
+    assert m.cu_seqlens.tolist() == [0, 5, 133, 262, 562]
+    assert m.scale_off.tolist() == [0, 1, 2, 4, 7]
+    assert (m.num_seqs, m.total_tokens, m.total_scale_blocks, m.max_seqlen) == (4, 562, 7, 300)
+    with pytest.raises(ValueError):
+        ometa.from_lengths([3, 0])
+    with pytest.raises(ValueError):
+        ometa.from_lengths([])
+
+
+def test_constant_v_gives_v():
+    g = np.random.default_rng(0)
+    q, k = g.standard_normal((7, 128)), g.standard_normal((33, 128))
+    vrow = g.standard_normal(128)
+    v = np.tile(vrow, (33, 1))
+    o, _ = oatt.attend_block(q, k, v)
+    assert np.allclose(o, vrow[None, :], atol=1e-12, rtol=0)
+
+
+def test_single_key():
+    g = np.random.default_rng(1)
+    q, k, v = g.standard_normal((5, 128)), g.standard_normal((1, 128)), g.standard_normal((1, 128))
+    o, lse = oatt.attend_block(q, k, v, qd=0.5, kd=3.0)
+    assert np.allclose(o, v, atol=1e-12, rtol=0)
+    s = (q @ k[0]) * 0.5 * 3.0 * SCALE
+    assert np.allclose(lse, s, atol=1e-12, rtol=0)
+
+
+def test_equal_logits():
+    g = np.random.default_rng(2)
+    n = 57
+    q = g.standard_normal((4, 128))
+    k = np.tile(g.standard_normal(128), (n, 1))
+    v = g.standard_normal((n, 128))
+    o, lse = oatt.attend_block(q, k, v)
+    s = (q @ k[0]) * SCALE
+    assert np.allclose(lse, np.log(n) + s, atol=1e-12, rtol=0)
+    assert np.allclose(o, v.mean(axis=0)[None, :], atol=1e-12, rtol=0)
+
+
+def _brute_attention(q, k, v, qd=1.0, kd=1.0, vd=1.0):
+    """Pure-Python loops: softmax(q.k * scale) v, natural-log LSE."""
+    out, lse = [], []
+    for r in range(len(q)):
+        s = []
+        for j in range(len(k)):
+            acc = 0.0
+            for d in range(128):
+                acc += float(q[r][d]) * float(k[j][d])
+            s.append(acc * qd * kd / math.sqrt(128.0))
+        mx = max(s)
+        w = [math.exp(x - mx) for x in s]
+        tot = sum(w)
+        row = []
+        for d in range(128):
+            acc = 0.0
+            for j in range(len(k)):
+                acc += w[j] * float(v[j][d])
+            row.append(acc / tot * vd)
+        out.append(row)
+        lse.append(mx + math.log(tot))
+    return np.array(out), np.array(lse)
+
+
+def test_brute_force_tiny_asymmetric():
+    g = np.random.default_rng(3)
+    q = g.standard_normal((3, 128)) * 2
+    k = g.standard_normal((5, 128)) * 1.5 + 0.3
+    v = g.standard_normal((5, 128)) - 0.2
+    o, lse = oatt.attend_block(q, k, v, qd=0.75, kd=1.25, vd=2.0)
+    ob, lb = _brute_attention(q, k, v, 0.75, 1.25, 2.0)
+    assert np.allclose(o, ob, atol=1e-12, rtol=1e-12)
+    assert np.allclose(lse, lb, atol=1e-12, rtol=1e-12)
+    s = (q @ k.T) * 0.75 * 1.25 * SCALE
+    assert np.allclose(lse, logsumexp(s, axis=1), atol=1e-12)
+
+
+def test_varlen_packing_equals_separate_and_cross_pairing():
+    g = np.random.default_rng(4)
+    lq, lk = [3, 9, 1], [4, 2, 11]
+    H = 2
+    q = g.standard_normal((sum(lq), H, 128))
+    k = g.standard_normal((sum(lk), H, 128))
+    v = g.standard_normal((sum(lk), H, 128))
+    o, lse = oatt.attention_fwd(q, k, v, lq, lk)
+    assert lse.shape == (H, sum(lq))
+    cq, ck = np.cumsum([0] + lq), np.cumsum([0] + lk)
+    for i in range(3):
+        for h in range(H):
+            ob, lb = _brute_attention(q[cq[i]:cq[i + 1], h], k[ck[i]:ck[i + 1], h], v[ck[i]:ck[i + 1], h])
+            assert np.allclose(o[cq[i]:cq[i + 1], h], ob, atol=1e-12)
+            assert np.allclose(lse[h, cq[i]:cq[i + 1]], lb, atol=1e-12)
+
+
+def test_key_permutation_invariance():
+    g = np.random.default_rng(5)
+    q, k, v = g.standard_normal((6, 128)), g.standard_normal((40, 128)), g.standard_normal((40, 128))
+    perm = g.permutation(40)
+    o1, l1 = oatt.attend_block(q, k, v)
+    o2, l2 = oatt.attend_block(q, k[perm], v[perm])
+    assert np.allclose(o1, o2, atol=1e-12) and np.allclose(l1, l2, atol=1e-12)
+
+
+def test_descale_two_equals_scale_bytes_plus_one():
+    """A q descale of 2 is the same as every Q scale byte raised by one."""
+    g = np.random.default_rng(6)
+    lens = [200]
+    x = g.standard_normal((200, 2, 128)).astype(np.float32)
+    kx = g.standard_normal((200, 2, 128)).astype(np.float32)
+    vx = g.standard_normal((200, 2, 128)).astype(np.float32)
+    pq, sq = omx.quantize_mxfp8_varlen(x, lens)
+    pk, sk = omx.quantize_mxfp8_varlen(kx, lens)
+    pv, sv = omx.quantize_mxfp8_varlen(vx, lens)
+    kh = omx.dequantize_mxfp8(pk, sk, lens, 2)
+    vh = omx.dequantize_mxfp8(pv, sv, lens, 2)
+    qh = omx.dequantize_mxfp8(pq, sq, lens, 2)
+    qh2 = omx.dequantize_mxfp8(pq, sq + np.uint8(1), lens, 2)
+    assert np.allclose(qh2, 2 * qh, atol=0)
+    o1, l1 = oatt.attention_fwd(qh, kh, vh, lens, lens, qd=2.0)
+    o2, l2 = oatt.attention_fwd(qh2, kh, vh, lens, lens)
+    assert np.allclose(o1, o2, atol=1e-12) and np.allclose(l1, l2, atol=1e-12)
+    o3, _ = oatt.attention_fwd(qh, kh, vh, lens, lens)
+    assert not np.allclose(o1, o3, atol=1e-3)
+
+
+def test_fp8_variant_equals_plain_when_weights_exact():
+    """Logits whose log2 values are integers give E4M3-exact weights: variant == definition."""
+    g = np.random.default_rng(7)
+    n = 24
+    ints = g.integers(-12, 1, size=n).astype(np.float64)
+    ints[3] = 0.0
+    # s_j = ints_j * ln 2 through a single query q = e_0 and keys k_j = (c_j, 0, ...)
+    q = np.zeros((1, 128)); q[0, 0] = 1.0
+    k = np.zeros((n, 128)); k[:, 0] = ints * math.log(2.0) * math.sqrt(128.0)
+    v = g.standard_normal((n, 128))
+    o_plain, l_plain = oatt.attend_block(q, k, v, p_mode="exact")
+    o_fp8, l_fp8 = oatt.attend_block(q, k, v, p_mode="fp8")
+    assert np.allclose(o_plain, o_fp8, atol=1e-12)
+    assert np.allclose(l_plain, l_fp8, atol=1e-12)
+
+
+def test_fp8_variant_shift_invariance_and_brute_force():
+    g = np.random.default_rng(8)
+    q, k, v = g.standard_normal((3, 128)), g.standard_normal((50, 128)), g.standard_normal((50, 128))
+    o1, _ = oatt.attend_block(q, k, v, p_mode="fp8")
+    # shifting every logit of a row by 3*ln2 (via descale on a constant extra channel)
+    qs = np.concatenate([q[:, :127], np.full((3, 1), 1.0)], axis=1)
+    ks = np.concatenate([k[:, :127], np.full((50, 1), 3 * math.log(2) * math.sqrt(128.0))], axis=1)
+    ob, _ = oatt.attend_block(qs, ks, v, p_mode="fp8")
+    ks0 = np.concatenate([k[:, :127], np.zeros((50, 1))], axis=1)
+    oa, _ = oatt.attend_block(qs, ks0, v, p_mode="fp8")
+    assert np.allclose(oa, ob, atol=1e-12)
+    # brute force with nearest-search rounding of 2^8 * 2^(t - ceil(max t))
+    vals = omx.e4m3_decode_table()
+    finite = [(c, vals[c]) for c in range(0x7F)]
+    for r in range(3):
+        t = [(q[r] @ k[j]) / math.sqrt(128) / math.log(2) for j in range(50)]
+        ms = math.ceil(max(t))
+        num = np.zeros(128)
+        den = 0.0
+        for j in range(50):
+            u = 2.0 ** (t[j] - ms)
+            den += u
+            target = 256.0 * u
+            best = min(finite, key=lambda cv: (abs(cv[1] - target), cv[0] % 2))
+            num += best[1] / 256.0 * v[j]
+        assert np.allclose(o1[r], num / den, atol=1e-12)
+
+
+def test_fp8_variant_differs_from_plain_on_random_logits():
+    """Negative control: the E4M3 rounding of P is visible on random inputs."""
+    g = np.random.default_rng(9)
+    q, k, v = g.standard_normal((64, 128)), g.standard_normal((512, 128)), g.standard_normal((512, 128))
+    o1, _ = oatt.attend_block(q, k, v, p_mode="exact")
+    o2, _ = oatt.attend_block(q, k, v, p_mode="fp8")
+    rel = np.linalg.norm(o1 - o2) / np.linalg.norm(o1)
+    assert 1e-3 < rel < 0.1
+
+
+def test_attention_rows_matches_full():
+    g = np.random.default_rng(10)
+    lq, lk = [5, 7], [9, 3]
+    q = g.standard_normal((12, 2, 128)); k = g.standard_normal((12, 2, 128)); v = g.standard_normal((12, 2, 128))
+    o, lse = oatt.attention_fwd(q, k, v, lq, lk)
+    rows = [0, 4, 5, 11]
+    seqs = [0, 0, 1, 1]
+    heads = [1, 0, 1, 0]
+    orow, lrow = oatt.attention_rows(q[rows, heads], seqs, heads, k, v, lk)
+    for i, (r, h) in enumerate(zip(rows, heads)):
+        assert np.allclose(orow[i], o[r, h], atol=1e-12)
+        assert np.isclose(lrow[i], lse[h, r], atol=1e-12)
