@@ -1,0 +1,194 @@
+/*
+ * lpfa.h -- C ABI of the block-scaled low-precision FlashAttention forward library
+ * (MXFP8 quantization of packed variable-length Q/K/V followed by a noncausal
+ * head-dim-128 multi-head attention forward with online softmax, BF16 O and fp32 LSE).
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * - All buffers are owned by the caller. The library never allocates device or
+ *   pinned memory. Pointers named *_dev, and every tensor argument, are device
+ *   pointers; lengths_host is a host pointer.
+ * - Work is enqueued asynchronously on `stream` (a cudaStream_t passed as void*;
+ *   NULL is the legacy default stream). Outputs are valid once the stream has
+ *   reached the call. Host arrays are read before the call returns.
+ * - Every call returns an lpfa_status. Nothing is thrown across the ABI. On a
+ *   non-OK status nothing has been enqueued, except for LPFA_ERR_CUDA after a
+ *   launch; lpfa_last_error_message() describes the last failure of the calling
+ *   thread.
+ * - Packed layout: a tensor of T tokens and H heads has shape (T, H, 128); the
+ *   tokens of sequence i are rows [cu_seqlens[i], cu_seqlens[i+1]).
+ * - Only head_dim 128 is supported; any other value returns LPFA_ERR_INVALID_ARG.
+ *
+ * Sources. "LP-FA4 README" is the README of the LP-FA4 low-precision FlashAttention-4
+ * kernels (facebookresearch ads_model_kernel_library, lp_fa4/README.md). "FastVideo
+ * #1654" is the FastVideo pull request "fp8 PV mode for the FA4-FP4 attention path".
+ * "vLLM #63232" is the vLLM pull request "FA4: no FP8 descale for a unit per-tensor
+ * scale".
+ */
+#ifndef LPFA_H
+#define LPFA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__) || defined(__clang__)
+#define LPFA_API __attribute__((visibility("default")))
+#else
+#define LPFA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  LPFA_OK = 0,
+  LPFA_ERR_INVALID_ARG = 1,   /* bad enum, size, pointer, alignment or metadata */
+  LPFA_ERR_UNSUPPORTED = 2,   /* current device is not sm_100 */
+  LPFA_ERR_CUDA = 3,          /* a CUDA runtime call or kernel launch failed */
+  LPFA_ERR_TIMEOUT = 4        /* a kernel gave up waiting on one of its own barriers */
+} lpfa_status;
+
+typedef enum { LPFA_IN_BF16 = 0, LPFA_IN_FP32 = 1 } lpfa_in_dtype;
+typedef enum { LPFA_SCALE_RCEIL = 0, LPFA_SCALE_FLOOR = 1 } lpfa_scaling_mode;
+typedef enum { LPFA_PV_BF16 = 0, LPFA_PV_FP8 = 1 } lpfa_pv_mode;
+
+/*
+ * Packed variable-length metadata (LP-FA4 README, "MXFP8 forward and backward":
+ * Mxfp8VarlenMeta.from_lengths; each sequence gets independent scale storage padded
+ * to a multiple of 128 tokens).
+ *
+ * `dev` points to a caller-owned device int32 buffer of lpfa_meta_dev_ints(num_seqs)
+ * entries holding two arrays of num_seqs + 1 entries each, in this order:
+ *   cu_seqlens[i]   first token of sequence i (cu_seqlens[n] = total_tokens);
+ *   scale_off[i]    first 128-token scale block of sequence i,
+ *                   scale_off[i+1] - scale_off[i] = ceil(len_i / 128). The same prefix
+ *                   numbers the 128-row attention tiles of each sequence.
+ */
+typedef struct {
+  int32_t num_seqs;
+  int32_t total_tokens;
+  int32_t total_scale_blocks;  /* scale_off[num_seqs] */
+  int32_t max_seqlen;
+  int32_t* dev;
+} lpfa_varlen_meta;
+
+/* Number of int32 entries `dev` must hold for num_seqs sequences: 2 * (num_seqs + 1). */
+LPFA_API size_t lpfa_meta_dev_ints(int32_t num_seqs);
+
+/*
+ * Host-only metadata builder: computes the scalar fields of `meta` and writes the two
+ * arrays (layout as for `dev`) into host_ints, which must hold lpfa_meta_dev_ints(num_seqs)
+ * entries. meta->dev is left unchanged. Errors: num_seqs < 1, a length < 1, a total that
+ * overflows int32, or a NULL pointer -> LPFA_ERR_INVALID_ARG.
+ */
+LPFA_API lpfa_status lpfa_varlen_meta_fill_host(const int32_t* lengths_host, int32_t num_seqs,
+                                       int32_t* host_ints, lpfa_varlen_meta* meta);
+
+/*
+ * Mxfp8VarlenMeta.from_lengths (LP-FA4 README, "MXFP8 forward and backward").
+ * On entry meta->dev must point to the caller's device buffer; on return the scalar
+ * fields are set and one host-to-device copy of the arrays is enqueued on `stream`.
+ * Errors as for lpfa_varlen_meta_fill_host, plus LPFA_ERR_INVALID_ARG for meta->dev NULL.
+ */
+LPFA_API lpfa_status lpfa_varlen_meta_from_lengths(const int32_t* lengths_host, int32_t num_seqs,
+                                          lpfa_varlen_meta* meta, void* stream);
+
+/* Bytes of scale storage for one quantized tensor: total_scale_blocks * heads * 512. */
+LPFA_API size_t lpfa_scale_bytes(const lpfa_varlen_meta* meta, int32_t heads);
+
+/*
+ * quantize_mxfp8_varlen (LP-FA4 README, "MXFP8 forward and backward": E4M3 payload plus
+ * one E8M0 scale per 32-element block along head_dim; RCEIL default, FLOOR optional;
+ * per-sequence 128-token-padded scale storage; quantization happens before the kernel).
+ *
+ * x          device, (T, H, 128) values of dtype `dt`; element (t, h, d) is at
+ *            x + t * tok_stride + h * head_stride + d (strides in elements; d is
+ *            contiguous). Values must be finite.
+ * payload    device, (T, H, 128) uint8 E4M3 codes, contiguous.
+ * scales     device, lpfa_scale_bytes(meta, heads) bytes. For sequence i, 128-token block b,
+ *            head h the 512-byte atom at ((scale_off[i] + b) * H + h) * 512 holds the scale
+ *            byte of token row r (0..127) and 32-element block kb (0..3) at
+ *            (r % 32) * 16 + (r / 32) * 4 + kb. Byte = e + 127 for the power of two 2^e.
+ *            Rows past the end of the sequence are written as 0x7F.
+ * Rules:     RCEIL: smallest e with amax <= 448 * 2^e; FLOOR: e = floor(log2 amax) - 8;
+ *            e clamped to [-127, 127]; amax == 0 gives byte 0x00. Payload is
+ *            E4M3(x * 2^-e), round to nearest even, saturating to +-448, sign kept.
+ * Alignment: x 16-byte aligned with tok_stride and head_stride multiples of 8 elements
+ *            (bf16) or 4 elements (fp32); payload 16-byte aligned.
+ * Errors:    LPFA_ERR_INVALID_ARG for NULL pointers, bad enums, head_dim != 128,
+ *            heads < 1, meta without a device buffer, or misalignment.
+ */
+LPFA_API lpfa_status lpfa_quantize_mxfp8_varlen(const void* x, lpfa_in_dtype dt, int64_t tok_stride,
+                                       int64_t head_stride, int32_t heads, int32_t head_dim,
+                                       const lpfa_varlen_meta* meta, lpfa_scaling_mode mode,
+                                       uint8_t* payload, uint8_t* scales, void* stream);
+
+/*
+ * fa4_v_to_fp8 (FastVideo #1654: the fp8 PV mode feeds V as an unscaled E4M3 cast, with no
+ * scale factors and an implicit dequant scale of 1.0).
+ *
+ * v          device, (tokens, H, 128) bf16 with strides as for the quantizer.
+ * out        device, (tokens, H, 128) uint8 E4M3 codes, contiguous; round to nearest even,
+ *            saturating to +-448, sign kept.
+ * Errors:    LPFA_ERR_INVALID_ARG for NULL pointers, tokens < 1, heads < 1,
+ *            head_dim != 128 or misalignment.
+ */
+LPFA_API lpfa_status lpfa_cast_e4m3(const void* v_bf16, int64_t tok_stride, int64_t head_stride,
+                           int64_t tokens, int32_t heads, int32_t head_dim, uint8_t* out,
+                           void* stream);
+
+/*
+ * mxfp8_flash_attn_varlen_forward (LP-FA4 README, "MXFP8 forward and backward": noncausal,
+ * head-dim-128 MHA over packed variable-length sequences, returning out and lse), with the
+ * fp8 PV mode of FastVideo #1654 and the per-tensor descales of vLLM #63232.
+ *
+ * q, q_sf          device, Q payload (Tq, H, 128) and its scale storage under meta_q.
+ * k, k_sf          device, K payload (Tk, H, 128) and its scale storage under meta_k.
+ * v, v_sf          device, V payload (Tk, H, 128). LPFA_PV_BF16: an MXFP8 payload whose scale
+ *                  storage (under meta_k) is v_sf; it is dequantized exactly to BF16 and P is
+ *                  rounded to BF16 for the PV product. LPFA_PV_FP8: unscaled E4M3 codes (see
+ *                  lpfa_cast_e4m3), v_sf must be NULL, P is rounded to E4M3 relative to a
+ *                  power-of-two running maximum.
+ * meta_q, meta_k   sequence i of meta_q attends to sequence i of meta_k (same num_seqs).
+ * q/k/v_descale    device pointers to one float each, or NULL. NULL means exactly 1.0: the
+ *                  kernel then uses the literal 1.0f on the same code path, so a descale of
+ *                  1.0 gives bit-identical output to NULL. Logits are scaled by
+ *                  q_descale * k_descale / sqrt(128), O by v_descale. Values must be finite.
+ * out_bf16         device, (Tq, H, 128) bf16, written for every real token row.
+ * lse              device, (H, Tq) fp32, natural-log logsumexp of the scaled logits.
+ * Alignment:       every tensor 16-byte aligned.
+ * Errors:          LPFA_ERR_INVALID_ARG for NULL required pointers, head_dim != 128,
+ *                  heads < 1, mismatched num_seqs, a bad pv_mode, or a non-NULL v_sf in fp8
+ *                  mode (and NULL v_sf in bf16 mode); LPFA_ERR_UNSUPPORTED off sm_100;
+ *                  LPFA_ERR_CUDA on launch failure. A kernel that gives up on a barrier wait
+ *                  records LPFA_ERR_TIMEOUT in the device status word (see below).
+ */
+LPFA_API lpfa_status lpfa_attn_fwd_varlen(const uint8_t* q, const uint8_t* q_sf, const uint8_t* k,
+                                 const uint8_t* k_sf, const uint8_t* v, const uint8_t* v_sf,
+                                 const lpfa_varlen_meta* meta_q, const lpfa_varlen_meta* meta_k,
+                                 int32_t heads, int32_t head_dim, lpfa_pv_mode pv_mode,
+                                 const float* q_descale, const float* k_descale,
+                                 const float* v_descale, void* out_bf16, float* lse,
+                                 void* stream);
+
+/*
+ * Device status word. Kernels that bound their barrier waits record a failure code in a
+ * library-owned device word instead of hanging. This call synchronizes `stream`, reads the
+ * word of the current device, resets it to zero, and returns LPFA_OK, LPFA_ERR_TIMEOUT, or
+ * LPFA_ERR_CUDA if the synchronization itself failed. *detail (may be NULL) receives the
+ * recorded diagnostic (which wait gave up), 0 if none.
+ */
+LPFA_API lpfa_status lpfa_device_status(void* stream, int32_t* detail);
+
+/* Message describing the last non-OK status returned on the calling thread ("" if none). */
+LPFA_API const char* lpfa_last_error_message(void);
+
+/* Library version string. */
+LPFA_API const char* lpfa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LPFA_H */

@@ -1,0 +1,234 @@
+"""Python binding of liblpfa: MXFP8 varlen quantization and block-scaled attention forward.
+
+Argument marshalling only: every step of the path runs in the library's CUDA kernels
+(``liblpfa.so``, built in-tree for sm_100a). PyTorch provides device memory and streams.
+Importing this package fails if the library has not been built; there is no CPU fallback.
+
+The functions carry the C ABI's names (``include/lpfa.h``); the LP-FA4 README names
+(``Mxfp8VarlenMeta.from_lengths``, ``quantize_mxfp8_varlen``,
+``mxfp8_flash_attn_varlen_forward``) are provided as aliases.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+import numpy as np
+import torch
+
+_PKG_DIR = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG_DIR, "liblpfa.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        "liblpfa.so is not built; run `python -m precision_attention_forward_b200.build` "
+        "(the library has no CPU fallback)")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+LPFA_OK, LPFA_ERR_INVALID_ARG, LPFA_ERR_UNSUPPORTED, LPFA_ERR_CUDA, LPFA_ERR_TIMEOUT = 0, 1, 2, 3, 4
+_STATUS_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "CUDA", 4: "TIMEOUT"}
+IN_DTYPES = {"bf16": 0, "fp32": 1}
+SCALING_MODES = {"rceil": 0, "floor": 1}
+PV_MODES = {"bf16": 0, "fp8": 1}
+
+# Symbols the header declares; the tests check that each one is exported.
+EXPORTED_SYMBOLS = (
+    "lpfa_meta_dev_ints", "lpfa_varlen_meta_fill_host", "lpfa_varlen_meta_from_lengths",
+    "lpfa_scale_bytes", "lpfa_quantize_mxfp8_varlen", "lpfa_cast_e4m3", "lpfa_attn_fwd_varlen",
+    "lpfa_device_status", "lpfa_last_error_message", "lpfa_version",
+)
+
+
+class LpfaError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"lpfa status {_STATUS_NAMES.get(status, status)}: {message}")
+        self.status = status
+
+
+class _Meta(ctypes.Structure):
+    _fields_ = [("num_seqs", ctypes.c_int32), ("total_tokens", ctypes.c_int32),
+                ("total_scale_blocks", ctypes.c_int32), ("max_seqlen", ctypes.c_int32),
+                ("dev", ctypes.c_void_p)]
+
+
+_vp, _i32, _i64, _f32p = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_void_p
+_lib.lpfa_meta_dev_ints.argtypes = [_i32]
+_lib.lpfa_meta_dev_ints.restype = ctypes.c_size_t
+_lib.lpfa_varlen_meta_fill_host.argtypes = [_vp, _i32, _vp, ctypes.POINTER(_Meta)]
+_lib.lpfa_varlen_meta_fill_host.restype = ctypes.c_int
+_lib.lpfa_varlen_meta_from_lengths.argtypes = [_vp, _i32, ctypes.POINTER(_Meta), _vp]
+_lib.lpfa_varlen_meta_from_lengths.restype = ctypes.c_int
+_lib.lpfa_scale_bytes.argtypes = [ctypes.POINTER(_Meta), _i32]
+_lib.lpfa_scale_bytes.restype = ctypes.c_size_t
+_lib.lpfa_quantize_mxfp8_varlen.argtypes = [_vp, ctypes.c_int, _i64, _i64, _i32, _i32, ctypes.POINTER(_Meta),
+                                            ctypes.c_int, _vp, _vp, _vp]
+_lib.lpfa_quantize_mxfp8_varlen.restype = ctypes.c_int
+_lib.lpfa_cast_e4m3.argtypes = [_vp, _i64, _i64, _i64, _i32, _i32, _vp, _vp]
+_lib.lpfa_cast_e4m3.restype = ctypes.c_int
+_lib.lpfa_attn_fwd_varlen.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, ctypes.POINTER(_Meta), ctypes.POINTER(_Meta),
+                                      _i32, _i32, ctypes.c_int, _f32p, _f32p, _f32p, _vp, _vp, _vp]
+_lib.lpfa_attn_fwd_varlen.restype = ctypes.c_int
+_lib.lpfa_device_status.argtypes = [_vp, ctypes.POINTER(_i32)]
+_lib.lpfa_device_status.restype = ctypes.c_int
+_lib.lpfa_last_error_message.argtypes = []
+_lib.lpfa_last_error_message.restype = ctypes.c_char_p
+_lib.lpfa_version.argtypes = []
+_lib.lpfa_version.restype = ctypes.c_char_p
+
+
+def _check(status: int) -> None:
+    if status != LPFA_OK:
+        raise LpfaError(status, _lib.lpfa_last_error_message().decode(errors="replace"))
+
+
+def _stream_ptr(stream) -> Optional[int]:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def lpfa_version() -> str:
+    return _lib.lpfa_version().decode()
+
+
+class VarlenMeta:
+    """Packed varlen metadata: host scalars plus a device int32 buffer (cu_seqlens | scale_off)."""
+
+    def __init__(self, lengths, c_meta: _Meta, dev: Optional[torch.Tensor], host_ints: np.ndarray):
+        self.lengths = np.asarray(lengths, dtype=np.int32)
+        self._c = c_meta
+        self.dev = dev
+        self.host_ints = host_ints
+
+    num_seqs = property(lambda self: self._c.num_seqs)
+    total_tokens = property(lambda self: self._c.total_tokens)
+    total_scale_blocks = property(lambda self: self._c.total_scale_blocks)
+    max_seqlen = property(lambda self: self._c.max_seqlen)
+
+    @property
+    def cu_seqlens(self) -> np.ndarray:
+        return self.host_ints[: self.num_seqs + 1]
+
+    @property
+    def scale_off(self) -> np.ndarray:
+        return self.host_ints[self.num_seqs + 1:]
+
+    def scale_bytes(self, heads: int) -> int:
+        return int(_lib.lpfa_scale_bytes(ctypes.byref(self._c), heads))
+
+    @classmethod
+    def from_lengths(cls, lengths: Sequence[int], device="cuda", stream=None) -> "VarlenMeta":
+        return lpfa_varlen_meta_from_lengths(lengths, device=device, stream=stream)
+
+
+def lpfa_varlen_meta_fill_host(lengths: Sequence[int]) -> VarlenMeta:
+    """Host-only metadata (no device buffer); usable without a GPU."""
+    lens = np.ascontiguousarray(np.asarray(lengths, dtype=np.int32))
+    n = int(lens.size)
+    host = np.zeros(max(int(_lib.lpfa_meta_dev_ints(n)), 1), dtype=np.int32)
+    m = _Meta()
+    _check(_lib.lpfa_varlen_meta_fill_host(lens.ctypes.data if n else None, n, host.ctypes.data, ctypes.byref(m)))
+    return VarlenMeta(lens, m, None, host)
+
+
+def lpfa_varlen_meta_from_lengths(lengths: Sequence[int], device="cuda", stream=None) -> VarlenMeta:
+    lens = np.ascontiguousarray(np.asarray(lengths, dtype=np.int32))
+    n = int(lens.size)
+    host_meta = lpfa_varlen_meta_fill_host(lens)
+    dev = torch.empty(int(_lib.lpfa_meta_dev_ints(n)), dtype=torch.int32, device=device)
+    m = _Meta()
+    m.dev = dev.data_ptr()
+    with torch.cuda.device(dev.device):
+        _check(_lib.lpfa_varlen_meta_from_lengths(lens.ctypes.data, n, ctypes.byref(m), _stream_ptr(stream)))
+    return VarlenMeta(lens, m, dev, host_meta.host_ints)
+
+
+def _strides(x: torch.Tensor):
+    if x.dim() != 3 or x.shape[2] != 128 or x.stride(2) != 1:
+        raise ValueError("expected a (tokens, heads, 128) tensor with a contiguous last dimension")
+    return x.stride(0), x.stride(1)
+
+
+def lpfa_quantize_mxfp8_varlen(x: torch.Tensor, meta: VarlenMeta, scaling_mode: str = "rceil",
+                               payload: Optional[torch.Tensor] = None, scales: Optional[torch.Tensor] = None,
+                               stream=None):
+    """Quantize packed (T, H, 128) bf16/fp32 to (payload uint8 (T,H,128), scales uint8 (blocks*H*512,))."""
+    dt = {torch.bfloat16: "bf16", torch.float32: "fp32"}.get(x.dtype)
+    if dt is None:
+        raise ValueError("x must be bf16 or fp32")
+    if scaling_mode not in SCALING_MODES:
+        raise ValueError("scaling_mode must be 'rceil' or 'floor'")
+    ts, hs = _strides(x)
+    T, H = x.shape[0], x.shape[1]
+    if T != meta.total_tokens:
+        raise ValueError("x has %d tokens but the metadata describes %d" % (T, meta.total_tokens))
+    if payload is None:
+        payload = torch.empty((T, H, 128), dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty(meta.scale_bytes(H), dtype=torch.uint8, device=x.device)
+    with torch.cuda.device(x.device):
+        _check(_lib.lpfa_quantize_mxfp8_varlen(x.data_ptr(), IN_DTYPES[dt], ts, hs, H, 128, ctypes.byref(meta._c),
+                                               SCALING_MODES[scaling_mode], payload.data_ptr(), scales.data_ptr(),
+                                               _stream_ptr(stream)))
+    return payload, scales
+
+
+def lpfa_cast_e4m3(v: torch.Tensor, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Unscaled E4M3 cast of a bf16 (T, H, 128) tensor (fp8 PV mode V)."""
+    if v.dtype != torch.bfloat16:
+        raise ValueError("v must be bf16")
+    ts, hs = _strides(v)
+    T, H = v.shape[0], v.shape[1]
+    if out is None:
+        out = torch.empty((T, H, 128), dtype=torch.uint8, device=v.device)
+    with torch.cuda.device(v.device):
+        _check(_lib.lpfa_cast_e4m3(v.data_ptr(), ts, hs, T, H, 128, out.data_ptr(), _stream_ptr(stream)))
+    return out
+
+
+def lpfa_attn_fwd_varlen(q: torch.Tensor, q_sf: torch.Tensor, k: torch.Tensor, k_sf: torch.Tensor,
+                         v: torch.Tensor, v_sf: Optional[torch.Tensor], meta_q: VarlenMeta, meta_k: VarlenMeta,
+                         pv_mode: str = "bf16", q_descale: Optional[torch.Tensor] = None,
+                         k_descale: Optional[torch.Tensor] = None, v_descale: Optional[torch.Tensor] = None,
+                         out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None, stream=None):
+    """Block-scaled attention forward; returns (out bf16 (Tq,H,128), lse fp32 (H,Tq))."""
+    if pv_mode not in PV_MODES:
+        raise ValueError("pv_mode must be 'bf16' or 'fp8'")
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if t.dtype != torch.uint8 or t.dim() != 3 or not t.is_contiguous():
+            raise ValueError("%s must be a contiguous uint8 (tokens, heads, 128) payload" % name)
+    for name, t in (("q_descale", q_descale), ("k_descale", k_descale), ("v_descale", v_descale)):
+        if t is not None and (t.dtype != torch.float32 or t.numel() != 1):
+            raise ValueError("%s must be a single-element float32 tensor" % name)
+    Tq, H = q.shape[0], q.shape[1]
+    if out is None:
+        out = torch.empty((Tq, H, 128), dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty((H, Tq), dtype=torch.float32, device=q.device)
+    with torch.cuda.device(q.device):
+        _check(_lib.lpfa_attn_fwd_varlen(
+            q.data_ptr(), q_sf.data_ptr(), k.data_ptr(), k_sf.data_ptr(), v.data_ptr(), _ptr(v_sf),
+            ctypes.byref(meta_q._c), ctypes.byref(meta_k._c), H, 128, PV_MODES[pv_mode],
+            _ptr(q_descale), _ptr(k_descale), _ptr(v_descale), out.data_ptr(), lse.data_ptr(),
+            _stream_ptr(stream)))
+    return out, lse
+
+
+def lpfa_device_status(stream=None):
+    """Synchronize `stream` and return (status, detail) of the device status word (then reset)."""
+    detail = _i32(0)
+    st = _lib.lpfa_device_status(_stream_ptr(stream), ctypes.byref(detail))
+    return st, detail.value
+
+
+# LP-FA4 README names.
+Mxfp8VarlenMeta = VarlenMeta
+quantize_mxfp8_varlen = lpfa_quantize_mxfp8_varlen
+mxfp8_flash_attn_varlen_forward = lpfa_attn_fwd_varlen
+fa4_v_to_fp8 = lpfa_cast_e4m3

@@ -1,0 +1,338 @@
+// lpfa.cu -- host side of the C ABI declared in include/lpfa.h: argument validation,
+// packed varlen metadata, TMA tensor maps and kernel launches. All kernels live in the
+// headers included below; this is the library's single translation unit.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdint>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "lpfa.h"
+#include "attn_fwd.cuh"
+#include "quantize.cuh"
+
+namespace {
+
+thread_local char g_msg[512] = "";
+
+lpfa_status fail(lpfa_status st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_msg, sizeof(g_msg), fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+lpfa_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(LPFA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  bool init = false;
+  bool sm100 = false;
+  int sms = 0;
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+// Returns LPFA_OK and fills *info for the current device, or an error status.
+lpfa_status current_device(DeviceInfo* info, int* dev_out = nullptr) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(LPFA_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.init) {
+    int major = 0, minor = 0, sms = 0;
+    if ((e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess)
+      return cuda_fail(e, "cudaDeviceGetAttribute");
+    if ((e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess)
+      return cuda_fail(e, "cudaDeviceGetAttribute");
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+      return cuda_fail(e, "cudaDeviceGetAttribute");
+    d.sm100 = (major == 10 && minor == 0);
+    d.sms = sms;
+    d.init = true;
+  }
+  *info = d;
+  if (dev_out) *dev_out = dev;
+  return LPFA_OK;
+}
+
+lpfa_status require_sm100(DeviceInfo* info) {
+  lpfa_status st = current_device(info);
+  if (st != LPFA_OK) return st;
+  if (!info->sm100) return fail(LPFA_ERR_UNSUPPORTED, "the current device is not sm_100 (B200)");
+  return LPFA_OK;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// Tensor map over a packed (tokens, heads, 128) uint8 payload; box = 128 tokens of one head,
+// 128-byte rows with the 128-byte swizzle the UMMA descriptors expect.
+lpfa_status payload_tmap(CUtensorMap* map, const void* base, int64_t tokens, int heads) {
+  auto fn = encode_fn();
+  if (!fn) return fail(LPFA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(heads), static_cast<cuuint64_t>(tokens)};
+  cuuint64_t strides[2] = {128, static_cast<cuuint64_t>(heads) * 128};
+  cuuint32_t box[3] = {128, 1, 128};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(LPFA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  return LPFA_OK;
+}
+
+lpfa_status check_meta(const lpfa_varlen_meta* m, const char* name) {
+  if (!m) return fail(LPFA_ERR_INVALID_ARG, "%s is NULL", name);
+  if (!m->dev) return fail(LPFA_ERR_INVALID_ARG, "%s has no device buffer", name);
+  if (m->num_seqs < 1 || m->total_tokens < 1 || m->total_scale_blocks < 1)
+    return fail(LPFA_ERR_INVALID_ARG, "%s is empty or was not filled", name);
+  return LPFA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* lpfa_last_error_message(void) { return g_msg; }
+
+const char* lpfa_version(void) { return "lpfa 0.1.0 (sm_100a)"; }
+
+size_t lpfa_meta_dev_ints(int32_t num_seqs) {
+  return num_seqs < 1 ? 0 : 2 * (static_cast<size_t>(num_seqs) + 1);
+}
+
+size_t lpfa_scale_bytes(const lpfa_varlen_meta* meta, int32_t heads) {
+  if (!meta || heads < 1 || meta->total_scale_blocks < 0) return 0;
+  return static_cast<size_t>(meta->total_scale_blocks) * static_cast<size_t>(heads) * 512u;
+}
+
+lpfa_status lpfa_varlen_meta_fill_host(const int32_t* lengths_host, int32_t num_seqs, int32_t* host_ints,
+                                       lpfa_varlen_meta* meta) {
+  if (!lengths_host || !host_ints || !meta) return fail(LPFA_ERR_INVALID_ARG, "NULL argument");
+  if (num_seqs < 1) return fail(LPFA_ERR_INVALID_ARG, "num_seqs must be >= 1 (got %d)", num_seqs);
+  int64_t cu = 0, so = 0;
+  int32_t mx = 0;
+  int32_t* cu_arr = host_ints;
+  int32_t* so_arr = host_ints + num_seqs + 1;
+  cu_arr[0] = 0;
+  so_arr[0] = 0;
+  for (int32_t i = 0; i < num_seqs; ++i) {
+    const int32_t len = lengths_host[i];
+    if (len < 1) return fail(LPFA_ERR_INVALID_ARG, "sequence %d has length %d; lengths must be >= 1", i, len);
+    cu += len;
+    so += (len + 127) / 128;
+    if (cu > INT32_MAX) return fail(LPFA_ERR_INVALID_ARG, "total token count overflows int32");
+    cu_arr[i + 1] = static_cast<int32_t>(cu);
+    so_arr[i + 1] = static_cast<int32_t>(so);
+    if (len > mx) mx = len;
+  }
+  meta->num_seqs = num_seqs;
+  meta->total_tokens = static_cast<int32_t>(cu);
+  meta->total_scale_blocks = static_cast<int32_t>(so);
+  meta->max_seqlen = mx;
+  return LPFA_OK;
+}
+
+lpfa_status lpfa_varlen_meta_from_lengths(const int32_t* lengths_host, int32_t num_seqs, lpfa_varlen_meta* meta,
+                                          void* stream) {
+  if (!meta) return fail(LPFA_ERR_INVALID_ARG, "meta is NULL");
+  if (!meta->dev) return fail(LPFA_ERR_INVALID_ARG, "meta->dev must point to a device buffer");
+  if (num_seqs < 1) return fail(LPFA_ERR_INVALID_ARG, "num_seqs must be >= 1 (got %d)", num_seqs);
+  std::vector<int32_t> host(lpfa_meta_dev_ints(num_seqs));
+  lpfa_varlen_meta tmp = *meta;
+  lpfa_status st = lpfa_varlen_meta_fill_host(lengths_host, num_seqs, host.data(), &tmp);
+  if (st != LPFA_OK) return st;
+  // Pageable source: the runtime stages the bytes before returning, so `host` may go away.
+  cudaError_t e = cudaMemcpyAsync(meta->dev, host.data(), host.size() * sizeof(int32_t), cudaMemcpyHostToDevice,
+                                  static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyAsync(meta)");
+  *meta = tmp;
+  return LPFA_OK;
+}
+
+lpfa_status lpfa_quantize_mxfp8_varlen(const void* x, lpfa_in_dtype dt, int64_t tok_stride, int64_t head_stride,
+                                       int32_t heads, int32_t head_dim, const lpfa_varlen_meta* meta,
+                                       lpfa_scaling_mode mode, uint8_t* payload, uint8_t* scales, void* stream) {
+  if (!x || !payload || !scales) return fail(LPFA_ERR_INVALID_ARG, "NULL tensor pointer");
+  if (dt != LPFA_IN_BF16 && dt != LPFA_IN_FP32) return fail(LPFA_ERR_INVALID_ARG, "invalid input dtype %d", dt);
+  if (mode != LPFA_SCALE_RCEIL && mode != LPFA_SCALE_FLOOR) return fail(LPFA_ERR_INVALID_ARG, "invalid scaling mode %d", mode);
+  if (head_dim != 128) return fail(LPFA_ERR_INVALID_ARG, "head_dim must be 128 (got %d)", head_dim);
+  if (heads < 1) return fail(LPFA_ERR_INVALID_ARG, "heads must be >= 1");
+  lpfa_status st = check_meta(meta, "meta");
+  if (st != LPFA_OK) return st;
+  const int vec = dt == LPFA_IN_BF16 ? 8 : 4;
+  if (!aligned16(x) || !aligned16(payload) || (tok_stride % vec) || (head_stride % vec))
+    return fail(LPFA_ERR_INVALID_ARG, "x/payload must be 16-byte aligned with strides multiple of %d elements", vec);
+  if (!aligned16(scales)) return fail(LPFA_ERR_INVALID_ARG, "scales must be 16-byte aligned");
+  if (heads > 65535) return fail(LPFA_ERR_INVALID_ARG, "at most 65535 heads per launch");
+  DeviceInfo info;
+  if ((st = require_sm100(&info)) != LPFA_OK) return st;
+  lpfa::QuantParams p;
+  p.x = x;
+  p.tok_stride = tok_stride;
+  p.head_stride = head_stride;
+  p.heads = heads;
+  p.num_seqs = meta->num_seqs;
+  p.cu_seqlens = meta->dev;
+  p.scale_off = meta->dev + meta->num_seqs + 1;
+  p.payload = payload;
+  p.scales = scales;
+  p.floor_mode = mode == LPFA_SCALE_FLOOR ? 1 : 0;
+  dim3 grid(meta->total_scale_blocks, heads);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (dt == LPFA_IN_BF16)
+    lpfa::quantize_mxfp8_kernel<__nv_bfloat16><<<grid, lpfa::kQuantThreads, 0, s>>>(p);
+  else
+    lpfa::quantize_mxfp8_kernel<float><<<grid, lpfa::kQuantThreads, 0, s>>>(p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "quantize launch");
+  return LPFA_OK;
+}
+
+lpfa_status lpfa_cast_e4m3(const void* v_bf16, int64_t tok_stride, int64_t head_stride, int64_t tokens,
+                           int32_t heads, int32_t head_dim, uint8_t* out, void* stream) {
+  if (!v_bf16 || !out) return fail(LPFA_ERR_INVALID_ARG, "NULL tensor pointer");
+  if (head_dim != 128) return fail(LPFA_ERR_INVALID_ARG, "head_dim must be 128 (got %d)", head_dim);
+  if (tokens < 1 || heads < 1) return fail(LPFA_ERR_INVALID_ARG, "tokens and heads must be >= 1");
+  if (!aligned16(v_bf16) || !aligned16(out) || (tok_stride % 8) || (head_stride % 8))
+    return fail(LPFA_ERR_INVALID_ARG, "v/out must be 16-byte aligned with strides multiple of 8 elements");
+  DeviceInfo info;
+  lpfa_status st = require_sm100(&info);
+  if (st != LPFA_OK) return st;
+  lpfa::CastParams p;
+  p.v = static_cast<const __nv_bfloat16*>(v_bf16);
+  p.tok_stride = tok_stride;
+  p.head_stride = head_stride;
+  p.rows = tokens * heads;
+  p.heads = heads;
+  p.out = out;
+  const int64_t lanes = p.rows * 16;
+  int64_t blocks = (lanes + 255) / 256;
+  const int64_t cap = static_cast<int64_t>(info.sms) * 16;
+  if (blocks > cap) blocks = cap;
+  lpfa::cast_e4m3_kernel<<<static_cast<unsigned>(blocks), 256, 0, static_cast<cudaStream_t>(stream)>>>(p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "cast launch");
+  return LPFA_OK;
+}
+
+// Internal entry shared with the test hook: debug_stall > 0 forces a bounded wait to run out.
+static lpfa_status attn_fwd_impl(const uint8_t* q, const uint8_t* q_sf, const uint8_t* k, const uint8_t* k_sf,
+                                 const uint8_t* v, const uint8_t* v_sf, const lpfa_varlen_meta* meta_q,
+                                 const lpfa_varlen_meta* meta_k, int32_t heads, int32_t head_dim,
+                                 lpfa_pv_mode pv_mode, const float* q_descale, const float* k_descale,
+                                 const float* v_descale, void* out_bf16, float* lse, void* stream,
+                                 int debug_stall) {
+  if (!q || !q_sf || !k || !k_sf || !v || !out_bf16 || !lse) return fail(LPFA_ERR_INVALID_ARG, "NULL tensor pointer");
+  if (pv_mode != LPFA_PV_BF16 && pv_mode != LPFA_PV_FP8) return fail(LPFA_ERR_INVALID_ARG, "invalid pv_mode %d", pv_mode);
+  if (pv_mode == LPFA_PV_FP8 && v_sf) return fail(LPFA_ERR_INVALID_ARG, "fp8 PV mode takes no V scale factors (v_sf must be NULL)");
+  if (pv_mode == LPFA_PV_BF16 && !v_sf) return fail(LPFA_ERR_INVALID_ARG, "bf16 PV mode needs the V scale factors (v_sf)");
+  if (head_dim != 128) return fail(LPFA_ERR_INVALID_ARG, "head_dim must be 128 (got %d)", head_dim);
+  if (heads < 1) return fail(LPFA_ERR_INVALID_ARG, "heads must be >= 1");
+  lpfa_status st;
+  if ((st = check_meta(meta_q, "meta_q")) != LPFA_OK) return st;
+  if ((st = check_meta(meta_k, "meta_k")) != LPFA_OK) return st;
+  if (meta_q->num_seqs != meta_k->num_seqs)
+    return fail(LPFA_ERR_INVALID_ARG, "meta_q has %d sequences but meta_k has %d", meta_q->num_seqs, meta_k->num_seqs);
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(q_sf) || !aligned16(k_sf) ||
+      (v_sf && !aligned16(v_sf)) || !aligned16(out_bf16) || !aligned16(lse))
+    return fail(LPFA_ERR_INVALID_ARG, "all tensors must be 16-byte aligned");
+  const int64_t units = static_cast<int64_t>(heads) * meta_q->total_scale_blocks;
+  if (units > INT32_MAX) return fail(LPFA_ERR_INVALID_ARG, "too many query tiles");
+  DeviceInfo info;
+  if ((st = require_sm100(&info)) != LPFA_OK) return st;
+
+  CUtensorMap tq, tk, tv;
+  if ((st = payload_tmap(&tq, q, meta_q->total_tokens, heads)) != LPFA_OK) return st;
+  if ((st = payload_tmap(&tk, k, meta_k->total_tokens, heads)) != LPFA_OK) return st;
+  if ((st = payload_tmap(&tv, v, meta_k->total_tokens, heads)) != LPFA_OK) return st;
+
+  lpfa::AttnParams p;
+  p.q_sf = q_sf;
+  p.k_sf = k_sf;
+  p.v_sf = v_sf;
+  p.cu_q = meta_q->dev;
+  p.so_q = meta_q->dev + meta_q->num_seqs + 1;
+  p.cu_k = meta_k->dev;
+  p.so_k = meta_k->dev + meta_k->num_seqs + 1;
+  p.q_descale = q_descale;
+  p.k_descale = k_descale;
+  p.v_descale = v_descale;
+  p.out = static_cast<__nv_bfloat16*>(out_bf16);
+  p.lse = lse;
+  p.num_seqs = meta_q->num_seqs;
+  p.heads = heads;
+  p.tq = meta_q->total_tokens;
+  p.total_q_tiles = meta_q->total_scale_blocks;
+  p.num_units = static_cast<int>(units);
+  p.debug_stall = debug_stall;
+
+  const int grid = static_cast<int>(units < info.sms ? units : info.sms);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  if (pv_mode == LPFA_PV_FP8) {
+    e = cudaFuncSetAttribute(lpfa::attn_fwd_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, lpfa::kAttnSmemBytes);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+    lpfa::attn_fwd_kernel<true><<<grid, lpfa::kAttnThreads, lpfa::kAttnSmemBytes, s>>>(tq, tk, tv, p);
+  } else {
+    e = cudaFuncSetAttribute(lpfa::attn_fwd_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, lpfa::kAttnSmemBytes);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+    lpfa::attn_fwd_kernel<false><<<grid, lpfa::kAttnThreads, lpfa::kAttnSmemBytes, s>>>(tq, tk, tv, p);
+  }
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "attention launch");
+  return LPFA_OK;
+}
+
+lpfa_status lpfa_attn_fwd_varlen(const uint8_t* q, const uint8_t* q_sf, const uint8_t* k, const uint8_t* k_sf,
+                                 const uint8_t* v, const uint8_t* v_sf, const lpfa_varlen_meta* meta_q,
+                                 const lpfa_varlen_meta* meta_k, int32_t heads, int32_t head_dim,
+                                 lpfa_pv_mode pv_mode, const float* q_descale, const float* k_descale,
+                                 const float* v_descale, void* out_bf16, float* lse, void* stream) {
+  return attn_fwd_impl(q, q_sf, k, k_sf, v, v_sf, meta_q, meta_k, heads, head_dim, pv_mode, q_descale, k_descale,
+                       v_descale, out_bf16, lse, stream, 0);
+}
+
+lpfa_status lpfa_device_status(void* stream, int32_t* detail) {
+  if (detail) *detail = 0;
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  int32_t word[2] = {0, 0};
+  e = cudaMemcpyFromSymbol(word, lpfa::g_lpfa_status, sizeof(word));
+  if (e != cudaSuccess) return cuda_fail(e, "reading the device status word");
+  if (word[0] != 0) {
+    const int32_t zero[2] = {0, 0};
+    e = cudaMemcpyToSymbol(lpfa::g_lpfa_status, zero, sizeof(zero));
+    if (e != cudaSuccess) return cuda_fail(e, "resetting the device status word");
+    if (detail) *detail = word[1];
+    return fail(LPFA_ERR_TIMEOUT, "a kernel gave up waiting on a barrier (site %d)", word[1]);
+  }
+  return LPFA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,176 @@
+"""Attention forward parity on the GPU against the fp64 oracle.
+
+Tolerances: O max-abs 2e-2 and rel-L2 1e-2 (oracle before BF16 rounding), LSE max-abs 1e-3.
+bf16 PV mode is compared with the plain definition; fp8 PV mode with the oracle's fp8-P
+grading variant (P rounded to E4M3 against a power-of-two reference).
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import workloads as wl
+from oracle import attention as oatt
+from tests import gpu_util as gu
+
+pytestmark = pytest.mark.gpu
+
+if torch.cuda.is_available():
+    import precision_attention_forward_b200 as lp
+
+
+def _status_ok():
+    st, detail = lp.lpfa_device_status()
+    assert st == lp.LPFA_OK, f"device status {st} (site {detail})"
+
+
+CASES = [
+    # (lens_q, lens_k, heads)
+    ([1], [1], 1),
+    ([5], [5], 2),
+    ([128], [128], 2),
+    ([129], [129], 1),
+    ([256], [256], 2),
+    ([300, 77, 1], [300, 77, 1], 3),
+    ([200], [1000], 2),                 # cross attention, several KV tiles
+    ([64, 700], [513, 129], 2),         # cross varlen with ragged tails
+]
+
+
+@pytest.mark.parametrize("pv_mode", ["bf16", "fp8"])
+@pytest.mark.parametrize("case", range(len(CASES)))
+def test_attention_small_cases(pv_mode, case):
+    lq, lk, H = CASES[case]
+    q, k, v = wl.small_random(100 + case, lq, lk, H)
+    if pv_mode == "fp8":
+        v = v * np.float32(2.0)
+    o, lse = gu.run_path(lp, q, k, v, lq, lk, H, pv_mode=pv_mode)
+    _status_ok()
+    o_ref, lse_ref = gu.oracle_full(q, k, v, lq, lk, H, pv_mode=pv_mode)
+    gu.assert_within(gu.compare_attention(o, lse, o_ref, lse_ref), f"{pv_mode} {lq}/{lk} H={H}")
+
+
+def test_attention_fp32_inputs():
+    lq = lk = [333]
+    q, k, v = wl.small_random(7, lq, lk, 2, dtype="fp32")
+    o, lse = gu.run_path(lp, q, k, v, lq, lk, 2, in_dtype="fp32")
+    o_ref, lse_ref = gu.oracle_full(q, k, v, lq, lk, 2)
+    gu.assert_within(gu.compare_attention(o, lse, o_ref, lse_ref), "fp32 inputs")
+
+
+@pytest.mark.parametrize("pv_mode", ["bf16", "fp8"])
+def test_closed_forms(pv_mode):
+    """Constant V gives V (bf16 PV) or V times one scalar per row (fp8 PV, where l sums the
+    unrounded weights); equal logits give LSE = ln n + s and O = the mean of V."""
+    H, n = 2, 300
+    g = np.random.default_rng(3)
+    q = wl.round_to_bf16(g.standard_normal((n, H, 128)).astype(np.float32))
+    krow = wl.round_to_bf16(g.standard_normal((1, H, 128)).astype(np.float32))
+    k = np.repeat(krow, n, axis=0)
+    v = wl.round_to_bf16(g.standard_normal((n, H, 128)).astype(np.float32))
+    vconst = np.repeat(v[:1], n, axis=0)
+    krand = wl.round_to_bf16(g.standard_normal((n, H, 128)).astype(np.float32))
+    # constant V (random keys)
+    o, lse = gu.run_path(lp, q, krand, vconst, [n], [n], H, pv_mode=pv_mode)
+    qh, kh, vh = gu.oracle_inputs(q, krand, vconst, [n], [n], H, pv_mode)
+    o_np = o.float().cpu().numpy().astype(np.float64)
+    if pv_mode == "bf16":
+        assert np.max(np.abs(o_np - vh[:1])) <= gu.O_MAX_ABS
+    else:
+        ratio = (o_np * vh[:1]).sum(axis=2) / (vh[:1] ** 2).sum(axis=2)      # (n, H)
+        assert np.all(np.abs(ratio - 1.0) < 0.02)
+        assert np.max(np.abs(o_np - ratio[..., None] * vh[:1])) <= gu.O_MAX_ABS / 2
+    # equal logits: all keys identical
+    o, lse = gu.run_path(lp, q, k, v, [n], [n], H, pv_mode=pv_mode)
+    qh, kh, vh = gu.oracle_inputs(q, k, v, [n], [n], H, pv_mode)
+    s = np.einsum("thd,hd->ht", qh, kh[0]) / math.sqrt(128)
+    assert np.max(np.abs(lse.cpu().numpy() - (np.log(n) + s))) < gu.LSE_MAX_ABS
+    if pv_mode == "bf16":
+        assert np.max(np.abs(o.float().cpu().numpy() - vh.mean(axis=0)[None])) <= gu.O_MAX_ABS
+
+
+def test_single_key():
+    q, k, v = wl.small_random(5, [77], [1], 2)
+    o, lse = gu.run_path(lp, q, k, v, [77], [1], 2)
+    qh, kh, vh = gu.oracle_inputs(q, k, v, [77], [1], 2)
+    assert np.max(np.abs(o.float().cpu().numpy() - vh[:1])) <= gu.O_MAX_ABS
+    s = np.einsum("thd,hd->ht", qh, kh[0]) / math.sqrt(128)
+    assert np.max(np.abs(lse.cpu().numpy() - s)) < gu.LSE_MAX_ABS
+
+
+@pytest.mark.parametrize("pv_mode", ["bf16", "fp8"])
+def test_unit_descale_is_bit_identical_and_two_changes_output(pv_mode):
+    """vLLM #63232 'Validation': absent descale == unit descale bit for bit; 2 changes it."""
+    w = wl.WORKLOADS["dense_4x2048_h16"]
+    lq, lk = wl.lengths(w)
+    q, k, v = (wl.make_tensor(w, x) for x in "qkv")
+    if pv_mode == "fp8":
+        v = v * np.float32(2.0)
+    o0, l0 = gu.run_path(lp, q, k, v, lq, lk, w.heads, pv_mode=pv_mode)
+    o1, l1 = gu.run_path(lp, q, k, v, lq, lk, w.heads, pv_mode=pv_mode, descales=(1.0, 1.0, 1.0))
+    assert torch.equal(o0.view(torch.int16), o1.view(torch.int16))
+    assert torch.equal(l0.view(torch.int32), l1.view(torch.int32))
+    o2, l2 = gu.run_path(lp, q, k, v, lq, lk, w.heads, pv_mode=pv_mode, descales=(2.0, 1.0, 1.0))
+    assert not torch.equal(o0, o2) and not torch.equal(l0, l2)
+    o3, l3 = gu.run_path(lp, q, k, v, lq, lk, w.heads, pv_mode=pv_mode, descales=(1.0, 1.0, 2.0))
+    assert not torch.equal(o0, o3)
+    _status_ok()
+
+
+@pytest.mark.parametrize("descales", [(2.0, 1.0, 1.0), (0.5, 3.0, 0.25), (-1.0, 1.0, 1.0), (1.0, 1.0, -2.0)])
+def test_descale_values_match_oracle(descales):
+    lq = lk = [400]
+    q, k, v = wl.small_random(17, lq, lk, 2)
+    o, lse = gu.run_path(lp, q, k, v, lq, lk, 2, descales=descales)
+    o_ref, lse_ref = gu.oracle_full(q, k, v, lq, lk, 2, descales=descales)
+    gu.assert_within(gu.compare_attention(o, lse, o_ref, lse_ref), f"descales {descales}")
+
+
+def test_negative_control_wrong_k_scales_fail():
+    """Scale bytes of K raised by one (K doubled) must fail the tolerance."""
+    lq = lk = [512]
+    q, k, v = wl.small_random(23, lq, lk, 2)
+    mq = lp.lpfa_varlen_meta_from_lengths(lq)
+    mk = lp.lpfa_varlen_meta_from_lengths(lk)
+    qp, qs = gu.gpu_quantize(lp, q, "bf16", mq)
+    kp, ks = gu.gpu_quantize(lp, k, "bf16", mk)
+    vp, vs = gu.gpu_quantize(lp, v, "bf16", mk)
+    o, lse = lp.lpfa_attn_fwd_varlen(qp, qs, kp, ks + 1, vp, vs, mq, mk)
+    o_ref, lse_ref = gu.oracle_full(q, k, v, lq, lk, 2)
+    max_abs, rel, lmax = gu.compare_attention(o, lse, o_ref, lse_ref)
+    assert lmax > gu.LSE_MAX_ABS and rel > gu.O_REL_L2
+
+
+@pytest.mark.parametrize("name", ["single_s256_h2", "dense_4x2048_h16"])
+@pytest.mark.parametrize("mode", ["rceil", "floor"])
+def test_workload_full_check(name, mode):
+    w = wl.WORKLOADS[name]
+    lq, lk = wl.lengths(w)
+    q, k, v = (wl.make_tensor(w, x) for x in "qkv")
+    o, lse = gu.run_path(lp, q, k, v, lq, lk, w.heads, in_dtype=w.in_dtype, pv_mode=w.pv_mode, mode=mode)
+    _status_ok()
+    o_ref, lse_ref = gu.oracle_full(q, k, v, lq, lk, w.heads, pv_mode=w.pv_mode, mode=mode)
+    print(gu.assert_within(gu.compare_attention(o, lse, o_ref, lse_ref), f"{name} {mode}"))
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name", ["varlen16_fp32_h16", "video_s32768_h24_fp8pv", "cross_varlen_outliers_h32"])
+def test_workload_sampled_check(name):
+    """Full-size run in the benchmarked launch configuration, checked on sampled rows that
+    cover every (sequence, head), each 128-row tile and every tail."""
+    w = wl.WORKLOADS[name]
+    lq, lk = wl.lengths(w)
+    q, k, v = (wl.make_tensor(w, x) for x in "qkv")
+    o, lse = gu.run_path(lp, q, k, v, lq, lk, w.heads, in_dtype=w.in_dtype, pv_mode=w.pv_mode)
+    _status_ok()
+    toks, hs = gu.sample_rows(lq, w.heads, seed=11, per_tile_random=0 if name.startswith("video") else 1)
+    if name.startswith("video"):
+        # 24 heads x 256 tiles: keep the oracle bounded to every 8th tile plus all edges.
+        keep = (toks % 1024 < 128) | (toks == toks.max())
+        toks, hs = toks[keep], hs[keep]
+    o_ref, lse_ref = gu.oracle_sampled(q, k, v, lq, lk, w.heads, toks, hs, pv_mode=w.pv_mode)
+    tt, hh = torch.from_numpy(toks).cuda(), torch.from_numpy(hs).cuda()
+    o_s = o[tt, hh]
+    lse_s = lse[hh, tt]
+    print(gu.assert_within(gu.compare_attention(o_s, lse_s, o_ref, lse_ref), f"{name} sampled"))
