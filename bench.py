@@ -1,0 +1,403 @@
+#!/usr/bin/env python3
+"""Benchmark of the MXFP8 attention forward hot path on B200.
+
+One step is one pass of the whole path over one batch of synthetic input already resident
+in HBM: varlen metadata, MXFP8 quantization of Q and K (and V in bf16 PV mode), the
+unscaled E4M3 cast of V (fp8 PV mode), and the attention forward. `value` is attention
+TFLOPS (sum of 4 * Sq * Sk * H * 128 over sequences, every rank) divided by the step time;
+the `roofline` object reports the attention kernel alone against the measured dense FP8
+peak, and `e2e` repeats the step with host buffers (pinned H2D of Q/K/V, D2H of O/LSE).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+For N > 1 run under torch.distributed.run: every rank processes its own copy of the
+workload (weak scaling; sequences and heads are independent, so there is no collective on
+the data path). `--impl reference` times the CPU oracle on a bounded sample instead.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as wl  # noqa: E402
+
+DEFAULT_WORKLOAD = "video_s32768_h24_fp8pv"
+METRIC = "MXFP8 attn-fwd TFLOPS (4*Sq*Sk*H*d) & % of dense FP8 peak; quantize GB/s"
+NOMINAL_FP8_TFLOPS = 4500.0          # dense, per GPU (context)
+FP8_OVER_BF16 = 2.0                  # nominal dense FP8 / BF16 tensor ratio
+FALLBACK_BF16_BURST = 1590.0         # used only when MEASURED_PEAKS.json is absent
+FALLBACK_HBM_GBS = 6650.0
+
+# DRAM traffic of one attention launch, from an ncu capture of the same command (see
+# profiles/attn_fwd_video_s32768_h24_fp8pv.md). Valid only for the kernel source whose
+# hash is recorded; any change to the kernel makes it null until re-captured.
+TRAFFIC = {
+    # workload: (sha256 of attn_fwd.cuh [:16], dram bytes read + written per launch)
+    "video_s32768_h24_fp8pv": ("b55837f60148cd68", 310.329088e6 + 176.407552e6),
+}
+
+
+def kernel_hash() -> str:
+    path = os.path.join(ROOT, "precision_attention_forward_b200", "csrc", "attn_fwd.cuh")
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except (OSError, ValueError):
+        return {"hbm_gbs": FALLBACK_HBM_GBS, "bf16_tflops": FALLBACK_BF16_BURST}, "fallback"
+
+
+def attention_flops(lq, lk, heads) -> float:
+    return float(sum(4.0 * a * b * heads * 128 for a, b in zip(lq, lk)))
+
+
+def quantizer_bytes(tokens, heads, in_bytes, scale_blocks) -> float:
+    return float(tokens) * heads * 128 * (in_bytes + 1) + float(scale_blocks) * heads * 512
+
+
+class ClockSampler:
+    """Samples nvidia-smi SM clocks and throttle reasons in the background."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.t = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.t = threading.Thread(target=self._read, daemon=True)
+        self.t.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.t:
+            self.t.join(timeout=2)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def cpu_oracle_sample(w, seconds: float, seed: int = 0):
+    """Time the CPU oracle on a bounded sample of the workload: for one head at a time,
+    quantize that head's K and V (or cast V), quantize a block of query rows, and run the
+    fp64 attention of those rows over all keys. Returns (tflops, desc, cores, elapsed)."""
+    from oracle import attention as oatt
+    from oracle import mxfp8 as omx
+
+    lq, lk = wl.lengths(w)
+    q = wl.make_tensor(w, "q")
+    k = wl.make_tensor(w, "k")
+    v = wl.make_tensor(w, "v")
+    cu_q = np.concatenate([[0], np.cumsum(lq)])
+    cu_k = np.concatenate([[0], np.cumsum(lk)])
+    rows_per = 128
+    done_flops = 0.0
+    units = 0
+    t0 = time.perf_counter()
+    while time.perf_counter() - t0 < seconds:
+        i = units % len(lq)
+        h = (units // len(lq)) % w.heads
+        k0, k1 = cu_k[i], cu_k[i + 1]
+        kp, ke = omx.quantize_rows(k[k0:k1, h].astype(np.float64), w.scaling_mode)
+        kh = (omx.e4m3_decode(kp).reshape(-1, 4, 32) * np.ldexp(1.0, ke)[..., None]).reshape(-1, 128)
+        if w.pv_mode == "fp8":
+            vh = omx.e4m3_decode(omx.cast_e4m3(v[k0:k1, h]))
+        else:
+            vp, ve = omx.quantize_rows(v[k0:k1, h].astype(np.float64), w.scaling_mode)
+            vh = (omx.e4m3_decode(vp).reshape(-1, 4, 32) * np.ldexp(1.0, ve)[..., None]).reshape(-1, 128)
+        r0 = cu_q[i] + (units * rows_per) % max(1, lq[i] - rows_per + 1)
+        r1 = min(cu_q[i + 1], r0 + rows_per)
+        qp, qe = omx.quantize_rows(q[r0:r1, h].astype(np.float64), w.scaling_mode)
+        qh = (omx.e4m3_decode(qp).reshape(-1, 4, 32) * np.ldexp(1.0, qe)[..., None]).reshape(-1, 128)
+        oatt.attend_block(qh, kh, vh, p_mode="fp8" if w.pv_mode == "fp8" else "exact")
+        done_flops += 4.0 * (r1 - r0) * (k1 - k0) * 128
+        units += 1
+    elapsed = time.perf_counter() - t0
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([d.get("num_threads", 1) for d in threadpool_info()] + [1])
+    except Exception:  # pragma: no cover
+        cores = os.cpu_count() or 1
+    desc = (f"{units} units of {rows_per} query rows x all keys of one (sequence, head), each with that "
+            f"head's K/V quantization, fp64 numpy oracle")
+    return done_flops / elapsed / 1e12, desc, cores, elapsed
+
+
+def run_reference(args, w):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    lq, lk = wl.lengths(w)
+    per_step = max(1.0, float(os.environ.get("LPFA_REF_STEP_SECONDS", "3.0")))
+    for _ in range(args.warmup):
+        cpu_oracle_sample(w, per_step)
+    vals, times, descs, cores = [], [], None, 1
+    for _ in range(args.steps):
+        tf, desc, cores, el = cpu_oracle_sample(w, per_step)
+        vals.append(tf)
+        times.append(el)
+        descs = desc
+    value = statistics.median(vals)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * statistics.mean(times),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": config_dict(w, lq, lk, args.gpus),
+        "cpu_baseline": {"value": value, "unit": "TFLOPS", "cores": cores, "kind": "oracle", "sample": descs},
+        "e2e": {"value": value, "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_dict(w, lq, lk, n):
+    return {
+        "workload": w.name, "description": w.description, "num_seqs": int(w.num_seqs),
+        "seq_len_q": int(max(lq)), "seq_len_k": int(max(lk)), "total_tokens_q": int(np.sum(lq)),
+        "total_tokens_k": int(np.sum(lk)), "heads": w.heads, "head_dim": 128, "pv_mode": w.pv_mode,
+        "in_dtype": w.in_dtype, "scaling_mode": w.scaling_mode, "global_batch": int(w.num_seqs) * n,
+        "parallelism": f"replicas{n}" if n > 1 else "single",
+        "l2": "inputs larger than L2 (no flush)" if np.sum(lk) * w.heads * 128 * 2 > 126e6
+              else "L2 flushed between steps",
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(wl.WORKLOADS))
+    ap.add_argument("--impl", default="lpfa", choices=["lpfa", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "lpfa":
+        sys.stderr.write("note: fewer than 3 warm-up steps; numbers are for smoke use only\n")
+    w = wl.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, w)
+
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local_rank)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local_rank))
+
+    import precision_attention_forward_b200 as lp
+
+    dev = torch.device("cuda", local_rank)
+    stream = torch.cuda.current_stream()
+    lq, lk = wl.lengths(w)
+    H = w.heads
+    flops = attention_flops(lq, lk, H)
+
+    # Inputs, resident in HBM.
+    host = {x: wl.make_tensor(w, x) for x in "qkv"}
+    dts = {x: wl.tensor_dtype(w, x) for x in "qkv"}
+    dev_in = {x: wl.to_torch(host[x], dts[x], device=dev) for x in "qkv"}
+    Tq, Tk = int(np.sum(lq)), int(np.sum(lk))
+    mq0 = lp.lpfa_varlen_meta_from_lengths(lq, device=dev)
+    sbq, sbk = mq0.total_scale_blocks, lp.lpfa_varlen_meta_from_lengths(lk, device=dev).total_scale_blocks
+    qp = torch.empty((Tq, H, 128), dtype=torch.uint8, device=dev)
+    kp = torch.empty((Tk, H, 128), dtype=torch.uint8, device=dev)
+    vp = torch.empty((Tk, H, 128), dtype=torch.uint8, device=dev)
+    qs = torch.empty(sbq * H * 512, dtype=torch.uint8, device=dev)
+    ks = torch.empty(sbk * H * 512, dtype=torch.uint8, device=dev)
+    vs = None if w.pv_mode == "fp8" else torch.empty(sbk * H * 512, dtype=torch.uint8, device=dev)
+    out = torch.empty((Tq, H, 128), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((H, Tq), dtype=torch.float32, device=dev)
+
+    def step(ins, timing=None):
+        mq = lp.lpfa_varlen_meta_from_lengths(lq, device=dev)
+        mk = lp.lpfa_varlen_meta_from_lengths(lk, device=dev)
+        if timing is not None:
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+        lp.lpfa_quantize_mxfp8_varlen(ins["q"], mq, w.scaling_mode, payload=qp, scales=qs)
+        lp.lpfa_quantize_mxfp8_varlen(ins["k"], mk, w.scaling_mode, payload=kp, scales=ks)
+        if w.pv_mode == "fp8":
+            lp.lpfa_cast_e4m3(ins["v"], out=vp)
+        else:
+            lp.lpfa_quantize_mxfp8_varlen(ins["v"], mk, w.scaling_mode, payload=vp, scales=vs)
+        if timing is not None:
+            c = torch.cuda.Event(enable_timing=True)
+            c.record(stream)
+        lp.lpfa_attn_fwd_varlen(qp, qs, kp, ks, vp, vs, mq, mk, pv_mode=w.pv_mode, out=out, lse=lse)
+        if timing is not None:
+            b.record(stream)
+            timing.append((a, c, b))
+        return 4  # kernels launched
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    smi_index = int(vis.split(",")[local_rank]) if vis and vis.split(",")[local_rank].strip().isdigit() else local_rank
+    sampler = ClockSampler(smi_index)
+    sampler.start()
+    for _ in range(args.warmup):
+        step(dev_in)
+    barrier()
+    timing = []
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    launches = 0
+    start.record(stream)
+    for _ in range(args.steps):
+        launches += step(dev_in, timing)
+    end.record(stream)
+    barrier()
+    clocks = sampler.stop()
+    total_ms = max_over_ranks(start.elapsed_time(end))
+    quant_ms = sum(a.elapsed_time(c) for a, c, b in timing) / args.steps
+    attn_ms = sum(c.elapsed_time(b) for a, c, b in timing) / args.steps
+    attn_ms = max_over_ranks(attn_ms)
+    quant_ms = max_over_ranks(quant_ms)
+    st, detail = lp.lpfa_device_status()
+    if st != lp.LPFA_OK:
+        raise RuntimeError(f"kernel reported status {st} (site {detail})")
+
+    ms_per_step = total_ms / args.steps
+    value = flops * world / (ms_per_step * 1e-3) / 1e12
+
+    # End to end through the public API with host buffers.
+    e2e = None
+    if not args.no_e2e:
+        pinned = {x: dev_in[x].cpu().pin_memory() for x in "qkv"}
+        o_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        l_host = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+        scratch = {x: torch.empty_like(dev_in[x]) for x in "qkv"}
+        h2d = sum(t.numel() * t.element_size() for t in pinned.values()) + 2 * 4 * (len(lq) + 1) * 2
+        d2h = o_host.numel() * o_host.element_size() + l_host.numel() * l_host.element_size()
+
+        def e2e_step():
+            for x in "qkv":
+                scratch[x].copy_(pinned[x], non_blocking=True)
+            step(scratch)
+            o_host.copy_(out, non_blocking=True)
+            l_host.copy_(lse, non_blocking=True)
+
+        for _ in range(max(1, args.warmup // 2)):
+            e2e_step()
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ne = max(3, args.steps // 2)
+        e0.record(stream)
+        for _ in range(ne):
+            e2e_step()
+        e1.record(stream)
+        barrier()
+        e_ms = max_over_ranks(e0.elapsed_time(e1)) / ne
+        e2e = {"value": flops * world / (e_ms * 1e-3) / 1e12, "unit": "TFLOPS", "ms_per_step": e_ms,
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+
+    peaks, peak_src = load_peaks()
+    # The attention kernel runs at full SM clock (it is not power capped like a dense GEMM), so
+    # the burst GEMM figure is the denominator: the larger, more conservative of the two.
+    fp8_peak = peaks.get("bf16_tflops", FALLBACK_BF16_BURST) * FP8_OVER_BF16
+    achieved = flops / (attn_ms * 1e-3) / 1e12
+    tr = TRAFFIC.get(w.name)
+    traffic = tr[1] if tr and tr[0] == kernel_hash() else None
+    qbytes = quantizer_bytes(Tq, H, 2 if dts["q"] == "bf16" else 4, sbq) + \
+        quantizer_bytes(Tk, H, 2 if dts["k"] == "bf16" else 4, sbk) + \
+        (Tk * H * 128 * 3.0 if w.pv_mode == "fp8" else quantizer_bytes(Tk, H, 2 if dts["v"] == "bf16" else 4, sbk))
+
+    if rank == 0:
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            tf, desc, cores, el = cpu_oracle_sample(w, float(os.environ.get("LPFA_CPU_SECONDS", "15")))
+            cpu = {"value": tf, "unit": "TFLOPS", "cores": cores, "kind": "oracle", "sample": desc,
+                   "seconds": el}
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "e4m3", "data": "synthetic",
+            "config": config_dict(w, lq, lk, world),
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": fp8_peak, "unit": "TFLOP/s",
+                         "frac": achieved / fp8_peak, "traffic": traffic,
+                         "peak_source": f"{peak_src} bf16 burst x {FP8_OVER_BF16:g} (nominal FP8/BF16 ratio)",
+                         "kernel": "attn_fwd_kernel", "flops_per_launch": flops},
+            "attn_kernel_ms": attn_ms,
+            "attn_pct_nominal_fp8": 100.0 * achieved / NOMINAL_FP8_TFLOPS,
+            "quantize": {"ms_per_step": quant_ms, "bytes_per_step": qbytes,
+                         "gbs": qbytes / (quant_ms * 1e-3) / 1e9,
+                         "frac_hbm": qbytes / (quant_ms * 1e-3) / 1e9 / peaks.get("hbm_gbs", FALLBACK_HBM_GBS)},
+            "e2e": e2e,
+            "gpu_launches": launches,
+            "clocks": clocks,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -24,10 +24,7 @@ LSE_MAX_ABS = 1e-3
 
 def to_device(x: np.ndarray, dtype: str, device="cuda") -> torch.Tensor:
     """Upload a float32 array as bf16 (exact values required) or fp32."""
-    if dtype == "bf16":
-        bits = wl.bf16_bits(x)
-        return torch.from_numpy(bits.view(np.int16)).to(device).view(torch.bfloat16)
-    return torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).to(device)
+    return wl.to_torch(x, dtype, device)
 
 
 def gpu_quantize(lp, x: np.ndarray, dtype: str, meta, mode="rceil"):

@@ -177,6 +177,15 @@ def tensor_dtype(w: Workload, which: str) -> str:
     return w.in_dtype
 
 
+def to_torch(x: np.ndarray, dtype: str, device="cuda"):
+    """Upload a float32 array to a torch device tensor as bf16 (values must be exact) or fp32."""
+    import torch
+
+    if dtype == "bf16":
+        return torch.from_numpy(bf16_bits(x).view(np.int16)).to(device).view(torch.bfloat16)
+    return torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).to(device)
+
+
 def small_random(seed: int, lengths_q, lengths_k, heads: int, scale: float = 1.0,
                  dtype: str = "bf16"):
     """Free-form seeded Q/K/V for edge-case tests (ragged lengths, few heads)."""
