@@ -13,24 +13,31 @@
 // running at the same time stream the same K/V through L2.
 //
 // Warp roles (512 threads):
-//   warp 0        TMA producer: Q tile + its scale atom, then K/V tiles (+ atoms) in the
-//                 order the MMA warp consumes them (K0, K1, V0, K2, V1, ...).
-//   warp 1        TMEM allocator and single-thread MMA issuer:
-//                   S[b] = Q K_j^T   tcgen05.mma kind::mxf8f6f4.block_scale (scales in TMEM)
-//                   O   += P_j V_j   tcgen05.mma kind::f16 (bf16 PV) or kind::f8f6f4 (fp8 PV)
-//                                    with P read from TMEM (it overwrites S in place).
+//   warp 0        TMA producer (whole warp, one lane issues): the Q tile + its scale atom once
+//                 per unit, then 128-key K/V tiles (+ atoms) in the order the MMA warp uses them
+//                 (K0, K1, V0, K2, V1, ...).
+//   warp 1        TMEM allocator and MMA issuer (whole warp, one lane issues):
+//                   S[b] = Q K_j^T   tcgen05.mma kind::mxf8f6f4.block_scale, M128 N128 K128
+//                   O   += P_j V_j   kind::f16 (bf16 PV) or kind::f8f6f4 (fp8 PV), P from TMEM
+//                 S is double buffered, so S(j+1) is computed while the softmax of S(j) runs.
+//                 A block-scaled MMA costs about as much issue time at N=64 as at N=128, so the
+//                 key tile is 128 wide.
 //   warps 4..7    softmax group 0: rows 0..127 of the tile, keys 0..63 of every S tile.
-//   warps 8..11   softmax group 1: the same rows, keys 64..127. The two groups exchange
-//                 row maxima through shared memory once per tile.
+//   warps 8..11   softmax group 1: the same rows, keys 64..127. The groups exchange row maxima
+//                 through shared memory once per tile, after computing their exponentials.
 //   warps 12..15  bf16 PV mode only: convert the V tile from MXFP8 to BF16 in shared memory.
 //
-// Online softmax keeps the running maximum m as an integer in log2 units (ceil of the
-// scaled row maximum), so every rescale factor 2^(m_old - m_new) is an exact power of two,
-// and rescaling of the O accumulator is needed only when the ceiling moves. In fp8 PV mode
-// P is stored as E4M3(2^8 * 2^(t - m)); the factor 2^8 cancels in the final division.
+// Online softmax keeps a reference m (an integer, log2 units) per row, shared by both
+// groups. Exponentials are computed against the current reference (or the group's own
+// ceiling if its keys exceed the reference by more than the lag) before the other group's
+// maximum arrives; the two groups then agree on the new reference and scale their P by an
+// exact power of two if it moved. The reference rises only when a tile exceeds it by more
+// than the lag, so rescaling of l and O is rare. In fp8 PV mode P is stored as
+// E4M3(2^(8 - lag) * 2^(t - m)) <= 256; the power of two cancels in the final division.
 //
-// TMEM columns (512 allocated): S/P buffer 0 [0,128), S/P buffer 1 [128,256), O [256,384),
-// Q scales (2 stages) [384,392), K scales (2 slots) [392,400).
+// TMEM columns (512 allocated): S buffer b at [128b, 128b + 128) (group g reads columns
+// [64g, 64g + 64) and writes its P over the first of them), O [256,384), Q scale atoms (2
+// stages) [384,392), K scale atoms (2 slots) [392,400).
 #pragma once
 
 #include <cstdint>
@@ -46,20 +53,21 @@ namespace lpfa {
 __device__ int g_lpfa_status[2];  // [0] = lpfa_status code of a failed kernel, [1] = detail
 
 constexpr int kAttnThreads = 512;
-constexpr int kTileM = 128;
-constexpr int kTileN = 128;
+constexpr int kTileM = 128;          // query rows per tile
+constexpr int kTileN = 128;          // keys per KV tile
 constexpr int kQStages = 2;
 constexpr int kKStages = 3;
 constexpr int kVStages = 3;
 constexpr int kVbfStages = 2;
-constexpr uint32_t kTileBytes = 128 * 128;  // one 128 x 128 fp8 tile
+constexpr uint32_t kTileBytes = 128 * 128;     // 128 rows x 128 fp8
+constexpr uint32_t kVbfBytes = 128 * 128 * 2;  // 128 keys x 128 bf16
 constexpr uint32_t kAtomBytes = 512;
 
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS0 = 0;
-constexpr uint32_t kColO = 256;
-constexpr uint32_t kColSFA = 384;
-constexpr uint32_t kColSFB = 392;
+constexpr uint32_t kColS = 0;        // + 128 * b  S buffer (fp32), P written over its columns
+constexpr uint32_t kColO = 256;      // O accumulator (fp32)
+constexpr uint32_t kColSFA = 384;    // + 4 * stage  Q scale atom
+constexpr uint32_t kColSFB = 392;    // + 4 * slot   K scale atom
 
 // log2(e) / sqrt(128) rounded to fp32: logits in log2 units per unit of Q.K.
 constexpr float kLog2eRsqrtD = 0.12751743082459868f;
@@ -98,14 +106,14 @@ struct SmemLayout {
   static constexpr uint32_t q = 0;
   static constexpr uint32_t k = q + kQStages * kTileBytes;
   static constexpr uint32_t v = k + kKStages * kTileBytes;
-  static constexpr uint32_t vbf = v + kVStages * kTileBytes;         // 2 x 32 KB (bf16 mode)
-  static constexpr uint32_t q_sf = vbf + kVbfStages * 2 * kTileBytes;
+  static constexpr uint32_t vbf = v + kVStages * kTileBytes;          // bf16 PV mode
+  static constexpr uint32_t q_sf = vbf + kVbfStages * kVbfBytes;
   static constexpr uint32_t k_sf = q_sf + kQStages * kAtomBytes;
   static constexpr uint32_t v_sf = k_sf + kKStages * kAtomBytes;
-  static constexpr uint32_t red = v_sf + kVStages * kAtomBytes;      // float [2 groups][2 slots][128]
+  static constexpr uint32_t red = v_sf + kVStages * kAtomBytes;       // float [2 groups][2 slots][128]
   static constexpr uint32_t lsum = red + 2 * 2 * 128 * 4;             // float [2 groups][128]
   static constexpr uint32_t bars = lsum + 2 * 128 * 4;                // uint64 barriers
-  static constexpr uint32_t num_bars = 32;
+  static constexpr uint32_t num_bars = 40;
   static constexpr uint32_t misc = bars + num_bars * 8;               // tmem base, abort flag
   static constexpr uint32_t total = misc + 64;
 };
@@ -115,7 +123,7 @@ constexpr uint32_t kAttnSmemBytes = SmemLayout::total + 1024;  // + alignment sl
 enum Bar : int {
   kBarQFull = 0, kBarQEmpty = 2, kBarKFull = 4, kBarKEmpty = 7, kBarVFull = 10, kBarVEmpty = 13,
   kBarVbfFull = 16, kBarVbfEmpty = 18, kBarSFull = 20, kBarPReady = 22, kBarRed = 24,
-  kBarPVDone = 26, kBarOEmpty = 27, kBarLReady = 28, kBarDrain = 29
+  kBarPVDone = 26, kBarOEmpty = 27, kBarLReady = 28, kBarDrain = 29, kBarOFull = 30
 };
 
 // UMMA shared-memory matrix descriptor (sm_100 format, version 1).
@@ -132,12 +140,108 @@ constexpr uint32_t kLayoutNone = 0;
 // Block-scaled E4M3 x E4M3 -> F32, M=128, N=128, both operands K-major, E8M0 scales.
 __device__ __forceinline__ uint32_t idesc_qk(int kb, int negate_a) {
   return (static_cast<uint32_t>(kb) << 4) | (static_cast<uint32_t>(negate_a) << 13) |
-         (16u << 17) | (1u << 23) | (8u << 24) | (static_cast<uint32_t>(kb) << 29);
+         ((kTileN >> 3) << 17) | (1u << 23) | (8u << 24) | (static_cast<uint32_t>(kb) << 29);
 }
 // E4M3 x E4M3 -> F32, M=128, N=128, A (P) K-major in TMEM, B (V) MN-major.
 constexpr uint32_t kIdescPV8 = (1u << 4) | (1u << 16) | (16u << 17) | (8u << 24);
 // BF16 x BF16 -> F32, M=128, N=128, A (P) K-major in TMEM, B (V) MN-major.
 constexpr uint32_t kIdescPV16 = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) | (16u << 17) | (8u << 24);
+
+// ---------------------------------------------------------------------------------------
+// Softmax helpers (one thread = one query row, 64 keys of an S tile held as 32 float2)
+// ---------------------------------------------------------------------------------------
+// Pairs of S elements, out of every 8, whose exp2 runs on the FMA pipe (polynomial) instead
+// of the MUFU unit. MUFU alone delivers 16 exp2 per clock per SM, half of what the FP8 tensor
+// core would need; moving part of the work to the FMA pipe balances the two.
+#ifndef LPFA_POLY_PAIRS
+#define LPFA_POLY_PAIRS 0
+#endif
+constexpr int kPolyPairs = LPFA_POLY_PAIRS;
+
+// 2^f on [-0.5, 0.5]: minimax-in-relative-error cubic, float32 coefficients produced by
+// csrc/exp2_poly_fit.py (max relative error 7.5e-5 in float32 Horner form).
+constexpr float kExp2P0 = 0.9999280571937561f;
+constexpr float kExp2P1 = 0.6932609677314758f;
+constexpr float kExp2P2 = 0.2426111251115799f;
+constexpr float kExp2P3 = 0.0551716685295105f;
+
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// 2^k for an integer-valued k <= 0 (or -inf), exactly; 0 below the normal range.
+__device__ __forceinline__ float exp2_int(float k) {
+  return k < -126.0f ? 0.0f : __uint_as_float(static_cast<uint32_t>(static_cast<int>(k) + 127) << 23);
+}
+
+__device__ __forceinline__ float2 exp2_mufu2(float2 x) {
+  return make_float2(ex2_approx(x.x), ex2_approx(x.y));
+}
+
+// 2^x = 2^j * q(x - j), j = round(x) by the 1.5 * 2^23 magic add; the exponent of q is
+// raised by j with one integer add on the bit pattern. x is clamped at -126 (results below
+// that are treated as zero downstream).
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  x.x = fmaxf(x.x, -126.0f);
+  x.y = fmaxf(x.y, -126.0f);
+  const float2 t = __fadd2_rn(x, make_float2(12582912.0f, 12582912.0f));
+  const float2 jf = __fadd2_rn(t, make_float2(-12582912.0f, -12582912.0f));
+  const float2 f = __ffma2_rn(jf, make_float2(-1.0f, -1.0f), x);
+  float2 q = __ffma2_rn(make_float2(kExp2P3, kExp2P3), f, make_float2(kExp2P2, kExp2P2));
+  q = __ffma2_rn(q, f, make_float2(kExp2P1, kExp2P1));
+  q = __ffma2_rn(q, f, make_float2(kExp2P0, kExp2P0));
+  return make_float2(__uint_as_float(__float_as_uint(q.x) + (__float_as_uint(t.x) << 23)),
+                     __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(t.y) << 23)));
+}
+
+__device__ __forceinline__ void load_s(uint32_t taddr, float2 (&s)[32]) {
+  uint32_t ra[32], rb[32];
+  tmem_ld64_sync(taddr, ra, rb);
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    s[i] = make_float2(__uint_as_float(ra[2 * i]), __uint_as_float(ra[2 * i + 1]));
+    s[16 + i] = make_float2(__uint_as_float(rb[2 * i]), __uint_as_float(rb[2 * i + 1]));
+  }
+}
+
+__device__ __forceinline__ void mask_keys(float2 (&s)[32], int key0, int klen) {
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    if (key0 + 2 * i >= klen) s[i].x = -INFINITY;
+    if (key0 + 2 * i + 1 >= klen) s[i].y = -INFINITY;
+  }
+}
+
+__device__ __forceinline__ float rowmax64(const float2 (&s)[32]) {
+  float a[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k)
+    a[k] = max3f(max3f(s[4 * k].x, s[4 * k].y, s[4 * k + 1].x), max3f(s[4 * k + 1].y, s[4 * k + 2].x, s[4 * k + 2].y),
+                 fmaxf(s[4 * k + 3].x, s[4 * k + 3].y));
+  return max3f(max3f(a[0], a[1], a[2]), max3f(a[3], a[4], a[5]), fmaxf(a[6], a[7]));
+}
+
+// p = 2^(s * c + nb) in place; masked keys (tail tiles) become exactly 0. Returns sum of p.
+template <bool kTail, int kPoly>
+__device__ __forceinline__ float exp_tile(float2 (&s)[32], float c, float nb, int key0, int klen) {
+  const float2 c2 = make_float2(c, c), nb2 = make_float2(nb, nb);
+  float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const float2 x = __ffma2_rn(s[i], c2, nb2);
+    float2 e = ((i & 7) < kPoly) ? exp2_poly2(x) : exp2_mufu2(x);
+    if (kTail) {
+      if (key0 + 2 * i >= klen) e.x = 0.0f;
+      if (key0 + 2 * i + 1 >= klen) e.y = 0.0f;
+    }
+    s[i] = e;
+    acc[i & 3] = __fadd2_rn(acc[i & 3], e);
+  }
+  const float2 t = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
+  return t.x + t.y;
+}
 
 struct UnitInfo {
   int h, seq, qtile, q_row0, q_len, k_row0, k_len, nkv, sbq, sbk;
@@ -169,10 +273,45 @@ __device__ __forceinline__ UnitInfo unit_info(const AttnParams& p, int w) {
   return u;
 }
 
+// Warp-uniform copies of values that every lane of a warp computes identically. Results of
+// warp votes and reductions live in uniform registers, which lets the compiler keep the
+// producer and MMA loops (trip counts, stage indices, descriptors) on the uniform datapath;
+// otherwise every tcgen05.mma operand would need a per-instruction register conversion.
+__device__ __forceinline__ int warp_uniform(int x) {
+  return static_cast<int>(__reduce_max_sync(0xFFFFFFFFu, static_cast<unsigned>(x)));
+}
+
+__device__ __forceinline__ UnitInfo warp_uniform(const UnitInfo& u) {
+  UnitInfo r;
+  r.h = warp_uniform(u.h);
+  r.seq = warp_uniform(u.seq);
+  r.qtile = warp_uniform(u.qtile);
+  r.q_row0 = warp_uniform(u.q_row0);
+  r.q_len = warp_uniform(u.q_len);
+  r.k_row0 = warp_uniform(u.k_row0);
+  r.k_len = warp_uniform(u.k_len);
+  r.nkv = warp_uniform(u.nkv);
+  r.sbq = warp_uniform(u.sbq);
+  r.sbk = warp_uniform(u.sbk);
+  return r;
+}
+
+// mbar_wait by a whole warp, with a warp-uniform result.
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, const volatile int* abort) {
+  return __all_sync(0xFFFFFFFFu, mbar_wait(bar, parity, abort));
+}
+
 __device__ __forceinline__ void record_failure(volatile int* abort_flag, int site) {
   *abort_flag = 1;
   if (atomicCAS(&g_lpfa_status[0], 0, 4 /* LPFA_ERR_TIMEOUT */) == 0) atomicExch(&g_lpfa_status[1], site);
 }
+
+// How far (log2 units) a row's logits may exceed its reference before the reference, P, l
+// and O are rescaled, and the power of two P is stored with. bf16 P keeps its 8-bit
+// mantissa at any scale, so it may lag 8 binades; fp8 P stores 2^(8 - lag) * p <= 256 < 448.
+template <bool kFp8PV> struct SoftmaxLag;
+template <> struct SoftmaxLag<true> { static constexpr float lag = 2.0f; static constexpr float bias = 6.0f; };
+template <> struct SoftmaxLag<false> { static constexpr float lag = 8.0f; static constexpr float bias = 0.0f; };
 
 template <bool kFp8PV>
 __global__ void __launch_bounds__(kAttnThreads, 1)
@@ -203,6 +342,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
       mbar_init(&bars[kBarRed + i], 8);
     }
     mbar_init(&bars[kBarPVDone], 1);
+    mbar_init(&bars[kBarOFull], 1);
     mbar_init(&bars[kBarOEmpty], 8);
     mbar_init(&bars[kBarLReady], 8);
     mbar_init(&bars[kBarDrain], 1);
@@ -224,146 +364,155 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      uint32_t u = 0, qc = 0, kc = 0, vc = 0;  // units, and fills issued per ring
-      bool ok = true;
-      auto load_v = [&](const UnitInfo& ui, int jj) -> bool {
-        const uint32_t s = vc % kVStages, ph = (vc / kVStages) & 1;
-        if (!mbar_wait(&bars[kBarVEmpty + s], ph ^ 1, abort_flag)) { record_failure(abort_flag, kSiteProducerV); return false; }
-        mbar_arrive_expect_tx(&bars[kBarVFull + s], kTileBytes + (kFp8PV ? 0 : kAtomBytes));
-        tma_load_3d(smem + SmemLayout::v + s * kTileBytes, &tmap_v, &bars[kBarVFull + s], 0, ui.h, ui.k_row0 + jj * kTileN);
-        if (!kFp8PV)
-          bulk_load(smem + SmemLayout::v_sf + s * kAtomBytes,
-                    p.v_sf + (static_cast<int64_t>(ui.sbk + jj) * p.heads + ui.h) * kAtomBytes, kAtomBytes,
-                    &bars[kBarVFull + s]);
-        ++vc;
-        return true;
-      };
-      for (int w = blockIdx.x; w < p.num_units && ok; w += G, ++u) {
-        const UnitInfo ui = unit_info(p, w);
-        const uint32_t qs = qc % kQStages, qph = (qc / kQStages) & 1;
-        if (!mbar_wait(&bars[kBarQEmpty + qs], qph ^ 1, abort_flag)) { record_failure(abort_flag, kSiteProducerQ); ok = false; break; }
-        mbar_arrive_expect_tx(&bars[kBarQFull + qs], kTileBytes + kAtomBytes);
-        tma_load_3d(smem + SmemLayout::q + qs * kTileBytes, &tmap_q, &bars[kBarQFull + qs], 0, ui.h, ui.q_row0);
-        bulk_load(smem + SmemLayout::q_sf + qs * kAtomBytes,
-                  p.q_sf + (static_cast<int64_t>(ui.sbq + ui.qtile) * p.heads + ui.h) * kAtomBytes, kAtomBytes,
-                  &bars[kBarQFull + qs]);
-        ++qc;
-        for (int j = 0; j < ui.nkv && ok; ++j) {
-          const uint32_t s = kc % kKStages, ph = (kc / kKStages) & 1;
-          if (!mbar_wait(&bars[kBarKEmpty + s], ph ^ 1, abort_flag)) { record_failure(abort_flag, kSiteProducerK); ok = false; break; }
-          mbar_arrive_expect_tx(&bars[kBarKFull + s], kTileBytes + kAtomBytes);
-          tma_load_3d(smem + SmemLayout::k + s * kTileBytes, &tmap_k, &bars[kBarKFull + s], 0, ui.h, ui.k_row0 + j * kTileN);
-          bulk_load(smem + SmemLayout::k_sf + s * kAtomBytes,
-                    p.k_sf + (static_cast<int64_t>(ui.sbk + j) * p.heads + ui.h) * kAtomBytes, kAtomBytes,
-                    &bars[kBarKFull + s]);
-          ++kc;
-          if (j >= 1) ok = load_v(ui, j - 1);
-        }
-        if (ok) ok = load_v(ui, ui.nkv - 1);
+    // The whole warp runs the loop (warp-uniform state); lane 0 issues the copies.
+    const uint32_t leader = lane == 0 ? 1u : 0u;
+    uint32_t qc = 0, kc = 0, vc = 0;  // fills issued per ring
+    bool ok = true;
+    auto load_v = [&](const UnitInfo& ui, int jj) -> bool {
+      const uint32_t s = vc % kVStages, ph = (vc / kVStages) & 1;
+      if (!mbar_wait_warp(&bars[kBarVEmpty + s], ph ^ 1, abort_flag)) { record_failure(abort_flag, kSiteProducerV); return false; }
+      mbar_arrive_expect_tx(&bars[kBarVFull + s], kTileBytes + (kFp8PV ? 0 : kAtomBytes), leader);
+      tma_load_3d(smem + SmemLayout::v + s * kTileBytes, &tmap_v, &bars[kBarVFull + s], 0, ui.h,
+                  ui.k_row0 + jj * kTileN, leader);
+      if (!kFp8PV)
+        bulk_load(smem + SmemLayout::v_sf + s * kAtomBytes,
+                  p.v_sf + (static_cast<int64_t>(ui.sbk + jj) * p.heads + ui.h) * kAtomBytes, kAtomBytes,
+                  &bars[kBarVFull + s], leader);
+      ++vc;
+      return true;
+    };
+    for (int w = blockIdx.x; w < p.num_units && ok; w += G) {
+      const UnitInfo ui = warp_uniform(unit_info(p, w));
+      if (ui.nkv == 0) continue;  // no keys: the softmax warps write the empty-sum result
+      const uint32_t qs = qc % kQStages, qph = (qc / kQStages) & 1;
+      if (!mbar_wait_warp(&bars[kBarQEmpty + qs], qph ^ 1, abort_flag)) { record_failure(abort_flag, kSiteProducerQ); ok = false; break; }
+      mbar_arrive_expect_tx(&bars[kBarQFull + qs], kTileBytes + kAtomBytes, leader);
+      tma_load_3d(smem + SmemLayout::q + qs * kTileBytes, &tmap_q, &bars[kBarQFull + qs], 0, ui.h, ui.q_row0, leader);
+      bulk_load(smem + SmemLayout::q_sf + qs * kAtomBytes,
+                p.q_sf + (static_cast<int64_t>(ui.sbq + ui.qtile) * p.heads + ui.h) * kAtomBytes, kAtomBytes,
+                &bars[kBarQFull + qs], leader);
+      ++qc;
+      for (int j = 0; j < ui.nkv && ok; ++j) {
+        const uint32_t s = kc % kKStages, ph = (kc / kKStages) & 1;
+        if (!mbar_wait_warp(&bars[kBarKEmpty + s], ph ^ 1, abort_flag)) { record_failure(abort_flag, kSiteProducerK); ok = false; break; }
+        mbar_arrive_expect_tx(&bars[kBarKFull + s], kTileBytes + kAtomBytes, leader);
+        tma_load_3d(smem + SmemLayout::k + s * kTileBytes, &tmap_k, &bars[kBarKFull + s], 0, ui.h,
+                    ui.k_row0 + j * kTileN, leader);
+        bulk_load(smem + SmemLayout::k_sf + s * kAtomBytes,
+                  p.k_sf + (static_cast<int64_t>(ui.sbk + j) * p.heads + ui.h) * kAtomBytes, kAtomBytes,
+                  &bars[kBarKFull + s], leader);
+        ++kc;
+        if (j >= 1) ok = load_v(ui, j - 1);
       }
-      // Drain: every copy issued here must land before the CTA exits. The newest fill of each
-      // stage is the last one issued into it; older fills of that stage were consumed already.
-      for (uint32_t i = (qc > kQStages ? qc - kQStages : 0); i < qc; ++i)
-        if (!mbar_wait(&bars[kBarQFull + i % kQStages], (i / kQStages) & 1, nullptr)) record_failure(abort_flag, kSiteDrain);
-      for (uint32_t i = (kc > kKStages ? kc - kKStages : 0); i < kc; ++i)
-        if (!mbar_wait(&bars[kBarKFull + i % kKStages], (i / kKStages) & 1, nullptr)) record_failure(abort_flag, kSiteDrain);
-      for (uint32_t i = (vc > kVStages ? vc - kVStages : 0); i < vc; ++i)
-        if (!mbar_wait(&bars[kBarVFull + i % kVStages], (i / kVStages) & 1, nullptr)) record_failure(abort_flag, kSiteDrain);
+      if (ok) ok = load_v(ui, ui.nkv - 1);
     }
+    // Drain: every copy issued here must land before the CTA exits. The newest fill of each
+    // stage is the last one issued into it; older fills of that stage were consumed already.
+    for (uint32_t i = (qc > kQStages ? qc - kQStages : 0); i < qc; ++i)
+      if (!mbar_wait(&bars[kBarQFull + i % kQStages], (i / kQStages) & 1, nullptr)) record_failure(abort_flag, kSiteDrain);
+    for (uint32_t i = (kc > kKStages ? kc - kKStages : 0); i < kc; ++i)
+      if (!mbar_wait(&bars[kBarKFull + i % kKStages], (i / kKStages) & 1, nullptr)) record_failure(abort_flag, kSiteDrain);
+    for (uint32_t i = (vc > kVStages ? vc - kVStages : 0); i < vc; ++i)
+      if (!mbar_wait(&bars[kBarVFull + i % kVStages], (i / kVStages) & 1, nullptr)) record_failure(abort_flag, kSiteDrain);
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      const float qd = p.q_descale ? __ldg(p.q_descale) : 1.0f;
-      const float kd = p.k_descale ? __ldg(p.k_descale) : 1.0f;
-      const int negate = (qd * kd) < 0.0f ? 1 : 0;
-      const uint32_t sm_q = smem_u32(smem + SmemLayout::q);
-      const uint32_t sm_k = smem_u32(smem + SmemLayout::k);
-      const uint32_t sm_v = smem_u32(smem + SmemLayout::v);
-      const uint32_t sm_vbf = smem_u32(smem + SmemLayout::vbf);
-      const uint32_t sm_qsf = smem_u32(smem + SmemLayout::q_sf);
-      const uint32_t sm_ksf = smem_u32(smem + SmemLayout::k_sf);
-      uint32_t u = 0, kc = 0, vc = 0, sc = 0;
-      bool ok = true;
-      if (p.debug_stall > 0) {
-        // Test hook: wait for a phase of the drain barrier that nothing completes before the
-        // drain below, so the wait runs out and the failure path is exercised.
-        if (!mbar_wait(&bars[kBarDrain], 0, abort_flag)) { record_failure(abort_flag, kSiteDebugStall); ok = false; }
-      }
-      // Issue O += P V for S tile `tile_sc` (tile jj of the current unit).
-      auto issue_pv = [&](uint32_t tile_sc, int jj) -> bool {
-        const uint32_t b = tile_sc & 1;
-        if (!mbar_wait(&bars[kBarPReady + b], (tile_sc >> 1) & 1, abort_flag)) { record_failure(abort_flag, kSiteMmaP); return false; }
-        if (jj == 0) {
-          if (!mbar_wait(&bars[kBarOEmpty], (u & 1) ^ 1, abort_flag)) { record_failure(abort_flag, kSiteMmaO); return false; }
-        }
-        const uint32_t p_col = tmem + kColS0 + b * 128;
-        if (kFp8PV) {
-          const uint32_t s = vc % kVStages, ph = (vc / kVStages) & 1;
-          if (!mbar_wait(&bars[kBarVFull + s], ph, abort_flag)) { record_failure(abort_flag, kSiteMmaV); return false; }
-          tc_fence_after();
-          const uint32_t vbase = sm_v + s * kTileBytes;
+    // The whole warp runs the loop (warp-uniform state); lane 0 issues the tcgen05 instructions.
+    const uint32_t leader = lane == 0 ? 1u : 0u;
+    const float qd = p.q_descale ? __ldg(p.q_descale) : 1.0f;
+    const float kd = p.k_descale ? __ldg(p.k_descale) : 1.0f;
+    const int negate = (qd * kd) < 0.0f ? 1 : 0;
+    // Descriptor bases; the start-address field is the low 14 bits (address >> 4), so a byte
+    // offset b inside shared memory advances a descriptor by b >> 4.
+    const uint64_t dq0 = umma_desc(smem_u32(smem + SmemLayout::q), 16, 1024, kLayoutSw128);
+    const uint64_t dk0 = umma_desc(smem_u32(smem + SmemLayout::k), 16, 1024, kLayoutSw128);
+    const uint64_t dv0 = kFp8PV ? umma_desc(smem_u32(smem + SmemLayout::v), kTileBytes, 1024, kLayoutSw128)
+                                : umma_desc(smem_u32(smem + SmemLayout::vbf), kTileBytes, 1024, kLayoutSw128);
+    const uint64_t dqsf0 = umma_desc(smem_u32(smem + SmemLayout::q_sf), 0, 128, kLayoutNone);
+    const uint64_t dksf0 = umma_desc(smem_u32(smem + SmemLayout::k_sf), 0, 128, kLayoutNone);
+    uint32_t idq[4];
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t bdesc = umma_desc(vbase + kk * 4096, kTileBytes, 1024, kLayoutSw128);
-            mma_f8f6f4_ts(tmem + kColO, p_col + kk * 8, bdesc, kIdescPV8, (jj > 0 || kk > 0) ? 1u : 0u);
-          }
-          mma_commit(&bars[kBarVEmpty + s]);
-        } else {
-          const uint32_t s = vc % kVbfStages, ph = (vc / kVbfStages) & 1;
-          if (!mbar_wait(&bars[kBarVbfFull + s], ph, abort_flag)) { record_failure(abort_flag, kSiteMmaV); return false; }
-          tc_fence_after();
-          const uint32_t vbase = sm_vbf + s * 2 * kTileBytes;
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint64_t bdesc = umma_desc(vbase + kk * 2048, kTileBytes, 1024, kLayoutSw128);
-            mma_f16_ts(tmem + kColO, p_col + kk * 8, bdesc, kIdescPV16, (jj > 0 || kk > 0) ? 1u : 0u);
-          }
-          mma_commit(&bars[kBarVbfEmpty + s]);
-        }
-        mma_commit(&bars[kBarPVDone]);
-        ++vc;
-        return true;
-      };
-      for (int w = blockIdx.x; w < p.num_units && ok; w += G, ++u) {
-        const UnitInfo ui = unit_info(p, w);
-        const uint32_t qs = u % kQStages, qph = (u / kQStages) & 1;
-        if (!mbar_wait(&bars[kBarQFull + qs], qph, abort_flag)) { record_failure(abort_flag, kSiteMmaQ); ok = false; break; }
-        tc_fence_after();
-        const uint32_t sfa = tmem + kColSFA + qs * 4;
-        tmem_cp_32x128b_x4(sfa, umma_desc(sm_qsf + qs * kAtomBytes, 0, 128, kLayoutNone));
-        const uint32_t qbase = sm_q + qs * kTileBytes;
-        for (int j = 0; j < ui.nkv; ++j) {
-          const uint32_t s = kc % kKStages, ph = (kc / kKStages) & 1;
-          if (!mbar_wait(&bars[kBarKFull + s], ph, abort_flag)) { record_failure(abort_flag, kSiteMmaK); ok = false; break; }
-          tc_fence_after();
-          const uint32_t sfb = tmem + kColSFB + (kc & 1) * 4;
-          tmem_cp_32x128b_x4(sfb, umma_desc(sm_ksf + s * kAtomBytes, 0, 128, kLayoutNone));
-          const uint32_t kbase = sm_k + s * kTileBytes;
-          const uint32_t d_col = tmem + kColS0 + (sc & 1) * 128;
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t adesc = umma_desc(qbase + kk * 32, 16, 1024, kLayoutSw128);
-            const uint64_t bdesc = umma_desc(kbase + kk * 32, 16, 1024, kLayoutSw128);
-            const uint32_t byte_sel = static_cast<uint32_t>(kk) << 30;
-            mma_mxf8f6f4_ss(d_col, adesc, bdesc, idesc_qk(kk, negate), sfa | byte_sel, sfb | byte_sel, kk > 0 ? 1u : 0u);
-          }
-          mma_commit(&bars[kBarSFull + (sc & 1)]);
-          mma_commit(&bars[kBarKEmpty + s]);
-          if (j == ui.nkv - 1) mma_commit(&bars[kBarQEmpty + qs]);
-          ++kc;
-          if (j >= 1 && !issue_pv(sc - 1, j - 1)) { ok = false; break; }
-          ++sc;
-        }
-        if (!ok) break;
-        if (!issue_pv(sc - 1, ui.nkv - 1)) { ok = false; break; }
-      }
-      // Drain: wait until every tcgen05 operation issued by this thread has completed.
-      mma_commit(&bars[kBarDrain]);
-      if (!mbar_wait(&bars[kBarDrain], 0, nullptr)) record_failure(abort_flag, kSiteDrain);
+    for (int kk = 0; kk < 4; ++kk) idq[kk] = idesc_qk(kk, negate);
+    uint32_t u = 0, kc = 0, vc = 0, sc = 0;
+    bool ok = true;
+    if (p.debug_stall > 0) {
+      // Test hook: wait for a phase of the drain barrier that nothing completes before the
+      // drain below, so the wait runs out and the failure path is exercised.
+      if (!mbar_wait_warp(&bars[kBarDrain], 0, abort_flag)) { record_failure(abort_flag, kSiteDebugStall); ok = false; }
     }
+    // O += P V for the S tile `tile_sc` (tile jj of the current unit).
+    auto issue_pv = [&](uint32_t tile_sc, int jj) -> bool {
+      const uint32_t b = tile_sc & 1;
+      if (!mbar_wait_warp(&bars[kBarPReady + b], (tile_sc >> 1) & 1, abort_flag)) { record_failure(abort_flag, kSiteMmaP); return false; }
+      if (jj == 0) {
+        if (!mbar_wait_warp(&bars[kBarOEmpty], (u & 1) ^ 1, abort_flag)) { record_failure(abort_flag, kSiteMmaO); return false; }
+      }
+      const bool got = kFp8PV ? mbar_wait_warp(&bars[kBarVFull + vc % kVStages], (vc / kVStages) & 1, abort_flag)
+                              : mbar_wait_warp(&bars[kBarVbfFull + vc % kVbfStages], (vc / kVbfStages) & 1, abort_flag);
+      if (!got) { record_failure(abort_flag, kSiteMmaV); return false; }
+      tc_fence_after();
+      const uint32_t p_col = tmem + kColS + b * 128;
+      if (kFp8PV) {
+        const uint64_t bdesc = dv0 + ((vc % kVStages) * kTileBytes >> 4);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)  // keys [32kk, 32kk+32): group kk/2's P, 8 columns per 32 keys
+          mma_f8f6f4_ts(tmem + kColO, p_col + (kk >> 1) * 64 + (kk & 1) * 8, bdesc + kk * 256, kIdescPV8,
+                        (jj > 0 || kk > 0) ? 1u : 0u, leader);
+        mma_commit(&bars[kBarVEmpty + vc % kVStages], leader);
+      } else {
+        const uint64_t bdesc = dv0 + ((vc % kVbfStages) * kVbfBytes >> 4);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)  // keys [16kk, 16kk+16): group kk/4's P, 8 columns per 16 keys
+          mma_f16_ts(tmem + kColO, p_col + (kk >> 2) * 64 + (kk & 3) * 8, bdesc + kk * 128, kIdescPV16,
+                     (jj > 0 || kk > 0) ? 1u : 0u, leader);
+        mma_commit(&bars[kBarVbfEmpty + vc % kVbfStages], leader);
+      }
+      mma_commit(&bars[kBarPVDone], leader);
+      ++vc;
+      return true;
+    };
+    for (int w = blockIdx.x; w < p.num_units && ok; w += G) {
+      const UnitInfo ui = warp_uniform(unit_info(p, w));
+      if (ui.nkv == 0) continue;
+      const uint32_t qs = u % kQStages;
+      if (!mbar_wait_warp(&bars[kBarQFull + qs], (u / kQStages) & 1, abort_flag)) { record_failure(abort_flag, kSiteMmaQ); ok = false; break; }
+      tc_fence_after();
+      const uint32_t sfa = tmem + kColSFA + qs * 4;
+      tmem_cp_32x128b_x4(sfa, dqsf0 + (qs * kAtomBytes >> 4), leader);
+      const uint64_t adesc = dq0 + (qs * kTileBytes >> 4);
+      for (int j = 0; j < ui.nkv; ++j) {
+        const uint32_t s = kc % kKStages;
+        if (!mbar_wait_warp(&bars[kBarKFull + s], (kc / kKStages) & 1, abort_flag)) { record_failure(abort_flag, kSiteMmaK); ok = false; break; }
+        tc_fence_after();
+        const uint32_t sfb = tmem + kColSFB + (kc & 1) * 4;
+        tmem_cp_32x128b_x4(sfb, dksf0 + (s * kAtomBytes >> 4), leader);
+        const uint64_t bdesc = dk0 + (s * kTileBytes >> 4);
+        const uint32_t d = tmem + kColS + (sc & 1) * 128;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {  // K = 32 bytes per MMA
+          const uint32_t byte_sel = static_cast<uint32_t>(kk) << 30;
+          mma_mxf8f6f4_ss(d, adesc + kk * 2, bdesc + kk * 2, idq[kk], sfa | byte_sel, sfb | byte_sel,
+                          kk > 0 ? 1u : 0u, leader);
+        }
+        mma_commit(&bars[kBarSFull + (sc & 1)], leader);
+        mma_commit(&bars[kBarKEmpty + s], leader);
+        if (j == ui.nkv - 1) mma_commit(&bars[kBarQEmpty + qs], leader);
+        ++kc;
+        // S buffer (sc+1) & 1 still holds P(j-1); its PV is issued before S(j+1) overwrites it.
+        if (j >= 1 && !issue_pv(sc - 1, j - 1)) { ok = false; break; }
+        ++sc;
+      }
+      if (!ok) break;
+      if (!issue_pv(sc - 1, ui.nkv - 1)) { ok = false; break; }
+      mma_commit(&bars[kBarOFull], leader);  // every PV of this unit is complete
+      ++u;
+    }
+    // Drain: wait until every tcgen05 operation issued by this warp has completed.
+    mma_commit(&bars[kBarDrain], leader);
+    if (!mbar_wait(&bars[kBarDrain], 0, nullptr)) record_failure(abort_flag, kSiteDrain);
   } else if (warp >= 4 && warp < 12) {
     // ------------------------------------------------------------------ softmax groups
+    constexpr float kLag = SoftmaxLag<kFp8PV>::lag;
+    constexpr float kBias = SoftmaxLag<kFp8PV>::bias;
     const int grp = (warp - 4) >> 2;             // 0: keys 0..63, 1: keys 64..127
     const int quarter = warp & 3;                // TMEM lane quarter of this warp
     const int row = quarter * 32 + lane;         // query row within the tile
@@ -372,82 +521,95 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
     const float kd = p.k_descale ? __ldg(p.k_descale) : 1.0f;
     const float vd = p.v_descale ? __ldg(p.v_descale) : 1.0f;
     const float cscale = fabsf((qd * kd) * kLog2eRsqrtD);  // sign folded into the QK MMA
-    const float pbias = kFp8PV ? 8.0f : 0.0f;
     uint32_t u = 0, sc = 0, pvn = 0;
     bool ok = true;
-    for (int w = blockIdx.x; w < p.num_units && ok; w += G, ++u) {
+    for (int w = blockIdx.x; w < p.num_units && ok; w += G) {
       const UnitInfo ui = unit_info(p, w);
-      float m = -INFINITY;  // running max, integer valued, log2 units
-      float l = 0.f;
+      if (ui.nkv == 0) {
+        const bool valid = ui.qtile * kTileM + row < ui.q_len;
+        const int64_t tok = ui.q_row0 + row;
+        // No keys: an empty sum, LSE = log 0 = -inf and O = 0.
+        if (valid) {
+          uint4* dst = reinterpret_cast<uint4*>(p.out + (tok * p.heads + ui.h) * 128 + grp * 64);
+#pragma unroll
+          for (int c = 0; c < 8; ++c) dst[c] = make_uint4(0u, 0u, 0u, 0u);
+          if (grp == 0) p.lse[static_cast<int64_t>(ui.h) * p.tq + tok] = -INFINITY;
+        }
+        continue;
+      }
+      float m = 0.f;   // shared reference of this row, integer valued, log2 units
+      float l = 0.f;   // this group's sum of p relative to m (times 2^kBias)
       for (int j = 0; j < ui.nkv; ++j) {
         const uint32_t b = sc & 1;
-        if (!mbar_wait(&bars[kBarSFull + b], (sc >> 1) & 1, abort_flag)) { record_failure(abort_flag, kSiteSoftS); ok = false; break; }
+        if (!mbar_wait_warp(&bars[kBarSFull + b], (sc >> 1) & 1, abort_flag)) { record_failure(abort_flag, kSiteSoftS); ok = false; break; }
         tc_fence_after();
-        const uint32_t s_addr = tmem + lane_addr + kColS0 + b * 128 + grp * 64;
-        uint32_t ra[32], rb[32];
-        tmem_ld32(s_addr, ra);
-        tmem_ld32(s_addr + 32, rb);
-        tmem_ld_wait();
-        float s[64];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) { s[i] = __uint_as_float(ra[i]); s[32 + i] = __uint_as_float(rb[i]); }
+        const uint32_t s_addr = tmem + lane_addr + kColS + b * 128 + grp * 64;
+        float2 sv[32];
+        load_s(s_addr, sv);
         const int key0 = j * kTileN + grp * 64;
         const bool tail = key0 + 64 > ui.k_len;
-        if (tail) {
-#pragma unroll
-          for (int i = 0; i < 64; ++i) if (key0 + i >= ui.k_len) s[i] = -INFINITY;
-        }
-        float pmax = s[0];
-#pragma unroll
-        for (int i = 1; i < 64; ++i) pmax = fmaxf(pmax, s[i]);
-        // Exchange the partial maxima of the two groups.
-        red[(grp * 2 + b) * 128 + row] = pmax;
+        if (tail) mask_keys(sv, key0, ui.k_len);
+        // This group's ceiling of the scaled row maximum (-inf if all its keys are masked).
+        const float smax = rowmax64(sv);
+        const float c_own = smax == -INFINITY ? -INFINITY : ceilf(smax * cscale);
+        red[(grp * 2 + b) * 128 + row] = c_own;
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars[kBarRed + b]);
-        if (!mbar_wait(&bars[kBarRed + b], (sc >> 1) & 1, abort_flag)) { record_failure(abort_flag, kSiteSoftRed); ok = false; break; }
-        const float tmax = fmaxf(pmax, red[((grp ^ 1) * 2 + b) * 128 + row]);
-        const float m_new = fmaxf(m, ceilf(tmax * cscale));
-        const float neg_off = pbias - m_new;
-        float psum = 0.f;
+        // Exponentials against the current reference, or this group's own ceiling when its
+        // keys exceed the reference by more than the lag (so p never overflows).
+        const float m_spec = (j == 0 || c_own > m + kLag) ? c_own : m;
+        // (m_spec is -inf only when all of this group's keys are masked, i.e. on a tail tile,
+        // where exp_tile zeroes every masked key.)
+        float psum = tail ? exp_tile<true, kPolyPairs>(sv, cscale, kBias - m_spec, key0, ui.k_len)
+                          : exp_tile<false, kPolyPairs>(sv, cscale, kBias - m_spec, key0, ui.k_len);
+        if (!mbar_wait_warp(&bars[kBarRed + b], (sc >> 1) & 1, abort_flag)) { record_failure(abort_flag, kSiteSoftRed); ok = false; break; }
+        const float c_row = fmaxf(c_own, red[((grp ^ 1) * 2 + b) * 128 + row]);  // row ceiling of this tile
+        // Both groups derive the same new reference from the same two ceilings.
+        const float m_new = (j == 0) ? c_row : (c_row > m + kLag ? c_row : m);
+        const float d = m_new - m_spec;  // >= 0, integer
+        if (__any_sync(0xFFFFFFFFu, d != 0.0f)) {
+          const float a = exp2_int(-d);
+          const float2 a2 = make_float2(a, a);
 #pragma unroll
-        for (int i = 0; i < 64; ++i) {
-          const float e = ex2_approx(fmaf(s[i], cscale, neg_off));
-          s[i] = (tail && key0 + i >= ui.k_len) ? 0.f : e;
-          psum += s[i];
+          for (int i = 0; i < 32; ++i) sv[i] = __fmul2_rn(sv[i], a2);
+          psum *= a;
         }
-        const float alpha = ex2_approx(m - m_new);
+        const float alpha = (j == 0) ? 0.0f : exp2_int(m - m_new);
         l = l * alpha + psum;
         m = m_new;
-        // P overwrites the S buffer: group g writes keys [64g, 64g+64).
+        // P overwrites the first columns of this group's own half of the S buffer.
         if (kFp8PV) {
           uint32_t pk[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i)
-            pk[i] = static_cast<uint32_t>(cvt_e4m3x2(s[4 * i], s[4 * i + 1])) |
-                    (static_cast<uint32_t>(cvt_e4m3x2(s[4 * i + 2], s[4 * i + 3])) << 16);
-          tmem_st16(tmem + lane_addr + kColS0 + b * 128 + grp * 16, pk);
+            pk[i] = static_cast<uint32_t>(cvt_e4m3x2(sv[2 * i].x, sv[2 * i].y)) |
+                    (static_cast<uint32_t>(cvt_e4m3x2(sv[2 * i + 1].x, sv[2 * i + 1].y)) << 16);
+          tmem_st16_sync(s_addr, pk);
         } else {
           uint32_t pk[32];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) pk[i] = cvt_bf16x2(s[2 * i], s[2 * i + 1]);
-          tmem_st32(tmem + lane_addr + kColS0 + b * 128 + grp * 32, pk);
+          for (int i = 0; i < 32; ++i) pk[i] = cvt_bf16x2(sv[i].x, sv[i].y);
+          tmem_st32_sync(s_addr, pk);
         }
-        // Rescale this group's half of O when the row ceiling moved (never on the first tile).
+        // Rescale this group's half of O when the reference moved (rare; never on tile 0).
         if (j > 0 && __any_sync(0xFFFFFFFFu, alpha != 1.0f)) {
-          if (!mbar_wait(&bars[kBarPVDone], (pvn - 1) & 1, abort_flag)) { record_failure(abort_flag, kSiteSoftPV); ok = false; break; }
+          if (!mbar_wait_warp(&bars[kBarPVDone], (pvn - 1) & 1, abort_flag)) { record_failure(abort_flag, kSiteSoftPV); ok = false; break; }
           tc_fence_after();
           const uint32_t o_addr = tmem + lane_addr + kColO + grp * 64;
+          const float2 a2 = make_float2(alpha, alpha);
 #pragma unroll
           for (int half = 0; half < 2; ++half) {
             uint32_t ro[32];
-            tmem_ld32(o_addr + half * 32, ro);
-            tmem_ld_wait();
+            tmem_ld32_sync(o_addr + half * 32, ro);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) ro[i] = __float_as_uint(__uint_as_float(ro[i]) * alpha);
-            tmem_st32(o_addr + half * 32, ro);
+            for (int i = 0; i < 16; ++i) {
+              const float2 o2 = __fmul2_rn(make_float2(__uint_as_float(ro[2 * i]), __uint_as_float(ro[2 * i + 1])), a2);
+              ro[2 * i] = __float_as_uint(o2.x);
+              ro[2 * i + 1] = __float_as_uint(o2.y);
+            }
+            tmem_st32_sync(o_addr + half * 32, ro);
           }
         }
-        tmem_st_wait();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars[kBarPReady + b]);
@@ -456,24 +618,24 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
       }
       if (!ok) break;
       // ---------------------------------------------------------------- epilogue
-      if (!mbar_wait(&bars[kBarPVDone], (pvn - 1) & 1, abort_flag)) { record_failure(abort_flag, kSiteSoftPV); ok = false; break; }
+      // OFull completes once per unit with keys, after the unit's last PV. (PVDone cannot be
+      // used here: its parity only tells apart two consecutive phases, and at this point the
+      // last two PVs may both be outstanding.)
+      if (!mbar_wait_warp(&bars[kBarOFull], u & 1, abort_flag)) { record_failure(abort_flag, kSiteSoftPV); ok = false; break; }
       tc_fence_after();
       lsum[grp * 128 + row] = l;
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars[kBarLReady]);
-      if (!mbar_wait(&bars[kBarLReady], u & 1, abort_flag)) { record_failure(abort_flag, kSiteSoftL); ok = false; break; }
+      if (!mbar_wait_warp(&bars[kBarLReady], u & 1, abort_flag)) { record_failure(abort_flag, kSiteSoftL); ok = false; break; }
       const float ltot = l + lsum[(grp ^ 1) * 128 + row];
       const float oscale = vd / ltot;
       const uint32_t o_addr = tmem + lane_addr + kColO + grp * 64;
       uint32_t ra[32], rb[32];
-      tmem_ld32(o_addr, ra);
-      tmem_ld32(o_addr + 32, rb);
-      tmem_ld_wait();
+      tmem_ld64_sync(o_addr, ra, rb);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars[kBarOEmpty]);
-      const bool valid = ui.qtile * kTileM + row < ui.q_len;
-      if (valid) {
+      if (ui.qtile * kTileM + row < ui.q_len) {
         const int64_t tok = ui.q_row0 + row;
         uint4* dst = reinterpret_cast<uint4*>(p.out + (tok * p.heads + ui.h) * 128 + grp * 64);
 #pragma unroll
@@ -494,28 +656,29 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
           v.w = cvt_bf16x2(__uint_as_float(rb[8 * c + 6]) * oscale, __uint_as_float(rb[8 * c + 7]) * oscale);
           dst[4 + c] = v;
         }
-        if (grp == 0) p.lse[static_cast<int64_t>(ui.h) * p.tq + tok] = (m - pbias + lg2_approx(ltot)) * kLn2;
+        if (grp == 0) p.lse[static_cast<int64_t>(ui.h) * p.tq + tok] = (m - kBias + lg2_approx(ltot)) * kLn2;
       }
+      ++u;
     }
   } else if (!kFp8PV && warp >= 12) {
     // ------------------------------------------------------------------ V converter (bf16 PV)
     const int t = threadIdx.x - 12 * 32;  // key row of the V tile, 0..127
     const uint32_t sw = static_cast<uint32_t>(t & 7);
-    uint32_t u = 0, vc = 0;
+    uint32_t vc = 0;
     bool ok = true;
-    for (int w = blockIdx.x; w < p.num_units && ok; w += G, ++u) {
+    for (int w = blockIdx.x; w < p.num_units && ok; w += G) {
       const UnitInfo ui = unit_info(p, w);
       for (int j = 0; j < ui.nkv; ++j) {
         const uint32_t s = vc % kVStages, ph = (vc / kVStages) & 1;
         const uint32_t sb = vc % kVbfStages, phb = (vc / kVbfStages) & 1;
-        if (!mbar_wait(&bars[kBarVFull + s], ph, abort_flag)) { record_failure(abort_flag, kSiteConvV); ok = false; break; }
-        if (!mbar_wait(&bars[kBarVbfEmpty + sb], phb ^ 1, abort_flag)) { record_failure(abort_flag, kSiteConvE); ok = false; break; }
+        if (!mbar_wait_warp(&bars[kBarVFull + s], ph, abort_flag)) { record_failure(abort_flag, kSiteConvV); ok = false; break; }
+        if (!mbar_wait_warp(&bars[kBarVbfEmpty + sb], phb ^ 1, abort_flag)) { record_failure(abort_flag, kSiteConvE); ok = false; break; }
         const uint8_t* src = smem + SmemLayout::v + s * kTileBytes + t * 128;
         const uint32_t sfw = reinterpret_cast<const uint32_t*>(smem + SmemLayout::v_sf + s * kAtomBytes)[(t & 31) * 4 + (t >> 5)];
-        uint8_t* dst = smem + SmemLayout::vbf + sb * 2 * kTileBytes + t * 128;
+        uint8_t* dst = smem + SmemLayout::vbf + sb * kVbfBytes + t * 128;
 #pragma unroll
         for (int c = 0; c < 8; ++c) {  // 16 fp8 values: head_dim [16c, 16c + 16)
-          const uint4 raw = *reinterpret_cast<const uint4*>(src + ((c ^ sw) << 4));
+          const uint4 raw = *reinterpret_cast<const uint4*>(src + ((static_cast<uint32_t>(c) ^ sw) << 4));
           const int e = static_cast<int>((sfw >> (8 * (c >> 1))) & 0xFFu) - 127;
           const float scale = e >= -126 ? __uint_as_float(static_cast<uint32_t>(e + 127) << 23)
                                         : __uint_as_float(0x00400000u);  // 2^-127

@@ -90,14 +90,14 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// Tensor map over a packed (tokens, heads, 128) uint8 payload; box = 128 tokens of one head,
-// 128-byte rows with the 128-byte swizzle the UMMA descriptors expect.
-lpfa_status payload_tmap(CUtensorMap* map, const void* base, int64_t tokens, int heads) {
+// Tensor map over a packed (tokens, heads, 128) uint8 payload; box = box_rows tokens of one
+// head, 128-byte rows with the 128-byte swizzle the UMMA descriptors expect.
+lpfa_status payload_tmap(CUtensorMap* map, const void* base, int64_t tokens, int heads, uint32_t box_rows) {
   auto fn = encode_fn();
   if (!fn) return fail(LPFA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
   cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(heads), static_cast<cuuint64_t>(tokens)};
   cuuint64_t strides[2] = {128, static_cast<cuuint64_t>(heads) * 128};
-  cuuint32_t box[3] = {128, 1, 128};
+  cuuint32_t box[3] = {128, 1, box_rows};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -268,9 +268,9 @@ static lpfa_status attn_fwd_impl(const uint8_t* q, const uint8_t* q_sf, const ui
   if ((st = require_sm100(&info)) != LPFA_OK) return st;
 
   CUtensorMap tq, tk, tv;
-  if ((st = payload_tmap(&tq, q, meta_q->total_tokens, heads)) != LPFA_OK) return st;
-  if ((st = payload_tmap(&tk, k, meta_k->total_tokens, heads)) != LPFA_OK) return st;
-  if ((st = payload_tmap(&tv, v, meta_k->total_tokens, heads)) != LPFA_OK) return st;
+  if ((st = payload_tmap(&tq, q, meta_q->total_tokens, heads, lpfa::kTileM)) != LPFA_OK) return st;
+  if ((st = payload_tmap(&tk, k, meta_k->total_tokens, heads, lpfa::kTileN)) != LPFA_OK) return st;
+  if ((st = payload_tmap(&tv, v, meta_k->total_tokens, heads, lpfa::kTileN)) != LPFA_OK) return st;
 
   lpfa::AttnParams p;
   p.q_sf = q_sf;
