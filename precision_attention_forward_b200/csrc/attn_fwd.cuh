@@ -12,32 +12,32 @@
 // per SM); CTA b takes units b, b + G, b + 2G, ... in head-major order so that the CTAs
 // running at the same time stream the same K/V through L2.
 //
-// Warp roles (512 threads):
+// Warp roles (512 threads, four warpgroups):
 //   warp 0        TMA producer (whole warp, one lane issues): the Q tile + its scale atom once
-//                 per unit, then 128-key K/V tiles (+ atoms) in the order the MMA warp uses them
-//                 (K0, K1, V0, K2, V1, ...).
+//                 per unit, then 128-key K/V tiles (+ atoms) in the order the MMA warp uses them.
 //   warp 1        TMEM allocator and MMA issuer (whole warp, one lane issues):
-//                   S[b] = Q K_j^T   tcgen05.mma kind::mxf8f6f4.block_scale, M128 N128 K128
-//                   O   += P_j V_j   kind::f16 (bf16 PV) or kind::f8f6f4 (fp8 PV), P from TMEM
-//                 S is double buffered, so S(j+1) is computed while the softmax of S(j) runs.
-//                 A block-scaled MMA costs about as much issue time at N=64 as at N=128, so the
-//                 key tile is 128 wide.
-//   warps 4..7    softmax group 0: rows 0..127 of the tile, keys 0..63 of every S tile.
-//   warps 8..11   softmax group 1: the same rows, keys 64..127. The groups exchange row maxima
-//                 through shared memory once per tile, after computing their exponentials.
+//                   S[t & 1] = Q K_t^T  tcgen05.mma kind::mxf8f6f4.block_scale, M128 N128 K128
+//                   O       += P_t V_t  kind::f8f6f4 (fp8 PV) or kind::f16 (bf16 PV), P in TMEM
+//                 QK of tile t is issued as soon as S buffer t & 1 has been read out, ahead of
+//                 the PV of the tiles before it, so a softmax group never waits for its next S.
+//   warps 4..7    softmax group 0: KV tiles t with t even (t counts all tiles of the CTA).
+//   warps 8..11   softmax group 1: KV tiles t with t odd. In both groups a thread owns one query
+//                 row and all 128 keys of the tile (192 registers after setmaxnreg). The groups
+//                 run half a tile apart, so one group's exponentials (MUFU) overlap the other's
+//                 load, max, packing and stores.
 //   warps 12..15  bf16 PV mode only: convert the V tile from MXFP8 to BF16 in shared memory.
 //
-// Online softmax keeps a reference m (an integer, log2 units) per row, shared by both
-// groups. Exponentials are computed against the current reference (or the group's own
-// ceiling if its keys exceed the reference by more than the lag) before the other group's
-// maximum arrives; the two groups then agree on the new reference and scale their P by an
-// exact power of two if it moved. The reference rises only when a tile exceeds it by more
-// than the lag, so rescaling of l and O is rare. In fp8 PV mode P is stored as
-// E4M3(2^(8 - lag) * 2^(t - m)) <= 256; the power of two cancels in the final division.
+// Online softmax keeps one reference m per row (an integer, log2 units) shared by the two
+// groups: tile t's reference is its own row-maximum ceiling if that exceeds tile t-1's
+// reference by more than a lag, else tile t-1's reference, so P <= 2^(lag + bias) and the
+// reference (and with it l and O) moves rarely and only by exact powers of two. Tile t-1's
+// reference reaches tile t through shared memory right after the other group's row max. In fp8
+// PV mode P is stored as E4M3(2^(bias - m) 2^s) <= 256; the power of two cancels in the final
+// division.
 //
-// TMEM columns (512 allocated): S buffer b at [128b, 128b + 128) (group g reads columns
-// [64g, 64g + 64) and writes its P over the first of them), O [256,384), Q scale atoms (2
-// stages) [384,392), K scale atoms (2 slots) [392,400).
+// TMEM columns (512 allocated): S buffer b at [128b, 128b + 128), O [256, 384), fp8 P buffer
+// b at [384 + 32b, 416 + 32b) (bf16 P is written over the first 64 columns of its S buffer),
+// Q scale atoms (2 stages) [448, 456), K scale atoms (2 slots) [456, 464).
 #pragma once
 
 #include <cstdint>
@@ -53,6 +53,10 @@ namespace lpfa {
 __device__ int g_lpfa_status[2];  // [0] = lpfa_status code of a failed kernel, [1] = detail
 
 constexpr int kAttnThreads = 512;
+constexpr int kLaunchRegs = 128;     // 65536 / 512: registers per thread at launch
+constexpr int kSoftmaxRegs = 192;    // softmax warpgroups after setmaxnreg.inc
+constexpr int kOtherRegs = 64;       // producer/MMA and converter warpgroups after setmaxnreg.dec
+static_assert(2 * kSoftmaxRegs + 2 * kOtherRegs == 4 * kLaunchRegs, "register split must use the launch budget");
 constexpr int kTileM = 128;          // query rows per tile
 constexpr int kTileN = 128;          // keys per KV tile
 constexpr int kQStages = 2;
@@ -64,10 +68,11 @@ constexpr uint32_t kVbfBytes = 128 * 128 * 2;  // 128 keys x 128 bf16
 constexpr uint32_t kAtomBytes = 512;
 
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS = 0;        // + 128 * b  S buffer (fp32), P written over its columns
+constexpr uint32_t kColS = 0;        // + 128 * b  S buffer (fp32); bf16 P over its first 64 columns
 constexpr uint32_t kColO = 256;      // O accumulator (fp32)
-constexpr uint32_t kColSFA = 384;    // + 4 * stage  Q scale atom
-constexpr uint32_t kColSFB = 392;    // + 4 * slot   K scale atom
+constexpr uint32_t kColP = 384;      // + 32 * b   fp8 P buffer
+constexpr uint32_t kColSFA = 448;    // + 4 * stage  Q scale atom
+constexpr uint32_t kColSFB = 456;    // + 4 * slot   K scale atom
 
 // log2(e) / sqrt(128) rounded to fp32: logits in log2 units per unit of Q.K.
 constexpr float kLog2eRsqrtD = 0.12751743082459868f;
@@ -77,7 +82,7 @@ constexpr float kLn2 = 0.69314718055994531f;
 enum WaitSite : int {
   kSiteProducerQ = 1, kSiteProducerK, kSiteProducerV, kSiteMmaQ, kSiteMmaK, kSiteMmaP,
   kSiteMmaV, kSiteMmaO, kSiteSoftS, kSiteSoftRed, kSiteSoftPV, kSiteSoftL, kSiteConvV,
-  kSiteConvE, kSiteDrain, kSiteDebugStall
+  kSiteConvE, kSiteDrain, kSiteDebugStall, kSiteMmaS, kSiteSoftO
 };
 
 struct AttnParams {
@@ -110,20 +115,29 @@ struct SmemLayout {
   static constexpr uint32_t q_sf = vbf + kVbfStages * kVbfBytes;
   static constexpr uint32_t k_sf = q_sf + kQStages * kAtomBytes;
   static constexpr uint32_t v_sf = k_sf + kKStages * kAtomBytes;
-  static constexpr uint32_t red = v_sf + kVStages * kAtomBytes;       // float [2 groups][2 slots][128]
-  static constexpr uint32_t lsum = red + 2 * 2 * 128 * 4;             // float [2 groups][128]
-  static constexpr uint32_t bars = lsum + 2 * 128 * 4;                // uint64 barriers
+  static constexpr uint32_t mref = v_sf + kVStages * kAtomBytes;      // float [2 groups][128] tile reference
+  static constexpr uint32_t lsum = mref + 2 * 128 * 4;                // float [2 groups][128] partial l
+  static constexpr uint32_t mfin = lsum + 2 * 128 * 4;                // float [2 groups][128] reference of l
+  static constexpr uint32_t bars = mfin + 2 * 128 * 4;                // uint64 barriers
   static constexpr uint32_t num_bars = 40;
   static constexpr uint32_t misc = bars + num_bars * 8;               // tmem base, abort flag
   static constexpr uint32_t total = misc + 64;
 };
 constexpr uint32_t kAttnSmemBytes = SmemLayout::total + 1024;  // + alignment slack
 
-// Barrier indices.
+// Barrier indices. [2]-sized entries are indexed by softmax group / S buffer b.
 enum Bar : int {
   kBarQFull = 0, kBarQEmpty = 2, kBarKFull = 4, kBarKEmpty = 7, kBarVFull = 10, kBarVEmpty = 13,
-  kBarVbfFull = 16, kBarVbfEmpty = 18, kBarSFull = 20, kBarPReady = 22, kBarRed = 24,
-  kBarPVDone = 26, kBarOEmpty = 27, kBarLReady = 28, kBarDrain = 29, kBarOFull = 30
+  kBarVbfFull = 16, kBarVbfEmpty = 18,
+  kBarSFull = 20,    // S(t) computed                       (MMA commit)
+  kBarSFree = 22,    // S(t) read out by its group            (4 warps)
+  kBarPReady = 24,   // P(t) stored, O rescaled if needed     (4 warps)
+  kBarPVDone = 26,   // PV(t) complete                        (MMA commit)
+  kBarMRef = 28,     // tile reference of t published         (4 warps)
+  kBarOFull = 30,    // every PV of the unit complete         (MMA commit)
+  kBarOEmpty = 31,   // O read out by both groups             (8 warps)
+  kBarLReady = 32,   // partial l / reference exchanged       (8 warps)
+  kBarDrain = 33
 };
 
 // UMMA shared-memory matrix descriptor (sm_100 format, version 1).
@@ -148,7 +162,7 @@ constexpr uint32_t kIdescPV8 = (1u << 4) | (1u << 16) | (16u << 17) | (8u << 24)
 constexpr uint32_t kIdescPV16 = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) | (16u << 17) | (8u << 24);
 
 // ---------------------------------------------------------------------------------------
-// Softmax helpers (one thread = one query row, 64 keys of an S tile held as 32 float2)
+// Softmax helpers (one thread = one query row, the 128 keys of an S tile held as 64 float2)
 // ---------------------------------------------------------------------------------------
 // Pairs of S elements, out of every 8, whose exp2 runs on the FMA pipe (polynomial) instead
 // of the MUFU unit. MUFU alone delivers 16 exp2 per clock per SM, half of what the FP8 tensor
@@ -196,40 +210,40 @@ __device__ __forceinline__ float2 exp2_poly2(float2 x) {
                      __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(t.y) << 23)));
 }
 
-__device__ __forceinline__ void load_s(uint32_t taddr, float2 (&s)[32]) {
-  uint32_t ra[32], rb[32];
-  tmem_ld64_sync(taddr, ra, rb);
+// The 128 S columns of this thread's row.
+__device__ __forceinline__ void load_row(uint32_t taddr, float2 (&s)[64]) {
+  uint32_t r[128];
+  tmem_ld128_sync(taddr, r);
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    s[i] = make_float2(__uint_as_float(ra[2 * i]), __uint_as_float(ra[2 * i + 1]));
-    s[16 + i] = make_float2(__uint_as_float(rb[2 * i]), __uint_as_float(rb[2 * i + 1]));
-  }
+  for (int i = 0; i < 64; ++i) s[i] = make_float2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
 }
 
-__device__ __forceinline__ void mask_keys(float2 (&s)[32], int key0, int klen) {
+__device__ __forceinline__ void mask_keys(float2 (&s)[64], int key0, int klen) {
 #pragma unroll
-  for (int i = 0; i < 32; ++i) {
+  for (int i = 0; i < 64; ++i) {
     if (key0 + 2 * i >= klen) s[i].x = -INFINITY;
     if (key0 + 2 * i + 1 >= klen) s[i].y = -INFINITY;
   }
 }
 
-__device__ __forceinline__ float rowmax64(const float2 (&s)[32]) {
-  float a[8];
+__device__ __forceinline__ float rowmax128(const float2 (&s)[64]) {
+  float a[16];
 #pragma unroll
-  for (int k = 0; k < 8; ++k)
+  for (int k = 0; k < 16; ++k)
     a[k] = max3f(max3f(s[4 * k].x, s[4 * k].y, s[4 * k + 1].x), max3f(s[4 * k + 1].y, s[4 * k + 2].x, s[4 * k + 2].y),
                  fmaxf(s[4 * k + 3].x, s[4 * k + 3].y));
-  return max3f(max3f(a[0], a[1], a[2]), max3f(a[3], a[4], a[5]), fmaxf(a[6], a[7]));
+  const float b0 = max3f(a[0], a[1], a[2]), b1 = max3f(a[3], a[4], a[5]), b2 = max3f(a[6], a[7], a[8]);
+  const float b3 = max3f(a[9], a[10], a[11]), b4 = max3f(a[12], a[13], a[14]);
+  return fmaxf(max3f(b0, b1, b2), max3f(b3, b4, a[15]));
 }
 
 // p = 2^(s * c + nb) in place; masked keys (tail tiles) become exactly 0. Returns sum of p.
 template <bool kTail, int kPoly>
-__device__ __forceinline__ float exp_tile(float2 (&s)[32], float c, float nb, int key0, int klen) {
+__device__ __forceinline__ float exp_row(float2 (&s)[64], float c, float nb, int key0, int klen) {
   const float2 c2 = make_float2(c, c), nb2 = make_float2(nb, nb);
   float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
-  for (int i = 0; i < 32; ++i) {
+  for (int i = 0; i < 64; ++i) {
     const float2 x = __ffma2_rn(s[i], c2, nb2);
     float2 e = ((i & 7) < kPoly) ? exp2_poly2(x) : exp2_mufu2(x);
     if (kTail) {
@@ -306,12 +320,17 @@ __device__ __forceinline__ void record_failure(volatile int* abort_flag, int sit
   if (atomicCAS(&g_lpfa_status[0], 0, 4 /* LPFA_ERR_TIMEOUT */) == 0) atomicExch(&g_lpfa_status[1], site);
 }
 
-// How far (log2 units) a row's logits may exceed its reference before the reference, P, l
-// and O are rescaled, and the power of two P is stored with. bf16 P keeps its 8-bit
-// mantissa at any scale, so it may lag 8 binades; fp8 P stores 2^(8 - lag) * p <= 256 < 448.
+// How far (log2 units) a row's logits may exceed its reference before the reference, l and
+// O move, and the power of two P is stored with. bf16 P keeps its 8-bit mantissa at any
+// scale, so it may lag 8 binades; fp8 P stores 2^(bias - m) 2^s <= 2^(lag + bias) = 256 < 448.
 template <bool kFp8PV> struct SoftmaxLag;
 template <> struct SoftmaxLag<true> { static constexpr float lag = 2.0f; static constexpr float bias = 6.0f; };
 template <> struct SoftmaxLag<false> { static constexpr float lag = 8.0f; static constexpr float bias = 0.0f; };
+
+// How many tiles the PV issue trails the QK issue. fp8 P has its own TMEM buffer, so QK(t)
+// may overwrite S buffer t & 1 before PV(t - 2) has run; bf16 P lives in the S buffer, so
+// PV(t - 2) must be issued before QK(t).
+template <bool kFp8PV> struct PvLag { static constexpr int value = kFp8PV ? 2 : 1; };
 
 template <bool kFp8PV>
 __global__ void __launch_bounds__(kAttnThreads, 1)
@@ -322,8 +341,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SmemLayout::bars);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + SmemLayout::misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + SmemLayout::misc + 16);
-  float* red = reinterpret_cast<float*>(smem + SmemLayout::red);
+  float* mref = reinterpret_cast<float*>(smem + SmemLayout::mref);
   float* lsum = reinterpret_cast<float*>(smem + SmemLayout::lsum);
+  float* mfin = reinterpret_cast<float*>(smem + SmemLayout::mfin);
+  constexpr int kLagPV = PvLag<kFp8PV>::value;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -338,10 +359,11 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
     for (int i = 0; i < kVbfStages; ++i) { mbar_init(&bars[kBarVbfFull + i], 4); mbar_init(&bars[kBarVbfEmpty + i], 1); }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bars[kBarSFull + i], 1);
-      mbar_init(&bars[kBarPReady + i], 8);
-      mbar_init(&bars[kBarRed + i], 8);
+      mbar_init(&bars[kBarSFree + i], 4);
+      mbar_init(&bars[kBarPReady + i], 4);
+      mbar_init(&bars[kBarPVDone + i], 1);
+      mbar_init(&bars[kBarMRef + i], 4);
     }
-    mbar_init(&bars[kBarPVDone], 1);
     mbar_init(&bars[kBarOFull], 1);
     mbar_init(&bars[kBarOEmpty], 8);
     mbar_init(&bars[kBarLReady], 8);
@@ -362,174 +384,187 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
 
   const int G = gridDim.x;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------------ TMA producer
-    // The whole warp runs the loop (warp-uniform state); lane 0 issues the copies.
-    const uint32_t leader = lane == 0 ? 1u : 0u;
-    uint32_t qc = 0, kc = 0, vc = 0;  // fills issued per ring
-    bool ok = true;
-    auto load_v = [&](const UnitInfo& ui, int jj) -> bool {
-      const uint32_t s = vc % kVStages, ph = (vc / kVStages) & 1;
-      if (!mbar_wait_warp(&bars[kBarVEmpty + s], ph ^ 1, abort_flag)) { record_failure(abort_flag, kSiteProducerV); return false; }
-      mbar_arrive_expect_tx(&bars[kBarVFull + s], kTileBytes + (kFp8PV ? 0 : kAtomBytes), leader);
-      tma_load_3d(smem + SmemLayout::v + s * kTileBytes, &tmap_v, &bars[kBarVFull + s], 0, ui.h,
-                  ui.k_row0 + jj * kTileN, leader);
-      if (!kFp8PV)
-        bulk_load(smem + SmemLayout::v_sf + s * kAtomBytes,
-                  p.v_sf + (static_cast<int64_t>(ui.sbk + jj) * p.heads + ui.h) * kAtomBytes, kAtomBytes,
-                  &bars[kBarVFull + s], leader);
-      ++vc;
-      return true;
-    };
-    for (int w = blockIdx.x; w < p.num_units && ok; w += G) {
-      const UnitInfo ui = warp_uniform(unit_info(p, w));
-      if (ui.nkv == 0) continue;  // no keys: the softmax warps write the empty-sum result
-      const uint32_t qs = qc % kQStages, qph = (qc / kQStages) & 1;
-      if (!mbar_wait_warp(&bars[kBarQEmpty + qs], qph ^ 1, abort_flag)) { record_failure(abort_flag, kSiteProducerQ); ok = false; break; }
-      mbar_arrive_expect_tx(&bars[kBarQFull + qs], kTileBytes + kAtomBytes, leader);
-      tma_load_3d(smem + SmemLayout::q + qs * kTileBytes, &tmap_q, &bars[kBarQFull + qs], 0, ui.h, ui.q_row0, leader);
-      bulk_load(smem + SmemLayout::q_sf + qs * kAtomBytes,
-                p.q_sf + (static_cast<int64_t>(ui.sbq + ui.qtile) * p.heads + ui.h) * kAtomBytes, kAtomBytes,
-                &bars[kBarQFull + qs], leader);
-      ++qc;
-      for (int j = 0; j < ui.nkv && ok; ++j) {
-        const uint32_t s = kc % kKStages, ph = (kc / kKStages) & 1;
-        if (!mbar_wait_warp(&bars[kBarKEmpty + s], ph ^ 1, abort_flag)) { record_failure(abort_flag, kSiteProducerK); ok = false; break; }
-        mbar_arrive_expect_tx(&bars[kBarKFull + s], kTileBytes + kAtomBytes, leader);
-        tma_load_3d(smem + SmemLayout::k + s * kTileBytes, &tmap_k, &bars[kBarKFull + s], 0, ui.h,
-                    ui.k_row0 + j * kTileN, leader);
-        bulk_load(smem + SmemLayout::k_sf + s * kAtomBytes,
-                  p.k_sf + (static_cast<int64_t>(ui.sbk + j) * p.heads + ui.h) * kAtomBytes, kAtomBytes,
-                  &bars[kBarKFull + s], leader);
-        ++kc;
-        if (j >= 1) ok = load_v(ui, j - 1);
-      }
-      if (ok) ok = load_v(ui, ui.nkv - 1);
-    }
-    // Drain: every copy issued here must land before the CTA exits. The newest fill of each
-    // stage is the last one issued into it; older fills of that stage were consumed already.
-    for (uint32_t i = (qc > kQStages ? qc - kQStages : 0); i < qc; ++i)
-      if (!mbar_wait(&bars[kBarQFull + i % kQStages], (i / kQStages) & 1, nullptr)) record_failure(abort_flag, kSiteDrain);
-    for (uint32_t i = (kc > kKStages ? kc - kKStages : 0); i < kc; ++i)
-      if (!mbar_wait(&bars[kBarKFull + i % kKStages], (i / kKStages) & 1, nullptr)) record_failure(abort_flag, kSiteDrain);
-    for (uint32_t i = (vc > kVStages ? vc - kVStages : 0); i < vc; ++i)
-      if (!mbar_wait(&bars[kBarVFull + i % kVStages], (i / kVStages) & 1, nullptr)) record_failure(abort_flag, kSiteDrain);
-  } else if (warp == 1) {
-    // ------------------------------------------------------------------ MMA issuer
-    // The whole warp runs the loop (warp-uniform state); lane 0 issues the tcgen05 instructions.
-    const uint32_t leader = lane == 0 ? 1u : 0u;
-    const float qd = p.q_descale ? __ldg(p.q_descale) : 1.0f;
-    const float kd = p.k_descale ? __ldg(p.k_descale) : 1.0f;
-    const int negate = (qd * kd) < 0.0f ? 1 : 0;
-    // Descriptor bases; the start-address field is the low 14 bits (address >> 4), so a byte
-    // offset b inside shared memory advances a descriptor by b >> 4.
-    const uint64_t dq0 = umma_desc(smem_u32(smem + SmemLayout::q), 16, 1024, kLayoutSw128);
-    const uint64_t dk0 = umma_desc(smem_u32(smem + SmemLayout::k), 16, 1024, kLayoutSw128);
-    const uint64_t dv0 = kFp8PV ? umma_desc(smem_u32(smem + SmemLayout::v), kTileBytes, 1024, kLayoutSw128)
-                                : umma_desc(smem_u32(smem + SmemLayout::vbf), kTileBytes, 1024, kLayoutSw128);
-    const uint64_t dqsf0 = umma_desc(smem_u32(smem + SmemLayout::q_sf), 0, 128, kLayoutNone);
-    const uint64_t dksf0 = umma_desc(smem_u32(smem + SmemLayout::k_sf), 0, 128, kLayoutNone);
-    uint32_t idq[4];
-#pragma unroll
-    for (int kk = 0; kk < 4; ++kk) idq[kk] = idesc_qk(kk, negate);
-    uint32_t u = 0, kc = 0, vc = 0, sc = 0;
-    bool ok = true;
-    if (p.debug_stall > 0) {
-      // Test hook: wait for a phase of the drain barrier that nothing completes before the
-      // drain below, so the wait runs out and the failure path is exercised.
-      if (!mbar_wait_warp(&bars[kBarDrain], 0, abort_flag)) { record_failure(abort_flag, kSiteDebugStall); ok = false; }
-    }
-    // O += P V for the S tile `tile_sc` (tile jj of the current unit).
-    auto issue_pv = [&](uint32_t tile_sc, int jj) -> bool {
-      const uint32_t b = tile_sc & 1;
-      if (!mbar_wait_warp(&bars[kBarPReady + b], (tile_sc >> 1) & 1, abort_flag)) { record_failure(abort_flag, kSiteMmaP); return false; }
-      if (jj == 0) {
-        if (!mbar_wait_warp(&bars[kBarOEmpty], (u & 1) ^ 1, abort_flag)) { record_failure(abort_flag, kSiteMmaO); return false; }
-      }
-      const bool got = kFp8PV ? mbar_wait_warp(&bars[kBarVFull + vc % kVStages], (vc / kVStages) & 1, abort_flag)
-                              : mbar_wait_warp(&bars[kBarVbfFull + vc % kVbfStages], (vc / kVbfStages) & 1, abort_flag);
-      if (!got) { record_failure(abort_flag, kSiteMmaV); return false; }
-      tc_fence_after();
-      const uint32_t p_col = tmem + kColS + b * 128;
-      if (kFp8PV) {
-        const uint64_t bdesc = dv0 + ((vc % kVStages) * kTileBytes >> 4);
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)  // keys [32kk, 32kk+32): group kk/2's P, 8 columns per 32 keys
-          mma_f8f6f4_ts(tmem + kColO, p_col + (kk >> 1) * 64 + (kk & 1) * 8, bdesc + kk * 256, kIdescPV8,
-                        (jj > 0 || kk > 0) ? 1u : 0u, leader);
-        mma_commit(&bars[kBarVEmpty + vc % kVStages], leader);
-      } else {
-        const uint64_t bdesc = dv0 + ((vc % kVbfStages) * kVbfBytes >> 4);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)  // keys [16kk, 16kk+16): group kk/4's P, 8 columns per 16 keys
-          mma_f16_ts(tmem + kColO, p_col + (kk >> 2) * 64 + (kk & 3) * 8, bdesc + kk * 128, kIdescPV16,
-                     (jj > 0 || kk > 0) ? 1u : 0u, leader);
-        mma_commit(&bars[kBarVbfEmpty + vc % kVbfStages], leader);
-      }
-      mma_commit(&bars[kBarPVDone], leader);
-      ++vc;
-      return true;
-    };
-    for (int w = blockIdx.x; w < p.num_units && ok; w += G) {
-      const UnitInfo ui = warp_uniform(unit_info(p, w));
-      if (ui.nkv == 0) continue;
-      const uint32_t qs = u % kQStages;
-      if (!mbar_wait_warp(&bars[kBarQFull + qs], (u / kQStages) & 1, abort_flag)) { record_failure(abort_flag, kSiteMmaQ); ok = false; break; }
-      tc_fence_after();
-      const uint32_t sfa = tmem + kColSFA + qs * 4;
-      tmem_cp_32x128b_x4(sfa, dqsf0 + (qs * kAtomBytes >> 4), leader);
-      const uint64_t adesc = dq0 + (qs * kTileBytes >> 4);
-      for (int j = 0; j < ui.nkv; ++j) {
-        const uint32_t s = kc % kKStages;
-        if (!mbar_wait_warp(&bars[kBarKFull + s], (kc / kKStages) & 1, abort_flag)) { record_failure(abort_flag, kSiteMmaK); ok = false; break; }
-        tc_fence_after();
-        const uint32_t sfb = tmem + kColSFB + (kc & 1) * 4;
-        tmem_cp_32x128b_x4(sfb, dksf0 + (s * kAtomBytes >> 4), leader);
-        const uint64_t bdesc = dk0 + (s * kTileBytes >> 4);
-        const uint32_t d = tmem + kColS + (sc & 1) * 128;
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {  // K = 32 bytes per MMA
-          const uint32_t byte_sel = static_cast<uint32_t>(kk) << 30;
-          mma_mxf8f6f4_ss(d, adesc + kk * 2, bdesc + kk * 2, idq[kk], sfa | byte_sel, sfb | byte_sel,
-                          kk > 0 ? 1u : 0u, leader);
+  if (warp < 4) {
+    setmaxnreg_dec<kOtherRegs>();
+    if (warp == 0) {
+      // ---------------------------------------------------------------- TMA producer
+      // The whole warp runs the loop (warp-uniform state); lane 0 issues the copies.
+      const uint32_t leader = lane == 0 ? 1u : 0u;
+      uint32_t qc = 0, kc = 0, vc = 0;  // fills issued per ring
+      bool ok = true;
+      auto load_v = [&](const UnitInfo& ui, int jj) -> bool {
+        const uint32_t s = vc % kVStages, ph = (vc / kVStages) & 1;
+        if (!mbar_wait_warp(&bars[kBarVEmpty + s], ph ^ 1, abort_flag)) { record_failure(abort_flag, kSiteProducerV); return false; }
+        mbar_arrive_expect_tx(&bars[kBarVFull + s], kTileBytes + (kFp8PV ? 0 : kAtomBytes), leader);
+        tma_load_3d(smem + SmemLayout::v + s * kTileBytes, &tmap_v, &bars[kBarVFull + s], 0, ui.h,
+                    ui.k_row0 + jj * kTileN, leader);
+        if (!kFp8PV)
+          bulk_load(smem + SmemLayout::v_sf + s * kAtomBytes,
+                    p.v_sf + (static_cast<int64_t>(ui.sbk + jj) * p.heads + ui.h) * kAtomBytes, kAtomBytes,
+                    &bars[kBarVFull + s], leader);
+        ++vc;
+        return true;
+      };
+      for (int w = blockIdx.x; w < p.num_units && ok; w += G) {
+        const UnitInfo ui = warp_uniform(unit_info(p, w));
+        if (ui.nkv == 0) continue;  // no keys: the softmax warps write the empty-sum result
+        const uint32_t qs = qc % kQStages, qph = (qc / kQStages) & 1;
+        if (!mbar_wait_warp(&bars[kBarQEmpty + qs], qph ^ 1, abort_flag)) { record_failure(abort_flag, kSiteProducerQ); ok = false; break; }
+        mbar_arrive_expect_tx(&bars[kBarQFull + qs], kTileBytes + kAtomBytes, leader);
+        tma_load_3d(smem + SmemLayout::q + qs * kTileBytes, &tmap_q, &bars[kBarQFull + qs], 0, ui.h, ui.q_row0, leader);
+        bulk_load(smem + SmemLayout::q_sf + qs * kAtomBytes,
+                  p.q_sf + (static_cast<int64_t>(ui.sbq + ui.qtile) * p.heads + ui.h) * kAtomBytes, kAtomBytes,
+                  &bars[kBarQFull + qs], leader);
+        ++qc;
+        for (int j = 0; j < ui.nkv && ok; ++j) {
+          const uint32_t s = kc % kKStages, ph = (kc / kKStages) & 1;
+          if (!mbar_wait_warp(&bars[kBarKEmpty + s], ph ^ 1, abort_flag)) { record_failure(abort_flag, kSiteProducerK); ok = false; break; }
+          mbar_arrive_expect_tx(&bars[kBarKFull + s], kTileBytes + kAtomBytes, leader);
+          tma_load_3d(smem + SmemLayout::k + s * kTileBytes, &tmap_k, &bars[kBarKFull + s], 0, ui.h,
+                      ui.k_row0 + j * kTileN, leader);
+          bulk_load(smem + SmemLayout::k_sf + s * kAtomBytes,
+                    p.k_sf + (static_cast<int64_t>(ui.sbk + j) * p.heads + ui.h) * kAtomBytes, kAtomBytes,
+                    &bars[kBarKFull + s], leader);
+          ++kc;
+          if (j >= kLagPV) ok = load_v(ui, j - kLagPV);
         }
-        mma_commit(&bars[kBarSFull + (sc & 1)], leader);
-        mma_commit(&bars[kBarKEmpty + s], leader);
-        if (j == ui.nkv - 1) mma_commit(&bars[kBarQEmpty + qs], leader);
-        ++kc;
-        // S buffer (sc+1) & 1 still holds P(j-1); its PV is issued before S(j+1) overwrites it.
-        if (j >= 1 && !issue_pv(sc - 1, j - 1)) { ok = false; break; }
-        ++sc;
+        for (int jj = ui.nkv > kLagPV ? ui.nkv - kLagPV : 0; jj < ui.nkv && ok; ++jj) ok = load_v(ui, jj);
       }
-      if (!ok) break;
-      if (!issue_pv(sc - 1, ui.nkv - 1)) { ok = false; break; }
-      mma_commit(&bars[kBarOFull], leader);  // every PV of this unit is complete
-      ++u;
+      // Drain: every copy issued here must land before the CTA exits. The newest fill of each
+      // stage is the last one issued into it; older fills of that stage were consumed already.
+      for (uint32_t i = (qc > kQStages ? qc - kQStages : 0); i < qc; ++i)
+        if (!mbar_wait(&bars[kBarQFull + i % kQStages], (i / kQStages) & 1, nullptr)) record_failure(abort_flag, kSiteDrain);
+      for (uint32_t i = (kc > kKStages ? kc - kKStages : 0); i < kc; ++i)
+        if (!mbar_wait(&bars[kBarKFull + i % kKStages], (i / kKStages) & 1, nullptr)) record_failure(abort_flag, kSiteDrain);
+      for (uint32_t i = (vc > kVStages ? vc - kVStages : 0); i < vc; ++i)
+        if (!mbar_wait(&bars[kBarVFull + i % kVStages], (i / kVStages) & 1, nullptr)) record_failure(abort_flag, kSiteDrain);
+    } else if (warp == 1) {
+      // ---------------------------------------------------------------- MMA issuer
+      // The whole warp runs the loop (warp-uniform state); lane 0 issues the tcgen05 instructions.
+      const uint32_t leader = lane == 0 ? 1u : 0u;
+      const float qd = p.q_descale ? __ldg(p.q_descale) : 1.0f;
+      const float kd = p.k_descale ? __ldg(p.k_descale) : 1.0f;
+      const int negate = (qd * kd) < 0.0f ? 1 : 0;
+      // Descriptor bases; the start-address field is the low 14 bits (address >> 4), so a byte
+      // offset b inside shared memory advances a descriptor by b >> 4.
+      const uint64_t dq0 = umma_desc(smem_u32(smem + SmemLayout::q), 16, 1024, kLayoutSw128);
+      const uint64_t dk0 = umma_desc(smem_u32(smem + SmemLayout::k), 16, 1024, kLayoutSw128);
+      const uint64_t dv0 = kFp8PV ? umma_desc(smem_u32(smem + SmemLayout::v), kTileBytes, 1024, kLayoutSw128)
+                                  : umma_desc(smem_u32(smem + SmemLayout::vbf), kTileBytes, 1024, kLayoutSw128);
+      const uint64_t dqsf0 = umma_desc(smem_u32(smem + SmemLayout::q_sf), 0, 128, kLayoutNone);
+      const uint64_t dksf0 = umma_desc(smem_u32(smem + SmemLayout::k_sf), 0, 128, kLayoutNone);
+      uint32_t idq[4];
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) idq[kk] = idesc_qk(kk, negate);
+      uint32_t u = 0, kc = 0, vc = 0, t0 = 0;  // units, K fills, V tiles, first tile of the unit
+      bool ok = true;
+      if (p.debug_stall > 0) {
+        // Test hook: wait for a phase of the drain barrier that nothing completes before the
+        // drain below, so the wait runs out and the failure path is exercised.
+        if (!mbar_wait_warp(&bars[kBarDrain], 0, abort_flag)) { record_failure(abort_flag, kSiteDebugStall); ok = false; }
+      }
+      // O += P(t) V(t); jj is t's index within the unit.
+      auto issue_pv = [&](uint32_t t, int jj) -> bool {
+        const uint32_t b = t & 1;
+        if (!mbar_wait_warp(&bars[kBarPReady + b], (t >> 1) & 1, abort_flag)) { record_failure(abort_flag, kSiteMmaP); return false; }
+        if (jj == 0) {
+          if (!mbar_wait_warp(&bars[kBarOEmpty], (u & 1) ^ 1, abort_flag)) { record_failure(abort_flag, kSiteMmaO); return false; }
+        }
+        const bool got = kFp8PV ? mbar_wait_warp(&bars[kBarVFull + vc % kVStages], (vc / kVStages) & 1, abort_flag)
+                                : mbar_wait_warp(&bars[kBarVbfFull + vc % kVbfStages], (vc / kVbfStages) & 1, abort_flag);
+        if (!got) { record_failure(abort_flag, kSiteMmaV); return false; }
+        tc_fence_after();
+        if (kFp8PV) {
+          const uint32_t p_col = tmem + kColP + b * 32;
+          const uint64_t bdesc = dv0 + ((vc % kVStages) * kTileBytes >> 4);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)  // keys [32kk, 32kk + 32): 8 columns of 4 E4M3 each
+            mma_f8f6f4_ts(tmem + kColO, p_col + kk * 8, bdesc + kk * 256, kIdescPV8,
+                          (jj > 0 || kk > 0) ? 1u : 0u, leader);
+          mma_commit(&bars[kBarVEmpty + vc % kVStages], leader);
+        } else {
+          const uint32_t p_col = tmem + kColS + b * 128;
+          const uint64_t bdesc = dv0 + ((vc % kVbfStages) * kVbfBytes >> 4);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)  // keys [16kk, 16kk + 16): 8 columns of 2 BF16 each
+            mma_f16_ts(tmem + kColO, p_col + kk * 8, bdesc + kk * 128, kIdescPV16,
+                       (jj > 0 || kk > 0) ? 1u : 0u, leader);
+          mma_commit(&bars[kBarVbfEmpty + vc % kVbfStages], leader);
+        }
+        mma_commit(&bars[kBarPVDone + b], leader);
+        ++vc;
+        return true;
+      };
+      for (int w = blockIdx.x; w < p.num_units && ok; w += G) {
+        const UnitInfo ui = warp_uniform(unit_info(p, w));
+        if (ui.nkv == 0) continue;
+        const uint32_t qs = u % kQStages;
+        if (!mbar_wait_warp(&bars[kBarQFull + qs], (u / kQStages) & 1, abort_flag)) { record_failure(abort_flag, kSiteMmaQ); ok = false; break; }
+        tc_fence_after();
+        const uint32_t sfa = tmem + kColSFA + qs * 4;
+        tmem_cp_32x128b_x4(sfa, dqsf0 + (qs * kAtomBytes >> 4), leader);
+        const uint64_t adesc = dq0 + (qs * kTileBytes >> 4);
+        for (int j = 0; j < ui.nkv; ++j) {
+          const uint32_t t = t0 + j;
+          const uint32_t b = t & 1;
+          // S buffer b was read out by its group (tile t - 2).
+          if (t >= 2 && !mbar_wait_warp(&bars[kBarSFree + b], ((t - 2) >> 1) & 1, abort_flag)) { record_failure(abort_flag, kSiteMmaS); ok = false; break; }
+          const uint32_t s = kc % kKStages;
+          if (!mbar_wait_warp(&bars[kBarKFull + s], (kc / kKStages) & 1, abort_flag)) { record_failure(abort_flag, kSiteMmaK); ok = false; break; }
+          tc_fence_after();
+          const uint32_t sfb = tmem + kColSFB + (kc & 1) * 4;
+          tmem_cp_32x128b_x4(sfb, dksf0 + (s * kAtomBytes >> 4), leader);
+          const uint64_t bdesc = dk0 + (s * kTileBytes >> 4);
+          const uint32_t d = tmem + kColS + b * 128;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {  // K = 32 bytes per MMA
+            const uint32_t byte_sel = static_cast<uint32_t>(kk) << 30;
+            mma_mxf8f6f4_ss(d, adesc + kk * 2, bdesc + kk * 2, idq[kk], sfa | byte_sel, sfb | byte_sel,
+                            kk > 0 ? 1u : 0u, leader);
+          }
+          mma_commit(&bars[kBarSFull + b], leader);
+          mma_commit(&bars[kBarKEmpty + s], leader);
+          if (j == ui.nkv - 1) mma_commit(&bars[kBarQEmpty + qs], leader);
+          ++kc;
+          if (j >= kLagPV && !issue_pv(t - kLagPV, j - kLagPV)) { ok = false; break; }
+        }
+        if (!ok) break;
+        // The unit's remaining PVs go out before the next unit's QK, which may wait for a
+        // softmax group that first has to finish this unit's epilogue.
+        for (int jj = ui.nkv > kLagPV ? ui.nkv - kLagPV : 0; jj < ui.nkv; ++jj)
+          if (!issue_pv(t0 + jj, jj)) { ok = false; break; }
+        if (!ok) break;
+        mma_commit(&bars[kBarOFull], leader);  // every PV of this unit is complete
+        t0 += ui.nkv;
+        ++u;
+      }
+      // Drain: wait until every tcgen05 operation issued by this warp has completed.
+      mma_commit(&bars[kBarDrain], leader);
+      if (!mbar_wait(&bars[kBarDrain], 0, nullptr)) record_failure(abort_flag, kSiteDrain);
     }
-    // Drain: wait until every tcgen05 operation issued by this warp has completed.
-    mma_commit(&bars[kBarDrain], leader);
-    if (!mbar_wait(&bars[kBarDrain], 0, nullptr)) record_failure(abort_flag, kSiteDrain);
-  } else if (warp >= 4 && warp < 12) {
+  } else if (warp < 12) {
+    setmaxnreg_inc<kSoftmaxRegs>();
     // ------------------------------------------------------------------ softmax groups
     constexpr float kLag = SoftmaxLag<kFp8PV>::lag;
     constexpr float kBias = SoftmaxLag<kFp8PV>::bias;
-    const int grp = (warp - 4) >> 2;             // 0: keys 0..63, 1: keys 64..127
-    const int quarter = warp & 3;                // TMEM lane quarter of this warp
-    const int row = quarter * 32 + lane;         // query row within the tile
+    const uint32_t grp = static_cast<uint32_t>(warp - 4) >> 2;  // tiles t with t & 1 == grp
+    const int quarter = warp & 3;                                // TMEM lane quarter of this warp
+    const int row = quarter * 32 + lane;                         // query row within the tile
     const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
     const float qd = p.q_descale ? __ldg(p.q_descale) : 1.0f;
     const float kd = p.k_descale ? __ldg(p.k_descale) : 1.0f;
     const float vd = p.v_descale ? __ldg(p.v_descale) : 1.0f;
     const float cscale = fabsf((qd * kd) * kLog2eRsqrtD);  // sign folded into the QK MMA
-    uint32_t u = 0, sc = 0, pvn = 0;
+    float* my_mref = mref + grp * 128 + row;
+    const float* other_mref = mref + (grp ^ 1) * 128 + row;
+    uint32_t u = 0, t0 = 0;
     bool ok = true;
     for (int w = blockIdx.x; w < p.num_units && ok; w += G) {
       const UnitInfo ui = unit_info(p, w);
       if (ui.nkv == 0) {
-        const bool valid = ui.qtile * kTileM + row < ui.q_len;
-        const int64_t tok = ui.q_row0 + row;
         // No keys: an empty sum, LSE = log 0 = -inf and O = 0.
-        if (valid) {
+        if (ui.qtile * kTileM + row < ui.q_len) {
+          const int64_t tok = ui.q_row0 + row;
           uint4* dst = reinterpret_cast<uint4*>(p.out + (tok * p.heads + ui.h) * 128 + grp * 64);
 #pragma unroll
           for (int c = 0; c < 8; ++c) dst[c] = make_uint4(0u, 0u, 0u, 0u);
@@ -537,101 +572,103 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
         }
         continue;
       }
-      float m = 0.f;   // shared reference of this row, integer valued, log2 units
-      float l = 0.f;   // this group's sum of p relative to m (times 2^kBias)
-      for (int j = 0; j < ui.nkv; ++j) {
-        const uint32_t b = sc & 1;
-        if (!mbar_wait_warp(&bars[kBarSFull + b], (sc >> 1) & 1, abort_flag)) { record_failure(abort_flag, kSiteSoftS); ok = false; break; }
+      float m_g = -INFINITY;  // reference this group's l is relative to (-inf: no tile yet)
+      float l_g = 0.0f;       // this group's sum of p over its tiles (times 2^kBias)
+      for (int j = static_cast<int>((t0 ^ grp) & 1); j < ui.nkv; j += 2) {
+        const uint32_t t = t0 + j;           // t & 1 == grp
+        const uint32_t kt = t >> 1;          // this group's tile ordinal
+        if (!mbar_wait_warp(&bars[kBarSFull + grp], kt & 1, abort_flag)) { record_failure(abort_flag, kSiteSoftS); ok = false; break; }
         tc_fence_after();
-        const uint32_t s_addr = tmem + lane_addr + kColS + b * 128 + grp * 64;
-        float2 sv[32];
-        load_s(s_addr, sv);
-        const int key0 = j * kTileN + grp * 64;
-        const bool tail = key0 + 64 > ui.k_len;
-        if (tail) mask_keys(sv, key0, ui.k_len);
-        // This group's ceiling of the scaled row maximum (-inf if all its keys are masked).
-        const float smax = rowmax64(sv);
-        const float c_own = smax == -INFINITY ? -INFINITY : ceilf(smax * cscale);
-        red[(grp * 2 + b) * 128 + row] = c_own;
+        float2 sv[64];
+        load_row(tmem + lane_addr + kColS + grp * 128, sv);
+        tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bars[kBarRed + b]);
-        // Exponentials against the current reference, or this group's own ceiling when its
-        // keys exceed the reference by more than the lag (so p never overflows).
-        const float m_spec = (j == 0 || c_own > m + kLag) ? c_own : m;
-        // (m_spec is -inf only when all of this group's keys are masked, i.e. on a tail tile,
-        // where exp_tile zeroes every masked key.)
-        float psum = tail ? exp_tile<true, kPolyPairs>(sv, cscale, kBias - m_spec, key0, ui.k_len)
-                          : exp_tile<false, kPolyPairs>(sv, cscale, kBias - m_spec, key0, ui.k_len);
-        if (!mbar_wait_warp(&bars[kBarRed + b], (sc >> 1) & 1, abort_flag)) { record_failure(abort_flag, kSiteSoftRed); ok = false; break; }
-        const float c_row = fmaxf(c_own, red[((grp ^ 1) * 2 + b) * 128 + row]);  // row ceiling of this tile
-        // Both groups derive the same new reference from the same two ceilings.
-        const float m_new = (j == 0) ? c_row : (c_row > m + kLag ? c_row : m);
-        const float d = m_new - m_spec;  // >= 0, integer
-        if (__any_sync(0xFFFFFFFFu, d != 0.0f)) {
-          const float a = exp2_int(-d);
-          const float2 a2 = make_float2(a, a);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) sv[i] = __fmul2_rn(sv[i], a2);
-          psum *= a;
+        if (lane == 0) mbar_arrive(&bars[kBarSFree + grp]);  // S buffer may be overwritten
+        const int key0 = j * kTileN;
+        const bool tail = key0 + kTileN > ui.k_len;
+        if (tail) mask_keys(sv, key0, ui.k_len);
+        // Every tile has a valid key, so the ceiling is finite.
+        const float c_t = ceilf(rowmax128(sv) * cscale);
+        // Reference of tile t - 1 (the other group's), published right after its row max.
+        // Every tile waits for it, even the first of a unit, which keeps the two groups' tile
+        // references in lockstep order.
+        float m_prev = 0.0f;
+        if (t >= 1) {
+          if (!mbar_wait_warp(&bars[kBarMRef + (grp ^ 1)], ((t - 1) >> 1) & 1, abort_flag)) { record_failure(abort_flag, kSiteSoftRed); ok = false; break; }
+          m_prev = *other_mref;
         }
-        const float alpha = (j == 0) ? 0.0f : exp2_int(m - m_new);
-        l = l * alpha + psum;
-        m = m_new;
-        // P overwrites the first columns of this group's own half of the S buffer.
+        const float m_t = (j == 0 || c_t > m_prev + kLag) ? c_t : m_prev;
+        *my_mref = m_t;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars[kBarMRef + grp]);
+        const float psum = tail ? exp_row<true, kPolyPairs>(sv, cscale, kBias - m_t, key0, ui.k_len)
+                                : exp_row<false, kPolyPairs>(sv, cscale, kBias - m_t, key0, ui.k_len);
+        l_g = l_g * exp2_int(m_g - m_t) + psum;
+        m_g = m_t;
+        // PV(t - 2) has read this group's previous P.
+        if (kt >= 1) {
+          if (!mbar_wait_warp(&bars[kBarPVDone + grp], (kt - 1) & 1, abort_flag)) { record_failure(abort_flag, kSiteSoftPV); ok = false; break; }
+          tc_fence_after();
+        }
         if (kFp8PV) {
-          uint32_t pk[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i)
-            pk[i] = static_cast<uint32_t>(cvt_e4m3x2(sv[2 * i].x, sv[2 * i].y)) |
-                    (static_cast<uint32_t>(cvt_e4m3x2(sv[2 * i + 1].x, sv[2 * i + 1].y)) << 16);
-          tmem_st16_sync(s_addr, pk);
-        } else {
           uint32_t pk[32];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) pk[i] = cvt_bf16x2(sv[i].x, sv[i].y);
-          tmem_st32_sync(s_addr, pk);
-        }
-        // Rescale this group's half of O when the reference moved (rare; never on tile 0).
-        if (j > 0 && __any_sync(0xFFFFFFFFu, alpha != 1.0f)) {
-          if (!mbar_wait_warp(&bars[kBarPVDone], (pvn - 1) & 1, abort_flag)) { record_failure(abort_flag, kSiteSoftPV); ok = false; break; }
-          tc_fence_after();
-          const uint32_t o_addr = tmem + lane_addr + kColO + grp * 64;
-          const float2 a2 = make_float2(alpha, alpha);
+          for (int i = 0; i < 32; ++i)
+            pk[i] = static_cast<uint32_t>(cvt_e4m3x2(sv[2 * i].x, sv[2 * i].y)) |
+                    (static_cast<uint32_t>(cvt_e4m3x2(sv[2 * i + 1].x, sv[2 * i + 1].y)) << 16);
+          tmem_st32_sync(tmem + lane_addr + kColP + grp * 32, pk);
+        } else {
 #pragma unroll
-          for (int half = 0; half < 2; ++half) {
+          for (int h = 0; h < 2; ++h) {
+            uint32_t pk[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) pk[i] = cvt_bf16x2(sv[32 * h + i].x, sv[32 * h + i].y);
+            tmem_st32_sync(tmem + lane_addr + kColS + grp * 128 + h * 32, pk);
+          }
+        }
+        // O holds tiles up to t - 1 relative to m_prev; rescale it when the reference moved
+        // (rare; never on a unit's first tile).
+        if (j > 0 && __any_sync(0xFFFFFFFFu, m_t != m_prev)) {
+          if (!mbar_wait_warp(&bars[kBarPVDone + (grp ^ 1)], ((t - 1) >> 1) & 1, abort_flag)) { record_failure(abort_flag, kSiteSoftO); ok = false; break; }
+          tc_fence_after();
+          const float alpha = exp2_int(m_prev - m_t);
+          const float2 a2 = make_float2(alpha, alpha);
+          const uint32_t o_addr = tmem + lane_addr + kColO;
+#pragma unroll 1
+          for (int c = 0; c < 4; ++c) {
             uint32_t ro[32];
-            tmem_ld32_sync(o_addr + half * 32, ro);
+            tmem_ld32_sync(o_addr + c * 32, ro);
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
               const float2 o2 = __fmul2_rn(make_float2(__uint_as_float(ro[2 * i]), __uint_as_float(ro[2 * i + 1])), a2);
               ro[2 * i] = __float_as_uint(o2.x);
               ro[2 * i + 1] = __float_as_uint(o2.y);
             }
-            tmem_st32_sync(o_addr + half * 32, ro);
+            tmem_st32_sync(o_addr + c * 32, ro);
           }
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bars[kBarPReady + b]);
-        ++sc;
-        ++pvn;
+        if (lane == 0) mbar_arrive(&bars[kBarPReady + grp]);
       }
       if (!ok) break;
+      t0 += ui.nkv;
       // ---------------------------------------------------------------- epilogue
-      // OFull completes once per unit with keys, after the unit's last PV. (PVDone cannot be
-      // used here: its parity only tells apart two consecutive phases, and at this point the
-      // last two PVs may both be outstanding.)
+      // OFull completes once per unit, after the unit's last PV (so after every rescale).
       if (!mbar_wait_warp(&bars[kBarOFull], u & 1, abort_flag)) { record_failure(abort_flag, kSiteSoftPV); ok = false; break; }
       tc_fence_after();
-      lsum[grp * 128 + row] = l;
+      lsum[grp * 128 + row] = l_g;
+      mfin[grp * 128 + row] = m_g;
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars[kBarLReady]);
       if (!mbar_wait_warp(&bars[kBarLReady], u & 1, abort_flag)) { record_failure(abort_flag, kSiteSoftL); ok = false; break; }
-      const float ltot = l + lsum[(grp ^ 1) * 128 + row];
+      const float m_o = mfin[(grp ^ 1) * 128 + row];
+      const float l_o = lsum[(grp ^ 1) * 128 + row];
+      const float m_f = fmaxf(m_g, m_o);  // the unit's last reference (references never fall)
+      const float ltot = l_g * exp2_int(m_g - m_f) + l_o * exp2_int(m_o - m_f);
       const float oscale = vd / ltot;
-      const uint32_t o_addr = tmem + lane_addr + kColO + grp * 64;
       uint32_t ra[32], rb[32];
-      tmem_ld64_sync(o_addr, ra, rb);
+      tmem_ld64_sync(tmem + lane_addr + kColO + grp * 64, ra, rb);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars[kBarOEmpty]);
@@ -656,60 +693,63 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
           v.w = cvt_bf16x2(__uint_as_float(rb[8 * c + 6]) * oscale, __uint_as_float(rb[8 * c + 7]) * oscale);
           dst[4 + c] = v;
         }
-        if (grp == 0) p.lse[static_cast<int64_t>(ui.h) * p.tq + tok] = (m - kBias + lg2_approx(ltot)) * kLn2;
+        if (grp == 0) p.lse[static_cast<int64_t>(ui.h) * p.tq + tok] = (m_f - kBias + lg2_approx(ltot)) * kLn2;
       }
       ++u;
     }
-  } else if (!kFp8PV && warp >= 12) {
-    // ------------------------------------------------------------------ V converter (bf16 PV)
-    const int t = threadIdx.x - 12 * 32;  // key row of the V tile, 0..127
-    const uint32_t sw = static_cast<uint32_t>(t & 7);
-    uint32_t vc = 0;
-    bool ok = true;
-    for (int w = blockIdx.x; w < p.num_units && ok; w += G) {
-      const UnitInfo ui = unit_info(p, w);
-      for (int j = 0; j < ui.nkv; ++j) {
-        const uint32_t s = vc % kVStages, ph = (vc / kVStages) & 1;
-        const uint32_t sb = vc % kVbfStages, phb = (vc / kVbfStages) & 1;
-        if (!mbar_wait_warp(&bars[kBarVFull + s], ph, abort_flag)) { record_failure(abort_flag, kSiteConvV); ok = false; break; }
-        if (!mbar_wait_warp(&bars[kBarVbfEmpty + sb], phb ^ 1, abort_flag)) { record_failure(abort_flag, kSiteConvE); ok = false; break; }
-        const uint8_t* src = smem + SmemLayout::v + s * kTileBytes + t * 128;
-        const uint32_t sfw = reinterpret_cast<const uint32_t*>(smem + SmemLayout::v_sf + s * kAtomBytes)[(t & 31) * 4 + (t >> 5)];
-        uint8_t* dst = smem + SmemLayout::vbf + sb * kVbfBytes + t * 128;
+  } else {
+    setmaxnreg_dec<kOtherRegs>();
+    if (!kFp8PV) {
+      // ---------------------------------------------------------------- V converter (bf16 PV)
+      const int t = threadIdx.x - 12 * 32;  // key row of the V tile, 0..127
+      const uint32_t sw = static_cast<uint32_t>(t & 7);
+      uint32_t vc = 0;
+      bool ok = true;
+      for (int w = blockIdx.x; w < p.num_units && ok; w += G) {
+        const UnitInfo ui = unit_info(p, w);
+        for (int j = 0; j < ui.nkv; ++j) {
+          const uint32_t s = vc % kVStages, ph = (vc / kVStages) & 1;
+          const uint32_t sb = vc % kVbfStages, phb = (vc / kVbfStages) & 1;
+          if (!mbar_wait_warp(&bars[kBarVFull + s], ph, abort_flag)) { record_failure(abort_flag, kSiteConvV); ok = false; break; }
+          if (!mbar_wait_warp(&bars[kBarVbfEmpty + sb], phb ^ 1, abort_flag)) { record_failure(abort_flag, kSiteConvE); ok = false; break; }
+          const uint8_t* src = smem + SmemLayout::v + s * kTileBytes + t * 128;
+          const uint32_t sfw = reinterpret_cast<const uint32_t*>(smem + SmemLayout::v_sf + s * kAtomBytes)[(t & 31) * 4 + (t >> 5)];
+          uint8_t* dst = smem + SmemLayout::vbf + sb * kVbfBytes + t * 128;
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {  // 16 fp8 values: head_dim [16c, 16c + 16)
-          const uint4 raw = *reinterpret_cast<const uint4*>(src + ((static_cast<uint32_t>(c) ^ sw) << 4));
-          const int e = static_cast<int>((sfw >> (8 * (c >> 1))) & 0xFFu) - 127;
-          const float scale = e >= -126 ? __uint_as_float(static_cast<uint32_t>(e + 127) << 23)
-                                        : __uint_as_float(0x00400000u);  // 2^-127
-          const uint32_t wv[4] = {raw.x, raw.y, raw.z, raw.w};
-          uint32_t outw[8];
+          for (int c = 0; c < 8; ++c) {  // 16 fp8 values: head_dim [16c, 16c + 16)
+            const uint4 raw = *reinterpret_cast<const uint4*>(src + ((static_cast<uint32_t>(c) ^ sw) << 4));
+            const int e = static_cast<int>((sfw >> (8 * (c >> 1))) & 0xFFu) - 127;
+            const float scale = e >= -126 ? __uint_as_float(static_cast<uint32_t>(e + 127) << 23)
+                                          : __uint_as_float(0x00400000u);  // 2^-127
+            const uint32_t wv[4] = {raw.x, raw.y, raw.z, raw.w};
+            uint32_t outw[8];
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const uint32_t h01 = cvt_e4m3x2_to_f16x2(static_cast<uint16_t>(wv[i] & 0xFFFFu));
-            const uint32_t h23 = cvt_e4m3x2_to_f16x2(static_cast<uint16_t>(wv[i] >> 16));
-            const float2 f01 = __half22float2(*reinterpret_cast<const __half2*>(&h01));
-            const float2 f23 = __half22float2(*reinterpret_cast<const __half2*>(&h23));
-            outw[2 * i] = cvt_bf16x2(f01.x * scale, f01.y * scale);
-            outw[2 * i + 1] = cvt_bf16x2(f23.x * scale, f23.y * scale);
+            for (int i = 0; i < 4; ++i) {
+              const uint32_t h01 = cvt_e4m3x2_to_f16x2(static_cast<uint16_t>(wv[i] & 0xFFFFu));
+              const uint32_t h23 = cvt_e4m3x2_to_f16x2(static_cast<uint16_t>(wv[i] >> 16));
+              const float2 f01 = __half22float2(*reinterpret_cast<const __half2*>(&h01));
+              const float2 f23 = __half22float2(*reinterpret_cast<const __half2*>(&h23));
+              outw[2 * i] = cvt_bf16x2(f01.x * scale, f01.y * scale);
+              outw[2 * i + 1] = cvt_bf16x2(f23.x * scale, f23.y * scale);
+            }
+            // bf16 chunks 2c and 2c+1 (8 elements each) of the MN-major SW128 layout:
+            // atom a = chunk / 8 holds head_dim [64a, 64a + 64); rows are keys.
+#pragma unroll
+            for (int hc = 0; hc < 2; ++hc) {
+              const uint32_t chunk = 2 * c + hc;
+              const uint32_t atom = chunk >> 3, cc = chunk & 7;
+              *reinterpret_cast<uint4*>(dst + atom * kTileBytes + ((cc ^ sw) << 4)) =
+                  make_uint4(outw[4 * hc], outw[4 * hc + 1], outw[4 * hc + 2], outw[4 * hc + 3]);
+            }
           }
-          // bf16 chunks 2c and 2c+1 (8 elements each) of the MN-major SW128 layout:
-          // atom a = chunk / 8 holds head_dim [64a, 64a + 64); rows are keys.
-#pragma unroll
-          for (int hc = 0; hc < 2; ++hc) {
-            const uint32_t chunk = 2 * c + hc;
-            const uint32_t atom = chunk >> 3, cc = chunk & 7;
-            *reinterpret_cast<uint4*>(dst + atom * kTileBytes + ((cc ^ sw) << 4)) =
-                make_uint4(outw[4 * hc], outw[4 * hc + 1], outw[4 * hc + 2], outw[4 * hc + 3]);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive(&bars[kBarVbfFull + sb]);
+            mbar_arrive(&bars[kBarVEmpty + s]);
           }
+          ++vc;
         }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(&bars[kBarVbfFull + sb]);
-          mbar_arrive(&bars[kBarVEmpty + s]);
-        }
-        ++vc;
       }
     }
   }

@@ -241,6 +241,22 @@ lpfa_status lpfa_cast_e4m3(const void* v_bf16, int64_t tok_stride, int64_t head_
   return LPFA_OK;
 }
 
+// The attention kernel moves registers between its warpgroups with setmaxnreg; the split
+// adds up to exactly the launch allocation of kLaunchRegs per thread, so a build whose
+// register count differs is refused here instead of launched (a larger split than the
+// allocation would never be granted). Also raises the dynamic shared memory limit.
+static lpfa_status check_attn_kernel(const void* fn) {
+  cudaFuncAttributes attr;
+  cudaError_t e = cudaFuncGetAttributes(&attr, fn);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncGetAttributes");
+  if (attr.numRegs != lpfa::kLaunchRegs)
+    return fail(LPFA_ERR_UNSUPPORTED, "attention kernel built with %d registers per thread; its warpgroup register "
+                "split needs exactly %d", attr.numRegs, lpfa::kLaunchRegs);
+  e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, lpfa::kAttnSmemBytes);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+  return LPFA_OK;
+}
+
 // Internal entry shared with the test hook: debug_stall > 0 forces a bounded wait to run out.
 static lpfa_status attn_fwd_impl(const uint8_t* q, const uint8_t* q_sf, const uint8_t* k, const uint8_t* k_sf,
                                  const uint8_t* v, const uint8_t* v_sf, const lpfa_varlen_meta* meta_q,
@@ -296,12 +312,10 @@ static lpfa_status attn_fwd_impl(const uint8_t* q, const uint8_t* q_sf, const ui
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e;
   if (pv_mode == LPFA_PV_FP8) {
-    e = cudaFuncSetAttribute(lpfa::attn_fwd_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, lpfa::kAttnSmemBytes);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+    if ((st = check_attn_kernel(reinterpret_cast<const void*>(lpfa::attn_fwd_kernel<true>))) != LPFA_OK) return st;
     lpfa::attn_fwd_kernel<true><<<grid, lpfa::kAttnThreads, lpfa::kAttnSmemBytes, s>>>(tq, tk, tv, p);
   } else {
-    e = cudaFuncSetAttribute(lpfa::attn_fwd_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, lpfa::kAttnSmemBytes);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+    if ((st = check_attn_kernel(reinterpret_cast<const void*>(lpfa::attn_fwd_kernel<false>))) != LPFA_OK) return st;
     lpfa::attn_fwd_kernel<false><<<grid, lpfa::kAttnThreads, lpfa::kAttnSmemBytes, s>>>(tq, tk, tv, p);
   }
   e = cudaGetLastError();

@@ -131,6 +131,14 @@ __device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t threads
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
+// Per-warpgroup register budget (every warp of the warpgroup executes the same call).
+template <uint32_t kRegs> __device__ __forceinline__ void setmaxnreg_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegs));
+}
+template <uint32_t kRegs> __device__ __forceinline__ void setmaxnreg_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegs));
+}
+
 // ---------------------------------------------------------------------------------------
 // tcgen05: tensor memory allocation
 // ---------------------------------------------------------------------------------------
@@ -247,6 +255,28 @@ __device__ __forceinline__ void tmem_ld64_sync(uint32_t taddr, uint32_t (&a)[32]
       : LPFA_O8(a, 0), LPFA_O8(a, 8), LPFA_O8(a, 16), LPFA_O8(a, 24),
         LPFA_O8(b, 0), LPFA_O8(b, 8), LPFA_O8(b, 16), LPFA_O8(b, 24)
       : "r"(taddr), "r"(taddr + 32u)
+      : "memory");
+}
+
+// 128 consecutive columns (two x64 loads in flight together), then one wait.
+__device__ __forceinline__ void tmem_ld128_sync(uint32_t taddr, uint32_t (&r)[128]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x64.b32 {"
+      "%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,"
+      "%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,"
+      "%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%128];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x64.b32 {"
+      "%64,%65,%66,%67,%68,%69,%70,%71,%72,%73,%74,%75,%76,%77,%78,%79,"
+      "%80,%81,%82,%83,%84,%85,%86,%87,%88,%89,%90,%91,%92,%93,%94,%95,"
+      "%96,%97,%98,%99,%100,%101,%102,%103,%104,%105,%106,%107,%108,%109,%110,%111,"
+      "%112,%113,%114,%115,%116,%117,%118,%119,%120,%121,%122,%123,%124,%125,%126,%127}, [%129];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : LPFA_O8(r, 0), LPFA_O8(r, 8), LPFA_O8(r, 16), LPFA_O8(r, 24),
+        LPFA_O8(r, 32), LPFA_O8(r, 40), LPFA_O8(r, 48), LPFA_O8(r, 56),
+        LPFA_O8(r, 64), LPFA_O8(r, 72), LPFA_O8(r, 80), LPFA_O8(r, 88),
+        LPFA_O8(r, 96), LPFA_O8(r, 104), LPFA_O8(r, 112), LPFA_O8(r, 120)
+      : "r"(taddr), "r"(taddr + 64u)
       : "memory");
 }
 
