@@ -13,13 +13,17 @@
 // running at the same time stream the same K/V through L2.
 //
 // Warp roles (512 threads, four warpgroups):
-//   warp 0        TMA producer (whole warp, one lane issues): the Q tile + its scale atom once
-//                 per unit, then 128-key K/V tiles (+ atoms) in the order the MMA warp uses them.
-//   warp 1        TMEM allocator and MMA issuer (whole warp, one lane issues):
+//   warp 0        Q/K producer (whole warp, one lane issues TMA): the Q tile + its scale atom
+//                 once per unit, then 128-key K tiles + their scale atoms.
+//   warp 3        V producer: 128-key V tiles (+ scale atoms in bf16 PV mode).
+//   warp 1        TMEM allocator and QK issuer (whole warp, one lane issues):
 //                   S[t & 1] = Q K_t^T  tcgen05.mma kind::mxf8f6f4.block_scale, M128 N128 K128
-//                   O       += P_t V_t  kind::f8f6f4 (fp8 PV) or kind::f16 (bf16 PV), P in TMEM
-//                 QK of tile t is issued as soon as S buffer t & 1 has been read out, ahead of
-//                 the PV of the tiles before it, so a softmax group never waits for its next S.
+//                 as soon as S buffer t & 1 has been read out by its softmax group.
+//   warp 2        PV issuer:  O += P_t V_t  kind::f8f6f4 (fp8 PV) or kind::f16 (bf16 PV), P in
+//                 TMEM. Issuing QK and PV from two warps keeps a wait for the softmax from
+//                 delaying the next QK, and overlaps one warp's barrier waits with the other's
+//                 MMA issue (a tcgen05.mma issue blocks for about as long as the tensor core
+//                 needs to execute the previous one).
 //   warps 4..7    softmax group 0: KV tiles t with t even (t counts all tiles of the CTA).
 //   warps 8..11   softmax group 1: KV tiles t with t odd. In both groups a thread owns one query
 //                 row and all 128 keys of the tile (192 registers after setmaxnreg). The groups
@@ -31,7 +35,7 @@
 // groups: tile t's reference is its own row-maximum ceiling if that exceeds tile t-1's
 // reference by more than a lag, else tile t-1's reference, so P <= 2^(lag + bias) and the
 // reference (and with it l and O) moves rarely and only by exact powers of two. Tile t-1's
-// reference reaches tile t through shared memory right after the other group's row max. In fp8
+// reference reaches tile t through shared memory after the other group's exponentials. In fp8
 // PV mode P is stored as E4M3(2^(bias - m) 2^s) <= 256; the power of two cancels in the final
 // division.
 //
@@ -60,9 +64,12 @@ static_assert(2 * kSoftmaxRegs + 2 * kOtherRegs == 4 * kLaunchRegs, "register sp
 constexpr int kTileM = 128;          // query rows per tile
 constexpr int kTileN = 128;          // keys per KV tile
 constexpr int kQStages = 2;
-constexpr int kKStages = 3;
-constexpr int kVStages = 3;
-constexpr int kVbfStages = 2;
+// K / V / BF16-V ring depths. K tiles are on the QK critical path and their loads see long
+// latencies while every SM streams the same head's K/V through L2, so in fp8 PV mode (no
+// BF16 V buffers) the shared memory goes to deeper K and V rings.
+template <bool kFp8PV> struct Stages;
+template <> struct Stages<true> { static constexpr int k = 6, v = 5, vbf = 1; };
+template <> struct Stages<false> { static constexpr int k = 3, v = 3, vbf = 2; };
 constexpr uint32_t kTileBytes = 128 * 128;     // 128 rows x 128 fp8
 constexpr uint32_t kVbfBytes = 128 * 128 * 2;  // 128 keys x 128 bf16
 constexpr uint32_t kAtomBytes = 512;
@@ -82,7 +89,7 @@ constexpr float kLn2 = 0.69314718055994531f;
 enum WaitSite : int {
   kSiteProducerQ = 1, kSiteProducerK, kSiteProducerV, kSiteMmaQ, kSiteMmaK, kSiteMmaP,
   kSiteMmaV, kSiteMmaO, kSiteSoftS, kSiteSoftRed, kSiteSoftPV, kSiteSoftL, kSiteConvV,
-  kSiteConvE, kSiteDrain, kSiteDebugStall, kSiteMmaS, kSiteSoftO
+  kSiteConvE, kSiteDrain, kSiteDebugStall, kSiteMmaS, kSiteSoftO, kSiteTmem
 };
 
 struct AttnParams {
@@ -107,38 +114,46 @@ struct AttnParams {
 };
 
 // Shared memory layout (offsets from a 1024-byte aligned base).
+template <bool kFp8PV>
 struct SmemLayout {
+  static constexpr int kK = Stages<kFp8PV>::k, kV = Stages<kFp8PV>::v, kVbf = Stages<kFp8PV>::vbf;
   static constexpr uint32_t q = 0;
   static constexpr uint32_t k = q + kQStages * kTileBytes;
-  static constexpr uint32_t v = k + kKStages * kTileBytes;
-  static constexpr uint32_t vbf = v + kVStages * kTileBytes;          // bf16 PV mode
-  static constexpr uint32_t q_sf = vbf + kVbfStages * kVbfBytes;
+  static constexpr uint32_t v = k + kK * kTileBytes;
+  static constexpr uint32_t vbf = v + kV * kTileBytes;                // bf16 PV mode
+  static constexpr uint32_t q_sf = vbf + (kFp8PV ? 0 : kVbf * kVbfBytes);
   static constexpr uint32_t k_sf = q_sf + kQStages * kAtomBytes;
-  static constexpr uint32_t v_sf = k_sf + kKStages * kAtomBytes;
-  static constexpr uint32_t mref = v_sf + kVStages * kAtomBytes;      // float [2 groups][128] tile reference
+  static constexpr uint32_t v_sf = k_sf + kK * kAtomBytes;
+  static constexpr uint32_t mref = v_sf + kV * kAtomBytes;            // float [2 groups][128] tile reference
   static constexpr uint32_t lsum = mref + 2 * 128 * 4;                // float [2 groups][128] partial l
   static constexpr uint32_t mfin = lsum + 2 * 128 * 4;                // float [2 groups][128] reference of l
   static constexpr uint32_t bars = mfin + 2 * 128 * 4;                // uint64 barriers
-  static constexpr uint32_t num_bars = 40;
+  static constexpr uint32_t num_bars = 64;
   static constexpr uint32_t misc = bars + num_bars * 8;               // tmem base, abort flag
   static constexpr uint32_t total = misc + 64;
 };
-constexpr uint32_t kAttnSmemBytes = SmemLayout::total + 1024;  // + alignment slack
+template <bool kFp8PV> constexpr uint32_t attn_smem_bytes() { return SmemLayout<kFp8PV>::total + 1024; }  // + alignment slack
+static_assert(attn_smem_bytes<true>() <= 227 * 1024 && attn_smem_bytes<false>() <= 227 * 1024, "shared memory");
 
 // Barrier indices. [2]-sized entries are indexed by softmax group / S buffer b.
 enum Bar : int {
-  kBarQFull = 0, kBarQEmpty = 2, kBarKFull = 4, kBarKEmpty = 7, kBarVFull = 10, kBarVEmpty = 13,
-  kBarVbfFull = 16, kBarVbfEmpty = 18,
-  kBarSFull = 20,    // S(t) computed                       (MMA commit)
-  kBarSFree = 22,    // S(t) read out by its group            (4 warps)
-  kBarPReady = 24,   // P(t) stored, O rescaled if needed     (4 warps)
-  kBarPVDone = 26,   // PV(t) complete                        (MMA commit)
-  kBarMRef = 28,     // tile reference of t published         (4 warps)
-  kBarOFull = 30,    // every PV of the unit complete         (MMA commit)
-  kBarOEmpty = 31,   // O read out by both groups             (8 warps)
-  kBarLReady = 32,   // partial l / reference exchanged       (8 warps)
-  kBarDrain = 33
+  kBarQFull = 0, kBarQEmpty = 2,         // [kQStages]
+  kBarKFull = 4, kBarKEmpty = 10,        // [up to 6]
+  kBarVFull = 16, kBarVEmpty = 22,       // [up to 6]
+  kBarVbfFull = 28, kBarVbfEmpty = 30,   // [2]
+  kBarSFull = 32,    // S(t) computed                       (MMA commit)
+  kBarSFree = 34,    // S(t) read out by its group            (4 warps)
+  kBarPReady = 36,   // P(t) stored, O rescaled if needed     (4 warps)
+  kBarPVDone = 38,   // PV(t) complete                        (MMA commit)
+  kBarOFull = 40,    // every PV of the unit complete         (MMA commit)
+  kBarOEmpty = 41,   // O read out by both groups             (8 warps)
+  kBarLReady = 42,   // partial l / reference exchanged       (8 warps)
+  kBarDrain = 43,    // QK issuer's own tcgen05 work done
+  kBarDrainPV = 44,  // PV issuer's own tcgen05 work done
+  kBarMRef = 48      // [group][lane quarter]: tile reference of t published and the MUFU
+                     // handed over to the other group (1 warp; 8 entries)
 };
+static_assert(Stages<true>::k <= 6 && Stages<true>::v <= 6 && Stages<false>::k <= 6 && Stages<false>::v <= 6, "ring barriers");
 
 // UMMA shared-memory matrix descriptor (sm_100 format, version 1).
 __device__ __forceinline__ uint64_t umma_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo, uint32_t layout) {
@@ -237,23 +252,44 @@ __device__ __forceinline__ float rowmax128(const float2 (&s)[64]) {
   return fmaxf(max3f(b0, b1, b2), max3f(b3, b4, a[15]));
 }
 
+// How many of a row's 64 exponential pairs are issued before a softmax group hands the MUFU
+// over to the other group (see the softmax loop). Handing over a little before the end
+// hides the hand-over latency behind the last exponentials.
+#ifndef LPFA_HANDOFF_PAIRS
+#define LPFA_HANDOFF_PAIRS 40
+#endif
+constexpr int kHandoffPairs = LPFA_HANDOFF_PAIRS;
+static_assert(kHandoffPairs >= 1 && kHandoffPairs <= 64, "hand-over point out of range");
+
 // p = 2^(s * c + nb) in place; masked keys (tail tiles) become exactly 0. Returns sum of p.
-template <bool kTail, int kPoly>
-__device__ __forceinline__ float exp_row(float2 (&s)[64], float c, float nb, int key0, int klen) {
+// Written in passes (exponents, exponentials, sum) so that the MUFU operations issue back to
+// back at the MUFU rate. handoff(x) runs after the first kHandoffPairs pairs, with x one of
+// their results (a data dependency that keeps it from being scheduled earlier).
+template <bool kTail, int kPoly, typename F>
+__device__ __forceinline__ float exp_row(float2 (&s)[64], float c, float nb, int key0, int klen, F&& handoff) {
   const float2 c2 = make_float2(c, c), nb2 = make_float2(nb, nb);
-  float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
-  for (int i = 0; i < 64; ++i) {
-    const float2 x = __ffma2_rn(s[i], c2, nb2);
-    float2 e = ((i & 7) < kPoly) ? exp2_poly2(x) : exp2_mufu2(x);
-    if (kTail) {
-      if (key0 + 2 * i >= klen) e.x = 0.0f;
-      if (key0 + 2 * i + 1 >= klen) e.y = 0.0f;
+  for (int i = 0; i < 64; ++i) s[i] = __ffma2_rn(s[i], c2, nb2);
+#pragma unroll
+  for (int i = 0; i < kHandoffPairs; ++i) s[i] = ((i & 7) < kPoly) ? exp2_poly2(s[i]) : exp2_mufu2(s[i]);
+  handoff(s[kHandoffPairs - 1].y);
+#pragma unroll
+  for (int i = kHandoffPairs; i < 64; ++i) s[i] = ((i & 7) < kPoly) ? exp2_poly2(s[i]) : exp2_mufu2(s[i]);
+  if (kTail) {
+#pragma unroll
+    for (int i = 0; i < 64; ++i) {
+      if (key0 + 2 * i >= klen) s[i].x = 0.0f;
+      if (key0 + 2 * i + 1 >= klen) s[i].y = 0.0f;
     }
-    s[i] = e;
-    acc[i & 3] = __fadd2_rn(acc[i & 3], e);
   }
-  const float2 t = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
+  float2 acc[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) acc[k] = s[k];
+#pragma unroll
+  for (int i = 8; i < 64; ++i) acc[i & 7] = __fadd2_rn(acc[i & 7], s[i]);
+  const float2 t0 = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
+  const float2 t1 = __fadd2_rn(__fadd2_rn(acc[4], acc[5]), __fadd2_rn(acc[6], acc[7]));
+  const float2 t = __fadd2_rn(t0, t1);
   return t.x + t.y;
 }
 
@@ -327,24 +363,21 @@ template <bool kFp8PV> struct SoftmaxLag;
 template <> struct SoftmaxLag<true> { static constexpr float lag = 2.0f; static constexpr float bias = 6.0f; };
 template <> struct SoftmaxLag<false> { static constexpr float lag = 8.0f; static constexpr float bias = 0.0f; };
 
-// How many tiles the PV issue trails the QK issue. fp8 P has its own TMEM buffer, so QK(t)
-// may overwrite S buffer t & 1 before PV(t - 2) has run; bf16 P lives in the S buffer, so
-// PV(t - 2) must be issued before QK(t).
-template <bool kFp8PV> struct PvLag { static constexpr int value = kFp8PV ? 2 : 1; };
 
 template <bool kFp8PV>
 __global__ void __launch_bounds__(kAttnThreads, 1)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                 const __grid_constant__ CUtensorMap tmap_v, const AttnParams p) {
+  using L = SmemLayout<kFp8PV>;
+  constexpr int kKStages = Stages<kFp8PV>::k, kVStages = Stages<kFp8PV>::v, kVbfStages = Stages<kFp8PV>::vbf;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SmemLayout::bars);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + SmemLayout::misc);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + SmemLayout::misc + 16);
-  float* mref = reinterpret_cast<float*>(smem + SmemLayout::mref);
-  float* lsum = reinterpret_cast<float*>(smem + SmemLayout::lsum);
-  float* mfin = reinterpret_cast<float*>(smem + SmemLayout::mfin);
-  constexpr int kLagPV = PvLag<kFp8PV>::value;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::bars);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::misc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::misc + 16);
+  float* mref = reinterpret_cast<float*>(smem + L::mref);
+  float* lsum = reinterpret_cast<float*>(smem + L::lsum);
+  float* mfin = reinterpret_cast<float*>(smem + L::mfin);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -362,12 +395,13 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
       mbar_init(&bars[kBarSFree + i], 4);
       mbar_init(&bars[kBarPReady + i], 4);
       mbar_init(&bars[kBarPVDone + i], 1);
-      mbar_init(&bars[kBarMRef + i], 4);
     }
     mbar_init(&bars[kBarOFull], 1);
     mbar_init(&bars[kBarOEmpty], 8);
     mbar_init(&bars[kBarLReady], 8);
     mbar_init(&bars[kBarDrain], 1);
+    mbar_init(&bars[kBarDrainPV], 1);
+    for (int i = 0; i < 8; ++i) mbar_init(&bars[kBarMRef + i], 1);
     *abort_flag = 0;
     mbar_fence_init();
   }
@@ -380,55 +414,47 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
+  // All 512 columns of the SM's tensor memory belong to this CTA (one CTA per SM), so the
+  // allocation starts at lane 0, column 0. Using the constant keeps every TMEM operand of
+  // the tcgen05 instructions a compile-time or warp-uniform value.
+  constexpr uint32_t tmem = 0;
+  const bool tmem_ok = *tmem_slot == tmem;
+  if (!tmem_ok && threadIdx.x == 0) record_failure(abort_flag, kSiteTmem);
 
   const int G = gridDim.x;
 
-  if (warp < 4) {
+  if (!tmem_ok) {
+    // nothing issued; fall through to the teardown
+  } else if (warp < 4) {
     setmaxnreg_dec<kOtherRegs>();
     if (warp == 0) {
-      // ---------------------------------------------------------------- TMA producer
+      // ---------------------------------------------------------------- Q/K producer
       // The whole warp runs the loop (warp-uniform state); lane 0 issues the copies.
       const uint32_t leader = lane == 0 ? 1u : 0u;
-      uint32_t qc = 0, kc = 0, vc = 0;  // fills issued per ring
+      uint32_t qc = 0, kc = 0;  // fills issued per ring
       bool ok = true;
-      auto load_v = [&](const UnitInfo& ui, int jj) -> bool {
-        const uint32_t s = vc % kVStages, ph = (vc / kVStages) & 1;
-        if (!mbar_wait_warp(&bars[kBarVEmpty + s], ph ^ 1, abort_flag)) { record_failure(abort_flag, kSiteProducerV); return false; }
-        mbar_arrive_expect_tx(&bars[kBarVFull + s], kTileBytes + (kFp8PV ? 0 : kAtomBytes), leader);
-        tma_load_3d(smem + SmemLayout::v + s * kTileBytes, &tmap_v, &bars[kBarVFull + s], 0, ui.h,
-                    ui.k_row0 + jj * kTileN, leader);
-        if (!kFp8PV)
-          bulk_load(smem + SmemLayout::v_sf + s * kAtomBytes,
-                    p.v_sf + (static_cast<int64_t>(ui.sbk + jj) * p.heads + ui.h) * kAtomBytes, kAtomBytes,
-                    &bars[kBarVFull + s], leader);
-        ++vc;
-        return true;
-      };
       for (int w = blockIdx.x; w < p.num_units && ok; w += G) {
         const UnitInfo ui = warp_uniform(unit_info(p, w));
         if (ui.nkv == 0) continue;  // no keys: the softmax warps write the empty-sum result
         const uint32_t qs = qc % kQStages, qph = (qc / kQStages) & 1;
         if (!mbar_wait_warp(&bars[kBarQEmpty + qs], qph ^ 1, abort_flag)) { record_failure(abort_flag, kSiteProducerQ); ok = false; break; }
         mbar_arrive_expect_tx(&bars[kBarQFull + qs], kTileBytes + kAtomBytes, leader);
-        tma_load_3d(smem + SmemLayout::q + qs * kTileBytes, &tmap_q, &bars[kBarQFull + qs], 0, ui.h, ui.q_row0, leader);
-        bulk_load(smem + SmemLayout::q_sf + qs * kAtomBytes,
+        tma_load_3d(smem + L::q + qs * kTileBytes, &tmap_q, &bars[kBarQFull + qs], 0, ui.h, ui.q_row0, leader);
+        bulk_load(smem + L::q_sf + qs * kAtomBytes,
                   p.q_sf + (static_cast<int64_t>(ui.sbq + ui.qtile) * p.heads + ui.h) * kAtomBytes, kAtomBytes,
                   &bars[kBarQFull + qs], leader);
         ++qc;
-        for (int j = 0; j < ui.nkv && ok; ++j) {
+        for (int j = 0; j < ui.nkv; ++j) {
           const uint32_t s = kc % kKStages, ph = (kc / kKStages) & 1;
           if (!mbar_wait_warp(&bars[kBarKEmpty + s], ph ^ 1, abort_flag)) { record_failure(abort_flag, kSiteProducerK); ok = false; break; }
           mbar_arrive_expect_tx(&bars[kBarKFull + s], kTileBytes + kAtomBytes, leader);
-          tma_load_3d(smem + SmemLayout::k + s * kTileBytes, &tmap_k, &bars[kBarKFull + s], 0, ui.h,
+          tma_load_3d(smem + L::k + s * kTileBytes, &tmap_k, &bars[kBarKFull + s], 0, ui.h,
                       ui.k_row0 + j * kTileN, leader);
-          bulk_load(smem + SmemLayout::k_sf + s * kAtomBytes,
+          bulk_load(smem + L::k_sf + s * kAtomBytes,
                     p.k_sf + (static_cast<int64_t>(ui.sbk + j) * p.heads + ui.h) * kAtomBytes, kAtomBytes,
                     &bars[kBarKFull + s], leader);
           ++kc;
-          if (j >= kLagPV) ok = load_v(ui, j - kLagPV);
         }
-        for (int jj = ui.nkv > kLagPV ? ui.nkv - kLagPV : 0; jj < ui.nkv && ok; ++jj) ok = load_v(ui, jj);
       }
       // Drain: every copy issued here must land before the CTA exits. The newest fill of each
       // stage is the last one issued into it; older fills of that stage were consumed already.
@@ -436,65 +462,55 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
         if (!mbar_wait(&bars[kBarQFull + i % kQStages], (i / kQStages) & 1, nullptr)) record_failure(abort_flag, kSiteDrain);
       for (uint32_t i = (kc > kKStages ? kc - kKStages : 0); i < kc; ++i)
         if (!mbar_wait(&bars[kBarKFull + i % kKStages], (i / kKStages) & 1, nullptr)) record_failure(abort_flag, kSiteDrain);
+    } else if (warp == 3) {
+      // ---------------------------------------------------------------- V producer
+      // A warp of its own, so that K loads (and with them QK) never wait behind a V stage
+      // that the PV of a slower softmax tile still holds.
+      const uint32_t leader = lane == 0 ? 1u : 0u;
+      uint32_t vc = 0;
+      bool ok = true;
+      for (int w = blockIdx.x; w < p.num_units && ok; w += G) {
+        const UnitInfo ui = warp_uniform(unit_info(p, w));
+        for (int j = 0; j < ui.nkv; ++j) {
+          const uint32_t s = vc % kVStages, ph = (vc / kVStages) & 1;
+          if (!mbar_wait_warp(&bars[kBarVEmpty + s], ph ^ 1, abort_flag)) { record_failure(abort_flag, kSiteProducerV); ok = false; break; }
+          mbar_arrive_expect_tx(&bars[kBarVFull + s], kTileBytes + (kFp8PV ? 0 : kAtomBytes), leader);
+          tma_load_3d(smem + L::v + s * kTileBytes, &tmap_v, &bars[kBarVFull + s], 0, ui.h,
+                      ui.k_row0 + j * kTileN, leader);
+          if (!kFp8PV)
+            bulk_load(smem + L::v_sf + s * kAtomBytes,
+                      p.v_sf + (static_cast<int64_t>(ui.sbk + j) * p.heads + ui.h) * kAtomBytes, kAtomBytes,
+                      &bars[kBarVFull + s], leader);
+          ++vc;
+        }
+      }
       for (uint32_t i = (vc > kVStages ? vc - kVStages : 0); i < vc; ++i)
         if (!mbar_wait(&bars[kBarVFull + i % kVStages], (i / kVStages) & 1, nullptr)) record_failure(abort_flag, kSiteDrain);
     } else if (warp == 1) {
-      // ---------------------------------------------------------------- MMA issuer
-      // The whole warp runs the loop (warp-uniform state); lane 0 issues the tcgen05 instructions.
+      // ---------------------------------------------------------------- QK issuer
+      // S(t) = Q K_t^T into S buffer t & 1. The whole warp runs the loop (warp-uniform state);
+      // lane 0 issues the tcgen05 instructions.
       const uint32_t leader = lane == 0 ? 1u : 0u;
       const float qd = p.q_descale ? __ldg(p.q_descale) : 1.0f;
       const float kd = p.k_descale ? __ldg(p.k_descale) : 1.0f;
       const int negate = (qd * kd) < 0.0f ? 1 : 0;
       // Descriptor bases; the start-address field is the low 14 bits (address >> 4), so a byte
       // offset b inside shared memory advances a descriptor by b >> 4.
-      const uint64_t dq0 = umma_desc(smem_u32(smem + SmemLayout::q), 16, 1024, kLayoutSw128);
-      const uint64_t dk0 = umma_desc(smem_u32(smem + SmemLayout::k), 16, 1024, kLayoutSw128);
-      const uint64_t dv0 = kFp8PV ? umma_desc(smem_u32(smem + SmemLayout::v), kTileBytes, 1024, kLayoutSw128)
-                                  : umma_desc(smem_u32(smem + SmemLayout::vbf), kTileBytes, 1024, kLayoutSw128);
-      const uint64_t dqsf0 = umma_desc(smem_u32(smem + SmemLayout::q_sf), 0, 128, kLayoutNone);
-      const uint64_t dksf0 = umma_desc(smem_u32(smem + SmemLayout::k_sf), 0, 128, kLayoutNone);
+      const uint32_t sb = static_cast<uint32_t>(warp_uniform(static_cast<int>(smem_u32(smem))));
+      const uint64_t dq0 = umma_desc(sb + L::q, 16, 1024, kLayoutSw128);
+      const uint64_t dk0 = umma_desc(sb + L::k, 16, 1024, kLayoutSw128);
+      const uint64_t dqsf0 = umma_desc(sb + L::q_sf, 0, 128, kLayoutNone);
+      const uint64_t dksf0 = umma_desc(sb + L::k_sf, 0, 128, kLayoutNone);
       uint32_t idq[4];
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk) idq[kk] = idesc_qk(kk, negate);
-      uint32_t u = 0, kc = 0, vc = 0, t0 = 0;  // units, K fills, V tiles, first tile of the unit
+      uint32_t u = 0, kc = 0, t = 0;  // units, K fills, tiles
       bool ok = true;
       if (p.debug_stall > 0) {
         // Test hook: wait for a phase of the drain barrier that nothing completes before the
-        // drain below, so the wait runs out and the failure path is exercised.
+        // drains below, so the wait runs out and the failure path is exercised.
         if (!mbar_wait_warp(&bars[kBarDrain], 0, abort_flag)) { record_failure(abort_flag, kSiteDebugStall); ok = false; }
       }
-      // O += P(t) V(t); jj is t's index within the unit.
-      auto issue_pv = [&](uint32_t t, int jj) -> bool {
-        const uint32_t b = t & 1;
-        if (!mbar_wait_warp(&bars[kBarPReady + b], (t >> 1) & 1, abort_flag)) { record_failure(abort_flag, kSiteMmaP); return false; }
-        if (jj == 0) {
-          if (!mbar_wait_warp(&bars[kBarOEmpty], (u & 1) ^ 1, abort_flag)) { record_failure(abort_flag, kSiteMmaO); return false; }
-        }
-        const bool got = kFp8PV ? mbar_wait_warp(&bars[kBarVFull + vc % kVStages], (vc / kVStages) & 1, abort_flag)
-                                : mbar_wait_warp(&bars[kBarVbfFull + vc % kVbfStages], (vc / kVbfStages) & 1, abort_flag);
-        if (!got) { record_failure(abort_flag, kSiteMmaV); return false; }
-        tc_fence_after();
-        if (kFp8PV) {
-          const uint32_t p_col = tmem + kColP + b * 32;
-          const uint64_t bdesc = dv0 + ((vc % kVStages) * kTileBytes >> 4);
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)  // keys [32kk, 32kk + 32): 8 columns of 4 E4M3 each
-            mma_f8f6f4_ts(tmem + kColO, p_col + kk * 8, bdesc + kk * 256, kIdescPV8,
-                          (jj > 0 || kk > 0) ? 1u : 0u, leader);
-          mma_commit(&bars[kBarVEmpty + vc % kVStages], leader);
-        } else {
-          const uint32_t p_col = tmem + kColS + b * 128;
-          const uint64_t bdesc = dv0 + ((vc % kVbfStages) * kVbfBytes >> 4);
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)  // keys [16kk, 16kk + 16): 8 columns of 2 BF16 each
-            mma_f16_ts(tmem + kColO, p_col + kk * 8, bdesc + kk * 128, kIdescPV16,
-                       (jj > 0 || kk > 0) ? 1u : 0u, leader);
-          mma_commit(&bars[kBarVbfEmpty + vc % kVbfStages], leader);
-        }
-        mma_commit(&bars[kBarPVDone + b], leader);
-        ++vc;
-        return true;
-      };
       for (int w = blockIdx.x; w < p.num_units && ok; w += G) {
         const UnitInfo ui = warp_uniform(unit_info(p, w));
         if (ui.nkv == 0) continue;
@@ -504,11 +520,14 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
         const uint32_t sfa = tmem + kColSFA + qs * 4;
         tmem_cp_32x128b_x4(sfa, dqsf0 + (qs * kAtomBytes >> 4), leader);
         const uint64_t adesc = dq0 + (qs * kTileBytes >> 4);
-        for (int j = 0; j < ui.nkv; ++j) {
-          const uint32_t t = t0 + j;
+        for (int j = 0; j < ui.nkv; ++j, ++t) {
           const uint32_t b = t & 1;
-          // S buffer b was read out by its group (tile t - 2).
-          if (t >= 2 && !mbar_wait_warp(&bars[kBarSFree + b], ((t - 2) >> 1) & 1, abort_flag)) { record_failure(abort_flag, kSiteMmaS); ok = false; break; }
+          if (t >= 2) {
+            // S buffer b has been read out by its group (tile t - 2); in bf16 PV mode it also
+            // holds P(t - 2), so PV(t - 2) must have completed.
+            if (!mbar_wait_warp(&bars[kBarSFree + b], ((t - 2) >> 1) & 1, abort_flag)) { record_failure(abort_flag, kSiteMmaS); ok = false; break; }
+            if (!kFp8PV && !mbar_wait_warp(&bars[kBarPVDone + b], ((t - 2) >> 1) & 1, abort_flag)) { record_failure(abort_flag, kSiteMmaS); ok = false; break; }
+          }
           const uint32_t s = kc % kKStages;
           if (!mbar_wait_warp(&bars[kBarKFull + s], (kc / kKStages) & 1, abort_flag)) { record_failure(abort_flag, kSiteMmaK); ok = false; break; }
           tc_fence_after();
@@ -526,21 +545,59 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
           mma_commit(&bars[kBarKEmpty + s], leader);
           if (j == ui.nkv - 1) mma_commit(&bars[kBarQEmpty + qs], leader);
           ++kc;
-          if (j >= kLagPV && !issue_pv(t - kLagPV, j - kLagPV)) { ok = false; break; }
         }
-        if (!ok) break;
-        // The unit's remaining PVs go out before the next unit's QK, which may wait for a
-        // softmax group that first has to finish this unit's epilogue.
-        for (int jj = ui.nkv > kLagPV ? ui.nkv - kLagPV : 0; jj < ui.nkv; ++jj)
-          if (!issue_pv(t0 + jj, jj)) { ok = false; break; }
-        if (!ok) break;
-        mma_commit(&bars[kBarOFull], leader);  // every PV of this unit is complete
-        t0 += ui.nkv;
         ++u;
       }
       // Drain: wait until every tcgen05 operation issued by this warp has completed.
       mma_commit(&bars[kBarDrain], leader);
       if (!mbar_wait(&bars[kBarDrain], 0, nullptr)) record_failure(abort_flag, kSiteDrain);
+    } else if (warp == 2) {
+      // ---------------------------------------------------------------- PV issuer
+      // O += P(t) V(t). A warp of its own, so that waiting for the softmax (PReady) never
+      // holds back the next QK.
+      const uint32_t leader = lane == 0 ? 1u : 0u;
+      const uint32_t sb = static_cast<uint32_t>(warp_uniform(static_cast<int>(smem_u32(smem))));
+      const uint64_t dv0 = kFp8PV ? umma_desc(sb + L::v, kTileBytes, 1024, kLayoutSw128)
+                                  : umma_desc(sb + L::vbf, kTileBytes, 1024, kLayoutSw128);
+      uint32_t u = 0, vc = 0, t = 0;  // units, V tiles, tiles
+      bool ok = true;
+      for (int w = blockIdx.x; w < p.num_units && ok; w += G) {
+        const UnitInfo ui = warp_uniform(unit_info(p, w));
+        if (ui.nkv == 0) continue;
+        for (int j = 0; j < ui.nkv; ++j, ++t) {
+          const uint32_t b = t & 1;
+          if (!mbar_wait_warp(&bars[kBarPReady + b], (t >> 1) & 1, abort_flag)) { record_failure(abort_flag, kSiteMmaP); ok = false; break; }
+          if (j == 0 && !mbar_wait_warp(&bars[kBarOEmpty], (u & 1) ^ 1, abort_flag)) { record_failure(abort_flag, kSiteMmaO); ok = false; break; }
+          const bool got = kFp8PV ? mbar_wait_warp(&bars[kBarVFull + vc % kVStages], (vc / kVStages) & 1, abort_flag)
+                                  : mbar_wait_warp(&bars[kBarVbfFull + vc % kVbfStages], (vc / kVbfStages) & 1, abort_flag);
+          if (!got) { record_failure(abort_flag, kSiteMmaV); ok = false; break; }
+          tc_fence_after();
+          if (kFp8PV) {
+            const uint32_t p_col = tmem + kColP + b * 32;
+            const uint64_t bdesc = dv0 + ((vc % kVStages) * kTileBytes >> 4);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)  // keys [32kk, 32kk + 32): 8 columns of 4 E4M3 each
+              mma_f8f6f4_ts(tmem + kColO, p_col + kk * 8, bdesc + kk * 256, kIdescPV8,
+                            (j > 0 || kk > 0) ? 1u : 0u, leader);
+            mma_commit(&bars[kBarVEmpty + vc % kVStages], leader);
+          } else {
+            const uint32_t p_col = tmem + kColS + b * 128;
+            const uint64_t bdesc = dv0 + ((vc % kVbfStages) * kVbfBytes >> 4);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)  // keys [16kk, 16kk + 16): 8 columns of 2 BF16 each
+              mma_f16_ts(tmem + kColO, p_col + kk * 8, bdesc + kk * 128, kIdescPV16,
+                         (j > 0 || kk > 0) ? 1u : 0u, leader);
+            mma_commit(&bars[kBarVbfEmpty + vc % kVbfStages], leader);
+          }
+          mma_commit(&bars[kBarPVDone + b], leader);
+          ++vc;
+        }
+        if (!ok) break;
+        mma_commit(&bars[kBarOFull], leader);  // every PV of this unit is complete
+        ++u;
+      }
+      mma_commit(&bars[kBarDrainPV], leader);
+      if (!mbar_wait(&bars[kBarDrainPV], 0, nullptr)) record_failure(abort_flag, kSiteDrain);
     }
   } else if (warp < 12) {
     setmaxnreg_inc<kSoftmaxRegs>();
@@ -589,20 +646,25 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
         if (tail) mask_keys(sv, key0, ui.k_len);
         // Every tile has a valid key, so the ceiling is finite.
         const float c_t = ceilf(rowmax128(sv) * cscale);
-        // Reference of tile t - 1 (the other group's), published right after its row max.
-        // Every tile waits for it, even the first of a unit, which keeps the two groups' tile
-        // references in lockstep order.
+        // Reference of tile t - 1 (the other group's). It is published after the other
+        // group's exponentials of tile t - 1, so this wait also hands the MUFU over from one
+        // group to the other: the two groups' exponential phases alternate instead of
+        // competing, and each group's load, max and P stores overlap the other's
+        // exponentials. Every tile waits, even the first of a unit, which keeps the hand-over
+        // (and the tile references) in tile order.
         float m_prev = 0.0f;
         if (t >= 1) {
-          if (!mbar_wait_warp(&bars[kBarMRef + (grp ^ 1)], ((t - 1) >> 1) & 1, abort_flag)) { record_failure(abort_flag, kSiteSoftRed); ok = false; break; }
+          if (!mbar_wait_warp(&bars[kBarMRef + (grp ^ 1) * 4 + quarter], ((t - 1) >> 1) & 1, abort_flag)) { record_failure(abort_flag, kSiteSoftRed); ok = false; break; }
           m_prev = *other_mref;
         }
         const float m_t = (j == 0 || c_t > m_prev + kLag) ? c_t : m_prev;
         *my_mref = m_t;
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars[kBarMRef + grp]);
-        const float psum = tail ? exp_row<true, kPolyPairs>(sv, cscale, kBias - m_t, key0, ui.k_len)
-                                : exp_row<false, kPolyPairs>(sv, cscale, kBias - m_t, key0, ui.k_len);
+        auto handoff = [&](float dep) {
+          __syncwarp();
+          if (lane == 0) mbar_arrive_after(&bars[kBarMRef + grp * 4 + quarter], dep);
+        };
+        const float psum = tail ? exp_row<true, kPolyPairs>(sv, cscale, kBias - m_t, key0, ui.k_len, handoff)
+                                : exp_row<false, kPolyPairs>(sv, cscale, kBias - m_t, key0, ui.k_len, handoff);
         l_g = l_g * exp2_int(m_g - m_t) + psum;
         m_g = m_t;
         // PV(t - 2) has read this group's previous P.
@@ -712,9 +774,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
           const uint32_t sb = vc % kVbfStages, phb = (vc / kVbfStages) & 1;
           if (!mbar_wait_warp(&bars[kBarVFull + s], ph, abort_flag)) { record_failure(abort_flag, kSiteConvV); ok = false; break; }
           if (!mbar_wait_warp(&bars[kBarVbfEmpty + sb], phb ^ 1, abort_flag)) { record_failure(abort_flag, kSiteConvE); ok = false; break; }
-          const uint8_t* src = smem + SmemLayout::v + s * kTileBytes + t * 128;
-          const uint32_t sfw = reinterpret_cast<const uint32_t*>(smem + SmemLayout::v_sf + s * kAtomBytes)[(t & 31) * 4 + (t >> 5)];
-          uint8_t* dst = smem + SmemLayout::vbf + sb * kVbfBytes + t * 128;
+          const uint8_t* src = smem + L::v + s * kTileBytes + t * 128;
+          const uint32_t sfw = reinterpret_cast<const uint32_t*>(smem + L::v_sf + s * kAtomBytes)[(t & 31) * 4 + (t >> 5)];
+          uint8_t* dst = smem + L::vbf + sb * kVbfBytes + t * 128;
 #pragma unroll
           for (int c = 0; c < 8; ++c) {  // 16 fp8 values: head_dim [16c, 16c + 16)
             const uint4 raw = *reinterpret_cast<const uint4*>(src + ((static_cast<uint32_t>(c) ^ sw) << 4));
@@ -758,7 +820,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, kTmemCols);
+    tmem_dealloc(*tmem_slot, kTmemCols);  // the address the allocation returned
   }
 }
 

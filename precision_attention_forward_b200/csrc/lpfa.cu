@@ -245,14 +245,14 @@ lpfa_status lpfa_cast_e4m3(const void* v_bf16, int64_t tok_stride, int64_t head_
 // adds up to exactly the launch allocation of kLaunchRegs per thread, so a build whose
 // register count differs is refused here instead of launched (a larger split than the
 // allocation would never be granted). Also raises the dynamic shared memory limit.
-static lpfa_status check_attn_kernel(const void* fn) {
+static lpfa_status check_attn_kernel(const void* fn, uint32_t smem_bytes) {
   cudaFuncAttributes attr;
   cudaError_t e = cudaFuncGetAttributes(&attr, fn);
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncGetAttributes");
   if (attr.numRegs != lpfa::kLaunchRegs)
     return fail(LPFA_ERR_UNSUPPORTED, "attention kernel built with %d registers per thread; its warpgroup register "
                 "split needs exactly %d", attr.numRegs, lpfa::kLaunchRegs);
-  e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, lpfa::kAttnSmemBytes);
+  e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem_bytes));
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
   return LPFA_OK;
 }
@@ -312,11 +312,11 @@ static lpfa_status attn_fwd_impl(const uint8_t* q, const uint8_t* q_sf, const ui
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e;
   if (pv_mode == LPFA_PV_FP8) {
-    if ((st = check_attn_kernel(reinterpret_cast<const void*>(lpfa::attn_fwd_kernel<true>))) != LPFA_OK) return st;
-    lpfa::attn_fwd_kernel<true><<<grid, lpfa::kAttnThreads, lpfa::kAttnSmemBytes, s>>>(tq, tk, tv, p);
+    if ((st = check_attn_kernel(reinterpret_cast<const void*>(lpfa::attn_fwd_kernel<true>), lpfa::attn_smem_bytes<true>())) != LPFA_OK) return st;
+    lpfa::attn_fwd_kernel<true><<<grid, lpfa::kAttnThreads, lpfa::attn_smem_bytes<true>(), s>>>(tq, tk, tv, p);
   } else {
-    if ((st = check_attn_kernel(reinterpret_cast<const void*>(lpfa::attn_fwd_kernel<false>))) != LPFA_OK) return st;
-    lpfa::attn_fwd_kernel<false><<<grid, lpfa::kAttnThreads, lpfa::kAttnSmemBytes, s>>>(tq, tk, tv, p);
+    if ((st = check_attn_kernel(reinterpret_cast<const void*>(lpfa::attn_fwd_kernel<false>), lpfa::attn_smem_bytes<false>())) != LPFA_OK) return st;
+    lpfa::attn_fwd_kernel<false><<<grid, lpfa::kAttnThreads, lpfa::attn_smem_bytes<false>(), s>>>(tq, tk, tv, p);
   }
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "attention launch");
