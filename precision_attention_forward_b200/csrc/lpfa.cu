@@ -106,6 +106,28 @@ lpfa_status payload_tmap(CUtensorMap* map, const void* base, int64_t tokens, int
   return LPFA_OK;
 }
 
+// Tensor map over a strided (tokens, heads, 128) input of bf16 or fp32 elements; box = 128
+// tokens of one head, no swizzle. A dimension of extent 1 gets a dummy stride (it is never
+// stepped over).
+lpfa_status input_tmap(CUtensorMap* map, const void* base, bool fp32, int64_t tokens, int heads, int64_t tok_stride,
+                       int64_t head_stride) {
+  auto fn = encode_fn();
+  if (!fn) return fail(LPFA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  const int64_t es = fp32 ? 4 : 2;
+  const int64_t hs = heads > 1 ? head_stride * es : 128 * es;
+  const int64_t ts = tokens > 1 ? tok_stride * es : 128 * es * heads;
+  if (hs <= 0 || ts <= 0) return fail(LPFA_ERR_INVALID_ARG, "strides must be positive");
+  cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(heads), static_cast<cuuint64_t>(tokens)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(hs), static_cast<cuuint64_t>(ts)};
+  cuuint32_t box[3] = {128, 1, 128};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, fp32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                  const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(LPFA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  return LPFA_OK;
+}
+
 lpfa_status check_meta(const lpfa_varlen_meta* m, const char* name) {
   if (!m) return fail(LPFA_ERR_INVALID_ARG, "%s is NULL", name);
   if (!m->dev) return fail(LPFA_ERR_INVALID_ARG, "%s has no device buffer", name);
@@ -175,6 +197,25 @@ lpfa_status lpfa_varlen_meta_from_lengths(const int32_t* lengths_host, int32_t n
   return LPFA_OK;
 }
 
+// Persistent launch of the streaming quantize/cast kernel: as many CTAs as fit on the SMs
+// (shared-memory bound), each walking tiles with the grid stride.
+static lpfa_status launch_quant(void (*kernel)(const CUtensorMap, lpfa::QuantParams), uint32_t smem, int threads,
+                                const CUtensorMap& tmap, const lpfa::QuantParams& p, int sms, cudaStream_t s,
+                                const char* what) {
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+  int per_sm = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, smem);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor");
+  if (per_sm < 1) return fail(LPFA_ERR_UNSUPPORTED, "%s: kernel does not fit on an SM", what);
+  const int64_t tiles = static_cast<int64_t>(p.num_blocks) * p.heads;
+  const int64_t grid = tiles < static_cast<int64_t>(per_sm) * sms ? tiles : static_cast<int64_t>(per_sm) * sms;
+  kernel<<<static_cast<unsigned>(grid), threads, smem, s>>>(tmap, p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, what);
+  return LPFA_OK;
+}
+
 lpfa_status lpfa_quantize_mxfp8_varlen(const void* x, lpfa_in_dtype dt, int64_t tok_stride, int64_t head_stride,
                                        int32_t heads, int32_t head_dim, const lpfa_varlen_meta* meta,
                                        lpfa_scaling_mode mode, uint8_t* payload, uint8_t* scales, void* stream) {
@@ -189,10 +230,9 @@ lpfa_status lpfa_quantize_mxfp8_varlen(const void* x, lpfa_in_dtype dt, int64_t 
   if (!aligned16(x) || !aligned16(payload) || (tok_stride % vec) || (head_stride % vec))
     return fail(LPFA_ERR_INVALID_ARG, "x/payload must be 16-byte aligned with strides multiple of %d elements", vec);
   if (!aligned16(scales)) return fail(LPFA_ERR_INVALID_ARG, "scales must be 16-byte aligned");
-  if (heads > 65535) return fail(LPFA_ERR_INVALID_ARG, "at most 65535 heads per launch");
   DeviceInfo info;
   if ((st = require_sm100(&info)) != LPFA_OK) return st;
-  lpfa::QuantParams p;
+  lpfa::QuantParams p = {};
   p.x = x;
   p.tok_stride = tok_stride;
   p.head_stride = head_stride;
@@ -200,18 +240,22 @@ lpfa_status lpfa_quantize_mxfp8_varlen(const void* x, lpfa_in_dtype dt, int64_t 
   p.num_seqs = meta->num_seqs;
   p.cu_seqlens = meta->dev;
   p.scale_off = meta->dev + meta->num_seqs + 1;
+  p.num_blocks = meta->total_scale_blocks;
   p.payload = payload;
   p.scales = scales;
   p.floor_mode = mode == LPFA_SCALE_FLOOR ? 1 : 0;
-  dim3 grid(meta->total_scale_blocks, heads);
+  if (static_cast<int64_t>(p.num_blocks) * heads > INT32_MAX) return fail(LPFA_ERR_INVALID_ARG, "too many tiles");
+  CUtensorMap tm;
+  if ((st = input_tmap(&tm, x, dt == LPFA_IN_FP32, meta->total_tokens, heads, tok_stride, head_stride)) != LPFA_OK)
+    return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (dt == LPFA_IN_BF16)
-    lpfa::quantize_mxfp8_kernel<__nv_bfloat16><<<grid, lpfa::kQuantThreads, 0, s>>>(p);
-  else
-    lpfa::quantize_mxfp8_kernel<float><<<grid, lpfa::kQuantThreads, 0, s>>>(p);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return cuda_fail(e, "quantize launch");
-  return LPFA_OK;
+    return launch_quant(lpfa::quantize_mxfp8_kernel<__nv_bfloat16, false>, lpfa::quant_smem_bytes<__nv_bfloat16>(),
+                        lpfa::quant_threads<__nv_bfloat16>(), tm,
+                        p, info.sms, s, "quantize launch");
+  return launch_quant(lpfa::quantize_mxfp8_kernel<float, false>, lpfa::quant_smem_bytes<float>(),
+                      lpfa::quant_threads<float>(), tm, p, info.sms, s,
+                      "quantize launch");
 }
 
 lpfa_status lpfa_cast_e4m3(const void* v_bf16, int64_t tok_stride, int64_t head_stride, int64_t tokens,
@@ -224,21 +268,21 @@ lpfa_status lpfa_cast_e4m3(const void* v_bf16, int64_t tok_stride, int64_t head_
   DeviceInfo info;
   lpfa_status st = require_sm100(&info);
   if (st != LPFA_OK) return st;
-  lpfa::CastParams p;
-  p.v = static_cast<const __nv_bfloat16*>(v_bf16);
+  lpfa::QuantParams p = {};
+  p.x = v_bf16;
   p.tok_stride = tok_stride;
   p.head_stride = head_stride;
-  p.rows = tokens * heads;
   p.heads = heads;
-  p.out = out;
-  const int64_t lanes = p.rows * 16;
-  int64_t blocks = (lanes + 255) / 256;
-  const int64_t cap = static_cast<int64_t>(info.sms) * 16;
-  if (blocks > cap) blocks = cap;
-  lpfa::cast_e4m3_kernel<<<static_cast<unsigned>(blocks), 256, 0, static_cast<cudaStream_t>(stream)>>>(p);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return cuda_fail(e, "cast launch");
-  return LPFA_OK;
+  p.tokens = tokens;
+  const int64_t blocks = (tokens + 127) / 128;
+  if (blocks * heads > INT32_MAX) return fail(LPFA_ERR_INVALID_ARG, "too many tiles");
+  p.num_blocks = static_cast<int>(blocks);
+  p.payload = out;
+  CUtensorMap tm;
+  if ((st = input_tmap(&tm, v_bf16, false, tokens, heads, tok_stride, head_stride)) != LPFA_OK) return st;
+  return launch_quant(lpfa::quantize_mxfp8_kernel<__nv_bfloat16, true>, lpfa::quant_smem_bytes<__nv_bfloat16>(),
+                        lpfa::quant_threads<__nv_bfloat16>(), tm, p,
+                      info.sms, static_cast<cudaStream_t>(stream), "cast launch");
 }
 
 // The attention kernel moves registers between its warpgroups with setmaxnreg; the split

@@ -10,11 +10,16 @@
 //
 // Cast (FastVideo #1654, "fp8 PV mode for the FA4-FP4 attention path"): E4M3(v) with no scale.
 //
-// Both kernels are HBM-bound streaming kernels: 16-byte vector loads, 8-byte vector stores,
-// warp-shuffle maxima over the 4 lanes that hold one 32-element block.
+// One persistent kernel serves both: each CTA walks (128-token block, head) tiles with a stride
+// of the grid size. One warp stages each tile (128 token rows of one head) into shared memory
+// with a single TMA box load, double buffered, so the next tile is in flight while the
+// converting warps work on the current one; they read 16 bytes per lane from shared memory,
+// find each 32-element block maximum over 4 lanes with warp shuffles, write 8 payload bytes per
+// lane (coalesced 128-byte rows) and one scale byte per block.
 #pragma once
 
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -22,19 +27,33 @@
 
 namespace lpfa {
 
-constexpr int kQuantThreads = 256;   // 8 warps; one CTA per (128-token block, head)
-constexpr int kRowsPerWarp = 16;     // 128 rows / 8 warps
+#ifndef LPFA_QUANT_STAGES_BF16
+#define LPFA_QUANT_STAGES_BF16 2
+#endif
+#ifndef LPFA_QUANT_STAGES_F32
+#define LPFA_QUANT_STAGES_F32 2
+#endif
+// Converting warps per CTA (one more warp stages the tiles): 8 for bf16 input (three CTAs fit
+// on an SM), 16 for fp32 input (one CTA per SM, twice the bytes per row).
+template <typename T> constexpr int quant_warps() { return sizeof(T) == 2 ? 8 : 16; }
+template <typename T> constexpr int quant_threads() { return 32 * quant_warps<T>() + 32; }
+// Tiles staged per CTA (input tile: 32 KB for bf16, 64 KB for fp32).
+template <typename T> constexpr int quant_stages() {
+  return sizeof(T) == 2 ? LPFA_QUANT_STAGES_BF16 : LPFA_QUANT_STAGES_F32;
+}
 
 struct QuantParams {
   const void* x;
   int64_t tok_stride;   // elements
   int64_t head_stride;  // elements
   int heads;
-  int num_seqs;
+  int num_seqs;               // quantizer: varlen metadata
   const int32_t* cu_seqlens;  // device, num_seqs + 1
   const int32_t* scale_off;   // device, num_seqs + 1
+  int64_t tokens;             // cast: plain token count (no metadata)
+  int num_blocks;             // 128-token blocks (quantizer: total_scale_blocks)
   uint8_t* payload;           // (T, H, 128)
-  uint8_t* scales;            // (blocks * H) * 512
+  uint8_t* scales;            // quantizer: (blocks * H) * 512
   int floor_mode;
 };
 
@@ -50,13 +69,13 @@ __device__ __forceinline__ int e8m0_exponent(float amax, int floor_mode) {
   return max(-127, min(127, e));
 }
 
-// Loads 8 consecutive elements as floats.
+// 8 consecutive elements of a staged row as floats.
 template <typename T>
-__device__ __forceinline__ void load8(const T* p, float (&v)[8]);
+__device__ __forceinline__ void smem_load8(const T* p, float (&v)[8]);
 
 template <>
-__device__ __forceinline__ void load8<__nv_bfloat16>(const __nv_bfloat16* p, float (&v)[8]) {
-  const uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
+__device__ __forceinline__ void smem_load8<__nv_bfloat16>(const __nv_bfloat16* p, float (&v)[8]) {
+  const uint4 u = *reinterpret_cast<const uint4*>(p);
   const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
@@ -66,9 +85,9 @@ __device__ __forceinline__ void load8<__nv_bfloat16>(const __nv_bfloat16* p, flo
 }
 
 template <>
-__device__ __forceinline__ void load8<float>(const float* p, float (&v)[8]) {
-  const float4 a = __ldg(reinterpret_cast<const float4*>(p));
-  const float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+__device__ __forceinline__ void smem_load8<float>(const float* p, float (&v)[8]) {
+  const float4 a = reinterpret_cast<const float4*>(p)[0];
+  const float4 b = reinterpret_cast<const float4*>(p)[1];
   v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
   v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
 }
@@ -83,95 +102,148 @@ __device__ __forceinline__ int find_seq(const int32_t* prefix, int n, int g) {
   return lo;
 }
 
-// grid = (total_scale_blocks, heads). Each CTA quantizes the 128 token rows of one scale
-// block of one head and writes that block's 512-byte scale atom.
-template <typename T>
-__global__ void __launch_bounds__(kQuantThreads)
-quantize_mxfp8_kernel(QuantParams p) {
-  const int g = blockIdx.x;
-  const int h = blockIdx.y;
-  const int seq = find_seq(p.scale_off, p.num_seqs, g);
-  const int blk = g - __ldg(p.scale_off + seq);
-  const int seq_start = __ldg(p.cu_seqlens + seq);
-  const int seq_len = __ldg(p.cu_seqlens + seq + 1) - seq_start;
-  const int rows_valid = min(128, seq_len - blk * 128);
+// A tile: 128 token rows of one head (rows >= rows_valid do not exist).
+struct QuantTile {
+  int64_t tok0;    // first token of the tile
+  int rows_valid;
+  int h;
+  int g;           // 128-token block index (the scale atom's block)
+};
+
+template <bool kCast>
+__device__ __forceinline__ QuantTile quant_tile(const QuantParams& p, int w) {
+  QuantTile t;
+  t.g = w / p.heads;
+  t.h = w - t.g * p.heads;
+  if (kCast) {
+    t.tok0 = static_cast<int64_t>(t.g) * 128;
+    const int64_t left = p.tokens - t.tok0;
+    t.rows_valid = left < 128 ? static_cast<int>(left) : 128;
+  } else {
+    const int seq = find_seq(p.scale_off, p.num_seqs, t.g);
+    const int blk = t.g - __ldg(p.scale_off + seq);
+    const int start = __ldg(p.cu_seqlens + seq);
+    const int len = __ldg(p.cu_seqlens + seq + 1) - start;
+    t.tok0 = start + blk * 128;
+    t.rows_valid = min(128, len - blk * 128);
+  }
+  return t;
+}
+
+// Persistent grid over tiles w = g * heads + h (heads of a token block are adjacent in
+// memory). Warps 0..7 convert; warp 8 stages tiles (its own warp, so that computing the next
+// tile's bounds and issuing its copies never holds up the converting warps). kCast: E4M3(x)
+// with no scale and no scale atoms.
+template <typename T, bool kCast>
+__global__ void __launch_bounds__(quant_threads<T>())
+quantize_mxfp8_kernel(const __grid_constant__ CUtensorMap tmap_x, QuantParams p) {
+  constexpr uint32_t kRowBytes = 128 * sizeof(T);
+  constexpr uint32_t kTileBytesIn = 128 * kRowBytes;
+  constexpr int kQuantStages = quant_stages<T>();
+  constexpr int kQuantWarps = quant_warps<T>();
+  constexpr int kQuantThreads = 32 * kQuantWarps;
+  constexpr int kRowsPerWarp = 128 / kQuantWarps;
+  static_assert(128 % (2 * kQuantWarps) == 0, "rows per converting warp");
+  extern __shared__ uint8_t qsmem_raw[];
+  uint8_t* qsmem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(qsmem_raw) + 127) & ~uintptr_t(127));
+  uint64_t* full = reinterpret_cast<uint64_t*>(qsmem + kQuantStages * kTileBytesIn);
+  uint64_t* empty = full + kQuantStages;
+  QuantTile* info = reinterpret_cast<QuantTile*>(empty + kQuantStages);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(info + kQuantStages);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int half = lane >> 4;        // which of the two rows of an iteration
-  const int col8 = (lane & 15) * 8;  // first of this lane's 8 elements
-  const T* x = static_cast<const T*>(p.x);
-  uint32_t* atom = reinterpret_cast<uint32_t*>(p.scales + (static_cast<int64_t>(g) * p.heads + h) * 512);
+  const int num_tiles = p.num_blocks * p.heads;
+  const int G = gridDim.x;
 
-  constexpr int kIters = kRowsPerWarp / 2;
-  float v[kIters][8];
-#pragma unroll
-  for (int it = 0; it < kIters; ++it) {
-    const int r = warp * kRowsPerWarp + it * 2 + half;
-    if (r < rows_valid) {
-      const int64_t t = seq_start + blk * 128 + r;
-      load8<T>(x + t * p.tok_stride + h * p.head_stride + col8, v[it]);
-    } else {
-#pragma unroll
-      for (int i = 0; i < 8; ++i) v[it][i] = 0.f;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kQuantStages; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], kQuantThreads / 32);
     }
+    *abort_flag = 0;
+    mbar_fence_init();
+  }
+  __syncthreads();
+
+  if (warp == kQuantThreads / 32) {
+    // ---------------------------------------------------------------- producer
+    // One TMA load per tile: the box is 128 rows (tokens) x 128 elements of one head; rows
+    // past the end of the tensor read as zero, rows of the next sequence are read but unused.
+    if (lane == 0) prefetch_tmap(&tmap_x);
+    int n = 0;  // tiles issued
+    for (int w = blockIdx.x; w < num_tiles; w += G, ++n) {
+      const int b = n % kQuantStages;
+      if (!mbar_wait(&empty[b], ((n / kQuantStages) & 1) ^ 1, abort_flag)) break;
+      const QuantTile t = quant_tile<kCast>(p, w);
+      if (lane == 0) {
+        info[b] = t;
+        fence_proxy_async_smem();  // the converters' reads of buffer b precede the copy below
+        mbar_arrive_expect_tx(&full[b], kTileBytesIn, 1u);
+        tma_load_3d(qsmem + b * kTileBytesIn, &tmap_x, &full[b], 0, t.h, static_cast<int32_t>(t.tok0), 1u);
+      }
+      __syncwarp();
+    }
+    // Copies still in flight must land before the CTA exits: wait (bounded) for the newest fill
+    // of each buffer. In normal operation the converters consumed them already.
+    for (int j = (n > kQuantStages ? n - kQuantStages : 0); j < n; ++j)
+      mbar_wait(&full[j % kQuantStages], (j / kQuantStages) & 1, nullptr);
+    return;
   }
 
-#pragma unroll
-  for (int it = 0; it < kIters; ++it) {
-    const int r = warp * kRowsPerWarp + it * 2 + half;
-    float amax = 0.f;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[it][i]));
-    amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
-    amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 2));
-    const int e = e8m0_exponent(amax, p.floor_mode);
-    const float inv = __uint_as_float(static_cast<uint32_t>(127 - e) << 23);  // 2^-e, normal
-    uint32_t w0 = cvt_e4m3x2(v[it][0] * inv, v[it][1] * inv) |
-                  (static_cast<uint32_t>(cvt_e4m3x2(v[it][2] * inv, v[it][3] * inv)) << 16);
-    uint32_t w1 = cvt_e4m3x2(v[it][4] * inv, v[it][5] * inv) |
-                  (static_cast<uint32_t>(cvt_e4m3x2(v[it][6] * inv, v[it][7] * inv)) << 16);
-    // Scale bytes of the row's four blocks live in lanes (row base) + 0, 4, 8, 12.
-    const uint32_t byte = static_cast<uint32_t>(e + 127);
-    const int base = lane & 16;
-    const uint32_t b0 = __shfl_sync(0xFFFFFFFFu, byte, base + 0);
-    const uint32_t b1 = __shfl_sync(0xFFFFFFFFu, byte, base + 4);
-    const uint32_t b2 = __shfl_sync(0xFFFFFFFFu, byte, base + 8);
-    const uint32_t b3 = __shfl_sync(0xFFFFFFFFu, byte, base + 12);
-    if (r < rows_valid) {
-      const int64_t t = seq_start + blk * 128 + r;
-      uint2* dst = reinterpret_cast<uint2*>(p.payload + (t * p.heads + h) * 128 + col8);
-      *dst = make_uint2(w0, w1);
-      if ((lane & 15) == 0) atom[(r & 31) * 4 + (r >> 5)] = b0 | (b1 << 8) | (b2 << 16) | (b3 << 24);
-    } else if ((lane & 15) == 0) {
-      atom[(r & 31) * 4 + (r >> 5)] = 0x7F7F7F7Fu;  // pad row: scale 1.0
+  // ------------------------------------------------------------------ converters
+  const int half = lane >> 4;        // which of the two rows of an iteration
+  const int col8 = (lane & 15) * 8;  // first of this lane's 8 elements
+  const int kb = (lane & 15) >> 2;   // this lane's 32-element block
+  int n = 0;
+  for (int w = blockIdx.x; w < num_tiles; w += G, ++n) {
+    const int b = n % kQuantStages;
+    if (!mbar_wait(&full[b], (n / kQuantStages) & 1, abort_flag)) {
+      *abort_flag = 1;
+      if (atomicCAS(&g_lpfa_status[0], 0, 4 /* LPFA_ERR_TIMEOUT */) == 0) atomicExch(&g_lpfa_status[1], 100);
+      break;
     }
+    const QuantTile t = info[b];
+    const T* src = reinterpret_cast<const T*>(qsmem + b * kTileBytesIn);
+    uint8_t* atom = kCast ? nullptr : p.scales + (static_cast<int64_t>(t.g) * p.heads + t.h) * 512;
+#pragma unroll 2
+    for (int k = 0; k < kRowsPerWarp / 2; ++k) {
+      const int r = warp * kRowsPerWarp + k * 2 + half;
+      float v[8];
+      if (r < t.rows_valid) {
+        smem_load8<T>(src + r * 128 + col8, v);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] = 0.f;
+      }
+      float inv = 1.0f;
+      int e = 0;
+      if (!kCast) {
+        float amax = 0.f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
+        amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
+        amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 2));
+        e = e8m0_exponent(amax, p.floor_mode);
+        inv = __uint_as_float(static_cast<uint32_t>(127 - e) << 23);  // 2^-e, normal
+      }
+      const uint32_t w0 = cvt_e4m3x2(v[0] * inv, v[1] * inv) |
+                          (static_cast<uint32_t>(cvt_e4m3x2(v[2] * inv, v[3] * inv)) << 16);
+      const uint32_t w1 = cvt_e4m3x2(v[4] * inv, v[5] * inv) |
+                          (static_cast<uint32_t>(cvt_e4m3x2(v[6] * inv, v[7] * inv)) << 16);
+      if (r < t.rows_valid)
+        *reinterpret_cast<uint2*>(p.payload + ((t.tok0 + r) * p.heads + t.h) * 128 + col8) = make_uint2(w0, w1);
+      // One lane per 32-element block writes its scale byte; rows past the sequence end
+      // hold 0x7F (scale 1.0).
+      if (!kCast && (lane & 3) == 0)
+        atom[(r & 31) * 16 + (r >> 5) * 4 + kb] = r < t.rows_valid ? static_cast<uint8_t>(e + 127) : uint8_t{0x7F};
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[b]);
   }
 }
 
-struct CastParams {
-  const __nv_bfloat16* v;
-  int64_t tok_stride;
-  int64_t head_stride;
-  int64_t rows;  // tokens * heads
-  int heads;
-  uint8_t* out;
-};
-
-// Grid-stride over (token, head) rows; 16 lanes per 128-element row.
-__global__ void __launch_bounds__(256) cast_e4m3_kernel(CastParams p) {
-  const int64_t lane_global = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  for (int64_t idx = lane_global; idx < p.rows * 16; idx += stride) {
-    const int64_t row = idx >> 4;
-    const int col8 = static_cast<int>(idx & 15) * 8;
-    const int64_t t = row / p.heads;
-    const int h = static_cast<int>(row - t * p.heads);
-    float v[8];
-    load8<__nv_bfloat16>(p.v + t * p.tok_stride + h * p.head_stride + col8, v);
-    const uint32_t w0 = cvt_e4m3x2(v[0], v[1]) | (static_cast<uint32_t>(cvt_e4m3x2(v[2], v[3])) << 16);
-    const uint32_t w1 = cvt_e4m3x2(v[4], v[5]) | (static_cast<uint32_t>(cvt_e4m3x2(v[6], v[7])) << 16);
-    *reinterpret_cast<uint2*>(p.out + row * 128 + col8) = make_uint2(w0, w1);
-  }
+template <typename T> constexpr uint32_t quant_smem_bytes() {
+  return quant_stages<T>() * (128 * 128 * sizeof(T) + 16 + sizeof(QuantTile)) + 16 + 128;  // + alignment
 }
 
 }  // namespace lpfa
