@@ -181,6 +181,23 @@ LPFA_API lpfa_status lpfa_attn_fwd_varlen(const uint8_t* q, const uint8_t* q_sf,
  */
 LPFA_API lpfa_status lpfa_device_status(void* stream, int32_t* detail);
 
+/*
+ * Test hook for the bounded-wait failure path (no counterpart on the pages). Same arguments
+ * and behaviour as lpfa_attn_fwd_varlen, plus debug_flags: with bit 0 set, the kernel's QK
+ * issuer first waits on a barrier phase that nothing completes, so its bounded wait runs out
+ * (about 2 s), the kernel records LPFA_ERR_TIMEOUT in the device status word (read it with
+ * lpfa_device_status) and every role exits after its in-flight copies and MMAs have landed;
+ * out_bf16 and lse are then unspecified. The GPU context stays usable. debug_flags = 0 is
+ * exactly lpfa_attn_fwd_varlen.
+ */
+LPFA_API lpfa_status lpfa_attn_fwd_varlen_debug(const uint8_t* q, const uint8_t* q_sf, const uint8_t* k,
+                                       const uint8_t* k_sf, const uint8_t* v, const uint8_t* v_sf,
+                                       const lpfa_varlen_meta* meta_q, const lpfa_varlen_meta* meta_k,
+                                       int32_t heads, int32_t head_dim, lpfa_pv_mode pv_mode,
+                                       const float* q_descale, const float* k_descale,
+                                       const float* v_descale, void* out_bf16, float* lse,
+                                       void* stream, int32_t debug_flags);
+
 /* Message describing the last non-OK status returned on the calling thread ("" if none). */
 LPFA_API const char* lpfa_last_error_message(void);
 

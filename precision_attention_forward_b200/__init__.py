@@ -22,7 +22,7 @@ LIB_PATH = os.path.join(_PKG_DIR, "liblpfa.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
-        "liblpfa.so is not built; run `python -m precision_attention_forward_b200.build` "
+        "liblpfa.so is not built; run `python precision_attention_forward_b200/build.py` "
         "(the library has no CPU fallback)")
 
 _lib = ctypes.CDLL(LIB_PATH)
@@ -37,7 +37,7 @@ PV_MODES = {"bf16": 0, "fp8": 1}
 EXPORTED_SYMBOLS = (
     "lpfa_meta_dev_ints", "lpfa_varlen_meta_fill_host", "lpfa_varlen_meta_from_lengths",
     "lpfa_scale_bytes", "lpfa_quantize_mxfp8_varlen", "lpfa_cast_e4m3", "lpfa_attn_fwd_varlen",
-    "lpfa_device_status", "lpfa_last_error_message", "lpfa_version",
+    "lpfa_device_status", "lpfa_last_error_message", "lpfa_version", "lpfa_attn_fwd_varlen_debug",
 )
 
 
@@ -70,6 +70,8 @@ _lib.lpfa_cast_e4m3.restype = ctypes.c_int
 _lib.lpfa_attn_fwd_varlen.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, ctypes.POINTER(_Meta), ctypes.POINTER(_Meta),
                                       _i32, _i32, ctypes.c_int, _f32p, _f32p, _f32p, _vp, _vp, _vp]
 _lib.lpfa_attn_fwd_varlen.restype = ctypes.c_int
+_lib.lpfa_attn_fwd_varlen_debug.argtypes = list(_lib.lpfa_attn_fwd_varlen.argtypes) + [_i32]
+_lib.lpfa_attn_fwd_varlen_debug.restype = ctypes.c_int
 _lib.lpfa_device_status.argtypes = [_vp, ctypes.POINTER(_i32)]
 _lib.lpfa_device_status.restype = ctypes.c_int
 _lib.lpfa_last_error_message.argtypes = []
@@ -196,8 +198,12 @@ def lpfa_attn_fwd_varlen(q: torch.Tensor, q_sf: torch.Tensor, k: torch.Tensor, k
                          v: torch.Tensor, v_sf: Optional[torch.Tensor], meta_q: VarlenMeta, meta_k: VarlenMeta,
                          pv_mode: str = "bf16", q_descale: Optional[torch.Tensor] = None,
                          k_descale: Optional[torch.Tensor] = None, v_descale: Optional[torch.Tensor] = None,
-                         out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None, stream=None):
-    """Block-scaled attention forward; returns (out bf16 (Tq,H,128), lse fp32 (H,Tq))."""
+                         out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None, stream=None,
+                         debug_flags: int = 0):
+    """Block-scaled attention forward; returns (out bf16 (Tq,H,128), lse fp32 (H,Tq)).
+
+    debug_flags != 0 goes through lpfa_attn_fwd_varlen_debug (test hook, see include/lpfa.h).
+    """
     if pv_mode not in PV_MODES:
         raise ValueError("pv_mode must be 'bf16' or 'fp8'")
     for name, t in (("q", q), ("k", k), ("v", v)):
@@ -211,12 +217,15 @@ def lpfa_attn_fwd_varlen(q: torch.Tensor, q_sf: torch.Tensor, k: torch.Tensor, k
         out = torch.empty((Tq, H, 128), dtype=torch.bfloat16, device=q.device)
     if lse is None:
         lse = torch.empty((H, Tq), dtype=torch.float32, device=q.device)
-    with torch.cuda.device(q.device):
-        _check(_lib.lpfa_attn_fwd_varlen(
-            q.data_ptr(), q_sf.data_ptr(), k.data_ptr(), k_sf.data_ptr(), v.data_ptr(), _ptr(v_sf),
+    args = (q.data_ptr(), q_sf.data_ptr(), k.data_ptr(), k_sf.data_ptr(), v.data_ptr(), _ptr(v_sf),
             ctypes.byref(meta_q._c), ctypes.byref(meta_k._c), H, 128, PV_MODES[pv_mode],
             _ptr(q_descale), _ptr(k_descale), _ptr(v_descale), out.data_ptr(), lse.data_ptr(),
-            _stream_ptr(stream)))
+            _stream_ptr(stream))
+    with torch.cuda.device(q.device):
+        if debug_flags:
+            _check(_lib.lpfa_attn_fwd_varlen_debug(*args, debug_flags))
+        else:
+            _check(_lib.lpfa_attn_fwd_varlen(*args))
     return out, lse
 
 

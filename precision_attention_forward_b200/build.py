@@ -1,7 +1,8 @@
 """Build the library (liblpfa.so) in-tree with nvcc for sm_100a.
 
-Usage: ``python -m precision_attention_forward_b200.build [--verbose]``. The shared
-library links the CUDA runtime statically and needs only the driver at run time.
+Usage: ``python precision_attention_forward_b200/build.py [--verbose]`` (run as a file: importing
+the package loads the library being built). The shared library links the CUDA runtime
+statically and needs only the driver at run time.
 """
 from __future__ import annotations
 

@@ -127,7 +127,8 @@ struct SmemLayout {
   static constexpr uint32_t mref = v_sf + kV * kAtomBytes;            // float [2 groups][128] tile reference
   static constexpr uint32_t lsum = mref + 2 * 128 * 4;                // float [2 groups][128] partial l
   static constexpr uint32_t mfin = lsum + 2 * 128 * 4;                // float [2 groups][128] reference of l
-  static constexpr uint32_t bars = mfin + 2 * 128 * 4;                // uint64 barriers
+  static constexpr uint32_t lsumr = mfin + 2 * 128 * 4;               // float [2 groups][128] partial sum of rounded P
+  static constexpr uint32_t bars = lsumr + 2 * 128 * 4;               // uint64 barriers
   static constexpr uint32_t num_bars = 64;
   static constexpr uint32_t misc = bars + num_bars * 8;               // tmem base, abort flag
   static constexpr uint32_t total = misc + 64;
@@ -378,6 +379,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
   float* mref = reinterpret_cast<float*>(smem + L::mref);
   float* lsum = reinterpret_cast<float*>(smem + L::lsum);
   float* mfin = reinterpret_cast<float*>(smem + L::mfin);
+  float* lsumr = reinterpret_cast<float*>(smem + L::lsumr);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -631,6 +633,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
       }
       float m_g = -INFINITY;  // reference this group's l is relative to (-inf: no tile yet)
       float l_g = 0.0f;       // this group's sum of p over its tiles (times 2^kBias)
+      float lr_g = 0.0f;      // bf16 PV mode: the same sum over the BF16-rounded P
       for (int j = static_cast<int>((t0 ^ grp) & 1); j < ui.nkv; j += 2) {
         const uint32_t t = t0 + j;           // t & 1 == grp
         const uint32_t kt = t >> 1;          // this group's tile ordinal
@@ -665,7 +668,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
         };
         const float psum = tail ? exp_row<true, kPolyPairs>(sv, cscale, kBias - m_t, key0, ui.k_len, handoff)
                                 : exp_row<false, kPolyPairs>(sv, cscale, kBias - m_t, key0, ui.k_len, handoff);
-        l_g = l_g * exp2_int(m_g - m_t) + psum;
+        const float l_scale = exp2_int(m_g - m_t);
+        l_g = l_g * l_scale + psum;
+        if (!kFp8PV) lr_g *= l_scale;
         m_g = m_t;
         // PV(t - 2) has read this group's previous P.
         if (kt >= 1) {
@@ -680,13 +685,22 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
                     (static_cast<uint32_t>(cvt_e4m3x2(sv[2 * i + 1].x, sv[2 * i + 1].y)) << 16);
           tmem_st32_sync(tmem + lane_addr + kColP + grp * 32, pk);
         } else {
+          // O is normalised by the sum of the P values the PV product actually uses, so a
+          // row dominated by one key gets that V row exactly (the LSE keeps the unrounded sum).
+          float2 racc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
             uint32_t pk[32];
 #pragma unroll
-            for (int i = 0; i < 32; ++i) pk[i] = cvt_bf16x2(sv[32 * h + i].x, sv[32 * h + i].y);
+            for (int i = 0; i < 32; ++i) {
+              pk[i] = cvt_bf16x2(sv[32 * h + i].x, sv[32 * h + i].y);
+              racc[i & 3] = __fadd2_rn(racc[i & 3], make_float2(__uint_as_float(pk[i] << 16),
+                                                               __uint_as_float(pk[i] & 0xFFFF0000u)));
+            }
             tmem_st32_sync(tmem + lane_addr + kColS + grp * 128 + h * 32, pk);
           }
+          const float2 rs = __fadd2_rn(__fadd2_rn(racc[0], racc[1]), __fadd2_rn(racc[2], racc[3]));
+          lr_g += rs.x + rs.y;
         }
         // O holds tiles up to t - 1 relative to m_prev; rescale it when the reference moved
         // (rare; never on a unit's first tile).
@@ -721,14 +735,16 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
       tc_fence_after();
       lsum[grp * 128 + row] = l_g;
       mfin[grp * 128 + row] = m_g;
+      if (!kFp8PV) lsumr[grp * 128 + row] = lr_g;
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars[kBarLReady]);
       if (!mbar_wait_warp(&bars[kBarLReady], u & 1, abort_flag)) { record_failure(abort_flag, kSiteSoftL); ok = false; break; }
       const float m_o = mfin[(grp ^ 1) * 128 + row];
       const float l_o = lsum[(grp ^ 1) * 128 + row];
       const float m_f = fmaxf(m_g, m_o);  // the unit's last reference (references never fall)
-      const float ltot = l_g * exp2_int(m_g - m_f) + l_o * exp2_int(m_o - m_f);
-      const float oscale = vd / ltot;
+      const float s_g = exp2_int(m_g - m_f), s_o = exp2_int(m_o - m_f);
+      const float ltot = l_g * s_g + l_o * s_o;
+      const float oscale = kFp8PV ? vd / ltot : vd / (lr_g * s_g + lsumr[(grp ^ 1) * 128 + row] * s_o);
       uint32_t ra[32], rb[32];
       tmem_ld64_sync(tmem + lane_addr + kColO + grp * 64, ra, rb);
       tc_fence_before();

@@ -376,6 +376,17 @@ lpfa_status lpfa_attn_fwd_varlen(const uint8_t* q, const uint8_t* q_sf, const ui
                        v_descale, out_bf16, lse, stream, 0);
 }
 
+lpfa_status lpfa_attn_fwd_varlen_debug(const uint8_t* q, const uint8_t* q_sf, const uint8_t* k, const uint8_t* k_sf,
+                                       const uint8_t* v, const uint8_t* v_sf, const lpfa_varlen_meta* meta_q,
+                                       const lpfa_varlen_meta* meta_k, int32_t heads, int32_t head_dim,
+                                       lpfa_pv_mode pv_mode, const float* q_descale, const float* k_descale,
+                                       const float* v_descale, void* out_bf16, float* lse, void* stream,
+                                       int32_t debug_flags) {
+  if (debug_flags & ~1) return fail(LPFA_ERR_INVALID_ARG, "unknown debug flags 0x%x", debug_flags);
+  return attn_fwd_impl(q, q_sf, k, k_sf, v, v_sf, meta_q, meta_k, heads, head_dim, pv_mode, q_descale, k_descale,
+                       v_descale, out_bf16, lse, stream, debug_flags & 1);
+}
+
 lpfa_status lpfa_device_status(void* stream, int32_t* detail) {
   if (detail) *detail = 0;
   cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));

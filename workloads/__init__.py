@@ -170,6 +170,16 @@ def make_tensor(w: Workload, which: str, seed: int = 0, tokens: Optional[int] = 
     return x
 
 
+def outlier_scale(w: Workload, which: str, seed: int = 0) -> np.ndarray:
+    """(heads, 128) float32: the outlier gain on the (head, channel) pairs ``make_tensor`` scales
+    for this tensor, 1 elsewhere."""
+    s = np.ones(w.heads * HEAD_DIM, dtype=np.float32)
+    if w.outlier_frac > 0.0:
+        ostream = {"q": _STREAM_OUT_Q, "k": _STREAM_OUT_K, "v": _STREAM_OUT_V}[which]
+        s[_outlier_pairs(seed, w, ostream)] = np.float32(w.outlier_gain)
+    return s.reshape(w.heads, HEAD_DIM)
+
+
 def tensor_dtype(w: Workload, which: str) -> str:
     """Input dtype of the tensor as handed to the library ("bf16" or "fp32")."""
     if which == "v" and w.pv_mode == "fp8":
