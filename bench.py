@@ -202,6 +202,45 @@ def run_reference(args, w):
     return 0
 
 
+class Ranks:
+    """Host-side bookkeeping across the ranks of a run (one process per GPU): a barrier and a
+    max over ranks of a float. There is no collective on the data path; the runs are replicas.
+
+    ``device`` is where the reduction tensor lives: the rank's GPU under NCCL, the CPU under
+    gloo (the CPU tests).
+    """
+
+    def __init__(self, world: int, device, sync_cuda: bool = True):
+        self.world = world
+        self.device = device
+        self.sync_cuda = sync_cuda
+
+    def barrier(self):
+        import torch
+        import torch.distributed as dist
+
+        if self.world > 1:
+            dist.barrier()
+        if self.sync_cuda:
+            torch.cuda.synchronize()
+
+    def max(self, x: float) -> float:
+        if self.world == 1:
+            return float(x)
+        import torch
+        import torch.distributed as dist
+
+        t = torch.tensor([x], dtype=torch.float64, device=self.device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+
+def job_tflops(flops_per_rank: float, world: int, ms_per_step: float) -> float:
+    """Whole-job throughput: every rank processes flops_per_rank per step (weak scaling), and
+    the step time is the slowest rank's."""
+    return flops_per_rank * world / (ms_per_step * 1e-3) / 1e12
+
+
 def config_dict(w, lq, lk, n):
     return {
         "workload": w.name, "description": w.description, "num_seqs": int(w.num_seqs),
@@ -286,17 +325,9 @@ def main():
             timing.append((a, c, b))
         return 4  # kernels launched
 
-    def barrier():
-        if world > 1:
-            dist.barrier()
-        torch.cuda.synchronize()
-
-    def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    ranks = Ranks(world, dev)
+    barrier = ranks.barrier
+    max_over_ranks = ranks.max
 
     vis = os.environ.get("CUDA_VISIBLE_DEVICES")
     smi_index = int(vis.split(",")[local_rank]) if vis and vis.split(",")[local_rank].strip().isdigit() else local_rank
@@ -324,7 +355,7 @@ def main():
         raise RuntimeError(f"kernel reported status {st} (site {detail})")
 
     ms_per_step = total_ms / args.steps
-    value = flops * world / (ms_per_step * 1e-3) / 1e12
+    value = job_tflops(flops, world, ms_per_step)
 
     # End to end through the public API with host buffers.
     e2e = None
@@ -354,7 +385,7 @@ def main():
         e1.record(stream)
         barrier()
         e_ms = max_over_ranks(e0.elapsed_time(e1)) / ne
-        e2e = {"value": flops * world / (e_ms * 1e-3) / 1e12, "unit": "TFLOPS", "ms_per_step": e_ms,
+        e2e = {"value": job_tflops(flops, world, e_ms), "unit": "TFLOPS", "ms_per_step": e_ms,
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
 
     peaks, peak_src = load_peaks()
