@@ -154,6 +154,8 @@ def cpu_oracle_sample(w, seconds: float, seed: int = 0):
         kh = (omx.e4m3_decode(kp).reshape(-1, 4, 32) * np.ldexp(1.0, ke)[..., None]).reshape(-1, 128)
         if w.pv_mode == "fp8":
             vh = omx.e4m3_decode(omx.cast_e4m3(v[k0:k1, h]))
+        elif w.pv_mode == "bf16v":
+            vh = v[k0:k1, h].astype(np.float64)
         else:
             vp, ve = omx.quantize_rows(v[k0:k1, h].astype(np.float64), w.scaling_mode)
             vh = (omx.e4m3_decode(vp).reshape(-1, 4, 32) * np.ldexp(1.0, ve)[..., None]).reshape(-1, 128)
@@ -297,10 +299,10 @@ def main():
     sbq, sbk = mq0.total_scale_blocks, lp.lpfa_varlen_meta_from_lengths(lk, device=dev).total_scale_blocks
     qp = torch.empty((Tq, H, 128), dtype=torch.uint8, device=dev)
     kp = torch.empty((Tk, H, 128), dtype=torch.uint8, device=dev)
-    vp = torch.empty((Tk, H, 128), dtype=torch.uint8, device=dev)
+    vp = torch.empty((Tk, H, 128), dtype=torch.uint8, device=dev) if w.pv_mode != "bf16v" else None
     qs = torch.empty(sbq * H * 512, dtype=torch.uint8, device=dev)
     ks = torch.empty(sbk * H * 512, dtype=torch.uint8, device=dev)
-    vs = None if w.pv_mode == "fp8" else torch.empty(sbk * H * 512, dtype=torch.uint8, device=dev)
+    vs = torch.empty(sbk * H * 512, dtype=torch.uint8, device=dev) if w.pv_mode == "bf16" else None
     out = torch.empty((Tq, H, 128), dtype=torch.bfloat16, device=dev)
     lse = torch.empty((H, Tq), dtype=torch.float32, device=dev)
 
@@ -314,16 +316,17 @@ def main():
         lp.lpfa_quantize_mxfp8_varlen(ins["k"], mk, w.scaling_mode, payload=kp, scales=ks)
         if w.pv_mode == "fp8":
             lp.lpfa_cast_e4m3(ins["v"], out=vp)
-        else:
+        elif w.pv_mode == "bf16":
             lp.lpfa_quantize_mxfp8_varlen(ins["v"], mk, w.scaling_mode, payload=vp, scales=vs)
         if timing is not None:
             c = torch.cuda.Event(enable_timing=True)
             c.record(stream)
-        lp.lpfa_attn_fwd_varlen(qp, qs, kp, ks, vp, vs, mq, mk, pv_mode=w.pv_mode, out=out, lse=lse)
+        v_in = ins["v"] if w.pv_mode == "bf16v" else vp   # BF16 V goes to the kernel as is
+        lp.lpfa_attn_fwd_varlen(qp, qs, kp, ks, v_in, vs, mq, mk, pv_mode=w.pv_mode, out=out, lse=lse)
         if timing is not None:
             b.record(stream)
             timing.append((a, c, b))
-        return 4  # kernels launched
+        return 3 if w.pv_mode == "bf16v" else 4  # kernels launched
 
     ranks = Ranks(world, dev)
     barrier = ranks.barrier
@@ -397,7 +400,8 @@ def main():
     traffic = tr[1] if tr and tr[0] == kernel_hash() else None
     qbytes = quantizer_bytes(Tq, H, 2 if dts["q"] == "bf16" else 4, sbq) + \
         quantizer_bytes(Tk, H, 2 if dts["k"] == "bf16" else 4, sbk) + \
-        (Tk * H * 128 * 3.0 if w.pv_mode == "fp8" else quantizer_bytes(Tk, H, 2 if dts["v"] == "bf16" else 4, sbk))
+        (Tk * H * 128 * 3.0 if w.pv_mode == "fp8" else
+         0.0 if w.pv_mode == "bf16v" else quantizer_bytes(Tk, H, 2 if dts["v"] == "bf16" else 4, sbk))
 
     if rank == 0:
         cpu = None

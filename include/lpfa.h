@@ -51,7 +51,7 @@ typedef enum {
 
 typedef enum { LPFA_IN_BF16 = 0, LPFA_IN_FP32 = 1 } lpfa_in_dtype;
 typedef enum { LPFA_SCALE_RCEIL = 0, LPFA_SCALE_FLOOR = 1 } lpfa_scaling_mode;
-typedef enum { LPFA_PV_BF16 = 0, LPFA_PV_FP8 = 1 } lpfa_pv_mode;
+typedef enum { LPFA_PV_BF16 = 0, LPFA_PV_FP8 = 1, LPFA_PV_BF16_V = 2 } lpfa_pv_mode;
 
 /*
  * Packed variable-length metadata (LP-FA4 README, "MXFP8 forward and backward":
@@ -149,7 +149,9 @@ LPFA_API lpfa_status lpfa_cast_e4m3(const void* v_bf16, int64_t tok_stride, int6
  *                  storage (under meta_k) is v_sf; it is dequantized exactly to BF16 and P is
  *                  rounded to BF16 for the PV product. LPFA_PV_FP8: unscaled E4M3 codes (see
  *                  lpfa_cast_e4m3), v_sf must be NULL, P is rounded to E4M3 relative to a
- *                  power-of-two running maximum.
+ *                  power-of-two running maximum. LPFA_PV_BF16_V: v points to BF16 values
+ *                  (Tk, H, 128), contiguous, never quantized (LP-FA4 README: V kept in BF16);
+ *                  v_sf must be NULL; P is rounded to BF16 as in LPFA_PV_BF16.
  * meta_q, meta_k   sequence i of meta_q attends to sequence i of meta_k (same num_seqs).
  * q/k/v_descale    device pointers to one float each, or NULL. NULL means exactly 1.0: the
  *                  kernel then uses the literal 1.0f on the same code path, so a descale of
@@ -160,7 +162,7 @@ LPFA_API lpfa_status lpfa_cast_e4m3(const void* v_bf16, int64_t tok_stride, int6
  * Alignment:       every tensor 16-byte aligned.
  * Errors:          LPFA_ERR_INVALID_ARG for NULL required pointers, head_dim != 128,
  *                  heads < 1, mismatched num_seqs, a bad pv_mode, or a non-NULL v_sf in fp8
- *                  mode (and NULL v_sf in bf16 mode); LPFA_ERR_UNSUPPORTED off sm_100;
+ *                  or BF16-V mode (and NULL v_sf in bf16 mode); LPFA_ERR_UNSUPPORTED off sm_100;
  *                  LPFA_ERR_CUDA on launch failure. A kernel that gives up on a barrier wait
  *                  records LPFA_ERR_TIMEOUT in the device status word (see below).
  */

@@ -31,7 +31,7 @@ LPFA_OK, LPFA_ERR_INVALID_ARG, LPFA_ERR_UNSUPPORTED, LPFA_ERR_CUDA, LPFA_ERR_TIM
 _STATUS_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "CUDA", 4: "TIMEOUT"}
 IN_DTYPES = {"bf16": 0, "fp32": 1}
 SCALING_MODES = {"rceil": 0, "floor": 1}
-PV_MODES = {"bf16": 0, "fp8": 1}
+PV_MODES = {"bf16": 0, "fp8": 1, "bf16v": 2}  # bf16v: BF16 V input, bf16 PV
 
 # Symbols the header declares; the tests check that each one is exported.
 EXPORTED_SYMBOLS = (
@@ -205,10 +205,11 @@ def lpfa_attn_fwd_varlen(q: torch.Tensor, q_sf: torch.Tensor, k: torch.Tensor, k
     debug_flags != 0 goes through lpfa_attn_fwd_varlen_debug (test hook, see include/lpfa.h).
     """
     if pv_mode not in PV_MODES:
-        raise ValueError("pv_mode must be 'bf16' or 'fp8'")
+        raise ValueError("pv_mode must be 'bf16', 'fp8' or 'bf16v'")
     for name, t in (("q", q), ("k", k), ("v", v)):
-        if t.dtype != torch.uint8 or t.dim() != 3 or not t.is_contiguous():
-            raise ValueError("%s must be a contiguous uint8 (tokens, heads, 128) payload" % name)
+        want = torch.bfloat16 if (name == "v" and pv_mode == "bf16v") else torch.uint8
+        if t.dtype != want or t.dim() != 3 or not t.is_contiguous():
+            raise ValueError("%s must be a contiguous %s (tokens, heads, 128) tensor" % (name, want))
     for name, t in (("q_descale", q_descale), ("k_descale", k_descale), ("v_descale", v_descale)):
         if t is not None and (t.dtype != torch.float32 or t.numel() != 1):
             raise ValueError("%s must be a single-element float32 tensor" % name)

@@ -357,6 +357,11 @@ __device__ __forceinline__ void record_failure(volatile int* abort_flag, int sit
   if (atomicCAS(&g_lpfa_status[0], 0, 4 /* LPFA_ERR_TIMEOUT */) == 0) atomicExch(&g_lpfa_status[1], site);
 }
 
+// PV variants of the kernel: V as MXFP8 dequantized to BF16 in shared memory (bf16 PV), V as
+// unscaled E4M3 (fp8 PV), or V given as BF16 and loaded by TMA straight into the layout the
+// BF16 PV MMA reads (bf16 PV with BF16 V; LP-FA4 README: the BF16 V path).
+enum PvKind : int { kPvBf16Mx = 0, kPvFp8 = 1, kPvBf16In = 2 };
+
 // How far (log2 units) a row's logits may exceed its reference before the reference, l and
 // O move, and the power of two P is stored with. bf16 P keeps its 8-bit mantissa at any
 // scale, so it may lag 8 binades; fp8 P stores 2^(bias - m) 2^s <= 2^(lag + bias) = 256 < 448.
@@ -365,10 +370,12 @@ template <> struct SoftmaxLag<true> { static constexpr float lag = 2.0f; static 
 template <> struct SoftmaxLag<false> { static constexpr float lag = 8.0f; static constexpr float bias = 0.0f; };
 
 
-template <bool kFp8PV>
+template <int kPv>
 __global__ void __launch_bounds__(kAttnThreads, 1)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                 const __grid_constant__ CUtensorMap tmap_v, const AttnParams p) {
+  constexpr bool kFp8PV = kPv == kPvFp8;
+  constexpr bool kVIn = kPv == kPvBf16In;  // BF16 V straight into the BF16 operand buffers
   using L = SmemLayout<kFp8PV>;
   constexpr int kKStages = Stages<kFp8PV>::k, kVStages = Stages<kFp8PV>::v, kVbfStages = Stages<kFp8PV>::vbf;
   extern __shared__ uint8_t smem_raw[];
@@ -391,7 +398,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
       mbar_init(&bars[kBarVFull + i], 1);
       mbar_init(&bars[kBarVEmpty + i], kFp8PV ? 1 : 4);   // MMA commit, or the 4 converter warps
     }
-    for (int i = 0; i < kVbfStages; ++i) { mbar_init(&bars[kBarVbfFull + i], 4); mbar_init(&bars[kBarVbfEmpty + i], 1); }
+    for (int i = 0; i < kVbfStages; ++i) {
+      mbar_init(&bars[kBarVbfFull + i], kVIn ? 1 : 4);  // the V producer's TMA, or the 4 converter warps
+      mbar_init(&bars[kBarVbfEmpty + i], 1);
+    }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bars[kBarSFull + i], 1);
       mbar_init(&bars[kBarSFree + i], 4);
@@ -464,6 +474,28 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
         if (!mbar_wait(&bars[kBarQFull + i % kQStages], (i / kQStages) & 1, nullptr)) record_failure(abort_flag, kSiteDrain);
       for (uint32_t i = (kc > kKStages ? kc - kKStages : 0); i < kc; ++i)
         if (!mbar_wait(&bars[kBarKFull + i % kKStages], (i / kKStages) & 1, nullptr)) record_failure(abort_flag, kSiteDrain);
+    } else if (warp == 3 && kVIn) {
+      // ---------------------------------------------------------------- V producer (BF16 V)
+      // Two TMA box loads per tile (head_dim [0, 64) and [64, 128), 128 keys each, 128-byte
+      // swizzle) produce exactly the MN-major BF16 operand layout the PV MMA reads.
+      const uint32_t leader = lane == 0 ? 1u : 0u;
+      uint32_t vc = 0;
+      bool ok = true;
+      for (int w = blockIdx.x; w < p.num_units && ok; w += G) {
+        const UnitInfo ui = warp_uniform(unit_info(p, w));
+        for (int j = 0; j < ui.nkv; ++j) {
+          const uint32_t sb = vc % kVbfStages, phb = (vc / kVbfStages) & 1;
+          if (!mbar_wait_warp(&bars[kBarVbfEmpty + sb], phb ^ 1, abort_flag)) { record_failure(abort_flag, kSiteProducerV); ok = false; break; }
+          mbar_arrive_expect_tx(&bars[kBarVbfFull + sb], kVbfBytes, leader);
+#pragma unroll
+          for (int a = 0; a < 2; ++a)
+            tma_load_3d(smem + L::vbf + sb * kVbfBytes + a * kTileBytes, &tmap_v, &bars[kBarVbfFull + sb], a * 64,
+                        ui.h, ui.k_row0 + j * kTileN, leader);
+          ++vc;
+        }
+      }
+      for (uint32_t i = (vc > kVbfStages ? vc - kVbfStages : 0); i < vc; ++i)
+        if (!mbar_wait(&bars[kBarVbfFull + i % kVbfStages], (i / kVbfStages) & 1, nullptr)) record_failure(abort_flag, kSiteDrain);
     } else if (warp == 3) {
       // ---------------------------------------------------------------- V producer
       // A warp of its own, so that K loads (and with them QK) never wait behind a V stage
@@ -777,7 +809,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
     }
   } else {
     setmaxnreg_dec<kOtherRegs>();
-    if (!kFp8PV) {
+    if (kPv == kPvBf16Mx) {
       // ---------------------------------------------------------------- V converter (bf16 PV)
       const int t = threadIdx.x - 12 * 32;  // key row of the V tile, 0..127
       const uint32_t sw = static_cast<uint32_t>(t & 7);

@@ -128,6 +128,23 @@ lpfa_status input_tmap(CUtensorMap* map, const void* base, bool fp32, int64_t to
   return LPFA_OK;
 }
 
+// Tensor map over a contiguous (tokens, heads, 128) BF16 V; box = 64 elements (128 bytes) of
+// one head x 128 tokens with the 128-byte swizzle: the two boxes of a 128-key tile are the two
+// MN-major swizzle atoms of the BF16 PV operand.
+lpfa_status bf16_v_tmap(CUtensorMap* map, const void* base, int64_t tokens, int heads) {
+  auto fn = encode_fn();
+  if (!fn) return fail(LPFA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(heads), static_cast<cuuint64_t>(tokens)};
+  cuuint64_t strides[2] = {256, static_cast<cuuint64_t>(heads) * 256};
+  cuuint32_t box[3] = {64, 1, 128};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(LPFA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  return LPFA_OK;
+}
+
 lpfa_status check_meta(const lpfa_varlen_meta* m, const char* name) {
   if (!m) return fail(LPFA_ERR_INVALID_ARG, "%s is NULL", name);
   if (!m->dev) return fail(LPFA_ERR_INVALID_ARG, "%s has no device buffer", name);
@@ -309,8 +326,10 @@ static lpfa_status attn_fwd_impl(const uint8_t* q, const uint8_t* q_sf, const ui
                                  const float* v_descale, void* out_bf16, float* lse, void* stream,
                                  int debug_stall) {
   if (!q || !q_sf || !k || !k_sf || !v || !out_bf16 || !lse) return fail(LPFA_ERR_INVALID_ARG, "NULL tensor pointer");
-  if (pv_mode != LPFA_PV_BF16 && pv_mode != LPFA_PV_FP8) return fail(LPFA_ERR_INVALID_ARG, "invalid pv_mode %d", pv_mode);
+  if (pv_mode != LPFA_PV_BF16 && pv_mode != LPFA_PV_FP8 && pv_mode != LPFA_PV_BF16_V)
+    return fail(LPFA_ERR_INVALID_ARG, "invalid pv_mode %d", pv_mode);
   if (pv_mode == LPFA_PV_FP8 && v_sf) return fail(LPFA_ERR_INVALID_ARG, "fp8 PV mode takes no V scale factors (v_sf must be NULL)");
+  if (pv_mode == LPFA_PV_BF16_V && v_sf) return fail(LPFA_ERR_INVALID_ARG, "BF16 V input takes no V scale factors (v_sf must be NULL)");
   if (pv_mode == LPFA_PV_BF16 && !v_sf) return fail(LPFA_ERR_INVALID_ARG, "bf16 PV mode needs the V scale factors (v_sf)");
   if (head_dim != 128) return fail(LPFA_ERR_INVALID_ARG, "head_dim must be 128 (got %d)", head_dim);
   if (heads < 1) return fail(LPFA_ERR_INVALID_ARG, "heads must be >= 1");
@@ -330,7 +349,12 @@ static lpfa_status attn_fwd_impl(const uint8_t* q, const uint8_t* q_sf, const ui
   CUtensorMap tq, tk, tv;
   if ((st = payload_tmap(&tq, q, meta_q->total_tokens, heads, lpfa::kTileM)) != LPFA_OK) return st;
   if ((st = payload_tmap(&tk, k, meta_k->total_tokens, heads, lpfa::kTileN)) != LPFA_OK) return st;
-  if ((st = payload_tmap(&tv, v, meta_k->total_tokens, heads, lpfa::kTileN)) != LPFA_OK) return st;
+  if (pv_mode == LPFA_PV_BF16_V) {
+    // BF16 V, contiguous (Tk, H, 128): boxes of 64 elements (128 bytes) x 128 keys, 128-byte swizzle.
+    if ((st = bf16_v_tmap(&tv, v, meta_k->total_tokens, heads)) != LPFA_OK) return st;
+  } else if ((st = payload_tmap(&tv, v, meta_k->total_tokens, heads, lpfa::kTileN)) != LPFA_OK) {
+    return st;
+  }
 
   lpfa::AttnParams p;
   p.q_sf = q_sf;
@@ -356,11 +380,17 @@ static lpfa_status attn_fwd_impl(const uint8_t* q, const uint8_t* q_sf, const ui
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e;
   if (pv_mode == LPFA_PV_FP8) {
-    if ((st = check_attn_kernel(reinterpret_cast<const void*>(lpfa::attn_fwd_kernel<true>), lpfa::attn_smem_bytes<true>())) != LPFA_OK) return st;
-    lpfa::attn_fwd_kernel<true><<<grid, lpfa::kAttnThreads, lpfa::attn_smem_bytes<true>(), s>>>(tq, tk, tv, p);
+    constexpr int kPv = lpfa::kPvFp8;
+    if ((st = check_attn_kernel(reinterpret_cast<const void*>(lpfa::attn_fwd_kernel<kPv>), lpfa::attn_smem_bytes<true>())) != LPFA_OK) return st;
+    lpfa::attn_fwd_kernel<kPv><<<grid, lpfa::kAttnThreads, lpfa::attn_smem_bytes<true>(), s>>>(tq, tk, tv, p);
+  } else if (pv_mode == LPFA_PV_BF16) {
+    constexpr int kPv = lpfa::kPvBf16Mx;
+    if ((st = check_attn_kernel(reinterpret_cast<const void*>(lpfa::attn_fwd_kernel<kPv>), lpfa::attn_smem_bytes<false>())) != LPFA_OK) return st;
+    lpfa::attn_fwd_kernel<kPv><<<grid, lpfa::kAttnThreads, lpfa::attn_smem_bytes<false>(), s>>>(tq, tk, tv, p);
   } else {
-    if ((st = check_attn_kernel(reinterpret_cast<const void*>(lpfa::attn_fwd_kernel<false>), lpfa::attn_smem_bytes<false>())) != LPFA_OK) return st;
-    lpfa::attn_fwd_kernel<false><<<grid, lpfa::kAttnThreads, lpfa::attn_smem_bytes<false>(), s>>>(tq, tk, tv, p);
+    constexpr int kPv = lpfa::kPvBf16In;
+    if ((st = check_attn_kernel(reinterpret_cast<const void*>(lpfa::attn_fwd_kernel<kPv>), lpfa::attn_smem_bytes<false>())) != LPFA_OK) return st;
+    lpfa::attn_fwd_kernel<kPv><<<grid, lpfa::kAttnThreads, lpfa::attn_smem_bytes<false>(), s>>>(tq, tk, tv, p);
   }
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "attention launch");

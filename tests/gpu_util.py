@@ -69,6 +69,8 @@ def run_path(lp, q, k, v, lens_q, lens_k, heads, in_dtype="bf16", pv_mode="bf16"
     kp, ks = gpu_quantize(lp, k, in_dtype, mk, mode)
     if pv_mode == "fp8":
         vp, vs = lp.lpfa_cast_e4m3(to_device(v, "bf16")), None
+    elif pv_mode == "bf16v":
+        vp, vs = to_device(v, "bf16"), None          # BF16 V input, never quantized
     else:
         vp, vs = gpu_quantize(lp, v, in_dtype, mk, mode)
     dd = [None if x is None else torch.tensor([x], dtype=torch.float32, device="cuda") for x in descales]
@@ -86,6 +88,8 @@ def oracle_inputs(q, k, v, lens_q, lens_k, heads, pv_mode="bf16", mode="rceil"):
     kh = omx.dequantize_mxfp8(pk, sk, lens_k, heads)
     if pv_mode == "fp8":
         vh = omx.e4m3_decode(omx.cast_e4m3(v))
+    elif pv_mode == "bf16v":
+        vh = np.asarray(v, dtype=np.float64)        # the BF16 values themselves
     else:
         pv, sv = omx.quantize_mxfp8_varlen(v, lens_k, mode)
         vh = omx.dequantize_mxfp8(pv, sv, lens_k, heads)
@@ -140,6 +144,8 @@ def oracle_sampled(q, k, v, lens_q, lens_k, heads, toks, hs, pv_mode="bf16", mod
             kh = (omx.e4m3_decode(kp).reshape(-1, 4, 32) * np.ldexp(1.0, ke)[..., None]).reshape(-1, 128)
             if pv_mode == "fp8":
                 vh = omx.e4m3_decode(omx.cast_e4m3(v[k0:k1, h]))
+            elif pv_mode == "bf16v":
+                vh = np.asarray(v[k0:k1, h], dtype=np.float64)
             else:
                 vp, ve = omx.quantize_rows(v[k0:k1, h].astype(np.float64), mode)
                 vh = (omx.e4m3_decode(vp).reshape(-1, 4, 32) * np.ldexp(1.0, ve)[..., None]).reshape(-1, 128)

@@ -38,7 +38,7 @@ CASES = [
 ]
 
 
-@pytest.mark.parametrize("pv_mode", ["bf16", "fp8"])
+@pytest.mark.parametrize("pv_mode", ["bf16", "fp8", "bf16v"])
 @pytest.mark.parametrize("case", range(len(CASES)))
 def test_attention_small_cases(pv_mode, case):
     lq, lk, H = CASES[case]
@@ -59,7 +59,7 @@ def test_attention_fp32_inputs():
     gu.assert_within(gu.compare_attention(o, lse, o_ref, lse_ref), "fp32 inputs")
 
 
-@pytest.mark.parametrize("pv_mode", ["bf16", "fp8"])
+@pytest.mark.parametrize("pv_mode", ["bf16", "fp8", "bf16v"])
 def test_closed_forms(pv_mode):
     """Constant V gives V (bf16 PV) or V times one scalar per row (fp8 PV, where l sums the
     unrounded weights); equal logits give LSE = ln n + s and O = the mean of V."""
@@ -75,7 +75,7 @@ def test_closed_forms(pv_mode):
     o, lse = gu.run_path(lp, q, krand, vconst, [n], [n], H, pv_mode=pv_mode)
     qh, kh, vh = gu.oracle_inputs(q, krand, vconst, [n], [n], H, pv_mode)
     o_np = o.float().cpu().numpy().astype(np.float64)
-    if pv_mode == "bf16":
+    if pv_mode != "fp8":
         assert np.max(np.abs(o_np - vh[:1])) <= gu.O_MAX_ABS
     else:
         ratio = (o_np * vh[:1]).sum(axis=2) / (vh[:1] ** 2).sum(axis=2)      # (n, H)
@@ -86,7 +86,7 @@ def test_closed_forms(pv_mode):
     qh, kh, vh = gu.oracle_inputs(q, k, v, [n], [n], H, pv_mode)
     s = np.einsum("thd,hd->ht", qh, kh[0]) / math.sqrt(128)
     assert np.max(np.abs(lse.cpu().numpy() - (np.log(n) + s))) < gu.LSE_MAX_ABS
-    if pv_mode == "bf16":
+    if pv_mode != "fp8":
         assert np.max(np.abs(o.float().cpu().numpy() - vh.mean(axis=0)[None])) <= gu.O_MAX_ABS
 
 
@@ -99,7 +99,7 @@ def test_single_key():
     assert np.max(np.abs(lse.cpu().numpy() - s)) < gu.LSE_MAX_ABS
 
 
-@pytest.mark.parametrize("pv_mode", ["bf16", "fp8"])
+@pytest.mark.parametrize("pv_mode", ["bf16", "fp8", "bf16v"])
 def test_unit_descale_is_bit_identical_and_two_changes_output(pv_mode):
     """vLLM #63232 'Validation': absent descale == unit descale bit for bit; 2 changes it."""
     w = wl.WORKLOADS["dense_4x2048_h16"]
@@ -142,7 +142,7 @@ def test_negative_control_wrong_k_scales_fail():
     assert lmax > gu.LSE_MAX_ABS and rel > gu.O_REL_L2
 
 
-@pytest.mark.parametrize("name", ["single_s256_h2", "dense_4x2048_h16"])
+@pytest.mark.parametrize("name", ["single_s256_h2", "dense_4x2048_h16", "dense_4x2048_h16_bf16v"])
 @pytest.mark.parametrize("mode", ["rceil", "floor"])
 def test_workload_full_check(name, mode):
     w = wl.WORKLOADS[name]

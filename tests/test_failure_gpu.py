@@ -37,7 +37,7 @@ def _guards_intact(buf: torch.Tensor, nbytes: int) -> bool:
     return bool(torch.all(head == PATTERN).item()) and bool(torch.all(tail == PATTERN).item())
 
 
-@pytest.mark.parametrize("pv_mode", ["fp8", "bf16"])
+@pytest.mark.parametrize("pv_mode", ["fp8", "bf16", "bf16v"])
 def test_bounded_wait_runs_out_and_context_survives(pv_mode):
     lens, H = [300, 77], 2
     q, k, v = wl.small_random(11, lens, lens, H)
@@ -49,6 +49,8 @@ def test_bounded_wait_runs_out_and_context_survives(pv_mode):
     kp, ks = gu.gpu_quantize(lp, k, "bf16", mk)
     if pv_mode == "fp8":
         vp, vs = lp.lpfa_cast_e4m3(gu.to_device(v, "bf16")), None
+    elif pv_mode == "bf16v":
+        vp, vs = gu.to_device(v, "bf16"), None
     else:
         vp, vs = gu.gpu_quantize(lp, v, "bf16", mk)
     assert lp.lpfa_device_status() == (lp.LPFA_OK, 0)
@@ -82,7 +84,7 @@ def test_unknown_debug_flag_rejected():
     assert e.value.status == lp.LPFA_ERR_INVALID_ARG
 
 
-@pytest.mark.parametrize("pv_mode", ["fp8", "bf16"])
+@pytest.mark.parametrize("pv_mode", ["fp8", "bf16", "bf16v"])
 @pytest.mark.parametrize("lens_q,lens_k,H", [([1], [1], 1), ([300, 77, 1], [129, 700, 3], 3), ([2048], [257], 2)])
 def test_outputs_stay_inside_their_buffers(pv_mode, lens_q, lens_k, H):
     q, k, v = wl.small_random(3, lens_q, lens_k, H)
@@ -99,8 +101,8 @@ def test_outputs_stay_inside_their_buffers(pv_mode, lens_q, lens_k, H):
     qs = alloc("qs", mq.scale_bytes(H))
     kp = alloc("kp", Tk * H * 128).view(Tk, H, 128)
     ks = alloc("ks", mk.scale_bytes(H))
-    vp = alloc("vp", Tk * H * 128).view(Tk, H, 128)
-    vs = None if pv_mode == "fp8" else alloc("vs", mk.scale_bytes(H))
+    vp = gu.to_device(v, "bf16") if pv_mode == "bf16v" else alloc("vp", Tk * H * 128).view(Tk, H, 128)
+    vs = None if pv_mode != "bf16" else alloc("vs", mk.scale_bytes(H))
     out = alloc("out", Tq * H * 128 * 2).view(torch.bfloat16).view(Tq, H, 128)
     lse = alloc("lse", H * Tq * 4).view(torch.float32).view(H, Tq)
 
@@ -108,7 +110,7 @@ def test_outputs_stay_inside_their_buffers(pv_mode, lens_q, lens_k, H):
     lp.lpfa_quantize_mxfp8_varlen(gu.to_device(k, "bf16"), mk, payload=kp, scales=ks)
     if pv_mode == "fp8":
         lp.lpfa_cast_e4m3(gu.to_device(v, "bf16"), out=vp)
-    else:
+    elif pv_mode == "bf16":
         lp.lpfa_quantize_mxfp8_varlen(gu.to_device(v, "bf16"), mk, payload=vp, scales=vs)
     lp.lpfa_attn_fwd_varlen(qp, qs, kp, ks, vp, vs, mq, mk, pv_mode=pv_mode, out=out, lse=lse)
     torch.cuda.synchronize()

@@ -41,7 +41,7 @@ class Workload:
     index: int                    # stable id mixed into the seed
     heads: int
     in_dtype: str                 # "bf16" or "fp32" (Q, K and the quantized V)
-    pv_mode: str                  # "bf16" or "fp8"
+    pv_mode: str                  # "bf16", "fp8", or "bf16v" (BF16 V input, bf16 PV)
     scaling_mode: str = "rceil"   # "rceil" or "floor"
     num_seqs: int = 1
     len_q: Optional[int] = None   # fixed length, or None for drawn lengths
@@ -86,7 +86,12 @@ _add(Workload("lpfa4_bundled_8x2048_h16", 5, heads=16, in_dtype="bf16", pv_mode=
               num_seqs=8, len_q=2048, len_k=2048,
               description="LP-FA4 bundled benchmark shape: 8 x 2048, 16 heads, RCEIL"))
 
-# The five evaluation workloads in order (the sixth is an extra benchmark row).
+_add(Workload("dense_4x2048_h16_bf16v", 6, heads=16, in_dtype="bf16", pv_mode="bf16v",
+              num_seqs=4, len_q=2048, len_k=2048,
+              description="4 x 2048 uniform packed offsets, 16 heads, bf16 N(0,1); Q/K MXFP8 RCEIL, "
+                          "V kept in BF16, bf16 PV"))
+
+# The five evaluation workloads in order (the others are extra benchmark rows).
 EVAL_ORDER: List[str] = [
     "single_s256_h2",
     "dense_4x2048_h16",
