@@ -3,9 +3,10 @@
 // Computes, per (sequence, head), O = softmax(Q K^T * qd * kd / sqrt(128)) V * vd and the
 // natural-log LSE, for noncausal head_dim 128 over packed variable-length sequences
 // (LP-FA4 README, "MXFP8 forward and backward"). Q and K are MXFP8 (E4M3 payload, one E8M0
-// scale per 32 elements along head_dim). V is either MXFP8 (bf16 PV mode: dequantized to
-// BF16 in shared memory, P rounded to BF16) or an unscaled E4M3 cast (fp8 PV mode of
-// FastVideo #1654: no V scales, implicit dequant scale 1.0, output still BF16).
+// scale per 32 elements along head_dim). V is MXFP8 (bf16 PV mode: dequantized to BF16 in
+// shared memory, P rounded to BF16), an unscaled E4M3 cast (fp8 PV mode of FastVideo #1654: no
+// V scales, implicit dequant scale 1.0, output still BF16), or BF16 that is never quantized
+// (bf16 PV with BF16 V, loaded by TMA straight into the BF16 operand layout).
 // Absent descales are the literal 1.0f on the same code path (vLLM #63232, "Claims").
 //
 // Work unit: one 128-row query tile of one (sequence, head). The grid is persistent (one CTA
@@ -29,7 +30,7 @@
 //                 row and all 128 keys of the tile (192 registers after setmaxnreg). The groups
 //                 run half a tile apart, so one group's exponentials (MUFU) overlap the other's
 //                 load, max, packing and stores.
-//   warps 12..15  bf16 PV mode only: convert the V tile from MXFP8 to BF16 in shared memory.
+//   warps 12..15  bf16 PV mode with MXFP8 V: convert the V tile to BF16 in shared memory.
 //
 // Online softmax keeps one reference m per row (an integer, log2 units) shared by the two
 // groups: tile t's reference is its own row-maximum ceiling if that exceeds tile t-1's
