@@ -114,6 +114,13 @@ struct AttnParams {
   int debug_stall;          // test hook: >0 makes the MMA warp wait on a phase that never comes
 };
 
+// Work order: up to this many sequences are ordered longest first (by key tiles) in shared
+// memory at the start of the kernel; beyond it units keep the plain head-major order.
+#ifndef LPFA_MAX_SORT_SEQS
+#define LPFA_MAX_SORT_SEQS 256
+#endif
+constexpr int kMaxSortSeqs = LPFA_MAX_SORT_SEQS;
+
 // Shared memory layout (offsets from a 1024-byte aligned base).
 template <bool kFp8PV>
 struct SmemLayout {
@@ -129,7 +136,8 @@ struct SmemLayout {
   static constexpr uint32_t lsum = mref + 2 * 128 * 4;                // float [2 groups][128] partial l
   static constexpr uint32_t mfin = lsum + 2 * 128 * 4;                // float [2 groups][128] reference of l
   static constexpr uint32_t lsumr = mfin + 2 * 128 * 4;               // float [2 groups][128] partial sum of rounded P
-  static constexpr uint32_t bars = lsumr + 2 * 128 * 4;               // uint64 barriers
+  static constexpr uint32_t sched = lsumr + 2 * 128 * 4;              // int: n, order[kMaxSortSeqs], prefix[kMaxSortSeqs + 1]
+  static constexpr uint32_t bars = sched + ((2 * kMaxSortSeqs + 2) * 4 + 15) / 16 * 16;  // uint64 barriers
   static constexpr uint32_t num_bars = 64;
   static constexpr uint32_t misc = bars + num_bars * 8;               // tmem base, abort flag
   static constexpr uint32_t total = misc + 64;
@@ -308,13 +316,42 @@ __device__ __forceinline__ int find_prefix(const int32_t* prefix, int n, int g) 
   return lo;
 }
 
-__device__ __forceinline__ UnitInfo unit_info(const AttnParams& p, int w) {
+// Unit order, kept in shared memory (sched[0] = n, sched[1 ..] = order, then the prefix) so that
+// nothing of it stays live in registers across the hot loops. Sorted (n > 0): sequences by
+// decreasing key-tile count, each taking heads * its query tiles consecutive units, query tiles
+// innermost so that the CTAs running together share one (sequence, head)'s K/V through L2; a
+// static round-robin over this longest-first list approximates longest-processing-time
+// scheduling. Unsorted (n = 0): unit w is head w / total_q_tiles, query tile w % total_q_tiles
+// of the packed order.
+__device__ __forceinline__ int find_prefix_smem(const int* prefix, int n, int g) {
+  int lo = 0, hi = n - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (prefix[mid] <= g) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+__device__ __forceinline__ UnitInfo unit_info(const AttnParams& p, const int* sched, int w) {
   UnitInfo u;
-  u.h = w / p.total_q_tiles;
-  const int g = w - u.h * p.total_q_tiles;
-  u.seq = find_prefix(p.so_q, p.num_seqs, g);
-  u.sbq = __ldg(p.so_q + u.seq);
-  u.qtile = g - u.sbq;
+  const int n = sched[0];
+  if (n > 0) {
+    const int* order = sched + 1;
+    const int* pre = sched + 1 + kMaxSortSeqs;
+    const int r = find_prefix_smem(pre, n, w);
+    u.seq = order[r];
+    u.sbq = __ldg(p.so_q + u.seq);
+    const int nq = __ldg(p.so_q + u.seq + 1) - u.sbq;
+    const int local = w - pre[r];
+    u.h = local / nq;
+    u.qtile = local - u.h * nq;
+  } else {
+    u.h = w / p.total_q_tiles;
+    const int g = w - u.h * p.total_q_tiles;
+    u.seq = find_prefix(p.so_q, p.num_seqs, g);
+    u.sbq = __ldg(p.so_q + u.seq);
+    u.qtile = g - u.sbq;
+  }
   const int cq0 = __ldg(p.cu_q + u.seq);
   u.q_row0 = cq0 + u.qtile * kTileM;
   u.q_len = __ldg(p.cu_q + u.seq + 1) - cq0;
@@ -323,6 +360,57 @@ __device__ __forceinline__ UnitInfo unit_info(const AttnParams& p, int w) {
   u.nkv = (u.k_len + kTileN - 1) / kTileN;
   u.sbk = __ldg(p.so_k + u.seq);
   return u;
+}
+
+// Builds the longest-first order in shared memory (all threads of the CTA; ends synchronized).
+// More than kMaxSortSeqs sequences, or a single one, keep the plain order (n = 0).
+__device__ __forceinline__ void build_unit_order(const AttnParams& p, int* sched) {
+  const int n = p.num_seqs;
+  int* s_order = sched + 1;
+  int* s_pre = sched + 1 + kMaxSortSeqs;
+  if (n > kMaxSortSeqs || n < 2) {
+    if (threadIdx.x == 0) sched[0] = 0;
+    __syncthreads();
+    return;
+  }
+  int* s_cost = s_pre;  // key tiles per sequence, before s_pre holds the prefix
+  for (int i = threadIdx.x; i < n; i += blockDim.x)
+    s_cost[i] = (__ldg(p.cu_k + i + 1) - __ldg(p.cu_k + i) + kTileN - 1) / kTileN;
+  __syncthreads();
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    const int ci = s_cost[i];
+    int rank = 0;
+    for (int j = 0; j < n; ++j) {
+      const int cj = s_cost[j];
+      rank += (cj > ci || (cj == ci && j < i)) ? 1 : 0;
+    }
+    s_order[rank] = i;
+  }
+  __syncthreads();
+  // Prefix of heads * query tiles over the sorted sequences (warp 0, 32 at a time).
+  if (threadIdx.x < 32) {
+    int carry = 0;
+    for (int base = 0; base < n; base += 32) {
+      const int r = base + static_cast<int>(threadIdx.x);
+      int v = 0;
+      if (r < n) {
+        const int sq = s_order[r];
+        v = p.heads * (__ldg(p.so_q + sq + 1) - __ldg(p.so_q + sq));
+      }
+#pragma unroll
+      for (int d = 1; d < 32; d <<= 1) {
+        const int o = __shfl_up_sync(0xFFFFFFFFu, v, d);
+        if (threadIdx.x >= static_cast<unsigned>(d)) v += o;
+      }
+      if (r < n) s_pre[r + 1] = carry + v;     // inclusive prefix -> entry r + 1
+      carry += __shfl_sync(0xFFFFFFFFu, v, 31);
+    }
+    if (threadIdx.x == 0) {
+      s_pre[0] = 0;
+      sched[0] = n;
+    }
+  }
+  __syncthreads();
 }
 
 // Warp-uniform copies of values that every lane of a warp computes identically. Results of
@@ -427,6 +515,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  build_unit_order(p, reinterpret_cast<int*>(smem + L::sched));
+  const int* sched = reinterpret_cast<const int*>(smem + L::sched);
   // All 512 columns of the SM's tensor memory belong to this CTA (one CTA per SM), so the
   // allocation starts at lane 0, column 0. Using the constant keeps every TMEM operand of
   // the tcgen05 instructions a compile-time or warp-uniform value.
@@ -447,7 +537,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
       uint32_t qc = 0, kc = 0;  // fills issued per ring
       bool ok = true;
       for (int w = blockIdx.x; w < p.num_units && ok; w += G) {
-        const UnitInfo ui = warp_uniform(unit_info(p, w));
+        const UnitInfo ui = warp_uniform(unit_info(p, sched, w));
         if (ui.nkv == 0) continue;  // no keys: the softmax warps write the empty-sum result
         const uint32_t qs = qc % kQStages, qph = (qc / kQStages) & 1;
         if (!mbar_wait_warp(&bars[kBarQEmpty + qs], qph ^ 1, abort_flag)) { record_failure(abort_flag, kSiteProducerQ); ok = false; break; }
@@ -483,7 +573,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
       uint32_t vc = 0;
       bool ok = true;
       for (int w = blockIdx.x; w < p.num_units && ok; w += G) {
-        const UnitInfo ui = warp_uniform(unit_info(p, w));
+        const UnitInfo ui = warp_uniform(unit_info(p, sched, w));
         for (int j = 0; j < ui.nkv; ++j) {
           const uint32_t sb = vc % kVbfStages, phb = (vc / kVbfStages) & 1;
           if (!mbar_wait_warp(&bars[kBarVbfEmpty + sb], phb ^ 1, abort_flag)) { record_failure(abort_flag, kSiteProducerV); ok = false; break; }
@@ -505,7 +595,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
       uint32_t vc = 0;
       bool ok = true;
       for (int w = blockIdx.x; w < p.num_units && ok; w += G) {
-        const UnitInfo ui = warp_uniform(unit_info(p, w));
+        const UnitInfo ui = warp_uniform(unit_info(p, sched, w));
         for (int j = 0; j < ui.nkv; ++j) {
           const uint32_t s = vc % kVStages, ph = (vc / kVStages) & 1;
           if (!mbar_wait_warp(&bars[kBarVEmpty + s], ph ^ 1, abort_flag)) { record_failure(abort_flag, kSiteProducerV); ok = false; break; }
@@ -547,7 +637,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
         if (!mbar_wait_warp(&bars[kBarDrain], 0, abort_flag)) { record_failure(abort_flag, kSiteDebugStall); ok = false; }
       }
       for (int w = blockIdx.x; w < p.num_units && ok; w += G) {
-        const UnitInfo ui = warp_uniform(unit_info(p, w));
+        const UnitInfo ui = warp_uniform(unit_info(p, sched, w));
         if (ui.nkv == 0) continue;
         const uint32_t qs = u % kQStages;
         if (!mbar_wait_warp(&bars[kBarQFull + qs], (u / kQStages) & 1, abort_flag)) { record_failure(abort_flag, kSiteMmaQ); ok = false; break; }
@@ -597,7 +687,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
       uint32_t u = 0, vc = 0, t = 0;  // units, V tiles, tiles
       bool ok = true;
       for (int w = blockIdx.x; w < p.num_units && ok; w += G) {
-        const UnitInfo ui = warp_uniform(unit_info(p, w));
+        const UnitInfo ui = warp_uniform(unit_info(p, sched, w));
         if (ui.nkv == 0) continue;
         for (int j = 0; j < ui.nkv; ++j, ++t) {
           const uint32_t b = t & 1;
@@ -652,7 +742,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
     uint32_t u = 0, t0 = 0;
     bool ok = true;
     for (int w = blockIdx.x; w < p.num_units && ok; w += G) {
-      const UnitInfo ui = unit_info(p, w);
+      const UnitInfo ui = unit_info(p, sched, w);
       if (ui.nkv == 0) {
         // No keys: an empty sum, LSE = log 0 = -inf and O = 0.
         if (ui.qtile * kTileM + row < ui.q_len) {
@@ -817,7 +907,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
       uint32_t vc = 0;
       bool ok = true;
       for (int w = blockIdx.x; w < p.num_units && ok; w += G) {
-        const UnitInfo ui = unit_info(p, w);
+        const UnitInfo ui = unit_info(p, sched, w);
         for (int j = 0; j < ui.nkv; ++j) {
           const uint32_t s = vc % kVStages, ph = (vc / kVStages) & 1;
           const uint32_t sb = vc % kVbfStages, phb = (vc / kVbfStages) & 1;

@@ -51,6 +51,18 @@ def test_attention_small_cases(pv_mode, case):
     gu.assert_within(gu.compare_attention(o, lse, o_ref, lse_ref), f"{pv_mode} {lq}/{lk} H={H}")
 
 
+@pytest.mark.parametrize("nseq", [200, 300])   # longest-first order (<= 256 sequences) and plain order
+def test_many_sequences(nseq):
+    g = np.random.default_rng(nseq)
+    lq = g.integers(1, 300, size=nseq).tolist()
+    lk = g.integers(1, 300, size=nseq).tolist()
+    q, k, v = wl.small_random(31, lq, lk, 1)
+    o, lse = gu.run_path(lp, q, k, v, lq, lk, 1, pv_mode="fp8")
+    _status_ok()
+    o_ref, lse_ref = gu.oracle_full(q, k, v, lq, lk, 1, pv_mode="fp8")
+    gu.assert_within(gu.compare_attention(o, lse, o_ref, lse_ref), f"{nseq} sequences")
+
+
 def test_attention_fp32_inputs():
     lq = lk = [333]
     q, k, v = wl.small_random(7, lq, lk, 2, dtype="fp32")
