@@ -40,9 +40,11 @@
 // PV mode P is stored as E4M3(2^(bias - m) 2^s) <= 256; the power of two cancels in the final
 // division.
 //
-// TMEM columns (512 allocated): S buffer b at [128b, 128b + 128), O [256, 384), fp8 P buffer
-// b at [384 + 32b, 416 + 32b) (bf16 P is written over the first 64 columns of its S buffer),
-// Q scale atoms (2 stages) [448, 456), K scale atoms (2 slots) [456, 464).
+// TMEM columns (512 allocated): S buffer b at [128b, 128b + 128), O [256, 384), fp8 P slot
+// t % 3 at [384 + 32 (t % 3), 416 + 32 (t % 3)) (bf16 P is written over the first 64 columns
+// of its S buffer), Q scale atoms (2 stages) [480, 488), K scale atoms (2 slots) [488, 496).
+// Three fp8 P slots let a group store P(t) once PV(t - 3) is done; with two, P(t) would wait
+// for PV(t - 2), which the tensor pipe is often still executing.
 #pragma once
 
 #include <cstdint>
@@ -78,9 +80,11 @@ constexpr uint32_t kAtomBytes = 512;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0;        // + 128 * b  S buffer (fp32); bf16 P over its first 64 columns
 constexpr uint32_t kColO = 256;      // O accumulator (fp32)
-constexpr uint32_t kColP = 384;      // + 32 * b   fp8 P buffer
-constexpr uint32_t kColSFA = 448;    // + 4 * stage  Q scale atom
-constexpr uint32_t kColSFB = 456;    // + 4 * slot   K scale atom
+constexpr uint32_t kColP = 384;      // + 32 * (t % kPSlots)  fp8 P slot
+constexpr uint32_t kPSlots = 3;
+constexpr uint32_t kColSFA = 480;    // + 4 * stage  Q scale atom
+constexpr uint32_t kColSFB = 488;    // + 4 * slot   K scale atom
+static_assert(kColP + 32 * kPSlots <= kColSFA && kColSFB + 8 <= kTmemCols, "TMEM columns");
 
 // log2(e) / sqrt(128) rounded to fp32: logits in log2 units per unit of Q.K.
 constexpr float kLog2eRsqrtD = 0.12751743082459868f;
@@ -154,12 +158,12 @@ enum Bar : int {
   kBarSFull = 32,    // S(t) computed                       (MMA commit)
   kBarSFree = 34,    // S(t) read out by its group            (4 warps)
   kBarPReady = 36,   // P(t) stored, O rescaled if needed     (4 warps)
-  kBarPVDone = 38,   // PV(t) complete                        (MMA commit)
-  kBarOFull = 40,    // every PV of the unit complete         (MMA commit)
-  kBarOEmpty = 41,   // O read out by both groups             (8 warps)
-  kBarLReady = 42,   // partial l / reference exchanged       (8 warps)
-  kBarDrain = 43,    // QK issuer's own tcgen05 work done
-  kBarDrainPV = 44,  // PV issuer's own tcgen05 work done
+  kBarPVDone = 38,   // [t % kPSlots] PV(t) complete           (MMA commit)
+  kBarOFull = 41,    // every PV of the unit complete         (MMA commit)
+  kBarOEmpty = 42,   // O read out by both groups             (8 warps)
+  kBarLReady = 43,   // partial l / reference exchanged       (8 warps)
+  kBarDrain = 44,    // QK issuer's own tcgen05 work done
+  kBarDrainPV = 45,  // PV issuer's own tcgen05 work done
   kBarMRef = 48      // [group][lane quarter]: tile reference of t published and the MUFU
                      // handed over to the other group (1 warp; 8 entries)
 };
@@ -495,8 +499,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
       mbar_init(&bars[kBarSFull + i], 1);
       mbar_init(&bars[kBarSFree + i], 4);
       mbar_init(&bars[kBarPReady + i], 4);
-      mbar_init(&bars[kBarPVDone + i], 1);
     }
+    for (uint32_t i = 0; i < kPSlots; ++i) mbar_init(&bars[kBarPVDone + i], 1);
     mbar_init(&bars[kBarOFull], 1);
     mbar_init(&bars[kBarOEmpty], 8);
     mbar_init(&bars[kBarLReady], 8);
@@ -651,7 +655,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
             // S buffer b has been read out by its group (tile t - 2); in bf16 PV mode it also
             // holds P(t - 2), so PV(t - 2) must have completed.
             if (!mbar_wait_warp(&bars[kBarSFree + b], ((t - 2) >> 1) & 1, abort_flag)) { record_failure(abort_flag, kSiteMmaS); ok = false; break; }
-            if (!kFp8PV && !mbar_wait_warp(&bars[kBarPVDone + b], ((t - 2) >> 1) & 1, abort_flag)) { record_failure(abort_flag, kSiteMmaS); ok = false; break; }
+            if (!kFp8PV && !mbar_wait_warp(&bars[kBarPVDone + (t - 2) % kPSlots], ((t - 2) / kPSlots) & 1, abort_flag)) { record_failure(abort_flag, kSiteMmaS); ok = false; break; }
           }
           const uint32_t s = kc % kKStages;
           if (!mbar_wait_warp(&bars[kBarKFull + s], (kc / kKStages) & 1, abort_flag)) { record_failure(abort_flag, kSiteMmaK); ok = false; break; }
@@ -698,7 +702,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
           if (!got) { record_failure(abort_flag, kSiteMmaV); ok = false; break; }
           tc_fence_after();
           if (kFp8PV) {
-            const uint32_t p_col = tmem + kColP + b * 32;
+            const uint32_t p_col = tmem + kColP + (t % kPSlots) * 32;
             const uint64_t bdesc = dv0 + ((vc % kVStages) * kTileBytes >> 4);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)  // keys [32kk, 32kk + 32): 8 columns of 4 E4M3 each
@@ -714,7 +718,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
                          (j > 0 || kk > 0) ? 1u : 0u, leader);
             mma_commit(&bars[kBarVbfEmpty + vc % kVbfStages], leader);
           }
-          mma_commit(&bars[kBarPVDone + b], leader);
+          mma_commit(&bars[kBarPVDone + t % kPSlots], leader);
           ++vc;
         }
         if (!ok) break;
@@ -795,18 +799,19 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
         l_g = l_g * l_scale + psum;
         if (!kFp8PV) lr_g *= l_scale;
         m_g = m_t;
-        // PV(t - 2) has read this group's previous P.
-        if (kt >= 1) {
-          if (!mbar_wait_warp(&bars[kBarPVDone + grp], (kt - 1) & 1, abort_flag)) { record_failure(abort_flag, kSiteSoftPV); ok = false; break; }
-          tc_fence_after();
-        }
         if (kFp8PV) {
+          // PV(t - 3) has read the previous P of this slot. (In bf16 PV mode P goes over the S
+          // buffer, which QK(t) only overwrote after PV(t - 2) had completed.)
+          if (t >= kPSlots) {
+            if (!mbar_wait_warp(&bars[kBarPVDone + t % kPSlots], ((t - kPSlots) / kPSlots) & 1, abort_flag)) { record_failure(abort_flag, kSiteSoftPV); ok = false; break; }
+            tc_fence_after();
+          }
           uint32_t pk[32];
 #pragma unroll
           for (int i = 0; i < 32; ++i)
             pk[i] = static_cast<uint32_t>(cvt_e4m3x2(sv[2 * i].x, sv[2 * i].y)) |
                     (static_cast<uint32_t>(cvt_e4m3x2(sv[2 * i + 1].x, sv[2 * i + 1].y)) << 16);
-          tmem_st32_sync(tmem + lane_addr + kColP + grp * 32, pk);
+          tmem_st32_sync(tmem + lane_addr + kColP + (t % kPSlots) * 32, pk);
         } else {
           // O is normalised by the sum of the P values the PV product actually uses, so a
           // row dominated by one key gets that V row exactly (the LSE keeps the unrounded sum).
@@ -828,7 +833,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
         // O holds tiles up to t - 1 relative to m_prev; rescale it when the reference moved
         // (rare; never on a unit's first tile).
         if (j > 0 && __any_sync(0xFFFFFFFFu, m_t != m_prev)) {
-          if (!mbar_wait_warp(&bars[kBarPVDone + (grp ^ 1)], ((t - 1) >> 1) & 1, abort_flag)) { record_failure(abort_flag, kSiteSoftO); ok = false; break; }
+          if (!mbar_wait_warp(&bars[kBarPVDone + (t - 1) % kPSlots], ((t - 1) / kPSlots) & 1, abort_flag)) { record_failure(abort_flag, kSiteSoftO); ok = false; break; }
           tc_fence_after();
           const float alpha = exp2_int(m_prev - m_t);
           const float2 a2 = make_float2(alpha, alpha);
