@@ -10,9 +10,13 @@ head_dim-128 MHA, ``out, lse = mxfp8_flash_attn_varlen_forward(...)``):
     LSE_r = m_r + ln(l_r)                          (natural log)
 
 Sequence i of the query metadata attends to sequence i of the key metadata
-(cross attention pairs sequences by index). Per-tensor descales qd, kd, vd
-default to exactly 1.0 when absent (vLLM PR #63232, "Claims": a missing descale
-is read as 1.0). qd and kd act on the logits, vd on the output.
+(cross attention pairs sequences by index). Descales qd, kd, vd default to
+exactly 1.0 when absent (vLLM PR #63232, "Claims": a missing descale is read as
+1.0). qd and kd act on the logits, vd on the output. Each is a scalar (per
+tensor) or an array indexed by (sequence, head): shape (H,) for per-head scales,
+(num_seqs, H) for FA4's (batch, kv_heads) descale layout, size-1 axes broadcast
+(same page: calibrated per-tensor and per-head scales keep their descale
+tensors). Reading: with MHA, the KV head of a query head is that head.
 
 fp8 PV grading variant (``p_mode="fp8"``). FastVideo PR #1654 feeds PV with
 plain fp8 operands but does not say how P is rounded. The reading used here,
@@ -55,6 +59,19 @@ def _fp8_weights(t: np.ndarray) -> np.ndarray:
     return w, u
 
 
+def descale_at(d, seq: int, head: int) -> float:
+    """The descale value for (sequence, head): d is a scalar, an (H,) array, or an (S, H) array
+    whose size-1 axes broadcast."""
+    a = np.asarray(d, dtype=np.float64)
+    if a.ndim == 0:
+        return float(a)
+    if a.ndim == 1:
+        return float(a[head if a.shape[0] > 1 else 0])
+    if a.ndim == 2:
+        return float(a[seq if a.shape[0] > 1 else 0, head if a.shape[1] > 1 else 0])
+    raise ValueError("a descale is a scalar, (H,) or (S, H)")
+
+
 def attend_block(q, k, v, qd=1.0, kd=1.0, vd=1.0, p_mode: str = "exact"):
     """Attention of query rows q (R,128) over keys k, v (N,128); returns (O (R,128), LSE (R,))."""
     q = np.asarray(q, dtype=np.float64)
@@ -93,7 +110,7 @@ def attention_fwd(qhat, khat, vhat, lengths_q, lengths_k, qd=1.0, kd=1.0, vd=1.0
         k0, k1 = int(mk.cu_seqlens[i]), int(mk.cu_seqlens[i + 1])
         for h in range(H):
             o, l = attend_block(qhat[q0:q1, h], khat[k0:k1, h], vhat[k0:k1, h],
-                                qd, kd, vd, p_mode)
+                                descale_at(qd, i, h), descale_at(kd, i, h), descale_at(vd, i, h), p_mode)
             out[q0:q1, h] = o
             lse[h, q0:q1] = l
     return out, lse
@@ -120,7 +137,8 @@ def attention_rows(qhat_rows, seq_of_row, head_of_row, khat, vhat, lengths_k,
         else:
             k0, k1 = int(mk.cu_seqlens[i]), int(mk.cu_seqlens[i + 1])
             kk, vv = khat[k0:k1, h], vhat[k0:k1, h]
-        o, l = attend_block(np.asarray(qhat_rows)[rows], kk, vv, qd, kd, vd, p_mode)
+        o, l = attend_block(np.asarray(qhat_rows)[rows], kk, vv, descale_at(qd, i, h),
+                            descale_at(kd, i, h), descale_at(vd, i, h), p_mode)
         out[rows] = o
         lse[rows] = l
     return out, lse

@@ -142,6 +142,60 @@ def test_descale_two_equals_scale_bytes_plus_one():
     assert not np.allclose(o1, o3, atol=1e-3)
 
 
+def _raise_scale_bytes(scales, lengths, heads, exps):
+    """Scale storage with the bytes of (sequence i, head h) raised by exps[i, h]."""
+    from oracle import meta as omt
+    m = omt.from_lengths(lengths)
+    out = scales.copy().reshape(-1, heads, 512)
+    for i in range(m.num_seqs):
+        for h in range(heads):
+            out[m.scale_off[i]:m.scale_off[i + 1], h, :] += np.uint8(exps[i, h])
+    return out.reshape(scales.shape)
+
+
+def test_per_head_and_per_sequence_descales_equal_raised_scale_bytes():
+    """vLLM PR #63232 ("Claims"): per-head scales keep their descale tensors. A per-head q descale
+    of 2^e_h is the same as raising head h's Q scale bytes by e_h, and an (S, H) k descale of
+    2^e_ih the same as raising the K bytes of sequence i, head h by e_ih; v descales scale O only."""
+    g = np.random.default_rng(9)
+    lens_q, lens_k, H = [150, 70], [90, 200], 3
+    x = g.standard_normal((sum(lens_q), H, 128)).astype(np.float32)
+    kx = g.standard_normal((sum(lens_k), H, 128)).astype(np.float32)
+    vx = g.standard_normal((sum(lens_k), H, 128)).astype(np.float32)
+    pq, sq = omx.quantize_mxfp8_varlen(x, lens_q)
+    pk, sk = omx.quantize_mxfp8_varlen(kx, lens_k)
+    pv, sv = omx.quantize_mxfp8_varlen(vx, lens_k)
+    qh = omx.dequantize_mxfp8(pq, sq, lens_q, H)
+    kh = omx.dequantize_mxfp8(pk, sk, lens_k, H)
+    vh = omx.dequantize_mxfp8(pv, sv, lens_k, H)
+    eq = np.array([1, -1, 2])
+    ek = np.array([[0, 1, -2], [2, 0, 1]])
+    qh2 = omx.dequantize_mxfp8(pq, _raise_scale_bytes(sq, lens_q, H, np.tile(eq, (2, 1))), lens_q, H)
+    kh2 = omx.dequantize_mxfp8(pk, _raise_scale_bytes(sk, lens_k, H, ek), lens_k, H)
+    o1, l1 = oatt.attention_fwd(qh, kh, vh, lens_q, lens_k, qd=2.0 ** eq, kd=2.0 ** ek)
+    o2, l2 = oatt.attention_fwd(qh2, kh2, vh, lens_q, lens_k)
+    assert np.allclose(o1, o2, atol=1e-12) and np.allclose(l1, l2, atol=1e-12)
+    # a per-head v descale multiplies that head's O and leaves the LSE alone
+    vd = np.array([1.0, 4.0, 0.5])
+    o3, l3 = oatt.attention_fwd(qh, kh, vh, lens_q, lens_k, vd=vd.reshape(1, 3))
+    o0, l0 = oatt.attention_fwd(qh, kh, vh, lens_q, lens_k)
+    assert np.allclose(o3, o0 * vd[None, :, None], atol=1e-12) and np.array_equal(l3, l0)
+    # broadcasting: (1, 1), (1,) and scalar are the same per-tensor value
+    for d in (np.array([[2.0]]), np.array([2.0]), 2.0):
+        o4, l4 = oatt.attention_fwd(qh, kh, vh, lens_q, lens_k, qd=d)
+        o5, l5 = oatt.attention_fwd(qh, kh, vh, lens_q, lens_k, qd=2.0)
+        assert np.array_equal(o4, o5) and np.array_equal(l4, l5)
+
+
+def test_descale_at_indexing():
+    d = np.arange(6, dtype=np.float64).reshape(2, 3)
+    assert oatt.descale_at(d, 1, 2) == 5.0 and oatt.descale_at(d, 0, 1) == 1.0
+    assert oatt.descale_at(np.array([7.0, 8.0, 9.0]), 1, 2) == 9.0
+    assert oatt.descale_at(np.array([[3.0, 4.0]]), 1, 1) == 4.0   # size-1 sequence axis broadcasts
+    assert oatt.descale_at(np.array([[3.0], [4.0]]), 1, 1) == 4.0  # size-1 head axis broadcasts
+    assert oatt.descale_at(1.5, 3, 3) == 1.5
+
+
 def test_fp8_variant_equals_plain_when_weights_exact():
     """Logits whose log2 values are integers give E4M3-exact weights: variant == definition."""
     g = np.random.default_rng(7)
