@@ -153,9 +153,10 @@ LPFA_API lpfa_status lpfa_cast_e4m3(const void* v_bf16, int64_t tok_stride, int6
  *                  (Tk, H, 128), contiguous, never quantized (LP-FA4 README: V kept in BF16);
  *                  v_sf must be NULL; P is rounded to BF16 as in LPFA_PV_BF16.
  * meta_q, meta_k   sequence i of meta_q attends to sequence i of meta_k (same num_seqs).
- * q/k/v_descale    device pointers to one float each, or NULL. NULL means exactly 1.0: the
- *                  kernel then uses the literal 1.0f on the same code path, so a descale of
- *                  1.0 gives bit-identical output to NULL. Logits are scaled by
+ * q/k/v_descale    device pointers to one float each, or NULL (per-tensor descales; see
+ *                  lpfa_attn_fwd_varlen_descaled for per-head ones). NULL means exactly 1.0:
+ *                  the kernel then uses the literal 1.0f on the same code path, so a descale
+ *                  of 1.0 gives bit-identical output to NULL. Logits are scaled by
  *                  q_descale * k_descale / sqrt(128), O by v_descale. Values must be finite.
  * out_bf16         device, (Tq, H, 128) bf16, written for every real token row.
  * lse              device, (H, Tq) fp32, natural-log logsumexp of the scaled logits.
@@ -173,6 +174,37 @@ LPFA_API lpfa_status lpfa_attn_fwd_varlen(const uint8_t* q, const uint8_t* q_sf,
                                  const float* q_descale, const float* k_descale,
                                  const float* v_descale, void* out_bf16, float* lse,
                                  void* stream);
+
+/*
+ * A descale tensor indexed by (sequence, head) (vLLM #63232, "Claims": calibrated per-tensor
+ * scales and per-head scales keep their descale tensors; FA4's descale views are
+ * (batch, kv_heads)). The value for sequence i, head h is ptr[i * seq_stride + h * head_stride]
+ * (strides in elements, >= 0): per tensor (0, 0), per head (0, 1), one value per sequence and
+ * head (heads, 1). ptr NULL means exactly 1.0 everywhere, the strides are then ignored. The
+ * caller owns the device buffer, which must hold every index the strides reach for
+ * i < num_seqs, h < heads.
+ */
+typedef struct {
+  const float* ptr;
+  int64_t seq_stride;
+  int64_t head_stride;
+} lpfa_descale;
+
+/*
+ * lpfa_attn_fwd_varlen with descales per (sequence, head). Arguments and behaviour as
+ * lpfa_attn_fwd_varlen, except that q/k/v_descale point to lpfa_descale descriptors (host
+ * memory, read before the call returns); a NULL descriptor or a NULL ptr means exactly 1.0 on
+ * the same code path, so descale values of 1.0 give bit-identical output to no descale.
+ * The logits of sequence i, head h are scaled by q(i,h) * k(i,h) / sqrt(128), its O rows by
+ * v(i,h). Errors: as lpfa_attn_fwd_varlen, plus LPFA_ERR_INVALID_ARG for a negative stride.
+ */
+LPFA_API lpfa_status lpfa_attn_fwd_varlen_descaled(const uint8_t* q, const uint8_t* q_sf, const uint8_t* k,
+                                          const uint8_t* k_sf, const uint8_t* v, const uint8_t* v_sf,
+                                          const lpfa_varlen_meta* meta_q, const lpfa_varlen_meta* meta_k,
+                                          int32_t heads, int32_t head_dim, lpfa_pv_mode pv_mode,
+                                          const lpfa_descale* q_descale, const lpfa_descale* k_descale,
+                                          const lpfa_descale* v_descale, void* out_bf16, float* lse,
+                                          void* stream);
 
 /*
  * Device status word. Kernels that bound their barrier waits record a failure code in a

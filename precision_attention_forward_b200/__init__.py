@@ -38,6 +38,7 @@ EXPORTED_SYMBOLS = (
     "lpfa_meta_dev_ints", "lpfa_varlen_meta_fill_host", "lpfa_varlen_meta_from_lengths",
     "lpfa_scale_bytes", "lpfa_quantize_mxfp8_varlen", "lpfa_cast_e4m3", "lpfa_attn_fwd_varlen",
     "lpfa_device_status", "lpfa_last_error_message", "lpfa_version", "lpfa_attn_fwd_varlen_debug",
+    "lpfa_attn_fwd_varlen_descaled",
 )
 
 
@@ -45,6 +46,10 @@ class LpfaError(RuntimeError):
     def __init__(self, status: int, message: str):
         super().__init__(f"lpfa status {_STATUS_NAMES.get(status, status)}: {message}")
         self.status = status
+
+
+class _Descale(ctypes.Structure):
+    _fields_ = [("ptr", ctypes.c_void_p), ("seq_stride", ctypes.c_int64), ("head_stride", ctypes.c_int64)]
 
 
 class _Meta(ctypes.Structure):
@@ -71,6 +76,9 @@ _lib.lpfa_attn_fwd_varlen.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, ctypes.POINT
                                       _i32, _i32, ctypes.c_int, _f32p, _f32p, _f32p, _vp, _vp, _vp]
 _lib.lpfa_attn_fwd_varlen.restype = ctypes.c_int
 _lib.lpfa_attn_fwd_varlen_debug.argtypes = list(_lib.lpfa_attn_fwd_varlen.argtypes) + [_i32]
+_lib.lpfa_attn_fwd_varlen_descaled.argtypes = (list(_lib.lpfa_attn_fwd_varlen.argtypes[:11]) +
+                                               [ctypes.POINTER(_Descale)] * 3 + [_vp, _vp, _vp])
+_lib.lpfa_attn_fwd_varlen_descaled.restype = ctypes.c_int
 _lib.lpfa_attn_fwd_varlen_debug.restype = ctypes.c_int
 _lib.lpfa_device_status.argtypes = [_vp, ctypes.POINTER(_i32)]
 _lib.lpfa_device_status.restype = ctypes.c_int
@@ -194,6 +202,25 @@ def lpfa_cast_e4m3(v: torch.Tensor, out: Optional[torch.Tensor] = None, stream=N
     return out
 
 
+def descale_strides(t: torch.Tensor, num_seqs: int, heads: int):
+    """(seq_stride, head_stride) in elements of a descale tensor indexed by (sequence, head).
+
+    Accepted shapes (vLLM #63232: per-tensor and per-head scales keep their descale tensors;
+    FA4's descale views are (batch, kv_heads)): one element (per tensor), (heads,) (per head),
+    and (S, Hd) with S in {1, num_seqs}, Hd in {1, heads}; size-1 axes broadcast (stride 0).
+    """
+    if t.dtype != torch.float32:
+        raise ValueError("a descale must be a float32 tensor")
+    if t.numel() == 1:
+        return 0, 0
+    if t.dim() == 1 and t.shape[0] == heads:
+        return 0, t.stride(0)
+    if t.dim() == 2 and t.shape[0] in (1, num_seqs) and t.shape[1] in (1, heads):
+        return (t.stride(0) if t.shape[0] > 1 else 0), (t.stride(1) if t.shape[1] > 1 else 0)
+    raise ValueError("a descale has one element, shape (heads,) or (num_seqs or 1, heads or 1); got %s"
+                     % (tuple(t.shape),))
+
+
 def lpfa_attn_fwd_varlen(q: torch.Tensor, q_sf: torch.Tensor, k: torch.Tensor, k_sf: torch.Tensor,
                          v: torch.Tensor, v_sf: Optional[torch.Tensor], meta_q: VarlenMeta, meta_k: VarlenMeta,
                          pv_mode: str = "bf16", q_descale: Optional[torch.Tensor] = None,
@@ -202,7 +229,10 @@ def lpfa_attn_fwd_varlen(q: torch.Tensor, q_sf: torch.Tensor, k: torch.Tensor, k
                          debug_flags: int = 0):
     """Block-scaled attention forward; returns (out bf16 (Tq,H,128), lse fp32 (H,Tq)).
 
-    debug_flags != 0 goes through lpfa_attn_fwd_varlen_debug (test hook, see include/lpfa.h).
+    q/k/v_descale: None (exactly 1.0), a one-element tensor (per tensor), (H,) (per head) or
+    (S, H) (per sequence and head), float32 on the device; see descale_strides.
+    debug_flags != 0 goes through lpfa_attn_fwd_varlen_debug (test hook, see include/lpfa.h),
+    which takes per-tensor descales only.
     """
     if pv_mode not in PV_MODES:
         raise ValueError("pv_mode must be 'bf16', 'fp8' or 'bf16v'")
@@ -210,10 +240,18 @@ def lpfa_attn_fwd_varlen(q: torch.Tensor, q_sf: torch.Tensor, k: torch.Tensor, k
         want = torch.bfloat16 if (name == "v" and pv_mode == "bf16v") else torch.uint8
         if t.dtype != want or t.dim() != 3 or not t.is_contiguous():
             raise ValueError("%s must be a contiguous %s (tokens, heads, 128) tensor" % (name, want))
-    for name, t in (("q_descale", q_descale), ("k_descale", k_descale), ("v_descale", v_descale)):
-        if t is not None and (t.dtype != torch.float32 or t.numel() != 1):
-            raise ValueError("%s must be a single-element float32 tensor" % name)
     Tq, H = q.shape[0], q.shape[1]
+    descs = []
+    for name, t in (("q_descale", q_descale), ("k_descale", k_descale), ("v_descale", v_descale)):
+        if t is None:
+            descs.append(_Descale(None, 0, 0))
+            continue
+        ss, hs = descale_strides(t, meta_q.num_seqs, H)
+        if debug_flags and (ss or hs):
+            raise ValueError("the debug entry point takes per-tensor descales only")
+        if t.device != q.device:
+            raise ValueError("%s must be on the device of q" % name)
+        descs.append(_Descale(t.data_ptr(), ss, hs))
     if out is None:
         out = torch.empty((Tq, H, 128), dtype=torch.bfloat16, device=q.device)
     if lse is None:
@@ -226,7 +264,8 @@ def lpfa_attn_fwd_varlen(q: torch.Tensor, q_sf: torch.Tensor, k: torch.Tensor, k
         if debug_flags:
             _check(_lib.lpfa_attn_fwd_varlen_debug(*args, debug_flags))
         else:
-            _check(_lib.lpfa_attn_fwd_varlen(*args))
+            _check(_lib.lpfa_attn_fwd_varlen_descaled(*args[:11], ctypes.byref(descs[0]), ctypes.byref(descs[1]),
+                                                      ctypes.byref(descs[2]), *args[14:]))
     return out, lse
 
 

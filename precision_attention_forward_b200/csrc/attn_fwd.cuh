@@ -97,6 +97,21 @@ enum WaitSite : int {
   kSiteConvE, kSiteDrain, kSiteDebugStall, kSiteMmaS, kSiteSoftO, kSiteTmem
 };
 
+// A descale indexed by (sequence, head): ptr[seq * seq_stride + h * head_stride] (vLLM #63232,
+// "Claims": per-head scales keep their descale tensors). A missing descale is read as exactly
+// 1.0 (same page): the host points it at g_lpfa_one with zero strides, so the kernel always
+// loads (no branch on the pointer) and 1.0 takes the same arithmetic path as any other value.
+struct Descale {
+  const float* ptr;
+  int64_t seq_stride, head_stride;
+};
+
+__device__ const float g_lpfa_one = 1.0f;
+
+__device__ __forceinline__ float descale_value(const Descale& d, int seq, int h) {
+  return __ldg(d.ptr + seq * d.seq_stride + h * d.head_stride);
+}
+
 struct AttnParams {
   const uint8_t* q_sf;
   const uint8_t* k_sf;
@@ -105,9 +120,7 @@ struct AttnParams {
   const int32_t* so_q;      // meta_q.dev + n + 1 (scale / tile prefix)
   const int32_t* cu_k;
   const int32_t* so_k;
-  const float* q_descale;   // nullable
-  const float* k_descale;
-  const float* v_descale;
+  Descale q_descale, k_descale, v_descale;
   __nv_bfloat16* out;       // (Tq, H, 128)
   float* lse;               // (H, Tq)
   int num_seqs;
@@ -157,13 +170,13 @@ enum Bar : int {
   kBarVbfFull = 28, kBarVbfEmpty = 30,   // [2]
   kBarSFull = 32,    // S(t) computed                       (MMA commit)
   kBarSFree = 34,    // S(t) read out by its group            (4 warps)
-  kBarPReady = 36,   // P(t) stored, O rescaled if needed     (4 warps)
-  kBarPVDone = 38,   // [t % kPSlots] PV(t) complete           (MMA commit)
-  kBarOFull = 41,    // every PV of the unit complete         (MMA commit)
-  kBarOEmpty = 42,   // O read out by both groups             (8 warps)
-  kBarLReady = 43,   // partial l / reference exchanged       (8 warps)
-  kBarDrain = 44,    // QK issuer's own tcgen05 work done
-  kBarDrainPV = 45,  // PV issuer's own tcgen05 work done
+  kBarPReady = 36,   // [t % kPSlots] P(t) stored, O rescaled if needed (4 warps)
+  kBarPVDone = 39,   // [t % kPSlots] PV(t) complete           (MMA commit)
+  kBarOFull = 42,    // every PV of the unit complete         (MMA commit)
+  kBarOEmpty = 43,   // O read out by both groups             (8 warps)
+  kBarLReady = 44,   // partial l / reference exchanged       (8 warps)
+  kBarDrain = 45,    // QK issuer's own tcgen05 work done
+  kBarDrainPV = 46,  // PV issuer's own tcgen05 work done
   kBarMRef = 48      // [group][lane quarter]: tile reference of t published and the MUFU
                      // handed over to the other group (1 warp; 8 entries)
 };
@@ -463,7 +476,10 @@ template <> struct SoftmaxLag<true> { static constexpr float lag = 2.0f; static 
 template <> struct SoftmaxLag<false> { static constexpr float lag = 8.0f; static constexpr float bias = 0.0f; };
 
 
-template <int kPv>
+// kPerUnitDescale: q/k descales that vary with (sequence, head) are read per unit by the softmax
+// (the QK issuer always reads them per unit). The host takes it only when a q or k descale has a
+// nonzero stride: reading the scale per unit costs the softmax loop several percent.
+template <int kPv, bool kPerUnitDescale>
 __global__ void __launch_bounds__(kAttnThreads, 1)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                 const __grid_constant__ CUtensorMap tmap_v, const AttnParams p) {
@@ -498,9 +514,16 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bars[kBarSFull + i], 1);
       mbar_init(&bars[kBarSFree + i], 4);
-      mbar_init(&bars[kBarPReady + i], 4);
     }
-    for (uint32_t i = 0; i < kPSlots; ++i) mbar_init(&bars[kBarPVDone + i], 1);
+    // PReady and PVDone are indexed by t % kPSlots. PReady counts the 4 warps of a group, which
+    // run independently of each other: a warp's arrival for tile t + 3 on the same barrier
+    // needs PV(t) complete (the P-slot wait), and so every arrival for tile t, which keeps the
+    // phases apart. (One barrier per group would let a fast warp's arrival for t + 2 complete
+    // the phase of t before a slow warp had stored its rows of P(t).)
+    for (uint32_t i = 0; i < kPSlots; ++i) {
+      mbar_init(&bars[kBarPReady + i], 4);
+      mbar_init(&bars[kBarPVDone + i], 1);
+    }
     mbar_init(&bars[kBarOFull], 1);
     mbar_init(&bars[kBarOEmpty], 8);
     mbar_init(&bars[kBarLReady], 8);
@@ -620,9 +643,6 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
       // S(t) = Q K_t^T into S buffer t & 1. The whole warp runs the loop (warp-uniform state);
       // lane 0 issues the tcgen05 instructions.
       const uint32_t leader = lane == 0 ? 1u : 0u;
-      const float qd = p.q_descale ? __ldg(p.q_descale) : 1.0f;
-      const float kd = p.k_descale ? __ldg(p.k_descale) : 1.0f;
-      const int negate = (qd * kd) < 0.0f ? 1 : 0;
       // Descriptor bases; the start-address field is the low 14 bits (address >> 4), so a byte
       // offset b inside shared memory advances a descriptor by b >> 4.
       const uint32_t sb = static_cast<uint32_t>(warp_uniform(static_cast<int>(smem_u32(smem))));
@@ -630,9 +650,6 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
       const uint64_t dk0 = umma_desc(sb + L::k, 16, 1024, kLayoutSw128);
       const uint64_t dqsf0 = umma_desc(sb + L::q_sf, 0, 128, kLayoutNone);
       const uint64_t dksf0 = umma_desc(sb + L::k_sf, 0, 128, kLayoutNone);
-      uint32_t idq[4];
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk) idq[kk] = idesc_qk(kk, negate);
       uint32_t u = 0, kc = 0, t = 0;  // units, K fills, tiles
       bool ok = true;
       if (p.debug_stall > 0) {
@@ -643,6 +660,13 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
       for (int w = blockIdx.x; w < p.num_units && ok; w += G) {
         const UnitInfo ui = warp_uniform(unit_info(p, sched, w));
         if (ui.nkv == 0) continue;
+        // The sign of the logit scale goes into the MMA (negated A); the softmax uses |scale|.
+        const float qd = descale_value(p.q_descale, ui.seq, ui.h);
+        const float kd = descale_value(p.k_descale, ui.seq, ui.h);
+        const int negate = (qd * kd) < 0.0f ? 1 : 0;
+        uint32_t idq[4];
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) idq[kk] = idesc_qk(kk, negate);
         const uint32_t qs = u % kQStages;
         if (!mbar_wait_warp(&bars[kBarQFull + qs], (u / kQStages) & 1, abort_flag)) { record_failure(abort_flag, kSiteMmaQ); ok = false; break; }
         tc_fence_after();
@@ -695,7 +719,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
         if (ui.nkv == 0) continue;
         for (int j = 0; j < ui.nkv; ++j, ++t) {
           const uint32_t b = t & 1;
-          if (!mbar_wait_warp(&bars[kBarPReady + b], (t >> 1) & 1, abort_flag)) { record_failure(abort_flag, kSiteMmaP); ok = false; break; }
+          if (!mbar_wait_warp(&bars[kBarPReady + t % kPSlots], (t / kPSlots) & 1, abort_flag)) { record_failure(abort_flag, kSiteMmaP); ok = false; break; }
           if (j == 0 && !mbar_wait_warp(&bars[kBarOEmpty], (u & 1) ^ 1, abort_flag)) { record_failure(abort_flag, kSiteMmaO); ok = false; break; }
           const bool got = kFp8PV ? mbar_wait_warp(&bars[kBarVFull + vc % kVStages], (vc / kVStages) & 1, abort_flag)
                                   : mbar_wait_warp(&bars[kBarVbfFull + vc % kVbfStages], (vc / kVbfStages) & 1, abort_flag);
@@ -737,12 +761,13 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
     const int quarter = warp & 3;                                // TMEM lane quarter of this warp
     const int row = quarter * 32 + lane;                         // query row within the tile
     const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
-    const float qd = p.q_descale ? __ldg(p.q_descale) : 1.0f;
-    const float kd = p.k_descale ? __ldg(p.k_descale) : 1.0f;
-    const float vd = p.v_descale ? __ldg(p.v_descale) : 1.0f;
-    const float cscale = fabsf((qd * kd) * kLog2eRsqrtD);  // sign folded into the QK MMA
     float* my_mref = mref + grp * 128 + row;
     const float* other_mref = mref + (grp ^ 1) * 128 + row;
+    // |logit scale|; the sign is folded into the QK MMA. With per-tensor q/k descales it is the
+    // same for every unit and is computed once here; kPerUnitDescale reads it per unit.
+    const float cscale_all = kPerUnitDescale ? 0.0f
+                                             : fabsf((descale_value(p.q_descale, 0, 0) *
+                                                      descale_value(p.k_descale, 0, 0)) * kLog2eRsqrtD);
     uint32_t u = 0, t0 = 0;
     bool ok = true;
     for (int w = blockIdx.x; w < p.num_units && ok; w += G) {
@@ -758,6 +783,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
         }
         continue;
       }
+      // (v's descale is read in the epilogue, so that nothing more stays live across the tiles.)
+      const float cscale = kPerUnitDescale ? fabsf((descale_value(p.q_descale, ui.seq, ui.h) *
+                                                    descale_value(p.k_descale, ui.seq, ui.h)) * kLog2eRsqrtD)
+                                           : cscale_all;
       float m_g = -INFINITY;  // reference this group's l is relative to (-inf: no tile yet)
       float l_g = 0.0f;       // this group's sum of p over its tiles (times 2^kBias)
       float lr_g = 0.0f;      // bf16 PV mode: the same sum over the BF16-rounded P
@@ -853,7 +882,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bars[kBarPReady + grp]);
+        if (lane == 0) mbar_arrive(&bars[kBarPReady + t % kPSlots]);
       }
       if (!ok) break;
       t0 += ui.nkv;
@@ -872,6 +901,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
       const float m_f = fmaxf(m_g, m_o);  // the unit's last reference (references never fall)
       const float s_g = exp2_int(m_g - m_f), s_o = exp2_int(m_o - m_f);
       const float ltot = l_g * s_g + l_o * s_o;
+      const float vd = descale_value(p.v_descale, ui.seq, ui.h);
       const float oscale = kFp8PV ? vd / ltot : vd / (lr_g * s_g + lsumr[(grp ^ 1) * 128 + row] * s_o);
       uint32_t ra[32], rb[32];
       tmem_ld64_sync(tmem + lane_addr + kColO + grp * 64, ra, rb);

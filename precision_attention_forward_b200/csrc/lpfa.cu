@@ -318,13 +318,26 @@ static lpfa_status check_attn_kernel(const void* fn, uint32_t smem_bytes) {
   return LPFA_OK;
 }
 
+extern "C++" {
+template <int kPv, bool kPerUnit>
+static lpfa_status launch_attn(int grid, cudaStream_t s, const CUtensorMap& tq, const CUtensorMap& tk,
+                               const CUtensorMap& tv, const lpfa::AttnParams& p) {
+  constexpr uint32_t smem = lpfa::attn_smem_bytes<kPv == lpfa::kPvFp8>();
+  const void* fn = reinterpret_cast<const void*>(lpfa::attn_fwd_kernel<kPv, kPerUnit>);
+  const lpfa_status st = check_attn_kernel(fn, smem);
+  if (st != LPFA_OK) return st;
+  lpfa::attn_fwd_kernel<kPv, kPerUnit><<<grid, lpfa::kAttnThreads, smem, s>>>(tq, tk, tv, p);
+  return LPFA_OK;
+}
+}  // extern "C++"
+
 // Internal entry shared with the test hook: debug_stall > 0 forces a bounded wait to run out.
 static lpfa_status attn_fwd_impl(const uint8_t* q, const uint8_t* q_sf, const uint8_t* k, const uint8_t* k_sf,
                                  const uint8_t* v, const uint8_t* v_sf, const lpfa_varlen_meta* meta_q,
                                  const lpfa_varlen_meta* meta_k, int32_t heads, int32_t head_dim,
-                                 lpfa_pv_mode pv_mode, const float* q_descale, const float* k_descale,
-                                 const float* v_descale, void* out_bf16, float* lse, void* stream,
-                                 int debug_stall) {
+                                 lpfa_pv_mode pv_mode, const lpfa_descale* q_descale,
+                                 const lpfa_descale* k_descale, const lpfa_descale* v_descale, void* out_bf16,
+                                 float* lse, void* stream, int debug_stall) {
   if (!q || !q_sf || !k || !k_sf || !v || !out_bf16 || !lse) return fail(LPFA_ERR_INVALID_ARG, "NULL tensor pointer");
   if (pv_mode != LPFA_PV_BF16 && pv_mode != LPFA_PV_FP8 && pv_mode != LPFA_PV_BF16_V)
     return fail(LPFA_ERR_INVALID_ARG, "invalid pv_mode %d", pv_mode);
@@ -333,6 +346,9 @@ static lpfa_status attn_fwd_impl(const uint8_t* q, const uint8_t* q_sf, const ui
   if (pv_mode == LPFA_PV_BF16 && !v_sf) return fail(LPFA_ERR_INVALID_ARG, "bf16 PV mode needs the V scale factors (v_sf)");
   if (head_dim != 128) return fail(LPFA_ERR_INVALID_ARG, "head_dim must be 128 (got %d)", head_dim);
   if (heads < 1) return fail(LPFA_ERR_INVALID_ARG, "heads must be >= 1");
+  for (const lpfa_descale* d : {q_descale, k_descale, v_descale})
+    if (d && d->ptr && (d->seq_stride < 0 || d->head_stride < 0))
+      return fail(LPFA_ERR_INVALID_ARG, "descale strides must be >= 0");
   lpfa_status st;
   if ((st = check_meta(meta_q, "meta_q")) != LPFA_OK) return st;
   if ((st = check_meta(meta_k, "meta_k")) != LPFA_OK) return st;
@@ -364,9 +380,19 @@ static lpfa_status attn_fwd_impl(const uint8_t* q, const uint8_t* q_sf, const ui
   p.so_q = meta_q->dev + meta_q->num_seqs + 1;
   p.cu_k = meta_k->dev;
   p.so_k = meta_k->dev + meta_k->num_seqs + 1;
-  p.q_descale = q_descale;
-  p.k_descale = k_descale;
-  p.v_descale = v_descale;
+  // A missing descale reads the library's device constant 1.0f with zero strides.
+  void* one_addr = nullptr;
+  cudaError_t e = cudaGetSymbolAddress(&one_addr, lpfa::g_lpfa_one);
+  const float* one = static_cast<const float*>(one_addr);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(g_lpfa_one)");
+  auto descale = [one](const lpfa_descale* d) {
+    lpfa::Descale r{one, 0, 0};
+    if (d && d->ptr) r = lpfa::Descale{d->ptr, d->seq_stride, d->head_stride};
+    return r;
+  };
+  p.q_descale = descale(q_descale);
+  p.k_descale = descale(k_descale);
+  p.v_descale = descale(v_descale);
   p.out = static_cast<__nv_bfloat16*>(out_bf16);
   p.lse = lse;
   p.num_seqs = meta_q->num_seqs;
@@ -378,20 +404,19 @@ static lpfa_status attn_fwd_impl(const uint8_t* q, const uint8_t* q_sf, const ui
 
   const int grid = static_cast<int>(units < info.sms ? units : info.sms);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  cudaError_t e;
+  const bool per_unit = (p.q_descale.seq_stride | p.q_descale.head_stride | p.k_descale.seq_stride |
+                         p.k_descale.head_stride) != 0;
   if (pv_mode == LPFA_PV_FP8) {
-    constexpr int kPv = lpfa::kPvFp8;
-    if ((st = check_attn_kernel(reinterpret_cast<const void*>(lpfa::attn_fwd_kernel<kPv>), lpfa::attn_smem_bytes<true>())) != LPFA_OK) return st;
-    lpfa::attn_fwd_kernel<kPv><<<grid, lpfa::kAttnThreads, lpfa::attn_smem_bytes<true>(), s>>>(tq, tk, tv, p);
+    st = per_unit ? launch_attn<lpfa::kPvFp8, true>(grid, s, tq, tk, tv, p)
+                  : launch_attn<lpfa::kPvFp8, false>(grid, s, tq, tk, tv, p);
   } else if (pv_mode == LPFA_PV_BF16) {
-    constexpr int kPv = lpfa::kPvBf16Mx;
-    if ((st = check_attn_kernel(reinterpret_cast<const void*>(lpfa::attn_fwd_kernel<kPv>), lpfa::attn_smem_bytes<false>())) != LPFA_OK) return st;
-    lpfa::attn_fwd_kernel<kPv><<<grid, lpfa::kAttnThreads, lpfa::attn_smem_bytes<false>(), s>>>(tq, tk, tv, p);
+    st = per_unit ? launch_attn<lpfa::kPvBf16Mx, true>(grid, s, tq, tk, tv, p)
+                  : launch_attn<lpfa::kPvBf16Mx, false>(grid, s, tq, tk, tv, p);
   } else {
-    constexpr int kPv = lpfa::kPvBf16In;
-    if ((st = check_attn_kernel(reinterpret_cast<const void*>(lpfa::attn_fwd_kernel<kPv>), lpfa::attn_smem_bytes<false>())) != LPFA_OK) return st;
-    lpfa::attn_fwd_kernel<kPv><<<grid, lpfa::kAttnThreads, lpfa::attn_smem_bytes<false>(), s>>>(tq, tk, tv, p);
+    st = per_unit ? launch_attn<lpfa::kPvBf16In, true>(grid, s, tq, tk, tv, p)
+                  : launch_attn<lpfa::kPvBf16In, false>(grid, s, tq, tk, tv, p);
   }
+  if (st != LPFA_OK) return st;
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "attention launch");
   return LPFA_OK;
@@ -402,6 +427,18 @@ lpfa_status lpfa_attn_fwd_varlen(const uint8_t* q, const uint8_t* q_sf, const ui
                                  const lpfa_varlen_meta* meta_k, int32_t heads, int32_t head_dim,
                                  lpfa_pv_mode pv_mode, const float* q_descale, const float* k_descale,
                                  const float* v_descale, void* out_bf16, float* lse, void* stream) {
+  const lpfa_descale qd{q_descale, 0, 0}, kd{k_descale, 0, 0}, vd{v_descale, 0, 0};
+  return attn_fwd_impl(q, q_sf, k, k_sf, v, v_sf, meta_q, meta_k, heads, head_dim, pv_mode, &qd, &kd, &vd,
+                       out_bf16, lse, stream, 0);
+}
+
+lpfa_status lpfa_attn_fwd_varlen_descaled(const uint8_t* q, const uint8_t* q_sf, const uint8_t* k,
+                                          const uint8_t* k_sf, const uint8_t* v, const uint8_t* v_sf,
+                                          const lpfa_varlen_meta* meta_q, const lpfa_varlen_meta* meta_k,
+                                          int32_t heads, int32_t head_dim, lpfa_pv_mode pv_mode,
+                                          const lpfa_descale* q_descale, const lpfa_descale* k_descale,
+                                          const lpfa_descale* v_descale, void* out_bf16, float* lse,
+                                          void* stream) {
   return attn_fwd_impl(q, q_sf, k, k_sf, v, v_sf, meta_q, meta_k, heads, head_dim, pv_mode, q_descale, k_descale,
                        v_descale, out_bf16, lse, stream, 0);
 }
@@ -413,8 +450,9 @@ lpfa_status lpfa_attn_fwd_varlen_debug(const uint8_t* q, const uint8_t* q_sf, co
                                        const float* v_descale, void* out_bf16, float* lse, void* stream,
                                        int32_t debug_flags) {
   if (debug_flags & ~1) return fail(LPFA_ERR_INVALID_ARG, "unknown debug flags 0x%x", debug_flags);
-  return attn_fwd_impl(q, q_sf, k, k_sf, v, v_sf, meta_q, meta_k, heads, head_dim, pv_mode, q_descale, k_descale,
-                       v_descale, out_bf16, lse, stream, debug_flags & 1);
+  const lpfa_descale qd{q_descale, 0, 0}, kd{k_descale, 0, 0}, vd{v_descale, 0, 0};
+  return attn_fwd_impl(q, q_sf, k, k_sf, v, v_sf, meta_q, meta_k, heads, head_dim, pv_mode, &qd, &kd, &vd,
+                       out_bf16, lse, stream, debug_flags & 1);
 }
 
 lpfa_status lpfa_device_status(void* stream, int32_t* detail) {

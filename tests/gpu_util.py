@@ -38,10 +38,10 @@ def compare_attention(o_gpu: torch.Tensor, lse_gpu: torch.Tensor, o_ref: np.ndar
     """Return (max_abs_O, rel_l2_O, max_abs_LSE) of the GPU result against the oracle.
 
     o_scale (broadcastable to O): the input scale of V's (head, channel) pairs where a workload
-    plants deliberate outliers. The max-abs bound is stated for unit-scale data, so the O error
-    of each channel is divided by that channel's scale before the maximum is taken (O in a
-    channel scaled x64 is x64 larger, and so are its BF16 rounding and every other error).
-    rel-L2 and LSE are unaffected.
+    plants deliberate outliers, or the magnitude of a per-head v descale. The max-abs bound is
+    stated for unit-scale data, so the O error of each channel is divided by that channel's
+    scale before the maximum is taken (O in a channel scaled x64 is x64 larger, and so are its
+    BF16 rounding and every other error). rel-L2 and LSE are unaffected.
     """
     o = o_gpu.float().cpu().numpy().astype(np.float64)
     l = lse_gpu.float().cpu().numpy().astype(np.float64)
@@ -60,6 +60,15 @@ def assert_within(stats, label=""):
     return msg
 
 
+def _descale_tensor(x):
+    """None, a float (one-element tensor), a numpy array (same shape) or a torch tensor (as is)."""
+    if x is None or isinstance(x, torch.Tensor):
+        return x
+    if np.ndim(x) == 0:
+        return torch.tensor([float(x)], dtype=torch.float32, device="cuda")
+    return torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).to("cuda")
+
+
 def run_path(lp, q, k, v, lens_q, lens_k, heads, in_dtype="bf16", pv_mode="bf16", mode="rceil",
              descales=(None, None, None)):
     """Library path: metadata, quantize Q/K (and V in bf16 PV mode) or cast V, attention."""
@@ -73,7 +82,7 @@ def run_path(lp, q, k, v, lens_q, lens_k, heads, in_dtype="bf16", pv_mode="bf16"
         vp, vs = to_device(v, "bf16"), None          # BF16 V input, never quantized
     else:
         vp, vs = gpu_quantize(lp, v, in_dtype, mk, mode)
-    dd = [None if x is None else torch.tensor([x], dtype=torch.float32, device="cuda") for x in descales]
+    dd = [_descale_tensor(x) for x in descales]
     o, lse = lp.lpfa_attn_fwd_varlen(qp, qs, kp, ks, vp, vs, mq, mk, pv_mode=pv_mode,
                                      q_descale=dd[0], k_descale=dd[1], v_descale=dd[2])
     torch.cuda.synchronize()

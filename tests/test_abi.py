@@ -8,6 +8,7 @@ import re
 
 import numpy as np
 import pytest
+import torch
 
 import precision_attention_forward_b200 as lp
 from oracle import meta as ometa
@@ -114,3 +115,39 @@ def test_cast_argument_validation():
     assert f(FAKE, 2048, 128, 10, 16, 100, FAKE, None) == lp.LPFA_ERR_INVALID_ARG
     assert f(FAKE, 2048, 128, 0, 16, 128, FAKE, None) == lp.LPFA_ERR_INVALID_ARG
     assert f(FAKE + 2, 2048, 128, 10, 16, 128, FAKE, None) == lp.LPFA_ERR_INVALID_ARG
+
+
+def test_descaled_entry_rejects_negative_strides():
+    good = lp._Descale(FAKE, 0, 1)
+    bad = lp._Descale(FAKE, -1, 0)
+    for descs in ((bad, None, None), (None, None, bad)):
+        ptrs = [ctypes.byref(d) if d is not None else None for d in descs]
+        st = lp._lib.lpfa_attn_fwd_varlen_descaled(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+                                                   ctypes.byref(_fake_meta(2, 300)), ctypes.byref(_fake_meta(2, 300)),
+                                                   4, 128, 0, *ptrs, FAKE, FAKE, None)
+        assert st == lp.LPFA_ERR_INVALID_ARG
+        assert "stride" in lp._lib.lpfa_last_error_message().decode()
+    # a valid descriptor passes descale validation and fails later (head_dim), not on the strides
+    st = lp._lib.lpfa_attn_fwd_varlen_descaled(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+                                               ctypes.byref(_fake_meta(2, 300)), ctypes.byref(_fake_meta(2, 300)),
+                                               4, 64, 0, ctypes.byref(good), None, None, FAKE, FAKE, None)
+    assert st == lp.LPFA_ERR_INVALID_ARG and "head_dim" in lp._lib.lpfa_last_error_message().decode()
+
+
+@pytest.mark.parametrize("shape,want", [
+    ((1,), (0, 0)), ((), (0, 0)), ((1, 1), (0, 0)), ((4,), (0, 1)), ((1, 4), (0, 1)),
+    ((3, 4), (4, 1)), ((3, 1), (1, 0)),
+])
+def test_descale_strides_shapes(shape, want):
+    t = torch.ones(shape, dtype=torch.float32)
+    assert lp.descale_strides(t, 3, 4) == want
+
+
+def test_descale_strides_views_and_rejects():
+    base = torch.arange(12, dtype=torch.float32).reshape(4, 3)
+    assert lp.descale_strides(base.t(), 3, 4) == (1, 3)            # transposed (S, H) view
+    assert lp.descale_strides(torch.ones(1).expand(3, 4), 3, 4) == (0, 0)
+    assert lp.descale_strides(torch.ones(4).expand(3, 4), 3, 4) == (0, 1)
+    for bad in (torch.ones(5), torch.ones(2, 4), torch.ones(3, 4, dtype=torch.float64), torch.ones(3, 4, 1)):
+        with pytest.raises(ValueError):
+            lp.descale_strides(bad, 3, 4)

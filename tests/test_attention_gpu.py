@@ -139,6 +139,59 @@ def test_descale_values_match_oracle(descales):
     gu.assert_within(gu.compare_attention(o, lse, o_ref, lse_ref), f"descales {descales}")
 
 
+@pytest.mark.parametrize("pv_mode", ["bf16", "fp8", "bf16v"])
+def test_per_head_and_per_sequence_descales_match_oracle(pv_mode):
+    """vLLM #63232 'Claims': per-head scales keep their descale tensors. q (H,), k (S, H) and
+    v (1, H) descales, with negative and non-power-of-two values, against the oracle."""
+    # At least 64 keys per sequence: with a handful of keys, one E4M3 rounding decision of P that
+    # falls differently in fp32 and fp64 moves O by more than the bound in fp8 PV mode, whatever
+    # the descales (the few-key cases are covered without descales elsewhere).
+    lq, lk, H = [300, 77, 129], [129, 700, 64], 3
+    q, k, v = wl.small_random(31, lq, lk, H)
+    if pv_mode == "fp8":
+        v = v * np.float32(2)
+    qd = np.array([0.5, -1.25, 2.0])
+    kd = np.array([[1.0, 0.75, 3.0], [2.0, 1.0, -0.5], [0.25, 1.5, 1.0]])
+    vd = np.array([[1.0, -2.0, 0.5]])
+    o, lse = gu.run_path(lp, q, k, v, lq, lk, H, pv_mode=pv_mode, descales=(qd, kd, vd))
+    o_ref, lse_ref = gu.oracle_full(q, k, v, lq, lk, H, pv_mode=pv_mode, descales=(qd, kd, vd))
+    # The O bound is stated at unit output scale: a v descale multiplies O, and with it every
+    # rounding error, exactly, so each head's O error is divided by |v descale| of that head.
+    o_scale = np.abs(vd).reshape(1, H, 1)
+    gu.assert_within(gu.compare_attention(o, lse, o_ref, lse_ref, o_scale=o_scale), f"per-head descales {pv_mode}")
+    _status_ok()
+
+
+@pytest.mark.parametrize("pv_mode", ["bf16", "fp8"])
+def test_per_head_unit_descales_bit_identical_and_one_head_changes(pv_mode):
+    """All-ones per-head descales == no descale bit for bit (vLLM #63232 'Validation'); a 2 on one
+    head changes that head only; an expanded per-tensor view equals the per-tensor value."""
+    lq = lk = [400, 200]
+    H = 4
+    q, k, v = wl.small_random(37, lq, lk, H)
+    if pv_mode == "fp8":
+        v = v * np.float32(2)
+    o0, l0 = gu.run_path(lp, q, k, v, lq, lk, H, pv_mode=pv_mode)
+    ones = np.ones(H)
+    o1, l1 = gu.run_path(lp, q, k, v, lq, lk, H, pv_mode=pv_mode, descales=(ones, ones.reshape(1, H), ones))
+    assert torch.equal(o0.view(torch.int16), o1.view(torch.int16))
+    assert torch.equal(l0.view(torch.int32), l1.view(torch.int32))
+    two_on_2 = np.array([1.0, 1.0, 2.0, 1.0])
+    o2, l2 = gu.run_path(lp, q, k, v, lq, lk, H, pv_mode=pv_mode, descales=(two_on_2, None, None))
+    for h in range(H):
+        same_o = torch.equal(o0[:, h].view(torch.int16), o2[:, h].view(torch.int16))
+        same_l = torch.equal(l0[h].view(torch.int32), l2[h].view(torch.int32))
+        assert (same_o and same_l) == (h != 2), h
+    # a per-tensor 2.0 given as a stride-0 (S, H) view equals the one-element tensor
+    d1 = torch.tensor([2.0], dtype=torch.float32, device="cuda")
+    o3, l3 = gu.run_path(lp, q, k, v, lq, lk, H, pv_mode=pv_mode, descales=(d1, None, d1))
+    o4, l4 = gu.run_path(lp, q, k, v, lq, lk, H, pv_mode=pv_mode, descales=(d1.view(1, 1).expand(2, H), None,
+                                                                          d1.expand(H)))
+    assert torch.equal(o3.view(torch.int16), o4.view(torch.int16))
+    assert torch.equal(l3.view(torch.int32), l4.view(torch.int32))
+    _status_ok()
+
+
 def test_negative_control_wrong_k_scales_fail():
     """Scale bytes of K raised by one (K doubled) must fail the tolerance."""
     lq = lk = [512]
