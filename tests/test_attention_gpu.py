@@ -192,6 +192,37 @@ def test_per_head_unit_descales_bit_identical_and_one_head_changes(pv_mode):
     _status_ok()
 
 
+@pytest.mark.parametrize("pv_mode", ["fp8", "bf16", "bf16v"])
+def test_repeated_runs_are_bit_identical(pv_mode):
+    """The kernel's result does not depend on timing: repeated calls on the same inputs give the
+    same bits (a barrier phase completed by the wrong warps once made fp8 PV rows differ)."""
+    w = wl.WORKLOADS["dense_4x2048_h16"]
+    lq, lk = wl.lengths(w)
+    q, k, v = (wl.make_tensor(w, x) for x in "qkv")
+    if pv_mode == "fp8":
+        v = v * np.float32(2.0)
+    mq = lp.lpfa_varlen_meta_from_lengths(lq)
+    mk = lp.lpfa_varlen_meta_from_lengths(lk)
+    qp, qs = gu.gpu_quantize(lp, q, "bf16", mq)
+    kp, ks = gu.gpu_quantize(lp, k, "bf16", mk)
+    if pv_mode == "fp8":
+        vp, vs = lp.lpfa_cast_e4m3(gu.to_device(v, "bf16")), None
+    elif pv_mode == "bf16v":
+        vp, vs = gu.to_device(v, "bf16"), None
+    else:
+        vp, vs = gu.gpu_quantize(lp, v, "bf16", mk)
+    ref = None
+    for _ in range(4):
+        o, lse = lp.lpfa_attn_fwd_varlen(qp, qs, kp, ks, vp, vs, mq, mk, pv_mode=pv_mode)
+        torch.cuda.synchronize()
+        if ref is None:
+            ref = (o.clone(), lse.clone())
+            continue
+        assert torch.equal(o.view(torch.int16), ref[0].view(torch.int16))
+        assert torch.equal(lse.view(torch.int32), ref[1].view(torch.int32))
+    _status_ok()
+
+
 def test_negative_control_wrong_k_scales_fail():
     """Scale bytes of K raised by one (K doubled) must fail the tolerance."""
     lq = lk = [512]
