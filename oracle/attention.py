@@ -30,6 +30,19 @@ and LSE as in the plain definition. Because E4M3 rounding commutes with exact
 power-of-two scaling outside the subnormal range, any schedule whose running
 maximum is an integer in log2 units reproduces these weights.
 
+Block-scaled MXFP8 PV variant (``p_mode="mxfp8"``; the block-scaled PV of LP-FA4, where P
+and V are both MXFP8 with their 32-element blocks along the keys). Reading: P is quantized
+exactly as the quantizer would quantize it, relative to any power-of-two reference:
+
+    u_j  = 2^(t_j - m*),  32-key groups aligned to the sequence's first key,
+    e_g  = RCEIL exponent of max_{j in g} u_j,
+    w~_j = E4M3(u_j * 2^-e_g) * 2^e_g,
+    O_r  = (sum_j w~_j v_j) / (sum_j u_j) * vd,
+
+with V the token-orientation dequantized values; the LSE as in the plain definition. The
+E8M0 scale absorbs the power of two, so the weights do not depend on m* or on a kernel's
+tile schedule (outside the clamp of e to [-127, 127]).
+
 Parity: the plain definition is pinned by closed forms (constant V, a single
 key, equal logits), by a brute-force pure-Python softmax on tiny inputs, by
 scipy's logsumexp, and by invariances (key permutation, packing vs separate
@@ -72,6 +85,18 @@ def descale_at(d, seq: int, head: int) -> float:
     raise ValueError("a descale is a scalar, (H,) or (S, H)")
 
 
+def _mx_weights(t: np.ndarray):
+    """Block-scaled MXFP8 P per row (see the module docstring): (w~, u), both relative to 2^m*."""
+    mstar = np.ceil(t.max(axis=-1, keepdims=True))
+    u = np.exp2(t - mstar)
+    R, N = u.shape
+    pad = (-N) % _mx.BLOCK
+    up = np.concatenate([u, np.zeros((R, pad))], axis=1).reshape(R, -1, _mx.BLOCK)
+    e = _mx.e8m0_exponent(up.max(axis=2), "rceil")                 # (R, groups)
+    w = _mx.e4m3_decode(_mx.e4m3_encode(up * np.ldexp(1.0, -e)[..., None])) * np.ldexp(1.0, e)[..., None]
+    return w.reshape(R, -1)[:, :N], u
+
+
 def attend_block(q, k, v, qd=1.0, kd=1.0, vd=1.0, p_mode: str = "exact"):
     """Attention of query rows q (R,128) over keys k, v (N,128); returns (O (R,128), LSE (R,))."""
     q = np.asarray(q, dtype=np.float64)
@@ -87,8 +112,11 @@ def attend_block(q, k, v, qd=1.0, kd=1.0, vd=1.0, p_mode: str = "exact"):
     elif p_mode == "fp8":
         wq, u = _fp8_weights(s * LOG2E)
         o = (wq @ v) / u.sum(axis=1)[:, None] * float(vd)
+    elif p_mode == "mxfp8":
+        wq, u = _mx_weights(s * LOG2E)
+        o = (wq @ v) / u.sum(axis=1)[:, None] * float(vd)
     else:
-        raise ValueError("p_mode must be 'exact' or 'fp8'")
+        raise ValueError("p_mode must be 'exact', 'fp8' or 'mxfp8'")
     return o, lse
 
 

@@ -20,17 +20,21 @@ Readings taken where the pages are silent (each is listed in the design doc):
   values in (448, 512) saturate to 448.
 * amax = 0: e = -127 (byte 0x00) and the payload is +-0.
 * Payload = E4M3(x * 2^-e), one rounding from the exact product.
-* Scale storage: for sequence i, 128-token block b, head h, the 512-byte atom at
+* Scale storage (head_dim orientation): for sequence i, 128-token block b, head h, the 512-byte atom at
   ``((scale_off[i] + b) * H + h) * 512``; inside it the 4 scales of token row r
   (0 <= r < 128) sit at ``(r % 32) * 16 + (r // 32) * 4 + kb``, kb = 0..3 the
   32-element block index along head_dim. Rows past the sequence end hold 0x7F
   (scale 1.0). This is the 32 x 4 x 4 atom the block-scaled tensor-core MMA
   reads its scale factors in.
 
+The token orientation (``quantize_mxfp8_varlen_tokens``) puts the 32-element blocks along
+the token axis instead (see its docstring).
+
 Parity: the codecs are pinned by exhaustive checks against brute-force nearest
 search over all 256 codes and by hand-picked values; the scale rules by
 brute-force search over all exponents; the quantizer by its round trip and by
-the invariance of the payload under power-of-two rescaling of the input.
+the invariance of the payload under power-of-two rescaling of the input; the token
+orientation by its identity with the head_dim orientation of the transposed 128 x 128 blocks.
 """
 from __future__ import annotations
 
@@ -169,6 +173,63 @@ def dequantize_mxfp8(payload, scales, lengths, heads: int) -> np.ndarray:
     e = scale_exponents(scales, lengths, heads)            # (T, H, 4)
     vals = e4m3_decode(payload).reshape(T, heads, 4, BLOCK)
     return (vals * np.ldexp(1.0, e)[..., None]).reshape(T, heads, HEAD_DIM)
+
+
+def quantize_mxfp8_varlen_tokens(x, lengths, mode: str = "rceil"):
+    """Token orientation: one E8M0 scale per 32 consecutive tokens of one (head, channel).
+
+    LP-FA4 README ("MXFP8 forward and backward"): Q, K and V keep both hardware orientations
+    needed across forward and backward; this is the second one, with the 32-element blocks along
+    the token axis, as the PV product (K = keys) and the backward's transposed products read
+    them. Readings: the 32-token groups are aligned to the start of each sequence,
+    4 per 128-token block; a group's amax is taken over the tokens the sequence has (a partial
+    last group is not padded with data); a group with no token of the sequence holds 0x7F.
+    Scale storage: the 512-byte atom of (sequence i, 128-token block b, head h) at
+    ``((scale_off[i] + b) * H + h) * 512`` as in the head_dim orientation, with channel n and
+    token group g at ``(n % 32) * 16 + (n // 32) * 4 + g``.
+    Returns (payload u8 (T, H, 128), scales u8 (blocks * H * 512,)).
+    """
+    x = np.asarray(x, dtype=np.float64)
+    T, H, D = x.shape
+    if D != HEAD_DIM:
+        raise ValueError("head_dim must be 128")
+    m = _meta.from_lengths(lengths)
+    if m.total_tokens != T:
+        raise ValueError("tensor token count does not match the lengths")
+    payload = np.empty((T, H, D), dtype=np.uint8)
+    scales = np.full(m.total_scale_blocks * H * ATOM_BYTES, 0x7F, dtype=np.uint8)
+    chan = np.arange(HEAD_DIM)
+    for i in range(m.num_seqs):
+        c0, n = int(m.cu_seqlens[i]), int(m.lengths[i])
+        for g0 in range(0, n, BLOCK):
+            g1 = min(n, g0 + BLOCK)
+            blk = x[c0 + g0:c0 + g1]                          # (tokens in group, H, 128)
+            e = e8m0_exponent(np.abs(blk).max(axis=0), mode)  # (H, 128)
+            payload[c0 + g0:c0 + g1] = e4m3_encode(blk * np.ldexp(1.0, -e)[None])
+            b, g = g0 // 128, (g0 % 128) // BLOCK
+            for h in range(H):
+                base = ((m.scale_off[i] + b) * H + h) * ATOM_BYTES
+                scales[base + (chan % 32) * 16 + (chan // 32) * 4 + g] = (e[h] + 127).astype(np.uint8)
+    return payload, scales
+
+
+def dequantize_mxfp8_tokens(payload, scales, lengths, heads: int) -> np.ndarray:
+    """x_hat of the token orientation: E4M3 value * 2^(byte - 127) of its (token group, channel)."""
+    payload = np.asarray(payload, dtype=np.uint8)
+    scales = np.asarray(scales, dtype=np.uint8)
+    m = _meta.from_lengths(lengths)
+    out = np.empty(payload.shape, dtype=np.float64)
+    chan = np.arange(HEAD_DIM)
+    for i in range(m.num_seqs):
+        c0, n = int(m.cu_seqlens[i]), int(m.lengths[i])
+        for tok in range(0, n, BLOCK):
+            t1 = min(n, tok + BLOCK)
+            b, g = tok // 128, (tok % 128) // BLOCK
+            for h in range(heads):
+                base = ((m.scale_off[i] + b) * heads + h) * ATOM_BYTES
+                e = scales[base + (chan % 32) * 16 + (chan // 32) * 4 + g].astype(np.int64) - 127
+                out[c0 + tok:c0 + t1, h] = e4m3_decode(payload[c0 + tok:c0 + t1, h]) * np.ldexp(1.0, e)[None]
+    return out
 
 
 def cast_e4m3(v) -> np.ndarray:

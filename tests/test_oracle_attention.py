@@ -262,3 +262,66 @@ def test_attention_rows_matches_full():
     for i, (r, h) in enumerate(zip(rows, heads)):
         assert np.allclose(orow[i], o[r, h], atol=1e-12)
         assert np.isclose(lrow[i], lse[h, r], atol=1e-12)
+
+
+def test_mxfp8_variant_equals_plain_when_weights_exact():
+    """Weights that are powers of two within one E4M3 scale range of their group maximum are exact
+    MXFP8 values: the block-scaled variant equals the plain definition."""
+    g = np.random.default_rng(41)
+    n = 70
+    ints = g.integers(-14, 1, size=n).astype(np.float64)
+    ints[[3, 40, 66]] = 0.0                                      # every 32-key group holds a 2^0
+    q = np.zeros((1, 128)); q[0, 0] = 1.0
+    k = np.zeros((n, 128)); k[:, 0] = ints * math.log(2.0) * math.sqrt(128.0)
+    v = g.standard_normal((n, 128))
+    o_plain, l_plain = oatt.attend_block(q, k, v, p_mode="exact")
+    o_mx, l_mx = oatt.attend_block(q, k, v, p_mode="mxfp8")
+    assert np.allclose(o_plain, o_mx, atol=1e-12) and np.allclose(l_plain, l_mx, atol=1e-12)
+
+
+def test_mxfp8_variant_shift_invariance_and_brute_force():
+    g = np.random.default_rng(42)
+    q, k, v = g.standard_normal((3, 128)), g.standard_normal((75, 128)) * 2, g.standard_normal((75, 128))
+    o1, _ = oatt.attend_block(q, k, v, p_mode="mxfp8")
+    qs = np.concatenate([q[:, :127], np.full((3, 1), 1.0)], axis=1)
+    ks = np.concatenate([k[:, :127], np.full((75, 1), 5 * math.log(2) * math.sqrt(128.0))], axis=1)
+    ks0 = np.concatenate([k[:, :127], np.zeros((75, 1))], axis=1)
+    oa, _ = oatt.attend_block(qs, ks0, v, p_mode="mxfp8")
+    ob, _ = oatt.attend_block(qs, ks, v, p_mode="mxfp8")
+    assert np.allclose(oa, ob, atol=1e-12)
+    # brute force: per 32-key group, the smallest e with max u <= 448 * 2^e by search, and
+    # nearest-value rounding (ties to even code) of u * 2^-e over the E4M3 table
+    vals = omx.e4m3_decode_table()
+    finite = [(c, vals[c]) for c in range(0x7F)]
+    for r in range(3):
+        t = [(q[r] @ k[j]) / math.sqrt(128) / math.log(2) for j in range(75)]
+        ms = math.ceil(max(t))
+        u = [2.0 ** (tj - ms) for tj in t]
+        num = np.zeros(128)
+        for g0 in range(0, 75, 32):
+            grp = range(g0, min(75, g0 + 32))
+            amax = max(u[j] for j in grp)
+            e = next(e for e in range(-140, 20) if amax <= 448.0 * 2.0 ** e)
+            for j in grp:
+                best = min(finite, key=lambda cv: (abs(cv[1] - u[j] * 2.0 ** -e), cv[0] % 2))
+                num += best[1] * 2.0 ** e * v[j]
+        assert np.allclose(o1[r], num / sum(u), atol=1e-12)
+
+
+def test_mxfp8_variant_differs_from_fp8_and_plain():
+    """Where a 32-key group's weights are far below the row maximum, the per-group scale keeps
+    their precision, while the fp8 variant's single power-of-two reference leaves them in the
+    E4M3 subnormal range: one key at t = -15.3 is 256 * 2^-15.3 = 3.25 * 2^-9 there (rounded to
+    3 * 2^-9, -7.7 %), but 1.625 * 2^-16 (exact to 0.03 %) under its own group scale."""
+    t = np.full(64, -40.0)
+    t[0] = 0.0                                          # group 0: the row maximum
+    t[40] = -15.3                                       # group 1: a single small weight
+    q = np.zeros((1, 128)); q[0, 0] = 1.0
+    k = np.zeros((64, 128)); k[:, 0] = t * math.log(2.0) * math.sqrt(128.0)
+    v = np.zeros((64, 128)); v[40, 1] = 1.0             # channel 1 sees key 40 only
+    o_e, _ = oatt.attend_block(q, k, v, p_mode="exact")
+    o_f, _ = oatt.attend_block(q, k, v, p_mode="fp8")
+    o_m, _ = oatt.attend_block(q, k, v, p_mode="mxfp8")
+    err_m = abs(o_m[0, 1] - o_e[0, 1]) / o_e[0, 1]
+    err_f = abs(o_f[0, 1] - o_e[0, 1]) / o_e[0, 1]
+    assert err_m < 2 ** -10 and 0.07 < err_f < 0.08, (err_m, err_f)

@@ -231,3 +231,51 @@ def test_cast_e4m3_matches_torch():
 def test_negative_tiny_keeps_sign():
     x = np.array([-1e-6, -0.0, 1e-6, -2.0 ** -11])
     assert omx.e4m3_encode(x).tolist() == [0x80, 0x80, 0x00, 0x80]
+
+
+def test_token_orientation_is_head_dim_orientation_of_the_transpose():
+    """Token-orientation quantization of a 128-token block equals the head_dim-orientation row
+    quantization of its transpose (channels as rows, tokens as the 128 elements), for every
+    32-token group that holds tokens; partial last blocks pad the transpose with zeros, which
+    leaves the group maxima alone."""
+    g = np.random.default_rng(40)
+    lens, H = [300, 37, 128], 2
+    x = (g.standard_normal((sum(lens), H, 128)) * np.exp2(g.integers(-6, 7, size=(1, H, 128)))).astype(np.float32)
+    p, s = omx.quantize_mxfp8_varlen_tokens(x, lens)
+    m = ometa.from_lengths(lens)
+    for i in range(m.num_seqs):
+        c0, n = int(m.cu_seqlens[i]), int(m.lengths[i])
+        for b in range(0, n, 128):
+            nb = min(128, n - b)
+            for h in range(H):
+                blk = np.zeros((128, 128))
+                blk[:, :nb] = x[c0 + b:c0 + b + nb, h].astype(np.float64).T   # (channel, token)
+                rp, re = omx.quantize_rows(blk)
+                assert np.array_equal(p[c0 + b:c0 + b + nb, h], rp[:, :nb].T)
+                base = ((m.scale_off[i] + b // 128) * H + h) * 512
+                for grp in range(4):
+                    for c in range(128):
+                        byte = s[base + (c % 32) * 16 + (c // 32) * 4 + grp]
+                        if grp * 32 < nb:
+                            assert byte == re[c, grp] + 127
+                        else:
+                            assert byte == 0x7F          # group with no token of the sequence
+
+
+def test_token_orientation_layout_by_hand():
+    """One channel with a known per-token magnitude: its group scales sit at the stated bytes."""
+    lens, H = [70], 1
+    x = np.zeros((70, 1, 128), dtype=np.float32)
+    x[:, 0, 5] = np.arange(1, 71, dtype=np.float32)            # channel 5: token t holds t + 1
+    x[:, 0, 100] = -3.0                                          # channel 100: constant
+    p, s = omx.quantize_mxfp8_varlen_tokens(x, lens)
+    # channel 5: group maxima 32, 64, 70 -> RCEIL e = -3, -2, -2 (448 * 2^-3 = 56 >= 32 ...)
+    for grp, want in ((0, omx.e8m0_exponent(32.0)), (1, omx.e8m0_exponent(64.0)), (2, omx.e8m0_exponent(70.0))):
+        assert s[(5 % 32) * 16 + (5 // 32) * 4 + grp] == int(want) + 127
+    assert s[(5 % 32) * 16 + (5 // 32) * 4 + 3] == 0x7F          # tokens 96..127 do not exist
+    assert s[(100 % 32) * 16 + (100 // 32) * 4 + 0] == int(omx.e8m0_exponent(3.0)) + 127
+    assert s[(0 % 32) * 16 + 0] == 0x00                          # an all-zero channel: amax 0
+    xh = omx.dequantize_mxfp8_tokens(p, s, lens, H)
+    assert np.array_equal(xh[:, 0, 100], np.full(70, -3.0))
+    assert np.array_equal(xh[:, 0, 5], np.arange(1, 71, dtype=np.float64) * 0 + xh[:, 0, 5])
+    assert np.all(np.abs(xh[:, 0, 5] - np.arange(1, 71)) <= np.arange(1, 71) / 16)
