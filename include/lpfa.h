@@ -125,6 +125,27 @@ LPFA_API lpfa_status lpfa_quantize_mxfp8_varlen(const void* x, lpfa_in_dtype dt,
                                        uint8_t* payload, uint8_t* scales, void* stream);
 
 /*
+ * The second hardware orientation of quantize_mxfp8_varlen (LP-FA4 README, "MXFP8 forward and
+ * backward": Q, K and V retain both hardware orientations needed across forward and backward):
+ * one E8M0 scale per 32 consecutive tokens of one (head, channel), groups aligned to the start
+ * of each sequence (4 per 128-token block). Arguments, alignment, errors and the scale rules
+ * are those of lpfa_quantize_mxfp8_varlen; only the blocking and the atom layout differ:
+ *
+ * payload    (T, H, 128) E4M3 codes, E4M3(x * 2^-e) with e the scale of the element's
+ *            (32-token group, channel).
+ * scales     the same storage size (lpfa_scale_bytes); the atom of (sequence i, 128-token
+ *            block b, head h) at ((scale_off[i] + b) * H + h) * 512 holds the scale of channel
+ *            n, token group g at byte (n % 32) * 16 + (n / 32) * 4 + g. A partial last group
+ *            takes its maximum over the tokens it has; a group with no token holds 0x7F.
+ *
+ * This is V's layout for LPFA_PV_MXFP8 (the PV product's K dimension is the keys).
+ */
+LPFA_API lpfa_status lpfa_quantize_mxfp8_varlen_tokens(const void* x, lpfa_in_dtype dt, int64_t tok_stride,
+                                              int64_t head_stride, int32_t heads, int32_t head_dim,
+                                              const lpfa_varlen_meta* meta, lpfa_scaling_mode mode,
+                                              uint8_t* payload, uint8_t* scales, void* stream);
+
+/*
  * fa4_v_to_fp8 (FastVideo #1654: the fp8 PV mode feeds V as an unscaled E4M3 cast, with no
  * scale factors and an implicit dequant scale of 1.0).
  *

@@ -38,7 +38,7 @@ EXPORTED_SYMBOLS = (
     "lpfa_meta_dev_ints", "lpfa_varlen_meta_fill_host", "lpfa_varlen_meta_from_lengths",
     "lpfa_scale_bytes", "lpfa_quantize_mxfp8_varlen", "lpfa_cast_e4m3", "lpfa_attn_fwd_varlen",
     "lpfa_device_status", "lpfa_last_error_message", "lpfa_version", "lpfa_attn_fwd_varlen_debug",
-    "lpfa_attn_fwd_varlen_descaled",
+    "lpfa_attn_fwd_varlen_descaled", "lpfa_quantize_mxfp8_varlen_tokens",
 )
 
 
@@ -70,6 +70,8 @@ _lib.lpfa_scale_bytes.restype = ctypes.c_size_t
 _lib.lpfa_quantize_mxfp8_varlen.argtypes = [_vp, ctypes.c_int, _i64, _i64, _i32, _i32, ctypes.POINTER(_Meta),
                                             ctypes.c_int, _vp, _vp, _vp]
 _lib.lpfa_quantize_mxfp8_varlen.restype = ctypes.c_int
+_lib.lpfa_quantize_mxfp8_varlen_tokens.argtypes = _lib.lpfa_quantize_mxfp8_varlen.argtypes
+_lib.lpfa_quantize_mxfp8_varlen_tokens.restype = ctypes.c_int
 _lib.lpfa_cast_e4m3.argtypes = [_vp, _i64, _i64, _i64, _i32, _i32, _vp, _vp]
 _lib.lpfa_cast_e4m3.restype = ctypes.c_int
 _lib.lpfa_attn_fwd_varlen.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, ctypes.POINTER(_Meta), ctypes.POINTER(_Meta),
@@ -167,8 +169,14 @@ def _strides(x: torch.Tensor):
 
 def lpfa_quantize_mxfp8_varlen(x: torch.Tensor, meta: VarlenMeta, scaling_mode: str = "rceil",
                                payload: Optional[torch.Tensor] = None, scales: Optional[torch.Tensor] = None,
-                               stream=None):
-    """Quantize packed (T, H, 128) bf16/fp32 to (payload uint8 (T,H,128), scales uint8 (blocks*H*512,))."""
+                               stream=None, orientation: str = "head_dim"):
+    """Quantize packed (T, H, 128) bf16/fp32 to (payload uint8 (T,H,128), scales uint8 (blocks*H*512,)).
+
+    orientation "head_dim": one scale per 32 elements along head_dim (Q and K, and V in bf16 PV
+    mode); "tokens": one scale per 32 tokens of a channel (V in mxfp8 PV mode).
+    """
+    if orientation not in ("head_dim", "tokens"):
+        raise ValueError("orientation must be 'head_dim' or 'tokens'")
     dt = {torch.bfloat16: "bf16", torch.float32: "fp32"}.get(x.dtype)
     if dt is None:
         raise ValueError("x must be bf16 or fp32")
@@ -183,9 +191,9 @@ def lpfa_quantize_mxfp8_varlen(x: torch.Tensor, meta: VarlenMeta, scaling_mode: 
     if scales is None:
         scales = torch.empty(meta.scale_bytes(H), dtype=torch.uint8, device=x.device)
     with torch.cuda.device(x.device):
-        _check(_lib.lpfa_quantize_mxfp8_varlen(x.data_ptr(), IN_DTYPES[dt], ts, hs, H, 128, ctypes.byref(meta._c),
-                                               SCALING_MODES[scaling_mode], payload.data_ptr(), scales.data_ptr(),
-                                               _stream_ptr(stream)))
+        fn = _lib.lpfa_quantize_mxfp8_varlen if orientation == "head_dim" else _lib.lpfa_quantize_mxfp8_varlen_tokens
+        _check(fn(x.data_ptr(), IN_DTYPES[dt], ts, hs, H, 128, ctypes.byref(meta._c),
+                  SCALING_MODES[scaling_mode], payload.data_ptr(), scales.data_ptr(), _stream_ptr(stream)))
     return payload, scales
 
 

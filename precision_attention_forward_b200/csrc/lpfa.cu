@@ -233,9 +233,11 @@ static lpfa_status launch_quant(void (*kernel)(const CUtensorMap, lpfa::QuantPar
   return LPFA_OK;
 }
 
-lpfa_status lpfa_quantize_mxfp8_varlen(const void* x, lpfa_in_dtype dt, int64_t tok_stride, int64_t head_stride,
-                                       int32_t heads, int32_t head_dim, const lpfa_varlen_meta* meta,
-                                       lpfa_scaling_mode mode, uint8_t* payload, uint8_t* scales, void* stream) {
+// Both orientations of the varlen quantizer: scales along head_dim or along the tokens.
+static lpfa_status quantize_impl(const void* x, lpfa_in_dtype dt, int64_t tok_stride, int64_t head_stride,
+                                 int32_t heads, int32_t head_dim, const lpfa_varlen_meta* meta,
+                                 lpfa_scaling_mode mode, uint8_t* payload, uint8_t* scales, void* stream,
+                                 bool tokens) {
   if (!x || !payload || !scales) return fail(LPFA_ERR_INVALID_ARG, "NULL tensor pointer");
   if (dt != LPFA_IN_BF16 && dt != LPFA_IN_FP32) return fail(LPFA_ERR_INVALID_ARG, "invalid input dtype %d", dt);
   if (mode != LPFA_SCALE_RCEIL && mode != LPFA_SCALE_FLOOR) return fail(LPFA_ERR_INVALID_ARG, "invalid scaling mode %d", mode);
@@ -266,13 +268,29 @@ lpfa_status lpfa_quantize_mxfp8_varlen(const void* x, lpfa_in_dtype dt, int64_t 
   if ((st = input_tmap(&tm, x, dt == LPFA_IN_FP32, meta->total_tokens, heads, tok_stride, head_stride)) != LPFA_OK)
     return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (dt == LPFA_IN_BF16)
-    return launch_quant(lpfa::quantize_mxfp8_kernel<__nv_bfloat16, false>, lpfa::quant_smem_bytes<__nv_bfloat16>(),
-                        lpfa::quant_threads<__nv_bfloat16>(), tm,
+  if (dt == LPFA_IN_BF16) {
+    auto kernel = tokens ? lpfa::quantize_mxfp8_kernel<__nv_bfloat16, lpfa::kQuantTokens>
+                         : lpfa::quantize_mxfp8_kernel<__nv_bfloat16, lpfa::kQuantHeadDim>;
+    return launch_quant(kernel, lpfa::quant_smem_bytes<__nv_bfloat16>(), lpfa::quant_threads<__nv_bfloat16>(), tm,
                         p, info.sms, s, "quantize launch");
-  return launch_quant(lpfa::quantize_mxfp8_kernel<float, false>, lpfa::quant_smem_bytes<float>(),
-                      lpfa::quant_threads<float>(), tm, p, info.sms, s,
+  }
+  auto kernel = tokens ? lpfa::quantize_mxfp8_kernel<float, lpfa::kQuantTokens>
+                       : lpfa::quantize_mxfp8_kernel<float, lpfa::kQuantHeadDim>;
+  return launch_quant(kernel, lpfa::quant_smem_bytes<float>(), lpfa::quant_threads<float>(), tm, p, info.sms, s,
                       "quantize launch");
+}
+
+lpfa_status lpfa_quantize_mxfp8_varlen(const void* x, lpfa_in_dtype dt, int64_t tok_stride, int64_t head_stride,
+                                       int32_t heads, int32_t head_dim, const lpfa_varlen_meta* meta,
+                                       lpfa_scaling_mode mode, uint8_t* payload, uint8_t* scales, void* stream) {
+  return quantize_impl(x, dt, tok_stride, head_stride, heads, head_dim, meta, mode, payload, scales, stream, false);
+}
+
+lpfa_status lpfa_quantize_mxfp8_varlen_tokens(const void* x, lpfa_in_dtype dt, int64_t tok_stride,
+                                              int64_t head_stride, int32_t heads, int32_t head_dim,
+                                              const lpfa_varlen_meta* meta, lpfa_scaling_mode mode,
+                                              uint8_t* payload, uint8_t* scales, void* stream) {
+  return quantize_impl(x, dt, tok_stride, head_stride, heads, head_dim, meta, mode, payload, scales, stream, true);
 }
 
 lpfa_status lpfa_cast_e4m3(const void* v_bf16, int64_t tok_stride, int64_t head_stride, int64_t tokens,
@@ -297,7 +315,7 @@ lpfa_status lpfa_cast_e4m3(const void* v_bf16, int64_t tok_stride, int64_t head_
   p.payload = out;
   CUtensorMap tm;
   if ((st = input_tmap(&tm, v_bf16, false, tokens, heads, tok_stride, head_stride)) != LPFA_OK) return st;
-  return launch_quant(lpfa::quantize_mxfp8_kernel<__nv_bfloat16, true>, lpfa::quant_smem_bytes<__nv_bfloat16>(),
+  return launch_quant(lpfa::quantize_mxfp8_kernel<__nv_bfloat16, lpfa::kQuantCast>, lpfa::quant_smem_bytes<__nv_bfloat16>(),
                         lpfa::quant_threads<__nv_bfloat16>(), tm, p,
                       info.sms, static_cast<cudaStream_t>(stream), "cast launch");
 }

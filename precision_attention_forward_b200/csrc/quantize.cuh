@@ -10,12 +10,21 @@
 //
 // Cast (FastVideo #1654, "fp8 PV mode for the FA4-FP4 attention path"): E4M3(v) with no scale.
 //
+// Token orientation (same README: Q, K and V keep both hardware orientations): one E8M0 scale per
+// 32 consecutive tokens of one (head, channel), the groups aligned to the sequence start, 4 per
+// 128-token block, in the same 512-byte atoms with channel n, group g at (n % 32) * 16 +
+// (n / 32) * 4 + g; a partial last group takes its maximum over the tokens it has, a group with
+// no token holds 0x7F. The block-scaled MXFP8 PV product reads V this way (K = keys).
+//
 // One persistent kernel serves both: each CTA walks (128-token block, head) tiles with a stride
 // of the grid size. One warp stages each tile (128 token rows of one head) into shared memory
 // with a single TMA box load, double buffered, so the next tile is in flight while the
 // converting warps work on the current one; they read 16 bytes per lane from shared memory,
 // find each 32-element block maximum over 4 lanes with warp shuffles, write 8 payload bytes per
-// lane (coalesced 128-byte rows) and one scale byte per block.
+// lane (coalesced 128-byte rows) and one scale byte per block. In the token orientation each
+// converting warp owns one 32-token group and a range of channels (consecutive channels on
+// consecutive lanes): one pass over the group's rows for the maxima, one to scale, convert and
+// store (contiguous payload bytes per row across the warp).
 #pragma once
 
 #include <cstdint>
@@ -26,6 +35,13 @@
 #include "ptx.cuh"
 
 namespace lpfa {
+
+// What quantize_mxfp8_kernel produces.
+enum QuantKind : int {
+  kQuantHeadDim = 0,  // scales per 32 elements along head_dim
+  kQuantCast = 1,     // unscaled E4M3, no scales
+  kQuantTokens = 2    // scales per 32 tokens of a channel
+};
 
 #ifndef LPFA_QUANT_STAGES_BF16
 #define LPFA_QUANT_STAGES_BF16 2
@@ -112,6 +128,7 @@ struct QuantTile {
 
 template <bool kCast>
 __device__ __forceinline__ QuantTile quant_tile(const QuantParams& p, int w) {
+  // (kCast: a plain token range without metadata.)
   QuantTile t;
   t.g = w / p.heads;
   t.h = w - t.g * p.heads;
@@ -132,11 +149,12 @@ __device__ __forceinline__ QuantTile quant_tile(const QuantParams& p, int w) {
 
 // Persistent grid over tiles w = g * heads + h (heads of a token block are adjacent in
 // memory). Warps 0..7 convert; warp 8 stages tiles (its own warp, so that computing the next
-// tile's bounds and issuing its copies never holds up the converting warps). kCast: E4M3(x)
-// with no scale and no scale atoms.
-template <typename T, bool kCast>
+// tile's bounds and issuing its copies never holds up the converting warps). kKind: see
+// QuantKind (the cast writes no scale atoms).
+template <typename T, int kKind>
 __global__ void __launch_bounds__(quant_threads<T>())
 quantize_mxfp8_kernel(const __grid_constant__ CUtensorMap tmap_x, QuantParams p) {
+  constexpr bool kCast = kKind == kQuantCast;
   constexpr uint32_t kRowBytes = 128 * sizeof(T);
   constexpr uint32_t kTileBytesIn = 128 * kRowBytes;
   constexpr int kQuantStages = quant_stages<T>();
@@ -191,6 +209,69 @@ quantize_mxfp8_kernel(const __grid_constant__ CUtensorMap tmap_x, QuantParams p)
   }
 
   // ------------------------------------------------------------------ converters
+  if (kKind == kQuantTokens) {
+    // Warp -> (32-token group g, channel range); lane -> kCh consecutive channels.
+    constexpr int kCh = 128 / (32 * (kQuantWarps / 4));  // bf16 (8 warps): 2, fp32 (16): 1
+    static_assert(kCh == 1 || kCh == 2, "channels per lane");
+    const int g = warp & 3;
+    const int c0 = (warp >> 2) * (32 * kCh) + lane * kCh;
+    int n = 0;
+    for (int w = blockIdx.x; w < num_tiles; w += G, ++n) {
+      const int b = n % kQuantStages;
+      if (!mbar_wait(&full[b], (n / kQuantStages) & 1, abort_flag)) {
+        *abort_flag = 1;
+        if (atomicCAS(&g_lpfa_status[0], 0, 4 /* LPFA_ERR_TIMEOUT */) == 0) atomicExch(&g_lpfa_status[1], 100);
+        break;
+      }
+      const QuantTile t = info[b];
+      const T* src = reinterpret_cast<const T*>(qsmem + b * kTileBytesIn);
+      uint8_t* atom = p.scales + (static_cast<int64_t>(t.g) * p.heads + t.h) * 512;
+      const int r0 = 32 * g;
+      const int r1 = min(t.rows_valid, r0 + 32);
+      float amax[kCh];
+#pragma unroll
+      for (int c = 0; c < kCh; ++c) amax[c] = 0.f;
+#pragma unroll 4
+      for (int r = r0; r < r1; ++r) {
+        float v[kCh];
+        if (kCh == 2) {
+          const uint32_t u = *reinterpret_cast<const uint32_t*>(src + r * 128 + c0);
+          v[0] = __uint_as_float(u << 16);
+          v[kCh - 1] = __uint_as_float(u & 0xFFFF0000u);
+        } else {
+          v[0] = static_cast<float>(src[r * 128 + c0]);
+        }
+#pragma unroll
+        for (int c = 0; c < kCh; ++c) amax[c] = fmaxf(amax[c], fabsf(v[c]));
+      }
+      int e[kCh];
+      float inv[kCh];
+#pragma unroll
+      for (int c = 0; c < kCh; ++c) {
+        e[c] = e8m0_exponent(amax[c], p.floor_mode);
+        inv[c] = __uint_as_float(static_cast<uint32_t>(127 - e[c]) << 23);  // 2^-e, normal
+      }
+#pragma unroll 4
+      for (int r = r0; r < r1; ++r) {
+        uint8_t* dst = p.payload + ((t.tok0 + r) * p.heads + t.h) * 128 + c0;
+        if (kCh == 2) {
+          const uint32_t u = *reinterpret_cast<const uint32_t*>(src + r * 128 + c0);
+          *reinterpret_cast<uint16_t*>(dst) =
+              cvt_e4m3x2(__uint_as_float(u << 16) * inv[0], __uint_as_float(u & 0xFFFF0000u) * inv[kCh - 1]);
+        } else {
+          *dst = static_cast<uint8_t>(cvt_e4m3x2(static_cast<float>(src[r * 128 + c0]) * inv[0], 0.0f) & 0xFF);
+        }
+      }
+#pragma unroll
+      for (int c = 0; c < kCh; ++c) {
+        const int ch = c0 + c;
+        atom[(ch & 31) * 16 + (ch >> 5) * 4 + g] = r0 < r1 ? static_cast<uint8_t>(e[c] + 127) : uint8_t{0x7F};
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[b]);
+    }
+    return;
+  }
   const int half = lane >> 4;        // which of the two rows of an iteration
   const int col8 = (lane & 15) * 8;  // first of this lane's 8 elements
   const int kb = (lane & 15) >> 2;   // this lane's 32-element block

@@ -158,3 +158,60 @@ def test_quantize_workload(name):
         toks, hs = gu.sample_rows(lk, w.heads, seed=8, per_tile_random=1)
         got = out[torch.from_numpy(toks).cuda(), torch.from_numpy(hs).cuda()].cpu().numpy()
         assert np.array_equal(got, omx.cast_e4m3(v[toks, hs]))
+
+
+def _check_tokens(x, lens, heads, dtype, mode, xd=None):
+    """Token orientation: whole payload and whole scale buffer against the oracle."""
+    meta = lp.lpfa_varlen_meta_from_lengths(lens)
+    if xd is None:
+        xd = gu.to_device(x, dtype)
+    payload, scales = lp.lpfa_quantize_mxfp8_varlen(xd, meta, scaling_mode=mode, orientation="tokens")
+    ref_p, ref_s = omx.quantize_mxfp8_varlen_tokens(x, lens, mode)
+    got_p, got_s = payload.cpu().numpy(), scales.cpu().numpy()
+    bad_p = np.argwhere(got_p != ref_p)
+    assert bad_p.size == 0, f"{len(bad_p)} payload bytes differ, first at {bad_p[:3].tolist()}"
+    bad_s = np.flatnonzero(got_s != ref_s)
+    assert bad_s.size == 0, f"{bad_s.size} scale bytes differ, first at {bad_s[:5].tolist()}"
+    return payload, scales
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+@pytest.mark.parametrize("mode", ["rceil", "floor"])
+def test_quantize_tokens_ragged_bit_exact(dtype, mode):
+    """Partial and empty 32-token groups, sequences shorter than a group, several blocks."""
+    lens = [1, 31, 32, 33, 127, 128, 129, 300, 64]
+    _check_tokens(_ragged_input(lens, 3, 12, dtype), lens, 3, dtype, mode)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+@pytest.mark.parametrize("mode", ["rceil", "floor"])
+def test_quantize_tokens_adversarial_bit_exact(dtype, mode):
+    """The adversarial rows laid along the tokens of each channel (128 tokens, 2 heads)."""
+    rows = _adversarial_rows().astype(np.float32)            # (5, 128): values along tokens
+    x = np.empty((128, 2, 128), dtype=np.float32)
+    for c in range(128):
+        x[:, 0, c] = rows[c % 5]
+        x[:, 1, c] = rows[(c + 2) % 5][::-1]
+    if dtype == "bf16":
+        x = wl.round_to_bf16(x)
+    _check_tokens(x, [128], 2, dtype, mode)
+    _check_tokens(x[:77], [77], 2, dtype, mode)
+
+
+def test_quantize_tokens_strided_input_matches_contiguous():
+    lens = [200, 57]
+    x = _ragged_input(lens, 4, 6, "bf16")
+    big = torch.zeros((257, 4, 384), dtype=torch.bfloat16, device="cuda")
+    big[:, :, 128:256] = gu.to_device(x, "bf16")
+    p1, s1 = _check_tokens(x, lens, 4, "bf16", "rceil", xd=big[:, :, 128:256])
+    hm = gu.to_device(np.ascontiguousarray(x.transpose(1, 0, 2)), "bf16").transpose(0, 1)
+    p2, s2 = _check_tokens(x, lens, 4, "bf16", "rceil", xd=hm)
+    assert torch.equal(p1, p2) and torch.equal(s1, s2)
+
+
+def test_quantize_tokens_workload_v():
+    """V of the dense workload (4 x 2048 tokens, 16 heads) at full size, every byte."""
+    w = wl.WORKLOADS["dense_4x2048_h16"]
+    lq, lk = wl.lengths(w)
+    v = wl.make_tensor(w, "v")
+    _check_tokens(v, lk, w.heads, "bf16", "rceil")
