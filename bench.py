@@ -156,6 +156,9 @@ def cpu_oracle_sample(w, seconds: float, seed: int = 0):
             vh = omx.e4m3_decode(omx.cast_e4m3(v[k0:k1, h]))
         elif w.pv_mode == "bf16v":
             vh = v[k0:k1, h].astype(np.float64)
+        elif w.pv_mode == "mxfp8":
+            vpt, vst = omx.quantize_mxfp8_varlen_tokens(v[k0:k1, h][:, None, :], [k1 - k0], w.scaling_mode)
+            vh = omx.dequantize_mxfp8_tokens(vpt, vst, [k1 - k0], 1)[:, 0]
         else:
             vp, ve = omx.quantize_rows(v[k0:k1, h].astype(np.float64), w.scaling_mode)
             vh = (omx.e4m3_decode(vp).reshape(-1, 4, 32) * np.ldexp(1.0, ve)[..., None]).reshape(-1, 128)
@@ -163,7 +166,7 @@ def cpu_oracle_sample(w, seconds: float, seed: int = 0):
         r1 = min(cu_q[i + 1], r0 + rows_per)
         qp, qe = omx.quantize_rows(q[r0:r1, h].astype(np.float64), w.scaling_mode)
         qh = (omx.e4m3_decode(qp).reshape(-1, 4, 32) * np.ldexp(1.0, qe)[..., None]).reshape(-1, 128)
-        oatt.attend_block(qh, kh, vh, p_mode="fp8" if w.pv_mode == "fp8" else "exact")
+        oatt.attend_block(qh, kh, vh, p_mode={"fp8": "fp8", "mxfp8": "mxfp8"}.get(w.pv_mode, "exact"))
         done_flops += 4.0 * (r1 - r0) * (k1 - k0) * 128
         units += 1
     elapsed = time.perf_counter() - t0
@@ -307,7 +310,7 @@ def main():
     vp = torch.empty((Tk, H, 128), dtype=torch.uint8, device=dev) if w.pv_mode != "bf16v" else None
     qs = torch.empty(sbq * H * 512, dtype=torch.uint8, device=dev)
     ks = torch.empty(sbk * H * 512, dtype=torch.uint8, device=dev)
-    vs = torch.empty(sbk * H * 512, dtype=torch.uint8, device=dev) if w.pv_mode == "bf16" else None
+    vs = torch.empty(sbk * H * 512, dtype=torch.uint8, device=dev) if w.pv_mode in ("bf16", "mxfp8") else None
     out = torch.empty((Tq, H, 128), dtype=torch.bfloat16, device=dev)
     lse = torch.empty((H, Tq), dtype=torch.float32, device=dev)
 
@@ -323,6 +326,8 @@ def main():
             lp.lpfa_cast_e4m3(ins["v"], out=vp)
         elif w.pv_mode == "bf16":
             lp.lpfa_quantize_mxfp8_varlen(ins["v"], mk, w.scaling_mode, payload=vp, scales=vs)
+        elif w.pv_mode == "mxfp8":   # V in the token orientation
+            lp.lpfa_quantize_mxfp8_varlen(ins["v"], mk, w.scaling_mode, payload=vp, scales=vs, orientation="tokens")
         if timing is not None:
             c = torch.cuda.Event(enable_timing=True)
             c.record(stream)

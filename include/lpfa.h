@@ -51,7 +51,7 @@ typedef enum {
 
 typedef enum { LPFA_IN_BF16 = 0, LPFA_IN_FP32 = 1 } lpfa_in_dtype;
 typedef enum { LPFA_SCALE_RCEIL = 0, LPFA_SCALE_FLOOR = 1 } lpfa_scaling_mode;
-typedef enum { LPFA_PV_BF16 = 0, LPFA_PV_FP8 = 1, LPFA_PV_BF16_V = 2 } lpfa_pv_mode;
+typedef enum { LPFA_PV_BF16 = 0, LPFA_PV_FP8 = 1, LPFA_PV_BF16_V = 2, LPFA_PV_MXFP8 = 3 } lpfa_pv_mode;
 
 /*
  * Packed variable-length metadata (LP-FA4 README, "MXFP8 forward and backward":
@@ -173,6 +173,10 @@ LPFA_API lpfa_status lpfa_cast_e4m3(const void* v_bf16, int64_t tok_stride, int6
  *                  power-of-two running maximum. LPFA_PV_BF16_V: v points to BF16 values
  *                  (Tk, H, 128), contiguous, never quantized (LP-FA4 README: V kept in BF16);
  *                  v_sf must be NULL; P is rounded to BF16 as in LPFA_PV_BF16.
+ *                  LPFA_PV_MXFP8: block-scaled MXFP8 PV; v and v_sf are V quantized in the
+ *                  token orientation (lpfa_quantize_mxfp8_varlen_tokens, under meta_k), and P
+ *                  is quantized to MXFP8 per 32 keys (RCEIL on each group's maximum) before a
+ *                  block-scaled E4M3 x E4M3 product; O is divided by the sum of the unrounded P.
  * meta_q, meta_k   sequence i of meta_q attends to sequence i of meta_k (same num_seqs).
  * q/k/v_descale    device pointers to one float each, or NULL (per-tensor descales; see
  *                  lpfa_attn_fwd_varlen_descaled for per-head ones). NULL means exactly 1.0:
@@ -184,7 +188,7 @@ LPFA_API lpfa_status lpfa_cast_e4m3(const void* v_bf16, int64_t tok_stride, int6
  * Alignment:       every tensor 16-byte aligned.
  * Errors:          LPFA_ERR_INVALID_ARG for NULL required pointers, head_dim != 128,
  *                  heads < 1, mismatched num_seqs, a bad pv_mode, or a non-NULL v_sf in fp8
- *                  or BF16-V mode (and NULL v_sf in bf16 mode); LPFA_ERR_UNSUPPORTED off sm_100;
+ *                  or BF16-V mode (and NULL v_sf in bf16 or MXFP8 mode); LPFA_ERR_UNSUPPORTED off sm_100;
  *                  LPFA_ERR_CUDA on launch failure. A kernel that gives up on a barrier wait
  *                  records LPFA_ERR_TIMEOUT in the device status word (see below).
  */

@@ -31,7 +31,7 @@ LPFA_OK, LPFA_ERR_INVALID_ARG, LPFA_ERR_UNSUPPORTED, LPFA_ERR_CUDA, LPFA_ERR_TIM
 _STATUS_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "CUDA", 4: "TIMEOUT"}
 IN_DTYPES = {"bf16": 0, "fp32": 1}
 SCALING_MODES = {"rceil": 0, "floor": 1}
-PV_MODES = {"bf16": 0, "fp8": 1, "bf16v": 2}  # bf16v: BF16 V input, bf16 PV
+PV_MODES = {"bf16": 0, "fp8": 1, "bf16v": 2, "mxfp8": 3}  # bf16v: BF16 V input, bf16 PV; mxfp8: block-scaled PV
 
 # Symbols the header declares; the tests check that each one is exported.
 EXPORTED_SYMBOLS = (
@@ -243,7 +243,7 @@ def lpfa_attn_fwd_varlen(q: torch.Tensor, q_sf: torch.Tensor, k: torch.Tensor, k
     which takes per-tensor descales only.
     """
     if pv_mode not in PV_MODES:
-        raise ValueError("pv_mode must be 'bf16', 'fp8' or 'bf16v'")
+        raise ValueError("pv_mode must be 'bf16', 'fp8', 'bf16v' or 'mxfp8'")
     for name, t in (("q", q), ("k", k), ("v", v)):
         want = torch.bfloat16 if (name == "v" and pv_mode == "bf16v") else torch.uint8
         if t.dtype != want or t.dim() != 3 or not t.is_contiguous():

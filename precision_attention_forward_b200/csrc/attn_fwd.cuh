@@ -84,7 +84,9 @@ constexpr uint32_t kColP = 384;      // + 32 * (t % kPSlots)  fp8 P slot
 constexpr uint32_t kPSlots = 3;
 constexpr uint32_t kColSFA = 480;    // + 4 * stage  Q scale atom
 constexpr uint32_t kColSFB = 488;    // + 4 * slot   K scale atom
-static_assert(kColP + 32 * kPSlots <= kColSFA && kColSFB + 8 <= kTmemCols, "TMEM columns");
+constexpr uint32_t kColSFP = 496;    // + 4 * (t & 1)   P scale atom (block-scaled MXFP8 PV)
+constexpr uint32_t kColSFV = 504;    // + 4 * (vc & 1)  V scale atom (block-scaled MXFP8 PV)
+static_assert(kColP + 32 * kPSlots <= kColSFA && kColSFV + 8 <= kTmemCols, "TMEM columns");
 
 // log2(e) / sqrt(128) rounded to fp32: logits in log2 units per unit of Q.K.
 constexpr float kLog2eRsqrtD = 0.12751743082459868f;
@@ -149,7 +151,8 @@ struct SmemLayout {
   static constexpr uint32_t q_sf = vbf + (kFp8PV ? 0 : kVbf * kVbfBytes);
   static constexpr uint32_t k_sf = q_sf + kQStages * kAtomBytes;
   static constexpr uint32_t v_sf = k_sf + kK * kAtomBytes;
-  static constexpr uint32_t mref = v_sf + kV * kAtomBytes;            // float [2 groups][128] tile reference
+  static constexpr uint32_t p_sf = v_sf + kV * kAtomBytes;            // [kPSlots] P scale atoms (MXFP8 PV)
+  static constexpr uint32_t mref = p_sf + kPSlots * kAtomBytes;       // float [2 groups][128] tile reference
   static constexpr uint32_t lsum = mref + 2 * 128 * 4;                // float [2 groups][128] partial l
   static constexpr uint32_t mfin = lsum + 2 * 128 * 4;                // float [2 groups][128] reference of l
   static constexpr uint32_t lsumr = mfin + 2 * 128 * 4;               // float [2 groups][128] partial sum of rounded P
@@ -200,6 +203,12 @@ __device__ __forceinline__ uint32_t idesc_qk(int kb, int negate_a) {
 }
 // E4M3 x E4M3 -> F32, M=128, N=128, A (P) K-major in TMEM, B (V) MN-major.
 constexpr uint32_t kIdescPV8 = (1u << 4) | (1u << 16) | (16u << 17) | (8u << 24);
+// Block-scaled E4M3 x E4M3 -> F32, M=128, N=128, A (P) K-major in TMEM, B (V) MN-major, E8M0
+// scales; kb selects the scale byte of the K step (keys [32kb, 32kb + 32)).
+__device__ __forceinline__ uint32_t idesc_pv_mx(int kb) {
+  return (static_cast<uint32_t>(kb) << 4) | (1u << 16) | ((128u >> 3) << 17) | (1u << 23) | (8u << 24) |
+         (static_cast<uint32_t>(kb) << 29);
+}
 // BF16 x BF16 -> F32, M=128, N=128, A (P) K-major in TMEM, B (V) MN-major.
 constexpr uint32_t kIdescPV16 = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) | (16u << 17) | (8u << 24);
 
@@ -466,7 +475,10 @@ __device__ __forceinline__ void record_failure(volatile int* abort_flag, int sit
 // PV variants of the kernel: V as MXFP8 dequantized to BF16 in shared memory (bf16 PV), V as
 // unscaled E4M3 (fp8 PV), or V given as BF16 and loaded by TMA straight into the layout the
 // BF16 PV MMA reads (bf16 PV with BF16 V; LP-FA4 README: the BF16 V path).
-enum PvKind : int { kPvBf16Mx = 0, kPvFp8 = 1, kPvBf16In = 2 };
+enum PvKind : int { kPvBf16Mx = 0, kPvFp8 = 1, kPvBf16In = 2, kPvMx = 3 };
+// P as 8-bit codes in the TMEM P slots and V used straight from its 8-bit tile: the fp8 PV mode
+// and the block-scaled MXFP8 PV mode share the shared-memory layout and stage counts.
+template <int kPv> constexpr bool pv_p8() { return kPv == kPvFp8 || kPv == kPvMx; }
 
 // How far (log2 units) a row's logits may exceed its reference before the reference, l and
 // O move, and the power of two P is stored with. bf16 P keeps its 8-bit mantissa at any
@@ -484,9 +496,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                 const __grid_constant__ CUtensorMap tmap_v, const AttnParams p) {
   constexpr bool kFp8PV = kPv == kPvFp8;
+  constexpr bool kMx = kPv == kPvMx;        // block-scaled MXFP8 PV: P and V scaled per 32 keys
+  constexpr bool kP8 = pv_p8<kPv>();        // P in the TMEM P slots, V from its 8-bit tile
   constexpr bool kVIn = kPv == kPvBf16In;  // BF16 V straight into the BF16 operand buffers
-  using L = SmemLayout<kFp8PV>;
-  constexpr int kKStages = Stages<kFp8PV>::k, kVStages = Stages<kFp8PV>::v, kVbfStages = Stages<kFp8PV>::vbf;
+  constexpr bool kVsf = kPv == kPvBf16Mx || kMx;  // V tiles come with a scale atom
+  using L = SmemLayout<kP8>;
+  constexpr int kKStages = Stages<kP8>::k, kVStages = Stages<kP8>::v, kVbfStages = Stages<kP8>::vbf;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::bars);
@@ -505,7 +520,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
     for (int i = 0; i < kKStages; ++i) { mbar_init(&bars[kBarKFull + i], 1); mbar_init(&bars[kBarKEmpty + i], 1); }
     for (int i = 0; i < kVStages; ++i) {
       mbar_init(&bars[kBarVFull + i], 1);
-      mbar_init(&bars[kBarVEmpty + i], kFp8PV ? 1 : 4);   // MMA commit, or the 4 converter warps
+      mbar_init(&bars[kBarVEmpty + i], kP8 ? 1 : 4);   // MMA commit, or the 4 converter warps
     }
     for (int i = 0; i < kVbfStages; ++i) {
       mbar_init(&bars[kBarVbfFull + i], kVIn ? 1 : 4);  // the V producer's TMA, or the 4 converter warps
@@ -626,10 +641,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
         for (int j = 0; j < ui.nkv; ++j) {
           const uint32_t s = vc % kVStages, ph = (vc / kVStages) & 1;
           if (!mbar_wait_warp(&bars[kBarVEmpty + s], ph ^ 1, abort_flag)) { record_failure(abort_flag, kSiteProducerV); ok = false; break; }
-          mbar_arrive_expect_tx(&bars[kBarVFull + s], kTileBytes + (kFp8PV ? 0 : kAtomBytes), leader);
+          mbar_arrive_expect_tx(&bars[kBarVFull + s], kTileBytes + (kVsf ? kAtomBytes : 0), leader);
           tma_load_3d(smem + L::v + s * kTileBytes, &tmap_v, &bars[kBarVFull + s], 0, ui.h,
                       ui.k_row0 + j * kTileN, leader);
-          if (!kFp8PV)
+          if (kVsf)
             bulk_load(smem + L::v_sf + s * kAtomBytes,
                       p.v_sf + (static_cast<int64_t>(ui.sbk + j) * p.heads + ui.h) * kAtomBytes, kAtomBytes,
                       &bars[kBarVFull + s], leader);
@@ -679,7 +694,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
             // S buffer b has been read out by its group (tile t - 2); in bf16 PV mode it also
             // holds P(t - 2), so PV(t - 2) must have completed.
             if (!mbar_wait_warp(&bars[kBarSFree + b], ((t - 2) >> 1) & 1, abort_flag)) { record_failure(abort_flag, kSiteMmaS); ok = false; break; }
-            if (!kFp8PV && !mbar_wait_warp(&bars[kBarPVDone + (t - 2) % kPSlots], ((t - 2) / kPSlots) & 1, abort_flag)) { record_failure(abort_flag, kSiteMmaS); ok = false; break; }
+            if (!kP8 && !mbar_wait_warp(&bars[kBarPVDone + (t - 2) % kPSlots], ((t - 2) / kPSlots) & 1, abort_flag)) { record_failure(abort_flag, kSiteMmaS); ok = false; break; }
           }
           const uint32_t s = kc % kKStages;
           if (!mbar_wait_warp(&bars[kBarKFull + s], (kc / kKStages) & 1, abort_flag)) { record_failure(abort_flag, kSiteMmaK); ok = false; break; }
@@ -710,8 +725,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
       // holds back the next QK.
       const uint32_t leader = lane == 0 ? 1u : 0u;
       const uint32_t sb = static_cast<uint32_t>(warp_uniform(static_cast<int>(smem_u32(smem))));
-      const uint64_t dv0 = kFp8PV ? umma_desc(sb + L::v, kTileBytes, 1024, kLayoutSw128)
-                                  : umma_desc(sb + L::vbf, kTileBytes, 1024, kLayoutSw128);
+      const uint64_t dv0 = kP8 ? umma_desc(sb + L::v, kTileBytes, 1024, kLayoutSw128)
+                               : umma_desc(sb + L::vbf, kTileBytes, 1024, kLayoutSw128);
+      const uint64_t dpsf0 = umma_desc(sb + L::p_sf, 0, 128, kLayoutNone);
+      const uint64_t dvsf0 = umma_desc(sb + L::v_sf, 0, 128, kLayoutNone);
       uint32_t u = 0, vc = 0, t = 0;  // units, V tiles, tiles
       bool ok = true;
       for (int w = blockIdx.x; w < p.num_units && ok; w += G) {
@@ -721,11 +738,27 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
           const uint32_t b = t & 1;
           if (!mbar_wait_warp(&bars[kBarPReady + t % kPSlots], (t / kPSlots) & 1, abort_flag)) { record_failure(abort_flag, kSiteMmaP); ok = false; break; }
           if (j == 0 && !mbar_wait_warp(&bars[kBarOEmpty], (u & 1) ^ 1, abort_flag)) { record_failure(abort_flag, kSiteMmaO); ok = false; break; }
-          const bool got = kFp8PV ? mbar_wait_warp(&bars[kBarVFull + vc % kVStages], (vc / kVStages) & 1, abort_flag)
-                                  : mbar_wait_warp(&bars[kBarVbfFull + vc % kVbfStages], (vc / kVbfStages) & 1, abort_flag);
+          const bool got = kP8 ? mbar_wait_warp(&bars[kBarVFull + vc % kVStages], (vc / kVStages) & 1, abort_flag)
+                               : mbar_wait_warp(&bars[kBarVbfFull + vc % kVbfStages], (vc / kVbfStages) & 1, abort_flag);
           if (!got) { record_failure(abort_flag, kSiteMmaV); ok = false; break; }
           tc_fence_after();
-          if (kFp8PV) {
+          if (kMx) {
+            // Scale atoms into TMEM (the copies run in order with the MMAs below): P's from the
+            // softmax's shared-memory atom of this slot, V's from the V stage.
+            const uint32_t sfp = tmem + kColSFP + (t & 1) * 4;
+            const uint32_t sfv = tmem + kColSFV + (vc & 1) * 4;
+            tmem_cp_32x128b_x4(sfp, dpsf0 + ((t % kPSlots) * kAtomBytes >> 4), leader);
+            tmem_cp_32x128b_x4(sfv, dvsf0 + ((vc % kVStages) * kAtomBytes >> 4), leader);
+            const uint32_t p_col = tmem + kColP + (t % kPSlots) * 32;
+            const uint64_t bdesc = dv0 + ((vc % kVStages) * kTileBytes >> 4);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {  // keys [32kk, 32kk + 32), scale byte kk
+              const uint32_t byte_sel = static_cast<uint32_t>(kk) << 30;
+              mma_mxf8f6f4_ts(tmem + kColO, p_col + kk * 8, bdesc + kk * 256, idesc_pv_mx(kk), sfp | byte_sel,
+                              sfv | byte_sel, (j > 0 || kk > 0) ? 1u : 0u, leader);
+            }
+            mma_commit(&bars[kBarVEmpty + vc % kVStages], leader);
+          } else if (kFp8PV) {
             const uint32_t p_col = tmem + kColP + (t % kPSlots) * 32;
             const uint64_t bdesc = dv0 + ((vc % kVStages) * kTileBytes >> 4);
 #pragma unroll
@@ -755,8 +788,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
   } else if (warp < 12) {
     setmaxnreg_inc<kSoftmaxRegs>();
     // ------------------------------------------------------------------ softmax groups
+    // (Block-scaled P has no E4M3 range limit to respect: it takes the bf16 mode's lag.)
     constexpr float kLag = SoftmaxLag<kFp8PV>::lag;
     constexpr float kBias = SoftmaxLag<kFp8PV>::bias;
+    uint32_t* p_sf_words = reinterpret_cast<uint32_t*>(smem + L::p_sf);
     const uint32_t grp = static_cast<uint32_t>(warp - 4) >> 2;  // tiles t with t & 1 == grp
     const int quarter = warp & 3;                                // TMEM lane quarter of this warp
     const int row = quarter * 32 + lane;                         // query row within the tile
@@ -826,14 +861,34 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
                                 : exp_row<false, kPolyPairs>(sv, cscale, kBias - m_t, key0, ui.k_len, handoff);
         const float l_scale = exp2_int(m_g - m_t);
         l_g = l_g * l_scale + psum;
-        if (!kFp8PV) lr_g *= l_scale;
+        if (!kP8) lr_g *= l_scale;
         m_g = m_t;
-        if (kFp8PV) {
+        if (kP8) {
           // PV(t - 3) has read the previous P of this slot. (In bf16 PV mode P goes over the S
           // buffer, which QK(t) only overwrote after PV(t - 2) had completed.)
           if (t >= kPSlots) {
             if (!mbar_wait_warp(&bars[kBarPVDone + t % kPSlots], ((t - kPSlots) / kPSlots) & 1, abort_flag)) { record_failure(abort_flag, kSiteSoftPV); ok = false; break; }
             tc_fence_after();
+          }
+          if (kMx) {
+            // MXFP8 P: per 32 keys the group maximum picks 2^e (RCEIL; p >= 0 and masked keys are
+            // 0, an all-zero group gives e = -127), P = E4M3(p * 2^-e). The 4 scale bytes of this
+            // row go to the slot's shared-memory atom (row r at (r % 32) * 16 + (r / 32) * 4).
+            uint32_t sfw = 0;
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+              float amax = 0.0f;
+#pragma unroll
+              for (int i = 16 * g; i < 16 * g + 16; ++i) amax = max3f(amax, sv[i].x, sv[i].y);
+              const int e = e8m0_exponent(amax, 0);
+              const float2 inv = make_float2(__uint_as_float(static_cast<uint32_t>(127 - e) << 23),
+                                             __uint_as_float(static_cast<uint32_t>(127 - e) << 23));
+#pragma unroll
+              for (int i = 16 * g; i < 16 * g + 16; ++i) sv[i] = __fmul2_rn(sv[i], inv);
+              sfw |= static_cast<uint32_t>(e + 127) << (8 * g);
+            }
+            p_sf_words[(t % kPSlots) * (kAtomBytes / 4) + (row & 31) * 4 + (row >> 5)] = sfw;
+            fence_proxy_async_smem();  // the PV issuer's tcgen05.cp reads the atom
           }
           uint32_t pk[32];
 #pragma unroll
@@ -892,7 +947,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
       tc_fence_after();
       lsum[grp * 128 + row] = l_g;
       mfin[grp * 128 + row] = m_g;
-      if (!kFp8PV) lsumr[grp * 128 + row] = lr_g;
+      if (!kP8) lsumr[grp * 128 + row] = lr_g;
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars[kBarLReady]);
       if (!mbar_wait_warp(&bars[kBarLReady], u & 1, abort_flag)) { record_failure(abort_flag, kSiteSoftL); ok = false; break; }
@@ -902,7 +957,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
       const float s_g = exp2_int(m_g - m_f), s_o = exp2_int(m_o - m_f);
       const float ltot = l_g * s_g + l_o * s_o;
       const float vd = descale_value(p.v_descale, ui.seq, ui.h);
-      const float oscale = kFp8PV ? vd / ltot : vd / (lr_g * s_g + lsumr[(grp ^ 1) * 128 + row] * s_o);
+      const float oscale = kP8 ? vd / ltot : vd / (lr_g * s_g + lsumr[(grp ^ 1) * 128 + row] * s_o);
       uint32_t ra[32], rb[32];
       tmem_ld64_sync(tmem + lane_addr + kColO + grp * 64, ra, rb);
       tc_fence_before();

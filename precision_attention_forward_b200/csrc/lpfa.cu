@@ -340,7 +340,7 @@ extern "C++" {
 template <int kPv, bool kPerUnit>
 static lpfa_status launch_attn(int grid, cudaStream_t s, const CUtensorMap& tq, const CUtensorMap& tk,
                                const CUtensorMap& tv, const lpfa::AttnParams& p) {
-  constexpr uint32_t smem = lpfa::attn_smem_bytes<kPv == lpfa::kPvFp8>();
+  constexpr uint32_t smem = lpfa::attn_smem_bytes<lpfa::pv_p8<kPv>()>();
   const void* fn = reinterpret_cast<const void*>(lpfa::attn_fwd_kernel<kPv, kPerUnit>);
   const lpfa_status st = check_attn_kernel(fn, smem);
   if (st != LPFA_OK) return st;
@@ -357,11 +357,13 @@ static lpfa_status attn_fwd_impl(const uint8_t* q, const uint8_t* q_sf, const ui
                                  const lpfa_descale* k_descale, const lpfa_descale* v_descale, void* out_bf16,
                                  float* lse, void* stream, int debug_stall) {
   if (!q || !q_sf || !k || !k_sf || !v || !out_bf16 || !lse) return fail(LPFA_ERR_INVALID_ARG, "NULL tensor pointer");
-  if (pv_mode != LPFA_PV_BF16 && pv_mode != LPFA_PV_FP8 && pv_mode != LPFA_PV_BF16_V)
+  if (pv_mode != LPFA_PV_BF16 && pv_mode != LPFA_PV_FP8 && pv_mode != LPFA_PV_BF16_V && pv_mode != LPFA_PV_MXFP8)
     return fail(LPFA_ERR_INVALID_ARG, "invalid pv_mode %d", pv_mode);
   if (pv_mode == LPFA_PV_FP8 && v_sf) return fail(LPFA_ERR_INVALID_ARG, "fp8 PV mode takes no V scale factors (v_sf must be NULL)");
   if (pv_mode == LPFA_PV_BF16_V && v_sf) return fail(LPFA_ERR_INVALID_ARG, "BF16 V input takes no V scale factors (v_sf must be NULL)");
   if (pv_mode == LPFA_PV_BF16 && !v_sf) return fail(LPFA_ERR_INVALID_ARG, "bf16 PV mode needs the V scale factors (v_sf)");
+  if (pv_mode == LPFA_PV_MXFP8 && !v_sf)
+    return fail(LPFA_ERR_INVALID_ARG, "MXFP8 PV mode needs V's token-orientation scale factors (v_sf)");
   if (head_dim != 128) return fail(LPFA_ERR_INVALID_ARG, "head_dim must be 128 (got %d)", head_dim);
   if (heads < 1) return fail(LPFA_ERR_INVALID_ARG, "heads must be >= 1");
   for (const lpfa_descale* d : {q_descale, k_descale, v_descale})
@@ -430,6 +432,9 @@ static lpfa_status attn_fwd_impl(const uint8_t* q, const uint8_t* q_sf, const ui
   } else if (pv_mode == LPFA_PV_BF16) {
     st = per_unit ? launch_attn<lpfa::kPvBf16Mx, true>(grid, s, tq, tk, tv, p)
                   : launch_attn<lpfa::kPvBf16Mx, false>(grid, s, tq, tk, tv, p);
+  } else if (pv_mode == LPFA_PV_MXFP8) {
+    st = per_unit ? launch_attn<lpfa::kPvMx, true>(grid, s, tq, tk, tv, p)
+                  : launch_attn<lpfa::kPvMx, false>(grid, s, tq, tk, tv, p);
   } else {
     st = per_unit ? launch_attn<lpfa::kPvBf16In, true>(grid, s, tq, tk, tv, p)
                   : launch_attn<lpfa::kPvBf16In, false>(grid, s, tq, tk, tv, p);

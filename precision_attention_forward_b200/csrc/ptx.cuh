@@ -346,6 +346,19 @@ __device__ __forceinline__ uint16_t cvt_e4m3x2(float lo, float hi) {
   return r;
 }
 
+// E8M0 exponent of a non-negative float block maximum (MXFP8 scale rule: RCEIL, the smallest e
+// with amax <= 448 * 2^e, or FLOOR, floor(log2 amax) - 8; clamped to [-127, 127]).
+__device__ __forceinline__ int e8m0_exponent(float amax, int floor_mode) {
+  const uint32_t bits = __float_as_uint(amax);
+  const int biased = static_cast<int>(bits >> 23);
+  if (biased == 0) return -127;  // zero or subnormal maximum: below 2^-126, clamps to -127
+  const int binade = biased - 127;
+  const uint32_t mant = bits & 0x7FFFFFu;
+  // 448 = 1.75 * 2^8: a block whose maximum has mantissa <= 0.75 fits at e = binade - 8.
+  int e = floor_mode ? binade - 8 : (mant <= 0x600000u ? binade - 8 : binade - 7);
+  return max(-127, min(127, e));
+}
+
 // Two floats -> packed bf16x2 (round to nearest even); lo in bits 0..15.
 __device__ __forceinline__ uint32_t cvt_bf16x2(float lo, float hi) {
   uint32_t r;

@@ -73,18 +73,6 @@ struct QuantParams {
   int floor_mode;
 };
 
-// E8M0 exponent of a non-negative float block maximum.
-__device__ __forceinline__ int e8m0_exponent(float amax, int floor_mode) {
-  const uint32_t bits = __float_as_uint(amax);
-  const int biased = static_cast<int>(bits >> 23);
-  if (biased == 0) return -127;  // zero or subnormal maximum: below 2^-126, clamps to -127
-  const int binade = biased - 127;
-  const uint32_t mant = bits & 0x7FFFFFu;
-  // 448 = 1.75 * 2^8: a block whose maximum has mantissa <= 0.75 fits at e = binade - 8.
-  int e = floor_mode ? binade - 8 : (mant <= 0x600000u ? binade - 8 : binade - 7);
-  return max(-127, min(127, e));
-}
-
 // 8 consecutive elements of a staged row as floats.
 template <typename T>
 __device__ __forceinline__ void smem_load8(const T* p, float (&v)[8]);

@@ -80,6 +80,8 @@ def run_path(lp, q, k, v, lens_q, lens_k, heads, in_dtype="bf16", pv_mode="bf16"
         vp, vs = lp.lpfa_cast_e4m3(to_device(v, "bf16")), None
     elif pv_mode == "bf16v":
         vp, vs = to_device(v, "bf16"), None          # BF16 V input, never quantized
+    elif pv_mode == "mxfp8":                          # V in the token orientation
+        vp, vs = lp.lpfa_quantize_mxfp8_varlen(to_device(v, in_dtype), mk, scaling_mode=mode, orientation="tokens")
     else:
         vp, vs = gpu_quantize(lp, v, in_dtype, mk, mode)
     dd = [_descale_tensor(x) for x in descales]
@@ -99,17 +101,24 @@ def oracle_inputs(q, k, v, lens_q, lens_k, heads, pv_mode="bf16", mode="rceil"):
         vh = omx.e4m3_decode(omx.cast_e4m3(v))
     elif pv_mode == "bf16v":
         vh = np.asarray(v, dtype=np.float64)        # the BF16 values themselves
+    elif pv_mode == "mxfp8":
+        pv, sv = omx.quantize_mxfp8_varlen_tokens(v, lens_k, mode)
+        vh = omx.dequantize_mxfp8_tokens(pv, sv, lens_k, heads)
     else:
         pv, sv = omx.quantize_mxfp8_varlen(v, lens_k, mode)
         vh = omx.dequantize_mxfp8(pv, sv, lens_k, heads)
     return qh, kh, vh
 
 
+def p_mode_of(pv_mode: str) -> str:
+    """The oracle variant that grades a PV mode."""
+    return {"fp8": "fp8", "mxfp8": "mxfp8"}.get(pv_mode, "exact")
+
+
 def oracle_full(q, k, v, lens_q, lens_k, heads, pv_mode="bf16", mode="rceil", descales=(None, None, None)):
     qh, kh, vh = oracle_inputs(q, k, v, lens_q, lens_k, heads, pv_mode, mode)
     qd, kd, vd = [1.0 if x is None else x for x in descales]
-    return oatt.attention_fwd(qh, kh, vh, lens_q, lens_k, qd, kd, vd,
-                              p_mode="fp8" if pv_mode == "fp8" else "exact")
+    return oatt.attention_fwd(qh, kh, vh, lens_q, lens_k, qd, kd, vd, p_mode=p_mode_of(pv_mode))
 
 
 def sample_rows(lens_q, heads, seed=0, per_tile_random=2):
@@ -155,6 +164,9 @@ def oracle_sampled(q, k, v, lens_q, lens_k, heads, toks, hs, pv_mode="bf16", mod
                 vh = omx.e4m3_decode(omx.cast_e4m3(v[k0:k1, h]))
             elif pv_mode == "bf16v":
                 vh = np.asarray(v[k0:k1, h], dtype=np.float64)
+            elif pv_mode == "mxfp8":
+                pv, sv = omx.quantize_mxfp8_varlen_tokens(v[k0:k1, h][:, None, :], [k1 - k0], mode)
+                vh = omx.dequantize_mxfp8_tokens(pv, sv, [k1 - k0], 1)[:, 0]
             else:
                 vp, ve = omx.quantize_rows(v[k0:k1, h].astype(np.float64), mode)
                 vh = (omx.e4m3_decode(vp).reshape(-1, 4, 32) * np.ldexp(1.0, ve)[..., None]).reshape(-1, 128)
@@ -168,7 +180,7 @@ def oracle_sampled(q, k, v, lens_q, lens_k, heads, toks, hs, pv_mode="bf16", mod
     l = np.zeros(len(toks))
     oo, ll = oatt.attention_rows(qhat[order], seq_of_tok[order], hs[order],
                                  lambda i, h: kv(i, h)[0], lambda i, h: kv(i, h)[1], lens_k,
-                                 qd, kd, vd, p_mode="fp8" if pv_mode == "fp8" else "exact")
+                                 qd, kd, vd, p_mode=p_mode_of(pv_mode))
     o[order] = oo
     l[order] = ll
     return o, l

@@ -38,7 +38,7 @@ CASES = [
 ]
 
 
-@pytest.mark.parametrize("pv_mode", ["bf16", "fp8", "bf16v"])
+@pytest.mark.parametrize("pv_mode", ["bf16", "fp8", "bf16v", "mxfp8"])
 @pytest.mark.parametrize("case", range(len(CASES)))
 def test_attention_small_cases(pv_mode, case):
     lq, lk, H = CASES[case]
@@ -71,7 +71,7 @@ def test_attention_fp32_inputs():
     gu.assert_within(gu.compare_attention(o, lse, o_ref, lse_ref), "fp32 inputs")
 
 
-@pytest.mark.parametrize("pv_mode", ["bf16", "fp8", "bf16v"])
+@pytest.mark.parametrize("pv_mode", ["bf16", "fp8", "bf16v", "mxfp8"])
 def test_closed_forms(pv_mode):
     """Constant V gives V (bf16 PV) or V times one scalar per row (fp8 PV, where l sums the
     unrounded weights); equal logits give LSE = ln n + s and O = the mean of V."""
@@ -87,7 +87,7 @@ def test_closed_forms(pv_mode):
     o, lse = gu.run_path(lp, q, krand, vconst, [n], [n], H, pv_mode=pv_mode)
     qh, kh, vh = gu.oracle_inputs(q, krand, vconst, [n], [n], H, pv_mode)
     o_np = o.float().cpu().numpy().astype(np.float64)
-    if pv_mode != "fp8":
+    if pv_mode not in ("fp8", "mxfp8"):   # P rounded to 8 bits, l the unrounded sum: a ratio
         assert np.max(np.abs(o_np - vh[:1])) <= gu.O_MAX_ABS
     else:
         ratio = (o_np * vh[:1]).sum(axis=2) / (vh[:1] ** 2).sum(axis=2)      # (n, H)
@@ -98,7 +98,7 @@ def test_closed_forms(pv_mode):
     qh, kh, vh = gu.oracle_inputs(q, k, v, [n], [n], H, pv_mode)
     s = np.einsum("thd,hd->ht", qh, kh[0]) / math.sqrt(128)
     assert np.max(np.abs(lse.cpu().numpy() - (np.log(n) + s))) < gu.LSE_MAX_ABS
-    if pv_mode != "fp8":
+    if pv_mode not in ("fp8", "mxfp8"):
         assert np.max(np.abs(o.float().cpu().numpy() - vh.mean(axis=0)[None])) <= gu.O_MAX_ABS
 
 
@@ -111,7 +111,7 @@ def test_single_key():
     assert np.max(np.abs(lse.cpu().numpy() - s)) < gu.LSE_MAX_ABS
 
 
-@pytest.mark.parametrize("pv_mode", ["bf16", "fp8", "bf16v"])
+@pytest.mark.parametrize("pv_mode", ["bf16", "fp8", "bf16v", "mxfp8"])
 def test_unit_descale_is_bit_identical_and_two_changes_output(pv_mode):
     """vLLM #63232 'Validation': absent descale == unit descale bit for bit; 2 changes it."""
     w = wl.WORKLOADS["dense_4x2048_h16"]
@@ -139,7 +139,7 @@ def test_descale_values_match_oracle(descales):
     gu.assert_within(gu.compare_attention(o, lse, o_ref, lse_ref), f"descales {descales}")
 
 
-@pytest.mark.parametrize("pv_mode", ["bf16", "fp8", "bf16v"])
+@pytest.mark.parametrize("pv_mode", ["bf16", "fp8", "bf16v", "mxfp8"])
 def test_per_head_and_per_sequence_descales_match_oracle(pv_mode):
     """vLLM #63232 'Claims': per-head scales keep their descale tensors. q (H,), k (S, H) and
     v (1, H) descales, with negative and non-power-of-two values, against the oracle."""
@@ -192,7 +192,7 @@ def test_per_head_unit_descales_bit_identical_and_one_head_changes(pv_mode):
     _status_ok()
 
 
-@pytest.mark.parametrize("pv_mode", ["fp8", "bf16", "bf16v"])
+@pytest.mark.parametrize("pv_mode", ["fp8", "bf16", "bf16v", "mxfp8"])
 def test_repeated_runs_are_bit_identical(pv_mode):
     """The kernel's result does not depend on timing: repeated calls on the same inputs give the
     same bits (a barrier phase completed by the wrong warps once made fp8 PV rows differ)."""
@@ -209,6 +209,8 @@ def test_repeated_runs_are_bit_identical(pv_mode):
         vp, vs = lp.lpfa_cast_e4m3(gu.to_device(v, "bf16")), None
     elif pv_mode == "bf16v":
         vp, vs = gu.to_device(v, "bf16"), None
+    elif pv_mode == "mxfp8":
+        vp, vs = lp.lpfa_quantize_mxfp8_varlen(gu.to_device(v, "bf16"), mk, orientation="tokens")
     else:
         vp, vs = gu.gpu_quantize(lp, v, "bf16", mk)
     ref = None
@@ -238,7 +240,7 @@ def test_negative_control_wrong_k_scales_fail():
     assert lmax > gu.LSE_MAX_ABS and rel > gu.O_REL_L2
 
 
-@pytest.mark.parametrize("name", ["single_s256_h2", "dense_4x2048_h16", "dense_4x2048_h16_bf16v"])
+@pytest.mark.parametrize("name", ["single_s256_h2", "dense_4x2048_h16", "dense_4x2048_h16_bf16v", "dense_4x2048_h16_mxpv"])
 @pytest.mark.parametrize("mode", ["rceil", "floor"])
 def test_workload_full_check(name, mode):
     w = wl.WORKLOADS[name]
@@ -251,7 +253,8 @@ def test_workload_full_check(name, mode):
 
 
 @pytest.mark.slow
-@pytest.mark.parametrize("name", ["varlen16_fp32_h16", "video_s32768_h24_fp8pv", "cross_varlen_outliers_h32"])
+@pytest.mark.parametrize("name", ["varlen16_fp32_h16", "video_s32768_h24_fp8pv", "cross_varlen_outliers_h32",
+                                  "video_s32768_h24_mxpv"])
 def test_workload_sampled_check(name):
     """Full-size run in the benchmarked launch configuration, checked on sampled rows that
     cover every (sequence, head), each 128-row tile and every tail."""

@@ -37,7 +37,7 @@ def _guards_intact(buf: torch.Tensor, nbytes: int) -> bool:
     return bool(torch.all(head == PATTERN).item()) and bool(torch.all(tail == PATTERN).item())
 
 
-@pytest.mark.parametrize("pv_mode", ["fp8", "bf16", "bf16v"])
+@pytest.mark.parametrize("pv_mode", ["fp8", "bf16", "bf16v", "mxfp8"])
 def test_bounded_wait_runs_out_and_context_survives(pv_mode):
     lens, H = [300, 77], 2
     q, k, v = wl.small_random(11, lens, lens, H)
@@ -51,6 +51,8 @@ def test_bounded_wait_runs_out_and_context_survives(pv_mode):
         vp, vs = lp.lpfa_cast_e4m3(gu.to_device(v, "bf16")), None
     elif pv_mode == "bf16v":
         vp, vs = gu.to_device(v, "bf16"), None
+    elif pv_mode == "mxfp8":
+        vp, vs = lp.lpfa_quantize_mxfp8_varlen(gu.to_device(v, "bf16"), mk, orientation="tokens")
     else:
         vp, vs = gu.gpu_quantize(lp, v, "bf16", mk)
     assert lp.lpfa_device_status() == (lp.LPFA_OK, 0)
@@ -84,7 +86,7 @@ def test_unknown_debug_flag_rejected():
     assert e.value.status == lp.LPFA_ERR_INVALID_ARG
 
 
-@pytest.mark.parametrize("pv_mode", ["fp8", "bf16", "bf16v"])
+@pytest.mark.parametrize("pv_mode", ["fp8", "bf16", "bf16v", "mxfp8"])
 @pytest.mark.parametrize("lens_q,lens_k,H", [([1], [1], 1), ([300, 77, 1], [129, 700, 3], 3), ([2048], [257], 2)])
 def test_outputs_stay_inside_their_buffers(pv_mode, lens_q, lens_k, H):
     q, k, v = wl.small_random(3, lens_q, lens_k, H)
@@ -102,7 +104,7 @@ def test_outputs_stay_inside_their_buffers(pv_mode, lens_q, lens_k, H):
     kp = alloc("kp", Tk * H * 128).view(Tk, H, 128)
     ks = alloc("ks", mk.scale_bytes(H))
     vp = gu.to_device(v, "bf16") if pv_mode == "bf16v" else alloc("vp", Tk * H * 128).view(Tk, H, 128)
-    vs = None if pv_mode != "bf16" else alloc("vs", mk.scale_bytes(H))
+    vs = alloc("vs", mk.scale_bytes(H)) if pv_mode in ("bf16", "mxfp8") else None
     out = alloc("out", Tq * H * 128 * 2).view(torch.bfloat16).view(Tq, H, 128)
     lse = alloc("lse", H * Tq * 4).view(torch.float32).view(H, Tq)
 
@@ -112,6 +114,8 @@ def test_outputs_stay_inside_their_buffers(pv_mode, lens_q, lens_k, H):
         lp.lpfa_cast_e4m3(gu.to_device(v, "bf16"), out=vp)
     elif pv_mode == "bf16":
         lp.lpfa_quantize_mxfp8_varlen(gu.to_device(v, "bf16"), mk, payload=vp, scales=vs)
+    elif pv_mode == "mxfp8":
+        lp.lpfa_quantize_mxfp8_varlen(gu.to_device(v, "bf16"), mk, payload=vp, scales=vs, orientation="tokens")
     lp.lpfa_attn_fwd_varlen(qp, qs, kp, ks, vp, vs, mq, mk, pv_mode=pv_mode, out=out, lse=lse)
     torch.cuda.synchronize()
     assert lp.lpfa_device_status() == (lp.LPFA_OK, 0)

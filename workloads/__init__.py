@@ -41,7 +41,7 @@ class Workload:
     index: int                    # stable id mixed into the seed
     heads: int
     in_dtype: str                 # "bf16" or "fp32" (Q, K and the quantized V)
-    pv_mode: str                  # "bf16", "fp8", or "bf16v" (BF16 V input, bf16 PV)
+    pv_mode: str                  # "bf16", "fp8", "bf16v" (BF16 V input, bf16 PV) or "mxfp8" (block-scaled PV)
     scaling_mode: str = "rceil"   # "rceil" or "floor"
     num_seqs: int = 1
     len_q: Optional[int] = None   # fixed length, or None for drawn lengths
@@ -90,6 +90,15 @@ _add(Workload("dense_4x2048_h16_bf16v", 6, heads=16, in_dtype="bf16", pv_mode="b
               num_seqs=4, len_q=2048, len_k=2048,
               description="4 x 2048 uniform packed offsets, 16 heads, bf16 N(0,1); Q/K MXFP8 RCEIL, "
                           "V kept in BF16, bf16 PV"))
+
+_add(Workload("dense_4x2048_h16_mxpv", 7, heads=16, in_dtype="bf16", pv_mode="mxfp8",
+              num_seqs=4, len_q=2048, len_k=2048,
+              description="4 x 2048 uniform packed offsets, 16 heads, bf16 N(0,1); Q/K MXFP8 RCEIL, V MXFP8 "
+                          "in the token orientation, block-scaled MXFP8 PV"))
+_add(Workload("video_s32768_h24_mxpv", 8, heads=24, in_dtype="bf16", pv_mode="mxfp8",
+              num_seqs=1, len_q=32768, len_k=32768,
+              description="batch 1, 32768 tokens, 24 heads; Q/K bf16 N(0,1) MXFP8 RCEIL; V bf16 N(0,1) MXFP8 "
+                          "in the token orientation, block-scaled MXFP8 PV"))
 
 # The five evaluation workloads in order (the others are extra benchmark rows).
 EVAL_ORDER: List[str] = [
