@@ -288,6 +288,18 @@ __device__ __forceinline__ float rowmax128(const float2 (&s)[64]) {
   return fmaxf(max3f(b0, b1, b2), max3f(b3, b4, a[15]));
 }
 
+// rowmax128 that also returns the maxima of the four 32-key groups (16 pairs each).
+__device__ __forceinline__ float rowmax128_groups(const float2 (&s)[64], float (&gmax)[4]) {
+  float a[16];
+#pragma unroll
+  for (int k = 0; k < 16; ++k)
+    a[k] = max3f(max3f(s[4 * k].x, s[4 * k].y, s[4 * k + 1].x), max3f(s[4 * k + 1].y, s[4 * k + 2].x, s[4 * k + 2].y),
+                 fmaxf(s[4 * k + 3].x, s[4 * k + 3].y));
+#pragma unroll
+  for (int g = 0; g < 4; ++g) gmax[g] = fmaxf(max3f(a[4 * g], a[4 * g + 1], a[4 * g + 2]), a[4 * g + 3]);
+  return max3f(max3f(gmax[0], gmax[1], gmax[2]), gmax[3], gmax[3]);
+}
+
 // How many of a row's 64 exponential pairs are issued before a softmax group hands the MUFU
 // over to the other group (see the softmax loop). Handing over a little before the end
 // hides the hand-over latency behind the last exponentials.
@@ -327,6 +339,39 @@ __device__ __forceinline__ float exp_row(float2 (&s)[64], float c, float nb, int
   const float2 t1 = __fadd2_rn(__fadd2_rn(acc[4], acc[5]), __fadd2_rn(acc[6], acc[7]));
   const float2 t = __fadd2_rn(t0, t1);
   return t.x + t.y;
+}
+
+// exp_row for block-scaled MXFP8 P: group g (pairs [16g, 16g + 16)) uses its own bias nbg[g]
+// = nb - e_g, so the exponentials come out already scaled by the group's 2^-e_g (an integer
+// shift of the exponent). gsum[g] receives the sum of the group's scaled p.
+template <bool kTail, typename F>
+__device__ __forceinline__ void exp_row_groups(float2 (&s)[64], float c, const float (&nbg)[4], int key0, int klen,
+                                               F&& handoff, float (&gsum)[4]) {
+  const float2 c2 = make_float2(c, c);
+#pragma unroll
+  for (int i = 0; i < 64; ++i) s[i] = __ffma2_rn(s[i], c2, make_float2(nbg[i >> 4], nbg[i >> 4]));
+#pragma unroll
+  for (int i = 0; i < kHandoffPairs; ++i) s[i] = exp2_mufu2(s[i]);
+  handoff(s[kHandoffPairs - 1].y);
+#pragma unroll
+  for (int i = kHandoffPairs; i < 64; ++i) s[i] = exp2_mufu2(s[i]);
+  if (kTail) {
+#pragma unroll
+    for (int i = 0; i < 64; ++i) {
+      if (key0 + 2 * i >= klen) s[i].x = 0.0f;
+      if (key0 + 2 * i + 1 >= klen) s[i].y = 0.0f;
+    }
+  }
+#pragma unroll
+  for (int g = 0; g < 4; ++g) {
+    float2 acc[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) acc[k] = s[16 * g + k];
+#pragma unroll
+    for (int i = 16 * g + 4; i < 16 * g + 16; ++i) acc[i & 3] = __fadd2_rn(acc[i & 3], s[i]);
+    const float2 t = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
+    gsum[g] = t.x + t.y;
+  }
 }
 
 struct UnitInfo {
@@ -839,7 +884,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
         const bool tail = key0 + kTileN > ui.k_len;
         if (tail) mask_keys(sv, key0, ui.k_len);
         // Every tile has a valid key, so the ceiling is finite.
-        const float c_t = ceilf(rowmax128(sv) * cscale);
+        float gmax[4];  // block-scaled MXFP8 P: the 32-key group maxima of S
+        const float c_t = ceilf((kMx ? rowmax128_groups(sv, gmax) : rowmax128(sv)) * cscale);
         // Reference of tile t - 1 (the other group's). It is published after the other
         // group's exponentials of tile t - 1, so this wait also hands the MUFU over from one
         // group to the other: the two groups' exponential phases alternate instead of
@@ -857,8 +903,30 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
           __syncwarp();
           if (lane == 0) mbar_arrive_after(&bars[kBarMRef + grp * 4 + quarter], dep);
         };
-        const float psum = tail ? exp_row<true, kPolyPairs>(sv, cscale, kBias - m_t, key0, ui.k_len, handoff)
-                                : exp_row<false, kPolyPairs>(sv, cscale, kBias - m_t, key0, ui.k_len, handoff);
+        float psum;
+        uint32_t mx_sfw = 0;  // block-scaled MXFP8 P: this row's four E8M0 scale bytes
+        if (kMx) {
+          // Group g: the largest p is ex2(gmax * c + nb) (ex2 and the fma are monotonic), which
+          // picks 2^e_g (RCEIL); the exponentials then run with bias nb - e_g, giving p * 2^-e_g.
+          const float nb = kBias - m_t;
+          float nbg[4], gsum[4];
+          int eg[4];
+#pragma unroll
+          for (int g = 0; g < 4; ++g) {
+            eg[g] = e8m0_exponent(ex2_approx(fmaf(gmax[g], cscale, nb)), 0);
+            nbg[g] = nb - static_cast<float>(eg[g]);
+            mx_sfw |= static_cast<uint32_t>(eg[g] + 127) << (8 * g);
+          }
+          if (tail) exp_row_groups<true>(sv, cscale, nbg, key0, ui.k_len, handoff, gsum);
+          else exp_row_groups<false>(sv, cscale, nbg, key0, ui.k_len, handoff, gsum);
+          psum = 0.0f;
+#pragma unroll
+          for (int g = 0; g < 4; ++g)  // sum of the unscaled p: exact powers of two (2^-126 for an empty group)
+            psum += gsum[g] * __uint_as_float(static_cast<uint32_t>(max(eg[g], -126) + 127) << 23);
+        } else {
+          psum = tail ? exp_row<true, kPolyPairs>(sv, cscale, kBias - m_t, key0, ui.k_len, handoff)
+                      : exp_row<false, kPolyPairs>(sv, cscale, kBias - m_t, key0, ui.k_len, handoff);
+        }
         const float l_scale = exp2_int(m_g - m_t);
         l_g = l_g * l_scale + psum;
         if (!kP8) lr_g *= l_scale;
@@ -871,23 +939,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
             tc_fence_after();
           }
           if (kMx) {
-            // MXFP8 P: per 32 keys the group maximum picks 2^e (RCEIL; p >= 0 and masked keys are
-            // 0, an all-zero group gives e = -127), P = E4M3(p * 2^-e). The 4 scale bytes of this
-            // row go to the slot's shared-memory atom (row r at (r % 32) * 16 + (r / 32) * 4).
-            uint32_t sfw = 0;
-#pragma unroll
-            for (int g = 0; g < 4; ++g) {
-              float amax = 0.0f;
-#pragma unroll
-              for (int i = 16 * g; i < 16 * g + 16; ++i) amax = max3f(amax, sv[i].x, sv[i].y);
-              const int e = e8m0_exponent(amax, 0);
-              const float2 inv = make_float2(__uint_as_float(static_cast<uint32_t>(127 - e) << 23),
-                                             __uint_as_float(static_cast<uint32_t>(127 - e) << 23));
-#pragma unroll
-              for (int i = 16 * g; i < 16 * g + 16; ++i) sv[i] = __fmul2_rn(sv[i], inv);
-              sfw |= static_cast<uint32_t>(e + 127) << (8 * g);
-            }
-            p_sf_words[(t % kPSlots) * (kAtomBytes / 4) + (row & 31) * 4 + (row >> 5)] = sfw;
+            // MXFP8 P (already p * 2^-e_g from the exponentials, so at most ~448 per group; the
+            // conversion below saturates): the row's four scale bytes go to the slot's
+            // shared-memory atom (row r at (r % 32) * 16 + (r / 32) * 4).
+            p_sf_words[(t % kPSlots) * (kAtomBytes / 4) + (row & 31) * 4 + (row >> 5)] = mx_sfw;
             fence_proxy_async_smem();  // the PV issuer's tcgen05.cp reads the atom
           }
           uint32_t pk[32];
