@@ -232,6 +232,40 @@ LPFA_API lpfa_status lpfa_attn_fwd_varlen_descaled(const uint8_t* q, const uint8
                                           void* stream);
 
 /*
+ * mxfp8_flash_attn_varlen_backward (LP-FA4 README, "MXFP8 forward and backward"): the gradients
+ * of lpfa_attn_fwd_varlen's output with respect to the dequantized Q, K, V (quantization is not
+ * differentiated), noncausal head-dim-128 MHA over packed variable-length sequences:
+ *   P = exp(S - lse), dV = vd P^T dO, dP = vd dO V^T, D = rowsum(dO * O), dS = P * (dP - D),
+ *   dQ = c dS K, dK = c dS^T Q, with S = Q K^T * c and c = qd * kd / sqrt(128).
+ *
+ * q, q_sf, k, k_sf, v, v_sf   MXFP8 Q, K, V with head_dim-orientation scale storage (as the
+ *                  quantizer writes them; v_sf required).
+ * out_bf16, dout_bf16   device, (Tq, H, 128) bf16: the forward's O and the incoming gradient.
+ * lse              device, (H, Tq) fp32, the forward's natural-log LSE.
+ * meta_q, meta_k, heads, head_dim   as for lpfa_attn_fwd_varlen.
+ * q/k/v_descale    as for lpfa_attn_fwd_varlen_descaled (NULL descriptors or pointers: 1.0).
+ * dq_bf16          device, (Tq, H, 128) bf16 output.
+ * dk, dv           device, (Tk, H, 128): bf16 when output_mxfp8_dkv is 0; E4M3 payloads when it
+ *                  is 1, with E8M0 scales (one per 32 elements along head_dim, RCEIL) written to
+ *                  dk_sf and dv_sf in the quantizer's scale storage layout under meta_k.
+ * Alignment:       every tensor 16-byte aligned.
+ * Errors:          LPFA_ERR_INVALID_ARG for NULL required pointers (dk_sf/dv_sf when
+ *                  output_mxfp8_dkv), head_dim != 128, heads < 1, mismatched num_seqs, misalignment
+ *                  or a negative descale stride; LPFA_ERR_UNSUPPORTED off sm_100; LPFA_ERR_CUDA on
+ *                  launch failure; a kernel whose bounded wait runs out records LPFA_ERR_TIMEOUT.
+ * The library allocates nothing; two kernels (dK/dV per key tile, dQ per query tile) run on
+ * `stream`.
+ */
+LPFA_API lpfa_status lpfa_attn_bwd_varlen(const uint8_t* q, const uint8_t* q_sf, const uint8_t* k,
+                                 const uint8_t* k_sf, const uint8_t* v, const uint8_t* v_sf,
+                                 const void* out_bf16, const void* dout_bf16, const float* lse,
+                                 const lpfa_varlen_meta* meta_q, const lpfa_varlen_meta* meta_k,
+                                 int32_t heads, int32_t head_dim, const lpfa_descale* q_descale,
+                                 const lpfa_descale* k_descale, const lpfa_descale* v_descale,
+                                 void* dq_bf16, void* dk, void* dv, uint8_t* dk_sf, uint8_t* dv_sf,
+                                 int32_t output_mxfp8_dkv, void* stream);
+
+/*
  * Device status word. Kernels that bound their barrier waits record a failure code in a
  * library-owned device word instead of hanging. This call synchronizes `stream`, reads the
  * word of the current device, resets it to zero, and returns LPFA_OK, LPFA_ERR_TIMEOUT, or

@@ -38,7 +38,7 @@ EXPORTED_SYMBOLS = (
     "lpfa_meta_dev_ints", "lpfa_varlen_meta_fill_host", "lpfa_varlen_meta_from_lengths",
     "lpfa_scale_bytes", "lpfa_quantize_mxfp8_varlen", "lpfa_cast_e4m3", "lpfa_attn_fwd_varlen",
     "lpfa_device_status", "lpfa_last_error_message", "lpfa_version", "lpfa_attn_fwd_varlen_debug",
-    "lpfa_attn_fwd_varlen_descaled", "lpfa_quantize_mxfp8_varlen_tokens",
+    "lpfa_attn_fwd_varlen_descaled", "lpfa_quantize_mxfp8_varlen_tokens", "lpfa_attn_bwd_varlen",
 )
 
 
@@ -72,6 +72,9 @@ _lib.lpfa_quantize_mxfp8_varlen.argtypes = [_vp, ctypes.c_int, _i64, _i64, _i32,
 _lib.lpfa_quantize_mxfp8_varlen.restype = ctypes.c_int
 _lib.lpfa_quantize_mxfp8_varlen_tokens.argtypes = _lib.lpfa_quantize_mxfp8_varlen.argtypes
 _lib.lpfa_quantize_mxfp8_varlen_tokens.restype = ctypes.c_int
+_lib.lpfa_attn_bwd_varlen.argtypes = ([_vp] * 9 + [ctypes.POINTER(_Meta), ctypes.POINTER(_Meta), _i32, _i32] +
+                                      [ctypes.POINTER(_Descale)] * 3 + [_vp] * 5 + [_i32, _vp])
+_lib.lpfa_attn_bwd_varlen.restype = ctypes.c_int
 _lib.lpfa_cast_e4m3.argtypes = [_vp, _i64, _i64, _i64, _i32, _i32, _vp, _vp]
 _lib.lpfa_cast_e4m3.restype = ctypes.c_int
 _lib.lpfa_attn_fwd_varlen.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, ctypes.POINTER(_Meta), ctypes.POINTER(_Meta),
@@ -277,6 +280,54 @@ def lpfa_attn_fwd_varlen(q: torch.Tensor, q_sf: torch.Tensor, k: torch.Tensor, k
     return out, lse
 
 
+def lpfa_attn_bwd_varlen(q: torch.Tensor, q_sf: torch.Tensor, k: torch.Tensor, k_sf: torch.Tensor,
+                         v: torch.Tensor, v_sf: torch.Tensor, out: torch.Tensor, dout: torch.Tensor,
+                         lse: torch.Tensor, meta_q: VarlenMeta, meta_k: VarlenMeta,
+                         q_descale: Optional[torch.Tensor] = None, k_descale: Optional[torch.Tensor] = None,
+                         v_descale: Optional[torch.Tensor] = None, output_mxfp8_dkv: bool = False, stream=None):
+    """Attention backward (see include/lpfa.h). q/k/v with their head_dim-orientation scales, out and
+    dout bf16 (Tq,H,128), lse fp32 (H,Tq). Returns (dq, dk, dv) in bf16, or with output_mxfp8_dkv
+    (dq, dk_payload, dv_payload, dk_scales, dv_scales) like LP-FA4's mxfp8_flash_attn_varlen_backward.
+    """
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if t.dtype != torch.uint8 or t.dim() != 3 or not t.is_contiguous():
+            raise ValueError("%s must be a contiguous uint8 (tokens, heads, 128) tensor" % name)
+    for name, t in (("out", out), ("dout", dout)):
+        if t.dtype != torch.bfloat16 or t.shape != q.shape or not t.is_contiguous():
+            raise ValueError("%s must be a contiguous bf16 tensor shaped like q" % name)
+    Tq, H = q.shape[0], q.shape[1]
+    Tk = k.shape[0]
+    if lse.dtype != torch.float32 or tuple(lse.shape) != (H, Tq) or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous float32 (heads, tokens) tensor")
+    descs = []
+    for name, t in (("q_descale", q_descale), ("k_descale", k_descale), ("v_descale", v_descale)):
+        if t is None:
+            descs.append(_Descale(None, 0, 0))
+        else:
+            ss, hs = descale_strides(t, meta_q.num_seqs, H)
+            descs.append(_Descale(t.data_ptr(), ss, hs))
+    dq = torch.empty((Tq, H, 128), dtype=torch.bfloat16, device=q.device)
+    if output_mxfp8_dkv:
+        dk = torch.empty((Tk, H, 128), dtype=torch.uint8, device=q.device)
+        dv = torch.empty((Tk, H, 128), dtype=torch.uint8, device=q.device)
+        dk_sf = torch.empty(meta_k.scale_bytes(H), dtype=torch.uint8, device=q.device)
+        dv_sf = torch.empty(meta_k.scale_bytes(H), dtype=torch.uint8, device=q.device)
+    else:
+        dk = torch.empty((Tk, H, 128), dtype=torch.bfloat16, device=q.device)
+        dv = torch.empty((Tk, H, 128), dtype=torch.bfloat16, device=q.device)
+        dk_sf = dv_sf = None
+    with torch.cuda.device(q.device):
+        _check(_lib.lpfa_attn_bwd_varlen(q.data_ptr(), q_sf.data_ptr(), k.data_ptr(), k_sf.data_ptr(), v.data_ptr(),
+                                         v_sf.data_ptr(), out.data_ptr(), dout.data_ptr(), lse.data_ptr(),
+                                         ctypes.byref(meta_q._c), ctypes.byref(meta_k._c), H, 128,
+                                         ctypes.byref(descs[0]), ctypes.byref(descs[1]), ctypes.byref(descs[2]),
+                                         dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), _ptr(dk_sf), _ptr(dv_sf),
+                                         1 if output_mxfp8_dkv else 0, _stream_ptr(stream)))
+    if output_mxfp8_dkv:
+        return dq, dk, dv, dk_sf, dv_sf
+    return dq, dk, dv
+
+
 def lpfa_device_status(stream=None):
     """Synchronize `stream` and return (status, detail) of the device status word (then reset)."""
     detail = _i32(0)
@@ -288,4 +339,5 @@ def lpfa_device_status(stream=None):
 Mxfp8VarlenMeta = VarlenMeta
 quantize_mxfp8_varlen = lpfa_quantize_mxfp8_varlen
 mxfp8_flash_attn_varlen_forward = lpfa_attn_fwd_varlen
+mxfp8_flash_attn_varlen_backward = lpfa_attn_bwd_varlen
 fa4_v_to_fp8 = lpfa_cast_e4m3

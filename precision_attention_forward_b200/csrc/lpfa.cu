@@ -15,6 +15,7 @@
 
 #include "lpfa.h"
 #include "attn_fwd.cuh"
+#include "attn_bwd.cuh"
 #include "quantize.cuh"
 
 namespace {
@@ -464,6 +465,84 @@ lpfa_status lpfa_attn_fwd_varlen_descaled(const uint8_t* q, const uint8_t* q_sf,
                                           void* stream) {
   return attn_fwd_impl(q, q_sf, k, k_sf, v, v_sf, meta_q, meta_k, heads, head_dim, pv_mode, q_descale, k_descale,
                        v_descale, out_bf16, lse, stream, 0);
+}
+
+lpfa_status lpfa_attn_bwd_varlen(const uint8_t* q, const uint8_t* q_sf, const uint8_t* k, const uint8_t* k_sf,
+                                 const uint8_t* v, const uint8_t* v_sf, const void* out_bf16, const void* dout_bf16,
+                                 const float* lse, const lpfa_varlen_meta* meta_q, const lpfa_varlen_meta* meta_k,
+                                 int32_t heads, int32_t head_dim, const lpfa_descale* q_descale,
+                                 const lpfa_descale* k_descale, const lpfa_descale* v_descale, void* dq_bf16,
+                                 void* dk, void* dv, uint8_t* dk_sf, uint8_t* dv_sf, int32_t output_mxfp8_dkv,
+                                 void* stream) {
+  if (!q || !q_sf || !k || !k_sf || !v || !v_sf || !out_bf16 || !dout_bf16 || !lse || !dq_bf16 || !dk || !dv)
+    return fail(LPFA_ERR_INVALID_ARG, "NULL tensor pointer");
+  if (output_mxfp8_dkv != 0 && output_mxfp8_dkv != 1) return fail(LPFA_ERR_INVALID_ARG, "output_mxfp8_dkv must be 0 or 1");
+  if (output_mxfp8_dkv && (!dk_sf || !dv_sf)) return fail(LPFA_ERR_INVALID_ARG, "MXFP8 dK/dV need dk_sf and dv_sf");
+  if (head_dim != 128) return fail(LPFA_ERR_INVALID_ARG, "head_dim must be 128 (got %d)", head_dim);
+  if (heads < 1) return fail(LPFA_ERR_INVALID_ARG, "heads must be >= 1");
+  for (const lpfa_descale* d : {q_descale, k_descale, v_descale})
+    if (d && d->ptr && (d->seq_stride < 0 || d->head_stride < 0))
+      return fail(LPFA_ERR_INVALID_ARG, "descale strides must be >= 0");
+  lpfa_status st;
+  if ((st = check_meta(meta_q, "meta_q")) != LPFA_OK) return st;
+  if ((st = check_meta(meta_k, "meta_k")) != LPFA_OK) return st;
+  if (meta_q->num_seqs != meta_k->num_seqs)
+    return fail(LPFA_ERR_INVALID_ARG, "meta_q has %d sequences but meta_k has %d", meta_q->num_seqs, meta_k->num_seqs);
+  for (const void* ptr : {static_cast<const void*>(q), static_cast<const void*>(q_sf), static_cast<const void*>(k),
+                          static_cast<const void*>(k_sf), static_cast<const void*>(v), static_cast<const void*>(v_sf),
+                          out_bf16, dout_bf16, static_cast<const void*>(lse), static_cast<const void*>(dq_bf16),
+                          static_cast<const void*>(dk), static_cast<const void*>(dv)})
+    if (!aligned16(ptr)) return fail(LPFA_ERR_INVALID_ARG, "all tensors must be 16-byte aligned");
+  if (output_mxfp8_dkv && (!aligned16(dk_sf) || !aligned16(dv_sf)))
+    return fail(LPFA_ERR_INVALID_ARG, "all tensors must be 16-byte aligned");
+  const int64_t ku = static_cast<int64_t>(heads) * meta_k->total_scale_blocks;
+  const int64_t qu = static_cast<int64_t>(heads) * meta_q->total_scale_blocks;
+  if (ku > INT32_MAX || qu > INT32_MAX) return fail(LPFA_ERR_INVALID_ARG, "too many tiles");
+  DeviceInfo info;
+  if ((st = require_sm100(&info)) != LPFA_OK) return st;
+  void* one_addr = nullptr;
+  cudaError_t e = cudaGetSymbolAddress(&one_addr, lpfa::g_lpfa_one);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(g_lpfa_one)");
+  const float* one = static_cast<const float*>(one_addr);
+  auto descale = [one](const lpfa_descale* d) {
+    lpfa::Descale r{one, 0, 0};
+    if (d && d->ptr) r = lpfa::Descale{d->ptr, d->seq_stride, d->head_stride};
+    return r;
+  };
+  lpfa::BwdParams p;
+  p.q = q; p.q_sf = q_sf; p.k = k; p.k_sf = k_sf; p.v = v; p.v_sf = v_sf;
+  p.o = static_cast<const __nv_bfloat16*>(out_bf16);
+  p.dout = static_cast<const __nv_bfloat16*>(dout_bf16);
+  p.lse = lse;
+  p.cu_q = meta_q->dev;
+  p.so_q = meta_q->dev + meta_q->num_seqs + 1;
+  p.cu_k = meta_k->dev;
+  p.so_k = meta_k->dev + meta_k->num_seqs + 1;
+  p.q_descale = descale(q_descale);
+  p.k_descale = descale(k_descale);
+  p.v_descale = descale(v_descale);
+  p.dq = static_cast<__nv_bfloat16*>(dq_bf16);
+  p.dk = dk;
+  p.dv = dv;
+  p.dk_sf = dk_sf;
+  p.dv_sf = dv_sf;
+  p.num_seqs = meta_q->num_seqs;
+  p.heads = heads;
+  p.tq = meta_q->total_tokens;
+  p.total_q_tiles = meta_q->total_scale_blocks;
+  p.total_k_tiles = meta_k->total_scale_blocks;
+  p.mxfp8_dkv = output_mxfp8_dkv;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  for (const void* fn : {reinterpret_cast<const void*>(lpfa::attn_bwd_dkdv_kernel),
+                         reinterpret_cast<const void*>(lpfa::attn_bwd_dq_kernel)}) {
+    e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(lpfa::kBwdSmem));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+  }
+  if (ku > 0) lpfa::attn_bwd_dkdv_kernel<<<static_cast<unsigned>(ku), lpfa::kBwdThreads, lpfa::kBwdSmem, s>>>(p);
+  if (qu > 0) lpfa::attn_bwd_dq_kernel<<<static_cast<unsigned>(qu), lpfa::kBwdThreads, lpfa::kBwdSmem, s>>>(p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "backward launch");
+  return LPFA_OK;
 }
 
 lpfa_status lpfa_attn_fwd_varlen_debug(const uint8_t* q, const uint8_t* q_sf, const uint8_t* k, const uint8_t* k_sf,
