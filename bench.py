@@ -263,6 +263,73 @@ def config_dict(w, lq, lk, n):
     }
 
 
+def run_backward(args, w):
+    """--pass bwd: the attention backward (lpfa_attn_bwd_varlen) on the workload, one GPU.
+
+    A step is one backward call (its two kernels) on inputs already in HBM: MXFP8 Q/K/V in the
+    head_dim orientation, the forward's O and LSE, a seeded BF16 dO. value = algorithmic
+    TFLOPS, 10 * Sq * Sk * H * 128 (the five products; the dQ kernel recomputes S and dP, which
+    is not counted); the products run as BF16 MMAs, so the peak is the measured BF16 burst.
+    """
+    import torch
+
+    import precision_attention_forward_b200 as lp
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(0)
+    stream = torch.cuda.current_stream()
+    lq, lk = wl.lengths(w)
+    H = w.heads
+    flops = 2.5 * attention_flops(lq, lk, H)
+    peaks, peak_src = load_peaks()
+    host = {x: wl.make_tensor(w, x) for x in "qkv"}
+    mq = lp.lpfa_varlen_meta_from_lengths(lq, device=dev)
+    mk = lp.lpfa_varlen_meta_from_lengths(lk, device=dev)
+    q8, qs = lp.lpfa_quantize_mxfp8_varlen(wl.to_torch(host["q"], wl.tensor_dtype(w, "q"), device=dev), mq, w.scaling_mode)
+    k8, ks = lp.lpfa_quantize_mxfp8_varlen(wl.to_torch(host["k"], wl.tensor_dtype(w, "k"), device=dev), mk, w.scaling_mode)
+    v8, vs = lp.lpfa_quantize_mxfp8_varlen(wl.to_torch(host["v"], "bf16" if w.pv_mode == "fp8" else w.in_dtype, device=dev),
+                                           mk, w.scaling_mode)
+    out, lse = lp.lpfa_attn_fwd_varlen(q8, qs, k8, ks, v8, vs, mq, mk, pv_mode="bf16")
+    g = np.random.default_rng(7)
+    dout = wl.to_torch(wl.round_to_bf16(g.standard_normal(out.shape, dtype=np.float32)), "bf16", device=dev)
+    flush = not l2_exceeded(lk, H)
+    flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=dev) if flush else None
+    sampler = ClockSampler(0)
+    sampler.start()
+    for _ in range(args.warmup):
+        lp.lpfa_attn_bwd_varlen(q8, qs, k8, ks, v8, vs, out, dout, lse, mq, mk)
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(args.steps):
+        if flush:
+            flush_buf.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        lp.lpfa_attn_bwd_varlen(q8, qs, k8, ks, v8, vs, out, dout, lse, mq, mk)
+        b.record(stream)
+        times.append((a, b))
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    st, detail = lp.lpfa_device_status()
+    if st != lp.LPFA_OK:
+        raise RuntimeError(f"kernel reported status {st} (site {detail})")
+    ms = sum(a.elapsed_time(b) for a, b in times) / args.steps
+    value = flops / (ms * 1e-3) / 1e12
+    bf16_peak = peaks.get("bf16_tflops", FALLBACK_BF16_BURST)
+    cfg = config_dict(w, lq, lk, 1)
+    cfg["pass"] = "backward (dQ BF16, dK/dV BF16; MXFP8 Q/K/V head_dim orientation)"
+    print(json.dumps({
+        "metric": "MXFP8 attn-bwd TFLOPS (10*Sq*Sk*H*d)", "value": value, "unit": "TFLOPS", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": cfg,
+        "roofline": {"bound": "tensor", "achieved": value, "peak": bf16_peak, "unit": "TFLOP/s",
+                     "frac": value / bf16_peak, "traffic": None,
+                     "peak_source": f"{peak_src} bf16 burst", "kernel": "attn_bwd_dkdv_kernel + attn_bwd_dq_kernel",
+                     "flops_per_launch": flops},
+        "e2e": None, "gpu_launches": 2 * args.steps, "clocks": clocks, "cpu_baseline": None,
+    }))
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -272,12 +339,16 @@ def main():
     ap.add_argument("--impl", default="lpfa", choices=["lpfa", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--pass", dest="which", default="fwd", choices=["fwd", "bwd"],
+                    help="bwd: time the attention backward on one GPU instead of the forward step")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "lpfa":
         sys.stderr.write("note: fewer than 3 warm-up steps; numbers are for smoke use only\n")
     w = wl.WORKLOADS[args.workload]
     if args.impl == "reference":
         return run_reference(args, w)
+    if args.which == "bwd":
+        return run_backward(args, w)
 
     import torch
     import torch.distributed as dist
