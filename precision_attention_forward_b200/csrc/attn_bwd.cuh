@@ -8,24 +8,27 @@
 //   P = exp(S - LSE),  dV = vd P^T dO,  dP = vd dO V^T,  D = rowsum(dO * O),
 //   dS = P * (dP - D),  dQ = c dS K,  dK = c dS^T Q.
 //
-// Two kernels, no scratch memory:
+// Three kernels, no scratch memory:
+//   attn_bwd_d_kernel     D for every (token, head), written as fp32 into the dQ output buffer,
+//                         which nothing else reads or writes until the dQ kernel overwrites it.
 //   attn_bwd_dkdv_kernel  one CTA per 128-key tile of a (sequence, head): over the sequence's
 //                         query tiles it recomputes S^T = K Q^T and dP^T = V dO^T, forms P^T and
 //                         dS^T (one thread per key row) and accumulates dV += P^T dO and
-//                         dK += dS^T Q in tensor memory (S^T, dP^T, dV, dK: all 512 columns).
+//                         dK += dS^T Q in tensor memory.
 //   attn_bwd_dq_kernel    one CTA per 128-row query tile: over the key tiles it recomputes S and
-//                         dP, forms dS (one thread per query row) and accumulates dQ += dS K.
+//                         dP, forms dS (one thread per query row) and accumulates dQ += dS K; it
+//                         computes its own tile's D from dO and O.
 // Each CTA dequantizes its MXFP8 tiles to BF16 in shared memory (exact: E4M3 * 2^e is a BF16
-// value) and runs BF16 tcgen05 MMAs, so no scale factors are needed in tensor memory. D is
-// computed in each CTA from dO and O rather than stored.
+// value) and runs BF16 tcgen05 MMAs, so no scale factors are needed in tensor memory.
 //
-// Warp roles (256 threads): warps 0-3 compute (one tile row per thread: the MMA issue from warp
-// 0, the TMEM reads and writes of the row updates), warps 4-7 load. The loaders fill a
-// two-stage ring of the streamed tiles (Q, dO, D, LSE in the dK/dV kernel; K, V in the dQ
-// kernel) with coalesced loads, one 16-byte piece per lane, converting as they store; a stage
-// is released by a tcgen05.commit after the last MMA that reads it. The first MMA pair of a
-// step runs as two N = 64 halves, so the row updates start after the first half; the second MMA
-// pair is issued 32 columns at a time behind the row updates.
+// Warp roles (288 threads): warps 0-3 compute (one tile row per thread: the TMEM reads and writes
+// of the row updates), warp 4 issues the MMAs, warps 5-8 load. The loaders fill a two-stage ring
+// of the streamed tiles (Q, dO, D, LSE in the dK/dV kernel; K, V in the dQ kernel) with
+// coalesced 16-byte loads, converting as they store. A step over one streamed tile runs as two
+// halves of 64 columns, each with its own TMEM region (columns 0-127 and 128-255: S and dP as
+// fp32, then P and dS as BF16 over the columns already read): while the compute warps work on
+// one half, the tensor core runs the other half's MMAs, so S/dP of the next half and the
+// accumulating MMAs of the previous one overlap the row updates.
 #pragma once
 
 #include <cstdint>
@@ -37,7 +40,9 @@
 
 namespace lpfa {
 
-constexpr int kBwdThreads = 256;                 // warps 0-3 compute, warps 4-7 load
+constexpr int kBwdThreads = 288;                 // warps 0-3 compute, warp 4 MMA issue, warps 5-8 load
+constexpr int kBwdIssueWarp = 4;
+constexpr int kBwdLoadWarp0 = 5;
 constexpr int kBwdCompute = 128;                 // one compute thread per tile row
 constexpr uint32_t kBfTile = 128 * 128 * 2;      // a 128 x 128 BF16 tile in shared memory
 constexpr uint32_t kBfAtom = 128 * 128;          // one 64-column half of it (SW128 atom column)
@@ -130,7 +135,7 @@ constexpr uint64_t kBfHalfRows = (64 * 128) >> 4;
 constexpr float kBwdLog2e = 1.4426950408889634f;
 constexpr float kBwdRsqrtD = 0.08838834764831845f;  // 1 / sqrt(128)
 
-// Shared memory of both kernels (offsets from the 1024-aligned base):
+// Shared memory of the two tile kernels (offsets from the 1024-aligned base):
 //   [0, 64K)        the resident pair: K, V (dK/dV kernel) or Q, dO (dQ kernel), BF16 tiles
 //   [64K, 192K)     two stages of the streamed pair: Q, dO or K, V
 //   [192K, +2K)     per stage: LSE (log2 units) and D, 128 floats each (dK/dV kernel); stage 0
@@ -140,9 +145,18 @@ constexpr uint32_t kBwdOffStage = 2 * kBfTile;
 constexpr uint32_t kBwdStageBytes = 2 * kBfTile;
 constexpr uint32_t kBwdOffVec = kBwdOffStage + 2 * kBwdStageBytes;
 constexpr uint32_t kBwdOffBar = kBwdOffVec + 2 * 2 * 128 * 4;
-constexpr uint32_t kBwdNumBars = 8;
+constexpr uint32_t kBwdNumBars = 12;
 constexpr uint32_t kBwdSmem = kBwdOffBar + kBwdNumBars * 8 + 16 + 1024;
 static_assert(kBwdSmem <= 227 * 1024, "backward shared memory over the per-CTA limit");
+
+// Barrier indices. Arrival counts: the loaders' 128 threads (resident, stage full), the compute
+// warps' 128 threads (half ready), one tcgen05.commit (the others).
+constexpr int kBbResident = 0;   // resident pair (and the dQ kernel's D, LSE) in shared memory
+constexpr int kBbFull = 1;       // + stage: streamed tile in shared memory
+constexpr int kBbEmpty = 3;      // + stage: the last MMA that reads the stage is done
+constexpr int kBbSFull = 5;      // + half: S and dP of the half in TMEM
+constexpr int kBbPReady = 7;     // + half: P and dS of the half in TMEM (compute threads)
+constexpr int kBbRFree = 9;      // + half: the half's accumulating MMAs are done (region free)
 
 struct BwdSmem {
   uint8_t* base;
@@ -152,7 +166,6 @@ struct BwdSmem {
   __device__ uint8_t* st1(int s) const { return base + kBwdOffStage + s * kBwdStageBytes + kBfTile; }
   __device__ float* lse(int s) const { return reinterpret_cast<float*>(base + kBwdOffVec + s * 1024); }
   __device__ float* dvec(int s) const { return reinterpret_cast<float*>(base + kBwdOffVec + s * 1024 + 512); }
-  // barriers: 0 resident full, 1-2 stage full, 3-4 stage empty, 5-6 first-MMA halves, 7 second MMA
   __device__ uint64_t* bar(int i) const { return reinterpret_cast<uint64_t*>(base + kBwdOffBar) + i; }
   __device__ uint32_t* tslot() const { return reinterpret_cast<uint32_t*>(base + kBwdOffBar + kBwdNumBars * 8); }
   __device__ int* abort_flag() const { return reinterpret_cast<int*>(base + kBwdOffBar + kBwdNumBars * 8 + 8); }
@@ -199,15 +212,46 @@ __device__ __forceinline__ void bwd_store_rows(uint32_t taddr, float scale, int 
   }
 }
 
+// D = rowsum(dO * O) for every (token, head), as fp32 at dbuf[h * Tq + token] (the layout of
+// LSE). 16 lanes per row, 8 values per lane; a warp covers two consecutive rows.
+__global__ void __launch_bounds__(256) attn_bwd_d_kernel(const BwdParams p) {
+  float* dbuf = reinterpret_cast<float*>(p.dq);
+  const int64_t rows = static_cast<int64_t>(p.tq) * p.heads;
+  const int lane = threadIdx.x & 31;
+  const int64_t warp_step = static_cast<int64_t>(gridDim.x) * (256 / 32) * 2;
+  for (int64_t wr = (static_cast<int64_t>(blockIdx.x) * (256 / 32) + (threadIdx.x >> 5)) * 2; wr < rows;
+       wr += warp_step) {
+    const int64_t rr = wr + (lane >> 4);
+    const bool valid = rr < rows;
+    uint4 a = make_uint4(0u, 0u, 0u, 0u), b = a;
+    if (valid) {
+      a = __ldg(reinterpret_cast<const uint4*>(p.dout + rr * 128) + (lane & 15));
+      b = __ldg(reinterpret_cast<const uint4*>(p.o + rr * 128) + (lane & 15));
+    }
+    float d = bf8_dot(a, b);
+    d += __shfl_xor_sync(0xFFFFFFFFu, d, 8);
+    d += __shfl_xor_sync(0xFFFFFFFFu, d, 4);
+    d += __shfl_xor_sync(0xFFFFFFFFu, d, 2);
+    d += __shfl_xor_sync(0xFFFFFFFFu, d, 1);
+    if (valid && (lane & 15) == 0) {
+      const int64_t tok = rr / p.heads;
+      const int64_t h = rr - tok * p.heads;
+      dbuf[h * p.tq + tok] = d;
+    }
+  }
+}
+
 // ---------------------------------------------------------------------------------------------
-// Loaders (warps 4-7; loader warp lw fills rows [32 lw, 32 lw + 32) of a 128-row tile). Every
-// load of a tile is issued before the first store, one 16-byte piece per lane, so a warp has 24
-// (query tile) or 16 (key tile) loads in flight; rows >= n are written as zeros.
+// Loaders (warps 5-8; loader warp lw fills rows [32 lw, 32 lw + 32) of a 128-row tile). Every
+// load of a tile is issued before the first store, one 16-byte piece per lane; rows >= n are
+// written as zeros.
 // ---------------------------------------------------------------------------------------------
 
 // A query tile of head h from token tok0 (n rows): Q dequantized to BF16 with its scale atom sf,
-// dO copied, D = dO . O (fp32, lanes of a row reduce by shuffles) and LSE in log2 units (+inf
-// past the end, so that p = 0 there).
+// dO copied, LSE in log2 units (+inf past the end, so that p = 0 there) and D, read from the D
+// kernel's output (kDFromBuffer) or computed here from dO and O (lanes of a row reduce by
+// shuffles).
+template <bool kDFromBuffer>
 __device__ __forceinline__ void bwd_load_q_tile(const BwdParams& p, int64_t tok0, const uint8_t* sf, int h, int n,
                                                 uint8_t* sQ, uint8_t* sDO, float* sD, float* sLse, int lw,
                                                 int lane) {
@@ -224,20 +268,25 @@ __device__ __forceinline__ void bwd_load_q_tile(const BwdParams& p, int64_t tok0
       qs[it] = __ldg(reinterpret_cast<const uint32_t*>(sf) + (r & 31) * 4 + (r >> 5));
     }
   }
-  uint4 dv[16], ov[16];
+  uint4 dv[16], ov[kDFromBuffer ? 1 : 16];
 #pragma unroll
-  for (int it = 0; it < 16; ++it) {  // dO and O: 2 rows per step, 16 lanes x 8 values per row
+  for (int it = 0; it < 16; ++it) {  // dO (and O): 2 rows per step, 16 lanes x 8 values per row
     const int r = rb + 2 * it + (lane >> 4);
     dv[it] = make_uint4(0u, 0u, 0u, 0u);
-    ov[it] = dv[it];
+    if constexpr (!kDFromBuffer) ov[it] = dv[it];
     if (r < n) {
       const int64_t off = ((tok0 + r) * p.heads + h) * 128;
       dv[it] = __ldg(reinterpret_cast<const uint4*>(p.dout + off) + (lane & 15));
-      ov[it] = __ldg(reinterpret_cast<const uint4*>(p.o + off) + (lane & 15));
+      if constexpr (!kDFromBuffer) ov[it] = __ldg(reinterpret_cast<const uint4*>(p.o + off) + (lane & 15));
     }
   }
   const int rl = rb + lane;
-  const float lse2 = rl < n ? __ldg(p.lse + static_cast<int64_t>(h) * p.tq + tok0 + rl) * kBwdLog2e : INFINITY;
+  const int64_t vi = static_cast<int64_t>(h) * p.tq + tok0 + rl;
+  const float lse2 = rl < n ? __ldg(p.lse + vi) * kBwdLog2e : INFINITY;
+  float dval = 0.0f;
+  if constexpr (kDFromBuffer) {
+    if (rl < n) dval = __ldg(reinterpret_cast<const float*>(p.dq) + vi);
+  }
 #pragma unroll
   for (int it = 0; it < 8; ++it) {
     const int r = rb + 4 * it + (lane >> 3), c = lane & 7;  // codes [16c, 16c + 16): block c / 2
@@ -250,13 +299,16 @@ __device__ __forceinline__ void bwd_load_q_tile(const BwdParams& p, int64_t tok0
   for (int it = 0; it < 16; ++it) {
     const int r = rb + 2 * it + (lane >> 4), c = lane & 15;
     *reinterpret_cast<uint4*>(sDO + bf_tile_offset(r, c)) = dv[it];
-    float d = bf8_dot(dv[it], ov[it]);
-    d += __shfl_xor_sync(0xFFFFFFFFu, d, 8);
-    d += __shfl_xor_sync(0xFFFFFFFFu, d, 4);
-    d += __shfl_xor_sync(0xFFFFFFFFu, d, 2);
-    d += __shfl_xor_sync(0xFFFFFFFFu, d, 1);
-    if (c == 0) sD[r] = d;
+    if constexpr (!kDFromBuffer) {
+      float d = bf8_dot(dv[it], ov[it]);
+      d += __shfl_xor_sync(0xFFFFFFFFu, d, 8);
+      d += __shfl_xor_sync(0xFFFFFFFFu, d, 4);
+      d += __shfl_xor_sync(0xFFFFFFFFu, d, 2);
+      d += __shfl_xor_sync(0xFFFFFFFFu, d, 1);
+      if (c == 0) sD[r] = d;
+    }
   }
+  if constexpr (kDFromBuffer) sD[rl] = dval;
   sLse[rl] = lse2;
 }
 
@@ -295,10 +347,13 @@ __device__ __forceinline__ void bwd_load_kv_tile(const BwdParams& p, int64_t tok
   }
 }
 
-// Barrier setup and TMEM allocation shared by both kernels; returns the TMEM base address.
+// Barrier setup and TMEM allocation shared by both tile kernels; returns the TMEM base address.
 __device__ __forceinline__ uint32_t bwd_setup(const BwdSmem& sm, int tid, int warp) {
   if (tid == 0) {
-    for (int b = 0; b < static_cast<int>(kBwdNumBars); ++b) mbar_init(sm.bar(b), b <= 2 ? 128u : 1u);
+    for (int b = 0; b < static_cast<int>(kBwdNumBars); ++b) {
+      const bool threads = b == kBbResident || b == kBbFull || b == kBbFull + 1 || b == kBbPReady || b == kBbPReady + 1;
+      mbar_init(sm.bar(b), threads ? 128u : 1u);
+    }
     *sm.abort_flag() = 0;
     mbar_fence_init();
   }
@@ -309,19 +364,181 @@ __device__ __forceinline__ uint32_t bwd_setup(const BwdSmem& sm, int tid, int wa
   return *sm.tslot();
 }
 
-// A wait whose outcome the 128 compute threads share: true when every one of them succeeded
-// (named barrier 1), so that all of them take the same branch and none is left at a barrier.
-__device__ __forceinline__ bool bwd_group_ok(bool waited) { return !bar_red_or(1, kBwdCompute, !waited); }
-
 __device__ __forceinline__ void bwd_report(const BwdSmem& sm, int site) {
   *reinterpret_cast<volatile int*>(sm.abort_flag()) = 1;
   if (atomicCAS(&g_lpfa_status[0], 0, 4 /* LPFA_ERR_TIMEOUT */) == 0) atomicExch(&g_lpfa_status[1], site);
 }
 
-// dK and dV of one 128-key tile of one (sequence, head). TMEM columns: S^T 0-127 (P^T as BF16
-// over 0-63), dP^T 128-255 (dS^T over 128-191), dV 256-383, dK 384-511.
-// Barriers: 0 K/V loaded, 1-2 query stage loaded, 3-4 stage free, 5-6 S^T/dP^T halves done,
-// 7 dV/dK step done.
+// ---------------------------------------------------------------------------------------------
+// The pipeline shared by both tile kernels. kDkDv: the dK/dV kernel (resident K, V are the A
+// operands of S^T and dP^T; the streamed Q, dO the B operands), else the dQ kernel (resident Q,
+// dO; streamed K, V). Step i streams tile i; its half x covers columns [64 x, 64 x + 64) of S
+// (queries in the dK/dV kernel, keys in the dQ kernel) in TMEM region x (columns 128 x ...):
+//   128 x + [0, 64)    S (fp32), then P as BF16 over [0, 32) (dK/dV kernel) or dS (dQ kernel)
+//   128 x + [64, 128)  dP (fp32), then dS as BF16 over [64, 96) (dK/dV kernel)
+// Accumulators: dV 256-383 and dK 384-511 (dK/dV kernel), dQ 256-383 (dQ kernel).
+// ---------------------------------------------------------------------------------------------
+
+// MMA issue (warp 4). Order: S/dP of step 0 (both halves); then per step i and half x: the
+// accumulating MMAs of (i, x) once its P/dS are in TMEM, and S/dP of (i + 1, x) once those are
+// done with region x. Returns false when a wait ran out.
+template <bool kDkDv>
+__device__ __forceinline__ bool bwd_issue(const BwdSmem& sm, uint32_t tm, int n, int lane,
+                                          const volatile int* abort_flag) {
+  const uint32_t leader = lane == 0 ? 1u : 0u;
+  const uint32_t sb = smem_u32(sm.base);
+  const uint64_t a1 = umma_desc(sb, 16, 1024, kLayoutSw128);            // K, or Q
+  const uint64_t a2 = umma_desc(sb + kBfTile, 16, 1024, kLayoutSw128);  // V, or dO
+  constexpr uint32_t idS = idesc_bf16(false, false, 64), idM = idesc_bf16(false, true);
+  auto mma_s = [&](int i, int x) {  // S (or S^T) and dP (or dP^T) of half x of step i
+    const uint32_t st = sb + kBwdOffStage + (i & 1) * kBwdStageBytes;
+    const uint64_t b1 = umma_desc(st, 16, 1024, kLayoutSw128) + x * kBfHalfRows;
+    const uint64_t b2 = umma_desc(st + kBfTile, 16, 1024, kLayoutSw128) + x * kBfHalfRows;
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk)
+      mma_f16_ss(tm + 128 * x, bf_kmajor_step(a1, kk), bf_kmajor_step(b1, kk), idS, kk > 0 ? 1u : 0u, leader);
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk)
+      mma_f16_ss(tm + 128 * x + 64, bf_kmajor_step(a2, kk), bf_kmajor_step(b2, kk), idS, kk > 0 ? 1u : 0u, leader);
+    mma_commit(sm.bar(kBbSFull + x), leader);
+  };
+  auto mma_acc = [&](int i, int x) {  // the accumulating MMAs over the 64 columns of half x
+    const uint32_t st = sb + kBwdOffStage + (i & 1) * kBwdStageBytes;
+    const uint64_t m0 = umma_desc(st, kBfAtom, 1024, kLayoutSw128);            // Q, or K (MN-major)
+    const uint64_t m1 = umma_desc(st + kBfTile, kBfAtom, 1024, kLayoutSw128);  // dO
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) {
+      const uint32_t acc = (i > 0 || x > 0 || kk > 0) ? 1u : 0u;
+      if constexpr (kDkDv) {
+        mma_f16_ts(tm + 256, tm + 128 * x + 8 * kk, bf_mnmajor_step(m1, 4 * x + kk), idM, acc, leader);  // dV/vd += P^T dO
+        mma_f16_ts(tm + 384, tm + 128 * x + 64 + 8 * kk, bf_mnmajor_step(m0, 4 * x + kk), idM, acc,
+                   leader);                                                                              // dK/c += dS^T Q
+      } else {
+        mma_f16_ts(tm + 256, tm + 128 * x + 8 * kk, bf_mnmajor_step(m0, 4 * x + kk), idM, acc, leader);  // dQ/c += dS K
+      }
+    }
+    mma_commit(sm.bar(kBbRFree + x), leader);
+  };
+  if (!mbar_wait_warp(sm.bar(kBbResident), 0, abort_flag)) return false;
+  if (n == 0) return true;
+  if (!mbar_wait_warp(sm.bar(kBbFull), 0, abort_flag)) return false;
+  tc_fence_after();
+  mma_s(0, 0);
+  mma_s(0, 1);
+#pragma unroll 1
+  for (int i = 0; i < n; ++i) {
+    const int s = i & 1;
+    const uint32_t ph = static_cast<uint32_t>(i & 1);
+    if (!mbar_wait_warp(sm.bar(kBbPReady), ph, abort_flag)) return false;
+    tc_fence_after();
+    mma_acc(i, 0);
+    if (i + 1 < n) {
+      if (!mbar_wait_warp(sm.bar(kBbFull + (s ^ 1)), ((i + 1) >> 1) & 1, abort_flag)) return false;
+      if (!mbar_wait_warp(sm.bar(kBbRFree), ph, abort_flag)) return false;
+      tc_fence_after();
+      mma_s(i + 1, 0);
+    }
+    if (!mbar_wait_warp(sm.bar(kBbPReady + 1), ph, abort_flag)) return false;
+    tc_fence_after();
+    mma_acc(i, 1);
+    mma_commit(sm.bar(kBbEmpty + s), leader);  // the last MMA reading stage s
+    if (i + 1 < n) {
+      if (!mbar_wait_warp(sm.bar(kBbRFree + 1), ph, abort_flag)) return false;
+      tc_fence_after();
+      mma_s(i + 1, 1);
+    }
+  }
+  return true;
+}
+
+// Row updates (warps 0-3, thread r = TMEM lane r): for each step and half, P = exp2(S c2 - LSE)
+// and dS = P (vd dP - D) from TMEM back to TMEM as BF16. dK/dV kernel: rows are keys, columns
+// queries (LSE and D per column, from the stage); dQ kernel: rows are queries (LSE and D per
+// row), columns keys, the last tile's columns past last_cols masked. Ends when every MMA is done.
+template <bool kDkDv>
+__device__ __forceinline__ bool bwd_compute(const BwdSmem& sm, uint32_t tm, int n, int warp, int lane, float c2,
+                                            float vd, int last_cols, const volatile int* abort_flag) {
+  const int r = warp * 32 + lane;
+  const uint32_t lane_addr = static_cast<uint32_t>(warp * 32) << 16;
+  if (!mbar_wait_warp(sm.bar(kBbResident), 0, abort_flag)) return false;
+  float d_r = 0.0f, lse2 = 0.0f;
+  if constexpr (!kDkDv) {
+    d_r = sm.dvec(0)[r];
+    lse2 = sm.lse(0)[r];  // +inf past the sequence: p = 0
+  }
+#pragma unroll 1
+  for (int i = 0; i < n; ++i) {
+    const int s = i & 1;
+    // The stage's LSE and D (dK/dV kernel) are read directly from shared memory.
+    if (kDkDv && !mbar_wait_warp(sm.bar(kBbFull + s), (i >> 1) & 1, abort_flag)) return false;
+    const int cols = (!kDkDv && i == n - 1) ? last_cols : 128;
+#pragma unroll 1
+    for (int x = 0; x < 2; ++x) {
+      if (!mbar_wait_warp(sm.bar(kBbSFull + x), i & 1, abort_flag)) return false;
+      tc_fence_after();
+      const uint32_t reg = tm + lane_addr + 128 * x;
+#pragma unroll 1
+      for (int c = 0; c < 2; ++c) {
+        uint32_t sv[32], dv[32];
+        tmem_ld32x2_sync(reg + 32 * c, reg + 64 + 32 * c, sv, dv);
+        uint32_t dw[16];
+        if constexpr (kDkDv) {
+          const float* L = sm.lse(s) + 64 * x + 32 * c;
+          const float* D = sm.dvec(s) + 64 * x + 32 * c;
+          uint32_t pw[16];
+#pragma unroll
+          for (int e = 0; e < 32; e += 4) {
+            const float4 l4 = *reinterpret_cast<const float4*>(L + e);
+            const float4 d4 = *reinterpret_cast<const float4*>(D + e);
+            const float p0 = ex2_approx(fmaf(__uint_as_float(sv[e]), c2, -l4.x));
+            const float p1 = ex2_approx(fmaf(__uint_as_float(sv[e + 1]), c2, -l4.y));
+            const float p2 = ex2_approx(fmaf(__uint_as_float(sv[e + 2]), c2, -l4.z));
+            const float p3 = ex2_approx(fmaf(__uint_as_float(sv[e + 3]), c2, -l4.w));
+            pw[e / 2] = cvt_bf16x2(p0, p1);
+            pw[e / 2 + 1] = cvt_bf16x2(p2, p3);
+            dw[e / 2] = cvt_bf16x2(p0 * fmaf(vd, __uint_as_float(dv[e]), -d4.x),
+                                   p1 * fmaf(vd, __uint_as_float(dv[e + 1]), -d4.y));
+            dw[e / 2 + 1] = cvt_bf16x2(p2 * fmaf(vd, __uint_as_float(dv[e + 2]), -d4.z),
+                                       p3 * fmaf(vd, __uint_as_float(dv[e + 3]), -d4.w));
+          }
+          tmem_st16(reg + 16 * c, pw);
+          tmem_st16(reg + 64 + 16 * c, dw);
+        } else {
+          const int j0 = 64 * x + 32 * c;  // first key of the chunk within the tile
+          if (cols >= j0 + 32) {
+#pragma unroll
+            for (int e = 0; e < 32; e += 2) {
+              const float p0 = ex2_approx(fmaf(__uint_as_float(sv[e]), c2, -lse2));
+              const float p1 = ex2_approx(fmaf(__uint_as_float(sv[e + 1]), c2, -lse2));
+              dw[e / 2] = cvt_bf16x2(p0 * fmaf(vd, __uint_as_float(dv[e]), -d_r),
+                                     p1 * fmaf(vd, __uint_as_float(dv[e + 1]), -d_r));
+            }
+          } else {  // keys past the sequence's end contribute nothing
+#pragma unroll
+            for (int e = 0; e < 32; e += 2) {
+              float p0 = ex2_approx(fmaf(__uint_as_float(sv[e]), c2, -lse2));
+              float p1 = ex2_approx(fmaf(__uint_as_float(sv[e + 1]), c2, -lse2));
+              if (j0 + e >= cols) p0 = 0.0f;
+              if (j0 + e + 1 >= cols) p1 = 0.0f;
+              dw[e / 2] = cvt_bf16x2(p0 * fmaf(vd, __uint_as_float(dv[e]), -d_r),
+                                     p1 * fmaf(vd, __uint_as_float(dv[e + 1]), -d_r));
+            }
+          }
+          tmem_st16(reg + 16 * c, dw);
+        }
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(sm.bar(kBbPReady + x));
+    }
+  }
+  // The last commit follows every MMA of the CTA.
+  if (n > 0 && !mbar_wait_warp(sm.bar(kBbRFree + 1), (n - 1) & 1, abort_flag)) return false;
+  tc_fence_after();
+  return true;
+}
+
+// dK and dV of one 128-key tile of one (sequence, head).
 __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dkdv_kernel(const BwdParams p) {
   extern __shared__ uint8_t bsmem_raw[];
   const BwdSmem sm{reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(bsmem_raw) + 1023) & ~uintptr_t(1023))};
@@ -340,114 +557,33 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dkdv_kernel(const Bwd
 
   const uint32_t tm = bwd_setup(sm, tid, warp);
   const volatile int* abort_flag = sm.abort_flag();
-  bool ok = true;
 
-  if (warp >= 4) {
+  if (warp >= kBwdLoadWarp0) {
     // Loaders: K and V once, then the sequence's query tiles through the two stages.
-    const int lw = warp - 4;
+    const int lw = warp - kBwdLoadWarp0;
     bwd_load_kv_tile(p, k0 + kt * 128, k_atom, h, keys, sm.res0(), sm.res1(), lw, lane);
     fence_proxy_async_smem();
-    mbar_arrive(sm.bar(0));
+    mbar_arrive(sm.bar(kBbResident));
+    bool ok = true;
+#pragma unroll 1
     for (int i = 0; i < nq; ++i) {
       const int s = i & 1;
-      if (i >= 2 && !mbar_wait(sm.bar(3 + s), ((i >> 1) - 1) & 1, abort_flag)) { ok = false; break; }
-      bwd_load_q_tile(p, q0 + i * 128, p.q_sf + (static_cast<int64_t>(so_q + i) * p.heads + h) * 512, h,
-                      min(128, q_len - i * 128), sm.st0(s), sm.st1(s), sm.dvec(s), sm.lse(s), lw, lane);
+      if (i >= 2 && !mbar_wait_warp(sm.bar(kBbEmpty + s), ((i >> 1) - 1) & 1, abort_flag)) { ok = false; break; }
+      bwd_load_q_tile<true>(p, q0 + i * 128, p.q_sf + (static_cast<int64_t>(so_q + i) * p.heads + h) * 512, h,
+                            min(128, q_len - i * 128), sm.st0(s), sm.st1(s), sm.dvec(s), sm.lse(s), lw, lane);
       fence_proxy_async_smem();
-      mbar_arrive(sm.bar(1 + s));
+      mbar_arrive(sm.bar(kBbFull + s));
     }
-    if (!ok) bwd_report(sm, 202);
+    if (!ok && lane == 0) bwd_report(sm, 202);
+  } else if (warp == kBwdIssueWarp) {
+    if (!bwd_issue<true>(sm, tm, nq, lane, abort_flag) && lane == 0) bwd_report(sm, 204);
   } else {
     const int r = tid;  // this thread's key row (TMEM lane)
-    const uint32_t leader = lane == 0 ? 1u : 0u;
     const uint32_t lane_addr = static_cast<uint32_t>(warp * 32) << 16;
     const float c = descale_value(p.q_descale, seq, h) * descale_value(p.k_descale, seq, h) * kBwdRsqrtD;
-    const float c2 = c * kBwdLog2e;
     const float vd = descale_value(p.v_descale, seq, h);
-    const uint32_t sb = smem_u32(sm.base);
-    const uint64_t kK = umma_desc(sb, 16, 1024, kLayoutSw128);
-    const uint64_t kV = umma_desc(sb + kBfTile, 16, 1024, kLayoutSw128);
-    constexpr uint32_t idS = idesc_bf16(false, false, 64), idM = idesc_bf16(false, true);
-    ok = bwd_group_ok(mbar_wait(sm.bar(0), 0, abort_flag));
-    for (int i = 0; i < nq && ok; ++i) {
-      const int s = i & 1;
-      const uint32_t stq = sb + kBwdOffStage + s * kBwdStageBytes, stdo = stq + kBfTile;
-      bool waited = mbar_wait(sm.bar(1 + s), (i >> 1) & 1, abort_flag);
-      // The previous step's dV/dK MMAs read P^T and dS^T from the columns S^T and dP^T overwrite.
-      if (i > 0) waited = mbar_wait(sm.bar(7), (i - 1) & 1, abort_flag) && waited;
-      if (!bwd_group_ok(waited)) { ok = false; break; }
-      tc_fence_after();
-      if (warp == 0) {
-        const uint64_t kQ = umma_desc(stq, 16, 1024, kLayoutSw128), kDO = umma_desc(stdo, 16, 1024, kLayoutSw128);
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {  // queries [64 half, 64 half + 64)
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)  // S^T = K Q^T
-            mma_f16_ss(tm + 64 * half, bf_kmajor_step(kK, kk), bf_kmajor_step(kQ + half * kBfHalfRows, kk), idS,
-                       kk > 0 ? 1u : 0u, leader);
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)  // dP^T / vd = V dO^T
-            mma_f16_ss(tm + 128 + 64 * half, bf_kmajor_step(kV, kk), bf_kmajor_step(kDO + half * kBfHalfRows, kk),
-                       idS, kk > 0 ? 1u : 0u, leader);
-          mma_commit(sm.bar(5 + half), leader);
-        }
-      }
-      const float* L = sm.lse(s);
-      const float* D = sm.dvec(s);
-      const uint64_t mQ = umma_desc(stq, kBfAtom, 1024, kLayoutSw128);
-      const uint64_t mDO = umma_desc(stdo, kBfAtom, 1024, kLayoutSw128);
-#pragma unroll 1
-      for (int half = 0; half < 2; ++half) {
-        if (!bwd_group_ok(mbar_wait(sm.bar(5 + half), i & 1, abort_flag))) { ok = false; break; }
-        tc_fence_after();
-#pragma unroll 1
-        for (int cb = 2 * half; cb < 2 * half + 2; ++cb) {
-          // Row r: P^T and dS^T for queries [32 cb, 32 cb + 32); their BF16 words land on
-          // columns already read.
-          uint32_t sv[32], dv[32];
-          tmem_ld32x2_sync(tm + lane_addr + cb * 32, tm + lane_addr + 128 + cb * 32, sv, dv);
-          uint32_t pw[16], dw[16];
-#pragma unroll
-          for (int x = 0; x < 32; x += 4) {
-            const float4 l4 = *reinterpret_cast<const float4*>(L + cb * 32 + x);
-            const float4 d4 = *reinterpret_cast<const float4*>(D + cb * 32 + x);
-            const float p0 = ex2_approx(fmaf(__uint_as_float(sv[x]), c2, -l4.x));
-            const float p1 = ex2_approx(fmaf(__uint_as_float(sv[x + 1]), c2, -l4.y));
-            const float p2 = ex2_approx(fmaf(__uint_as_float(sv[x + 2]), c2, -l4.z));
-            const float p3 = ex2_approx(fmaf(__uint_as_float(sv[x + 3]), c2, -l4.w));
-            pw[x / 2] = cvt_bf16x2(p0, p1);
-            pw[x / 2 + 1] = cvt_bf16x2(p2, p3);
-            dw[x / 2] = cvt_bf16x2(p0 * fmaf(vd, __uint_as_float(dv[x]), -d4.x),
-                                   p1 * fmaf(vd, __uint_as_float(dv[x + 1]), -d4.y));
-            dw[x / 2 + 1] = cvt_bf16x2(p2 * fmaf(vd, __uint_as_float(dv[x + 2]), -d4.z),
-                                       p3 * fmaf(vd, __uint_as_float(dv[x + 3]), -d4.w));
-          }
-          tmem_st16(tm + lane_addr + cb * 16, pw);
-          tmem_st16(tm + lane_addr + 128 + cb * 16, dw);
-          tmem_wait_st();
-          tc_fence_before();
-          named_barrier_sync(2, kBwdCompute);
-          if (warp == 0) {
-            tc_fence_after();
-#pragma unroll
-            for (int kk = 2 * cb; kk < 2 * cb + 2; ++kk) {
-              const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
-              mma_f16_ts(tm + 256, tm + kk * 8, bf_mnmajor_step(mDO, kk), idM, acc, leader);        // dV/vd += P^T dO
-              mma_f16_ts(tm + 384, tm + 128 + kk * 8, bf_mnmajor_step(mQ, kk), idM, acc, leader);  // dK/c += dS^T Q
-            }
-            if (cb == 3) {
-              mma_commit(sm.bar(3 + s), leader);
-              mma_commit(sm.bar(7), leader);
-            }
-          }
-        }
-      }
-    }
-    if (ok && nq > 0) {
-      ok = bwd_group_ok(mbar_wait(sm.bar(7), (nq - 1) & 1, abort_flag));
-      tc_fence_after();
-    }
-    if (!ok && r == 0) bwd_report(sm, 200);
+    const bool ok = bwd_compute<true>(sm, tm, nq, warp, lane, c * kBwdLog2e, vd, 128, abort_flag);
+    if (!ok && lane == 0) bwd_report(sm, 200);
     // Epilogue: row r of dV and dK (no query tile: zeros).
     const int64_t out_row = static_cast<int64_t>(k0 + kt * 128 + r) * p.heads + h;
     if (!ok) {
@@ -478,10 +614,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dkdv_kernel(const Bwd
   }
 }
 
-// dQ of one 128-row query tile of one (sequence, head). TMEM columns: S 0-127, dP 128-255,
-// dQ 256-383, dS as BF16 384-447 (apart from S, so that the next step's S and dP MMAs need not
-// wait for this step's dQ MMAs). Barriers: 0 Q/dO/D/LSE loaded, 1-2 key stage loaded, 3-4 stage
-// free, 5-6 S/dP halves done, 7 dQ step done.
+// dQ of one 128-row query tile of one (sequence, head).
 __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dq_kernel(const BwdParams p) {
   extern __shared__ uint8_t bsmem_raw[];
   const BwdSmem sm{reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(bsmem_raw) + 1023) & ~uintptr_t(1023))};
@@ -499,115 +632,36 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dq_kernel(const BwdPa
 
   const uint32_t tm = bwd_setup(sm, tid, warp);
   const volatile int* abort_flag = sm.abort_flag();
-  bool ok = true;
 
-  if (warp >= 4) {
+  if (warp >= kBwdLoadWarp0) {
     // Loaders: the query tile (Q, dO, D, LSE) once, then the key tiles through the two stages.
-    const int lw = warp - 4;
-    bwd_load_q_tile(p, q0 + qt * 128, p.q_sf + (static_cast<int64_t>(__ldg(p.so_q + seq) + qt) * p.heads + h) * 512,
-                    h, qrows, sm.res0(), sm.res1(), sm.dvec(0), sm.lse(0), lw, lane);
+    const int lw = warp - kBwdLoadWarp0;
+    bwd_load_q_tile<false>(p, q0 + qt * 128,
+                           p.q_sf + (static_cast<int64_t>(__ldg(p.so_q + seq) + qt) * p.heads + h) * 512, h, qrows,
+                           sm.res0(), sm.res1(), sm.dvec(0), sm.lse(0), lw, lane);
     fence_proxy_async_smem();
-    mbar_arrive(sm.bar(0));
+    mbar_arrive(sm.bar(kBbResident));
+    bool ok = true;
+#pragma unroll 1
     for (int j = 0; j < nk; ++j) {
       const int s = j & 1;
-      if (j >= 2 && !mbar_wait(sm.bar(3 + s), ((j >> 1) - 1) & 1, abort_flag)) { ok = false; break; }
+      if (j >= 2 && !mbar_wait_warp(sm.bar(kBbEmpty + s), ((j >> 1) - 1) & 1, abort_flag)) { ok = false; break; }
       bwd_load_kv_tile(p, k0 + j * 128, (static_cast<int64_t>(so_k + j) * p.heads + h) * 512, h,
                        min(128, k_len - j * 128), sm.st0(s), sm.st1(s), lw, lane);
       fence_proxy_async_smem();
-      mbar_arrive(sm.bar(1 + s));
+      mbar_arrive(sm.bar(kBbFull + s));
     }
-    if (!ok) bwd_report(sm, 203);
+    if (!ok && lane == 0) bwd_report(sm, 203);
+  } else if (warp == kBwdIssueWarp) {
+    if (!bwd_issue<false>(sm, tm, nk, lane, abort_flag) && lane == 0) bwd_report(sm, 205);
   } else {
     const int r = tid;  // this thread's query row (TMEM lane)
-    const uint32_t leader = lane == 0 ? 1u : 0u;
     const uint32_t lane_addr = static_cast<uint32_t>(warp * 32) << 16;
     const float c = descale_value(p.q_descale, seq, h) * descale_value(p.k_descale, seq, h) * kBwdRsqrtD;
-    const float c2 = c * kBwdLog2e;
     const float vd = descale_value(p.v_descale, seq, h);
-    const uint32_t sb = smem_u32(sm.base);
-    const uint64_t kQ = umma_desc(sb, 16, 1024, kLayoutSw128);
-    const uint64_t kDO = umma_desc(sb + kBfTile, 16, 1024, kLayoutSw128);
-    constexpr uint32_t idS = idesc_bf16(false, false, 64), idM = idesc_bf16(false, true);
-    ok = bwd_group_ok(mbar_wait(sm.bar(0), 0, abort_flag));
-    const float d_r = sm.dvec(0)[r];
-    const float lse2 = sm.lse(0)[r];  // +inf past the sequence: p = 0
-    for (int j = 0; j < nk && ok; ++j) {
-      const int s = j & 1;
-      const int keys = min(128, k_len - j * 128);
-      const uint32_t stk = sb + kBwdOffStage + s * kBwdStageBytes, stv = stk + kBfTile;
-      if (!bwd_group_ok(mbar_wait(sm.bar(1 + s), (j >> 1) & 1, abort_flag))) { ok = false; break; }
-      tc_fence_after();
-      if (warp == 0) {
-        const uint64_t kK = umma_desc(stk, 16, 1024, kLayoutSw128), kV = umma_desc(stv, 16, 1024, kLayoutSw128);
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {  // keys [64 half, 64 half + 64)
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)  // S = Q K^T
-            mma_f16_ss(tm + 64 * half, bf_kmajor_step(kQ, kk), bf_kmajor_step(kK + half * kBfHalfRows, kk), idS,
-                       kk > 0 ? 1u : 0u, leader);
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)  // dP / vd = dO V^T
-            mma_f16_ss(tm + 128 + 64 * half, bf_kmajor_step(kDO, kk), bf_kmajor_step(kV + half * kBfHalfRows, kk),
-                       idS, kk > 0 ? 1u : 0u, leader);
-          mma_commit(sm.bar(5 + half), leader);
-        }
-      }
-      const uint64_t mK = umma_desc(stk, kBfAtom, 1024, kLayoutSw128);
-#pragma unroll 1
-      for (int half = 0; half < 2; ++half) {
-        bool waited = mbar_wait(sm.bar(5 + half), j & 1, abort_flag);
-        // The previous step's dQ MMAs read dS from the columns this step's dS overwrites.
-        if (half == 0 && j > 0) waited = mbar_wait(sm.bar(7), (j - 1) & 1, abort_flag) && waited;
-        if (!bwd_group_ok(waited)) { ok = false; break; }
-        tc_fence_after();
-#pragma unroll 1
-        for (int cb = 2 * half; cb < 2 * half + 2; ++cb) {
-          uint32_t sv[32], dv[32];
-          tmem_ld32x2_sync(tm + lane_addr + cb * 32, tm + lane_addr + 128 + cb * 32, sv, dv);
-          uint32_t dw[16];
-          if (keys >= 128) {
-#pragma unroll
-            for (int x = 0; x < 32; x += 2) {
-              const float p0 = ex2_approx(fmaf(__uint_as_float(sv[x]), c2, -lse2));
-              const float p1 = ex2_approx(fmaf(__uint_as_float(sv[x + 1]), c2, -lse2));
-              dw[x / 2] = cvt_bf16x2(p0 * fmaf(vd, __uint_as_float(dv[x]), -d_r),
-                                     p1 * fmaf(vd, __uint_as_float(dv[x + 1]), -d_r));
-            }
-          } else {  // the sequence's last key tile: keys past its end contribute nothing
-#pragma unroll
-            for (int x = 0; x < 32; x += 2) {
-              const int kj = cb * 32 + x;
-              float p0 = ex2_approx(fmaf(__uint_as_float(sv[x]), c2, -lse2));
-              float p1 = ex2_approx(fmaf(__uint_as_float(sv[x + 1]), c2, -lse2));
-              if (kj >= keys) p0 = 0.0f;
-              if (kj + 1 >= keys) p1 = 0.0f;
-              dw[x / 2] = cvt_bf16x2(p0 * fmaf(vd, __uint_as_float(dv[x]), -d_r),
-                                     p1 * fmaf(vd, __uint_as_float(dv[x + 1]), -d_r));
-            }
-          }
-          tmem_st16(tm + lane_addr + 384 + cb * 16, dw);
-          tmem_wait_st();
-          tc_fence_before();
-          named_barrier_sync(2, kBwdCompute);
-          if (warp == 0) {
-            tc_fence_after();
-#pragma unroll
-            for (int kk = 2 * cb; kk < 2 * cb + 2; ++kk)  // dQ / c += dS K
-              mma_f16_ts(tm + 256, tm + 384 + kk * 8, bf_mnmajor_step(mK, kk), idM, (j > 0 || kk > 0) ? 1u : 0u,
-                         leader);
-            if (cb == 3) {
-              mma_commit(sm.bar(3 + s), leader);
-              mma_commit(sm.bar(7), leader);
-            }
-          }
-        }
-      }
-    }
-    if (ok && nk > 0) {
-      ok = bwd_group_ok(mbar_wait(sm.bar(7), (nk - 1) & 1, abort_flag));
-      tc_fence_after();
-    }
-    if (!ok && r == 0) bwd_report(sm, 201);
+    const int last_cols = k_len - (nk - 1) * 128;
+    const bool ok = bwd_compute<false>(sm, tm, nk, warp, lane, c * kBwdLog2e, vd, last_cols, abort_flag);
+    if (!ok && lane == 0) bwd_report(sm, 201);
     const int64_t tok = q0 + qt * 128 + r;
     if (!ok) {
       // (outputs unspecified; the status word reports the failure)

@@ -6,6 +6,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cstdarg>
 #include <cstdint>
 #include <cstdio>
@@ -538,7 +539,13 @@ lpfa_status lpfa_attn_bwd_varlen(const uint8_t* q, const uint8_t* q_sf, const ui
     e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(lpfa::kBwdSmem));
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
   }
-  if (ku > 0) lpfa::attn_bwd_dkdv_kernel<<<static_cast<unsigned>(ku), lpfa::kBwdThreads, lpfa::kBwdSmem, s>>>(p);
+  if (ku > 0) {
+    // D into the dQ buffer first (read by the dK/dV kernel; the dQ kernel then overwrites it).
+    const int64_t rows = static_cast<int64_t>(meta_q->total_tokens) * heads;
+    const int64_t blocks = std::min<int64_t>((rows + 15) / 16, static_cast<int64_t>(info.sms) * 16);
+    if (blocks > 0) lpfa::attn_bwd_d_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(p);
+    lpfa::attn_bwd_dkdv_kernel<<<static_cast<unsigned>(ku), lpfa::kBwdThreads, lpfa::kBwdSmem, s>>>(p);
+  }
   if (qu > 0) lpfa::attn_bwd_dq_kernel<<<static_cast<unsigned>(qu), lpfa::kBwdThreads, lpfa::kBwdSmem, s>>>(p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "backward launch");
