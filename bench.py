@@ -266,7 +266,7 @@ def config_dict(w, lq, lk, n):
 def run_backward(args, w):
     """--pass bwd: the attention backward (lpfa_attn_bwd_varlen) on the workload, one GPU.
 
-    A step is one backward call (its two kernels) on inputs already in HBM: MXFP8 Q/K/V in the
+    A step is one backward call (its three kernels) on inputs already in HBM: MXFP8 Q/K/V in the
     head_dim orientation, the forward's O and LSE, a seeded BF16 dO. value = algorithmic
     TFLOPS, 10 * Sq * Sk * H * 128 (the five products; the dQ kernel recomputes S and dP, which
     is not counted); the products run as BF16 MMAs, so the peak is the measured BF16 burst.
@@ -324,9 +324,9 @@ def run_backward(args, w):
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": cfg,
         "roofline": {"bound": "tensor", "achieved": value, "peak": bf16_peak, "unit": "TFLOP/s",
                      "frac": value / bf16_peak, "traffic": None,
-                     "peak_source": f"{peak_src} bf16 burst", "kernel": "attn_bwd_dkdv_kernel + attn_bwd_dq_kernel",
+                     "peak_source": f"{peak_src} bf16 burst", "kernel": "attn_bwd_d_kernel + attn_bwd_dkdv_kernel + attn_bwd_dq_kernel",
                      "flops_per_launch": flops},
-        "e2e": None, "gpu_launches": 2 * args.steps, "clocks": clocks, "cpu_baseline": None,
+        "e2e": None, "gpu_launches": 3 * args.steps, "clocks": clocks, "cpu_baseline": None,
     }))
 
 

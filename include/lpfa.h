@@ -244,7 +244,9 @@ LPFA_API lpfa_status lpfa_attn_fwd_varlen_descaled(const uint8_t* q, const uint8
  * lse              device, (H, Tq) fp32, the forward's natural-log LSE.
  * meta_q, meta_k, heads, head_dim   as for lpfa_attn_fwd_varlen.
  * q/k/v_descale    as for lpfa_attn_fwd_varlen_descaled (NULL descriptors or pointers: 1.0).
- * dq_bf16          device, (Tq, H, 128) bf16 output.
+ * dq_bf16          device, (Tq, H, 128) bf16 output. Before dQ is written, its first Tq * H * 4
+ *                  bytes hold D = rowsum(dO * O) as fp32 for the dK/dV kernel, so it must not
+ *                  overlap any input.
  * dk, dv           device, (Tk, H, 128): bf16 when output_mxfp8_dkv is 0; E4M3 payloads when it
  *                  is 1, with E8M0 scales (one per 32 elements along head_dim, RCEIL) written to
  *                  dk_sf and dv_sf in the quantizer's scale storage layout under meta_k.
@@ -253,8 +255,8 @@ LPFA_API lpfa_status lpfa_attn_fwd_varlen_descaled(const uint8_t* q, const uint8
  *                  output_mxfp8_dkv), head_dim != 128, heads < 1, mismatched num_seqs, misalignment
  *                  or a negative descale stride; LPFA_ERR_UNSUPPORTED off sm_100; LPFA_ERR_CUDA on
  *                  launch failure; a kernel whose bounded wait runs out records LPFA_ERR_TIMEOUT.
- * The library allocates nothing; two kernels (dK/dV per key tile, dQ per query tile) run on
- * `stream`.
+ * The library allocates nothing; three kernels (D per row, dK/dV per key tile, dQ per query
+ * tile) run on `stream`.
  */
 LPFA_API lpfa_status lpfa_attn_bwd_varlen(const uint8_t* q, const uint8_t* q_sf, const uint8_t* k,
                                  const uint8_t* k_sf, const uint8_t* v, const uint8_t* v_sf,
