@@ -151,3 +151,34 @@ def test_descale_strides_views_and_rejects():
     for bad in (torch.ones(5), torch.ones(2, 4), torch.ones(3, 4, dtype=torch.float64), torch.ones(3, 4, 1)):
         with pytest.raises(ValueError):
             lp.descale_strides(bad, 3, 4)
+
+
+def _bwd(**over):
+    args = dict(q=FAKE, q_sf=FAKE, k=FAKE, k_sf=FAKE, v=FAKE, v_sf=FAKE, out=FAKE, dout=FAKE, lse=FAKE,
+                mq=_fake_meta(2, 300), mk=_fake_meta(2, 300), heads=4, head_dim=128, qd=None, kd=None, vd=None,
+                dq=FAKE, dk=FAKE, dv=FAKE, dk_sf=None, dv_sf=None, mx=0)
+    args.update(over)
+    st = lp._lib.lpfa_attn_bwd_varlen(args["q"], args["q_sf"], args["k"], args["k_sf"], args["v"], args["v_sf"],
+                                      args["out"], args["dout"], args["lse"], ctypes.byref(args["mq"]),
+                                      ctypes.byref(args["mk"]), args["heads"], args["head_dim"], args["qd"],
+                                      args["kd"], args["vd"], args["dq"], args["dk"], args["dv"], args["dk_sf"],
+                                      args["dv_sf"], args["mx"], None)
+    return st, lp._lib.lpfa_last_error_message().decode()
+
+
+@pytest.mark.parametrize("over,needle", [
+    (dict(q=None), "NULL"),
+    (dict(v_sf=None), "NULL"),
+    (dict(dq=None), "NULL"),
+    (dict(mx=2), "output_mxfp8_dkv"),
+    (dict(mx=1), "dk_sf"),                      # MXFP8 dK/dV without their scale buffers
+    (dict(head_dim=64), "head_dim"),
+    (dict(heads=0), "heads"),
+    (dict(mk=_fake_meta(3, 300)), "sequences"),
+    (dict(dq=FAKE + 8), "aligned"),
+    (dict(qd=ctypes.pointer(lp._Descale(FAKE, -1, 0))), "stride"),
+])
+def test_backward_argument_validation(over, needle):
+    st, msg = _bwd(**over)
+    assert st == lp.LPFA_ERR_INVALID_ARG
+    assert needle in msg
