@@ -24,11 +24,10 @@
 // Warp roles (288 threads): warps 0-3 compute (one tile row per thread: the TMEM reads and writes
 // of the row updates), warp 4 issues the MMAs, warps 5-8 load. The loaders fill a two-stage ring
 // of the streamed tiles (Q, dO, D, LSE in the dK/dV kernel; K, V in the dQ kernel) with
-// coalesced 16-byte loads, converting as they store. A step over one streamed tile runs as two
-// halves of 64 columns, each with its own TMEM region (columns 0-127 and 128-255: S and dP as
-// fp32, then P and dS as BF16 over the columns already read): while the compute warps work on
-// one half, the tensor core runs the other half's MMAs, so S/dP of the next half and the
-// accumulating MMAs of the previous one overlap the row updates.
+// coalesced 16-byte loads, converting as they store. Per step the S and dP MMAs run with N = 128
+// (a 64-column split measured 2-3x slower per flop on the tensor core); the accumulating MMAs
+// follow the row updates 32 columns at a time, and the next step's S/dP MMAs are issued as soon
+// as their TMEM columns are free.
 #pragma once
 
 #include <cstdint>
@@ -129,8 +128,6 @@ __device__ __forceinline__ uint64_t bf_kmajor_step(uint64_t base, int kk) {
 __device__ __forceinline__ uint64_t bf_mnmajor_step(uint64_t base, int kk) {
   return base + static_cast<uint64_t>(kk * (16 * 128 >> 4));
 }
-// Rows 64..127 of a K-major tile (the second N = 64 half): 64 rows of 128 bytes into each atom.
-constexpr uint64_t kBfHalfRows = (64 * 128) >> 4;
 
 constexpr float kBwdLog2e = 1.4426950408889634f;
 constexpr float kBwdRsqrtD = 0.08838834764831845f;  // 1 / sqrt(128)
@@ -150,13 +147,13 @@ constexpr uint32_t kBwdSmem = kBwdOffBar + kBwdNumBars * 8 + 16 + 1024;
 static_assert(kBwdSmem <= 227 * 1024, "backward shared memory over the per-CTA limit");
 
 // Barrier indices. Arrival counts: the loaders' 128 threads (resident, stage full), the compute
-// warps' 128 threads (half ready), one tcgen05.commit (the others).
+// warps' 128 threads (chunk ready), one tcgen05.commit (the others).
 constexpr int kBbResident = 0;   // resident pair (and the dQ kernel's D, LSE) in shared memory
 constexpr int kBbFull = 1;       // + stage: streamed tile in shared memory
 constexpr int kBbEmpty = 3;      // + stage: the last MMA that reads the stage is done
-constexpr int kBbSFull = 5;      // + half: S and dP of the half in TMEM
-constexpr int kBbPReady = 7;     // + half: P and dS of the half in TMEM (compute threads)
-constexpr int kBbRFree = 9;      // + half: the half's accumulating MMAs are done (region free)
+constexpr int kBbSFull = 5;      // S and dP of the step in TMEM
+constexpr int kBbChunk = 6;      // + chunk (4): the chunk's P and dS in TMEM (compute threads)
+constexpr int kBbRFree = 10;     // the step's accumulating MMAs are done
 
 struct BwdSmem {
   uint8_t* base;
@@ -351,7 +348,7 @@ __device__ __forceinline__ void bwd_load_kv_tile(const BwdParams& p, int64_t tok
 __device__ __forceinline__ uint32_t bwd_setup(const BwdSmem& sm, int tid, int warp) {
   if (tid == 0) {
     for (int b = 0; b < static_cast<int>(kBwdNumBars); ++b) {
-      const bool threads = b == kBbResident || b == kBbFull || b == kBbFull + 1 || b == kBbPReady || b == kBbPReady + 1;
+      const bool threads = b == kBbResident || b == kBbFull || b == kBbFull + 1 || (b >= kBbChunk && b < kBbChunk + 4);
       mbar_init(sm.bar(b), threads ? 128u : 1u);
     }
     *sm.abort_flag() = 0;
@@ -372,16 +369,21 @@ __device__ __forceinline__ void bwd_report(const BwdSmem& sm, int site) {
 // ---------------------------------------------------------------------------------------------
 // The pipeline shared by both tile kernels. kDkDv: the dK/dV kernel (resident K, V are the A
 // operands of S^T and dP^T; the streamed Q, dO the B operands), else the dQ kernel (resident Q,
-// dO; streamed K, V). Step i streams tile i; its half x covers columns [64 x, 64 x + 64) of S
-// (queries in the dK/dV kernel, keys in the dQ kernel) in TMEM region x (columns 128 x ...):
-//   128 x + [0, 64)    S (fp32), then P as BF16 over [0, 32) (dK/dV kernel) or dS (dQ kernel)
-//   128 x + [64, 128)  dP (fp32), then dS as BF16 over [64, 96) (dK/dV kernel)
-// Accumulators: dV 256-383 and dK 384-511 (dK/dV kernel), dQ 256-383 (dQ kernel).
+// dO; streamed K, V). Step i streams tile i. TMEM columns:
+//   0-127      S (fp32, 128 columns: queries in the dK/dV kernel, keys in the dQ kernel); the
+//              dK/dV kernel writes P^T as BF16 over 0-63
+//   128-255    dP (fp32); the dK/dV kernel writes dS^T as BF16 over 128-191
+//   256-383    dV (dK/dV kernel) or dQ (dQ kernel), fp32 accumulators
+//   384-511    dK (dK/dV kernel); the dQ kernel writes dS as BF16 over 384-447, apart from S and
+//              dP, so that the next step's S/dP MMAs only wait for the row updates to read them
+// The row updates go 32 columns at a time; each chunk's accumulating MMAs are issued as soon as
+// the chunk is in TMEM, behind the row updates of the next one.
 // ---------------------------------------------------------------------------------------------
 
-// MMA issue (warp 4). Order: S/dP of step 0 (both halves); then per step i and half x: the
-// accumulating MMAs of (i, x) once its P/dS are in TMEM, and S/dP of (i + 1, x) once those are
-// done with region x. Returns false when a wait ran out.
+// MMA issue (warp 4): S/dP of step 0; then per step i the accumulating MMAs chunk by chunk, and
+// S/dP of step i + 1 once region 0-255 is free (dK/dV kernel: the accumulating MMAs that read
+// P^T and dS^T there are done; dQ kernel: the row updates have read S and dP). Returns false
+// when a wait ran out.
 template <bool kDkDv>
 __device__ __forceinline__ bool bwd_issue(const BwdSmem& sm, uint32_t tm, int n, int lane,
                                           const volatile int* abort_flag) {
@@ -389,77 +391,69 @@ __device__ __forceinline__ bool bwd_issue(const BwdSmem& sm, uint32_t tm, int n,
   const uint32_t sb = smem_u32(sm.base);
   const uint64_t a1 = umma_desc(sb, 16, 1024, kLayoutSw128);            // K, or Q
   const uint64_t a2 = umma_desc(sb + kBfTile, 16, 1024, kLayoutSw128);  // V, or dO
-  constexpr uint32_t idS = idesc_bf16(false, false, 64), idM = idesc_bf16(false, true);
-  auto mma_s = [&](int i, int x) {  // S (or S^T) and dP (or dP^T) of half x of step i
+  constexpr uint32_t idS = idesc_bf16(false, false), idM = idesc_bf16(false, true);
+  auto mma_s = [&](int i) {  // S (or S^T) and dP (or dP^T) of step i, N = 128
     const uint32_t st = sb + kBwdOffStage + (i & 1) * kBwdStageBytes;
-    const uint64_t b1 = umma_desc(st, 16, 1024, kLayoutSw128) + x * kBfHalfRows;
-    const uint64_t b2 = umma_desc(st + kBfTile, 16, 1024, kLayoutSw128) + x * kBfHalfRows;
+    const uint64_t b1 = umma_desc(st, 16, 1024, kLayoutSw128);
+    const uint64_t b2 = umma_desc(st + kBfTile, 16, 1024, kLayoutSw128);
 #pragma unroll
     for (int kk = 0; kk < 8; ++kk)
-      mma_f16_ss(tm + 128 * x, bf_kmajor_step(a1, kk), bf_kmajor_step(b1, kk), idS, kk > 0 ? 1u : 0u, leader);
+      mma_f16_ss(tm, bf_kmajor_step(a1, kk), bf_kmajor_step(b1, kk), idS, kk > 0 ? 1u : 0u, leader);
 #pragma unroll
     for (int kk = 0; kk < 8; ++kk)
-      mma_f16_ss(tm + 128 * x + 64, bf_kmajor_step(a2, kk), bf_kmajor_step(b2, kk), idS, kk > 0 ? 1u : 0u, leader);
-    mma_commit(sm.bar(kBbSFull + x), leader);
-  };
-  auto mma_acc = [&](int i, int x) {  // the accumulating MMAs over the 64 columns of half x
-    const uint32_t st = sb + kBwdOffStage + (i & 1) * kBwdStageBytes;
-    const uint64_t m0 = umma_desc(st, kBfAtom, 1024, kLayoutSw128);            // Q, or K (MN-major)
-    const uint64_t m1 = umma_desc(st + kBfTile, kBfAtom, 1024, kLayoutSw128);  // dO
-#pragma unroll
-    for (int kk = 0; kk < 4; ++kk) {
-      const uint32_t acc = (i > 0 || x > 0 || kk > 0) ? 1u : 0u;
-      if constexpr (kDkDv) {
-        mma_f16_ts(tm + 256, tm + 128 * x + 8 * kk, bf_mnmajor_step(m1, 4 * x + kk), idM, acc, leader);  // dV/vd += P^T dO
-        mma_f16_ts(tm + 384, tm + 128 * x + 64 + 8 * kk, bf_mnmajor_step(m0, 4 * x + kk), idM, acc,
-                   leader);                                                                              // dK/c += dS^T Q
-      } else {
-        mma_f16_ts(tm + 256, tm + 128 * x + 8 * kk, bf_mnmajor_step(m0, 4 * x + kk), idM, acc, leader);  // dQ/c += dS K
-      }
-    }
-    mma_commit(sm.bar(kBbRFree + x), leader);
+      mma_f16_ss(tm + 128, bf_kmajor_step(a2, kk), bf_kmajor_step(b2, kk), idS, kk > 0 ? 1u : 0u, leader);
+    mma_commit(sm.bar(kBbSFull), leader);
   };
   if (!mbar_wait_warp(sm.bar(kBbResident), 0, abort_flag)) return false;
   if (n == 0) return true;
   if (!mbar_wait_warp(sm.bar(kBbFull), 0, abort_flag)) return false;
   tc_fence_after();
-  mma_s(0, 0);
-  mma_s(0, 1);
+  mma_s(0);
 #pragma unroll 1
   for (int i = 0; i < n; ++i) {
     const int s = i & 1;
     const uint32_t ph = static_cast<uint32_t>(i & 1);
-    if (!mbar_wait_warp(sm.bar(kBbPReady), ph, abort_flag)) return false;
-    tc_fence_after();
-    mma_acc(i, 0);
-    if (i + 1 < n) {
-      if (!mbar_wait_warp(sm.bar(kBbFull + (s ^ 1)), ((i + 1) >> 1) & 1, abort_flag)) return false;
-      if (!mbar_wait_warp(sm.bar(kBbRFree), ph, abort_flag)) return false;
+    const uint32_t st = sb + kBwdOffStage + s * kBwdStageBytes;
+    const uint64_t m0 = umma_desc(st, kBfAtom, 1024, kLayoutSw128);            // Q, or K (MN-major)
+    const uint64_t m1 = umma_desc(st + kBfTile, kBfAtom, 1024, kLayoutSw128);  // dO
+#pragma unroll 1
+    for (int c = 0; c < 4; ++c) {
+      if (!mbar_wait_warp(sm.bar(kBbChunk + c), ph, abort_flag)) return false;
       tc_fence_after();
-      mma_s(i + 1, 0);
+#pragma unroll
+      for (int kk = 2 * c; kk < 2 * c + 2; ++kk) {
+        const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
+        if constexpr (kDkDv) {
+          mma_f16_ts(tm + 256, tm + 8 * kk, bf_mnmajor_step(m1, kk), idM, acc, leader);        // dV/vd += P^T dO
+          mma_f16_ts(tm + 384, tm + 128 + 8 * kk, bf_mnmajor_step(m0, kk), idM, acc, leader);  // dK/c += dS^T Q
+        } else {
+          mma_f16_ts(tm + 256, tm + 384 + 8 * kk, bf_mnmajor_step(m0, kk), idM, acc, leader);  // dQ/c += dS K
+        }
+      }
     }
-    if (!mbar_wait_warp(sm.bar(kBbPReady + 1), ph, abort_flag)) return false;
-    tc_fence_after();
-    mma_acc(i, 1);
+    mma_commit(sm.bar(kBbRFree), leader);
     mma_commit(sm.bar(kBbEmpty + s), leader);  // the last MMA reading stage s
     if (i + 1 < n) {
-      if (!mbar_wait_warp(sm.bar(kBbRFree + 1), ph, abort_flag)) return false;
+      if (!mbar_wait_warp(sm.bar(kBbFull + (s ^ 1)), ((i + 1) >> 1) & 1, abort_flag)) return false;
+      if (kDkDv && !mbar_wait_warp(sm.bar(kBbRFree), ph, abort_flag)) return false;
       tc_fence_after();
-      mma_s(i + 1, 1);
+      mma_s(i + 1);
     }
   }
   return true;
 }
 
-// Row updates (warps 0-3, thread r = TMEM lane r): for each step and half, P = exp2(S c2 - LSE)
-// and dS = P (vd dP - D) from TMEM back to TMEM as BF16. dK/dV kernel: rows are keys, columns
-// queries (LSE and D per column, from the stage); dQ kernel: rows are queries (LSE and D per
-// row), columns keys, the last tile's columns past last_cols masked. Ends when every MMA is done.
+// Row updates (warps 0-3, thread r = TMEM lane r): per step, 32 columns at a time,
+// P = exp2(S c2 - LSE) and dS = P (vd dP - D) from TMEM back to TMEM as BF16. dK/dV kernel: rows
+// are keys, columns queries (LSE and D per column, from the stage); dQ kernel: rows are queries
+// (LSE and D per row), columns keys, the last tile's columns past last_cols masked. Ends when
+// every MMA is done.
 template <bool kDkDv>
 __device__ __forceinline__ bool bwd_compute(const BwdSmem& sm, uint32_t tm, int n, int warp, int lane, float c2,
                                             float vd, int last_cols, const volatile int* abort_flag) {
   const int r = warp * 32 + lane;
   const uint32_t lane_addr = static_cast<uint32_t>(warp * 32) << 16;
+  const uint32_t trow = tm + lane_addr;
   if (!mbar_wait_warp(sm.bar(kBbResident), 0, abort_flag)) return false;
   float d_r = 0.0f, lse2 = 0.0f;
   if constexpr (!kDkDv) {
@@ -471,69 +465,68 @@ __device__ __forceinline__ bool bwd_compute(const BwdSmem& sm, uint32_t tm, int 
     const int s = i & 1;
     // The stage's LSE and D (dK/dV kernel) are read directly from shared memory.
     if (kDkDv && !mbar_wait_warp(sm.bar(kBbFull + s), (i >> 1) & 1, abort_flag)) return false;
+    if (!mbar_wait_warp(sm.bar(kBbSFull), i & 1, abort_flag)) return false;
+    // dQ kernel: the previous step's dQ MMAs read dS from the columns this step's dS overwrites.
+    if (!kDkDv && i > 0 && !mbar_wait_warp(sm.bar(kBbRFree), (i - 1) & 1, abort_flag)) return false;
+    tc_fence_after();
     const int cols = (!kDkDv && i == n - 1) ? last_cols : 128;
 #pragma unroll 1
-    for (int x = 0; x < 2; ++x) {
-      if (!mbar_wait_warp(sm.bar(kBbSFull + x), i & 1, abort_flag)) return false;
-      tc_fence_after();
-      const uint32_t reg = tm + lane_addr + 128 * x;
-#pragma unroll 1
-      for (int c = 0; c < 2; ++c) {
-        uint32_t sv[32], dv[32];
-        tmem_ld32x2_sync(reg + 32 * c, reg + 64 + 32 * c, sv, dv);
-        uint32_t dw[16];
-        if constexpr (kDkDv) {
-          const float* L = sm.lse(s) + 64 * x + 32 * c;
-          const float* D = sm.dvec(s) + 64 * x + 32 * c;
-          uint32_t pw[16];
+    for (int c = 0; c < 4; ++c) {
+      uint32_t sv[32], dv[32];
+      tmem_ld32x2_sync(trow + 32 * c, trow + 128 + 32 * c, sv, dv);
+      uint32_t dw[16];
+      if constexpr (kDkDv) {
+        const float* L = sm.lse(s) + 32 * c;
+        const float* D = sm.dvec(s) + 32 * c;
+        uint32_t pw[16];
 #pragma unroll
-          for (int e = 0; e < 32; e += 4) {
-            const float4 l4 = *reinterpret_cast<const float4*>(L + e);
-            const float4 d4 = *reinterpret_cast<const float4*>(D + e);
-            const float p0 = ex2_approx(fmaf(__uint_as_float(sv[e]), c2, -l4.x));
-            const float p1 = ex2_approx(fmaf(__uint_as_float(sv[e + 1]), c2, -l4.y));
-            const float p2 = ex2_approx(fmaf(__uint_as_float(sv[e + 2]), c2, -l4.z));
-            const float p3 = ex2_approx(fmaf(__uint_as_float(sv[e + 3]), c2, -l4.w));
-            pw[e / 2] = cvt_bf16x2(p0, p1);
-            pw[e / 2 + 1] = cvt_bf16x2(p2, p3);
-            dw[e / 2] = cvt_bf16x2(p0 * fmaf(vd, __uint_as_float(dv[e]), -d4.x),
-                                   p1 * fmaf(vd, __uint_as_float(dv[e + 1]), -d4.y));
-            dw[e / 2 + 1] = cvt_bf16x2(p2 * fmaf(vd, __uint_as_float(dv[e + 2]), -d4.z),
-                                       p3 * fmaf(vd, __uint_as_float(dv[e + 3]), -d4.w));
-          }
-          tmem_st16(reg + 16 * c, pw);
-          tmem_st16(reg + 64 + 16 * c, dw);
-        } else {
-          const int j0 = 64 * x + 32 * c;  // first key of the chunk within the tile
-          if (cols >= j0 + 32) {
-#pragma unroll
-            for (int e = 0; e < 32; e += 2) {
-              const float p0 = ex2_approx(fmaf(__uint_as_float(sv[e]), c2, -lse2));
-              const float p1 = ex2_approx(fmaf(__uint_as_float(sv[e + 1]), c2, -lse2));
-              dw[e / 2] = cvt_bf16x2(p0 * fmaf(vd, __uint_as_float(dv[e]), -d_r),
-                                     p1 * fmaf(vd, __uint_as_float(dv[e + 1]), -d_r));
-            }
-          } else {  // keys past the sequence's end contribute nothing
-#pragma unroll
-            for (int e = 0; e < 32; e += 2) {
-              float p0 = ex2_approx(fmaf(__uint_as_float(sv[e]), c2, -lse2));
-              float p1 = ex2_approx(fmaf(__uint_as_float(sv[e + 1]), c2, -lse2));
-              if (j0 + e >= cols) p0 = 0.0f;
-              if (j0 + e + 1 >= cols) p1 = 0.0f;
-              dw[e / 2] = cvt_bf16x2(p0 * fmaf(vd, __uint_as_float(dv[e]), -d_r),
-                                     p1 * fmaf(vd, __uint_as_float(dv[e + 1]), -d_r));
-            }
-          }
-          tmem_st16(reg + 16 * c, dw);
+        for (int e = 0; e < 32; e += 4) {
+          const float4 l4 = *reinterpret_cast<const float4*>(L + e);
+          const float4 d4 = *reinterpret_cast<const float4*>(D + e);
+          const float p0 = ex2_approx(fmaf(__uint_as_float(sv[e]), c2, -l4.x));
+          const float p1 = ex2_approx(fmaf(__uint_as_float(sv[e + 1]), c2, -l4.y));
+          const float p2 = ex2_approx(fmaf(__uint_as_float(sv[e + 2]), c2, -l4.z));
+          const float p3 = ex2_approx(fmaf(__uint_as_float(sv[e + 3]), c2, -l4.w));
+          pw[e / 2] = cvt_bf16x2(p0, p1);
+          pw[e / 2 + 1] = cvt_bf16x2(p2, p3);
+          dw[e / 2] = cvt_bf16x2(p0 * fmaf(vd, __uint_as_float(dv[e]), -d4.x),
+                                 p1 * fmaf(vd, __uint_as_float(dv[e + 1]), -d4.y));
+          dw[e / 2 + 1] = cvt_bf16x2(p2 * fmaf(vd, __uint_as_float(dv[e + 2]), -d4.z),
+                                     p3 * fmaf(vd, __uint_as_float(dv[e + 3]), -d4.w));
         }
+        // Over columns already read: chunk c writes [16 c, 16 c + 16) of S^T and of dP^T.
+        tmem_st16(trow + 16 * c, pw);
+        tmem_st16(trow + 128 + 16 * c, dw);
+      } else {
+        const int j0 = 32 * c;  // first key of the chunk within the tile
+        if (cols >= j0 + 32) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const float p0 = ex2_approx(fmaf(__uint_as_float(sv[e]), c2, -lse2));
+            const float p1 = ex2_approx(fmaf(__uint_as_float(sv[e + 1]), c2, -lse2));
+            dw[e / 2] = cvt_bf16x2(p0 * fmaf(vd, __uint_as_float(dv[e]), -d_r),
+                                   p1 * fmaf(vd, __uint_as_float(dv[e + 1]), -d_r));
+          }
+        } else {  // keys past the sequence's end contribute nothing
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            float p0 = ex2_approx(fmaf(__uint_as_float(sv[e]), c2, -lse2));
+            float p1 = ex2_approx(fmaf(__uint_as_float(sv[e + 1]), c2, -lse2));
+            if (j0 + e >= cols) p0 = 0.0f;
+            if (j0 + e + 1 >= cols) p1 = 0.0f;
+            dw[e / 2] = cvt_bf16x2(p0 * fmaf(vd, __uint_as_float(dv[e]), -d_r),
+                                   p1 * fmaf(vd, __uint_as_float(dv[e + 1]), -d_r));
+          }
+        }
+        tmem_st16(trow + 384 + 16 * c, dw);
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(sm.bar(kBbPReady + x));
+      mbar_arrive(sm.bar(kBbChunk + c));
     }
   }
   // The last commit follows every MMA of the CTA.
-  if (n > 0 && !mbar_wait_warp(sm.bar(kBbRFree + 1), (n - 1) & 1, abort_flag)) return false;
+  if (n > 0 && !mbar_wait_warp(sm.bar(kBbRFree), (n - 1) & 1, abort_flag)) return false;
   tc_fence_after();
   return true;
 }
