@@ -42,7 +42,6 @@ namespace lpfa {
 constexpr int kBwdThreads = 288;                 // warps 0-3 compute, warp 4 MMA issue, warps 5-8 load
 constexpr int kBwdIssueWarp = 4;
 constexpr int kBwdLoadWarp0 = 5;
-constexpr int kBwdCompute = 128;                 // one compute thread per tile row
 constexpr uint32_t kBfTile = 128 * 128 * 2;      // a 128 x 128 BF16 tile in shared memory
 constexpr uint32_t kBfAtom = 128 * 128;          // one 64-column half of it (SW128 atom column)
 
