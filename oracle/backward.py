@@ -89,3 +89,26 @@ def attention_bwd(qhat, khat, vhat, o, do, lse, lengths_q, lengths_k, qd=1.0, kd
 def quantize_dkv(dk, dv, lengths_k, mode: str = "rceil"):
     """output_mxfp8_dkv: dK and dV as MXFP8 in the head_dim orientation (payload, scales) each."""
     return _mx.quantize_mxfp8_varlen(dk, lengths_k, mode), _mx.quantize_mxfp8_varlen(dv, lengths_k, mode)
+
+
+def attend_block_backward_sampled(q, k, v, o, do, lse, key_idx, row_idx, qd=1.0, kd=1.0, vd=1.0):
+    """Selected gradient rows of one (sequence, head), each from the same definition as
+    attend_block_backward, without forming the whole score matrix: dK and dV for the keys
+    key_idx (each needs one column of S over all query rows), dQ for the query rows row_idx (each
+    needs one row of S over all keys). Returns (dQ[row_idx], dK[key_idx], dV[key_idx])."""
+    q, k, v, o, do = (np.asarray(a, dtype=np.float64) for a in (q, k, v, o, do))
+    lse = np.asarray(lse, dtype=np.float64)
+    key_idx = np.asarray(key_idx, dtype=np.int64)
+    row_idx = np.asarray(row_idx, dtype=np.int64)
+    c = float(qd) * float(kd) / math.sqrt(HEAD_DIM)
+    d = np.sum(do * o, axis=1)
+    # columns j of S, P, dP, dS over every query row
+    p_c = np.exp((q @ k[key_idx].T) * c - lse[:, None])
+    ds_c = p_c * (float(vd) * (do @ v[key_idx].T) - d[:, None])
+    dv = float(vd) * (p_c.T @ do)
+    dk = c * (ds_c.T @ q)
+    # rows r of S, P, dP, dS over every key
+    p_r = np.exp((q[row_idx] @ k.T) * c - lse[row_idx, None])
+    ds_r = p_r * (float(vd) * (do[row_idx] @ v.T) - d[row_idx, None])
+    dq = c * (ds_r @ k)
+    return dq, dk, dv

@@ -12,6 +12,7 @@ import torch
 
 import workloads as wl
 from oracle import attention as oatt
+from oracle import backward as obwd
 from oracle import meta as ometa
 from oracle import mxfp8 as omx
 
@@ -184,3 +185,17 @@ def oracle_sampled(q, k, v, lens_q, lens_k, heads, toks, hs, pv_mode="bf16", mod
     o[order] = oo
     l[order] = ll
     return o, l
+
+
+def sampled_backward_reference(q, k, v, o, do, lse, lens_q, lens_k, h, keys, rows, mode="rceil"):
+    """Oracle dQ[rows], dK[keys], dV[keys] of head h of a one-sequence problem, from the oracle's
+    own MXFP8 quantization of that head (scales are per (token, head, 32 elements), so one head
+    quantizes alone) and the definition evaluated row by row. o, do: (T, H, 128); lse: (H, T)."""
+    assert len(lens_q) == 1 and len(lens_k) == 1, "one sequence"
+    deq = []
+    for x, lens in ((q, lens_q), (k, lens_k), (v, lens_k)):
+        p, s = omx.quantize_mxfp8_varlen(np.ascontiguousarray(x[:, h:h + 1, :]), lens, mode)
+        deq.append(omx.dequantize_mxfp8(p, s, lens, 1)[:, 0, :])
+    return obwd.attend_block_backward_sampled(deq[0], deq[1], deq[2], np.asarray(o[:, h], dtype=np.float64),
+                                              np.asarray(do[:, h], dtype=np.float64),
+                                              np.asarray(lse[h], dtype=np.float64), keys, rows)

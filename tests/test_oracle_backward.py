@@ -92,3 +92,53 @@ def test_mxfp8_dkv_output_round_trip():
         bmax = np.abs(x).reshape(103, 2, 4, 32).max(axis=3, keepdims=True)
         err = np.abs(xh - x).reshape(103, 2, 4, 32)
         assert np.all(err <= bmax * 2.0 ** -4 + 1e-300)
+
+
+def test_sampled_rows_match_full_backward_and_finite_differences():
+    """attend_block_backward_sampled: its rows equal the full backward's on a case with descales,
+    and its dK/dQ rows match central differences of the forward definition."""
+    g = np.random.default_rng(71)
+    q, k, v = g.standard_normal((37, 128)), g.standard_normal((29, 128)), g.standard_normal((29, 128))
+    do = g.standard_normal((37, 128))
+    qd, kd, vd = 0.8, 1.1, -0.6
+    o, lse = oatt.attend_block(q, k, v, qd, kd, vd)
+    keys, rows = [0, 5, 28], [0, 17, 36]
+    sq, sk, sv = obwd.attend_block_backward_sampled(q, k, v, o, do, lse, keys, rows, qd, kd, vd)
+    fq, fk, fv = obwd.attend_block_backward(q, k, v, o, do, lse, qd, kd, vd)
+    np.testing.assert_allclose(sq, fq[rows], rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(sk, fk[keys], rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(sv, fv[keys], rtol=1e-12, atol=1e-12)
+    eps = 1e-6
+    for name, x, grad, idx_rows in (("q", q, sq, rows), ("k", k, sk, keys), ("v", v, sv, keys)):
+        for t, row in enumerate(idx_rows):
+            col = int(g.integers(128))
+            xp, xm = x.copy(), x.copy()
+            xp[row, col] += eps
+            xm[row, col] -= eps
+            args = {"q": q, "k": k, "v": v}
+            lp_ = _loss(*(xp if n == name else args[n] for n in "qkv"), do, qd, kd, vd)
+            lm_ = _loss(*(xm if n == name else args[n] for n in "qkv"), do, qd, kd, vd)
+            num = (lp_ - lm_) / (2 * eps)
+            assert abs(num - grad[t, col]) <= 1e-6 * max(1.0, abs(num)), (name, row, col, num, grad[t, col])
+
+
+def test_sampled_reference_helper_matches_full_oracle():
+    """tests.gpu_util.sampled_backward_reference (used at the video shape on the GPU): per-head
+    quantization and sampled rows equal the full varlen oracle's rows on a small two-head case."""
+    from tests import gpu_util as gu
+    import workloads as wl
+
+    lq, lk, H = [300], [260], 2
+    q, k, v = wl.small_random(5, lq, lk, H)
+    qh, kh, vh = gu.oracle_inputs(q, k, v, lq, lk, H)
+    o_full, lse = oatt.attention_fwd(qh, kh, vh, lq, lk)
+    g = np.random.default_rng(6)
+    o = o_full.astype(np.float32)
+    do = g.standard_normal(q.shape).astype(np.float32)
+    fq, fk, fv = obwd.attention_bwd(qh, kh, vh, o.astype(np.float64), do.astype(np.float64), lse, lq, lk)
+    keys, rows = [0, 127, 128, 259], [0, 1, 255, 299]
+    for h in range(H):
+        sq, sk, sv = gu.sampled_backward_reference(q, k, v, o, do, lse, lq, lk, h, keys, rows)
+        np.testing.assert_allclose(sq, fq[rows, h], rtol=1e-10, atol=1e-12)
+        np.testing.assert_allclose(sk, fk[keys, h], rtol=1e-10, atol=1e-12)
+        np.testing.assert_allclose(sv, fv[keys, h], rtol=1e-10, atol=1e-12)
