@@ -18,7 +18,7 @@ to the dequantized inputs, for one (sequence, head) with query rows r and keys j
     dS_rj = p_rj * (dP_rj - D_r)
     dQ_r  = c * sum_j dS_rj k_j,    dK_j = c * sum_r dS_rj q_r
 
-Readings: quantization is not differentiated (the gradients are those of the
+Readings taken where the pages are silent: quantization is not differentiated (the gradients are those of the
 dequantized inputs, the straight-through reading); MXFP8 dK and dV use the head_dim orientation
 (one scale per 32 elements along head_dim of a token row, as the forward's inputs) and RCEIL
 (the README's default scaling).

@@ -7,7 +7,7 @@ What the pages fix (LP-FA4 README, "MXFP8 forward and backward"):
 FastVideo PR #1654 (description): the fp8 PV mode feeds V as an unscaled E4M3
 cast, with no scale factors and an implicit dequant scale of 1.0.
 
-Readings taken where the pages are silent (each is listed in the design doc):
+Readings taken where the pages are silent:
 * E4M3 is the OCP "fn" variant: bias 7, no infinities, 0x7F/0xFF are NaN,
   largest finite 448, smallest normal 2^-6, subnormals k * 2^-9.
 * Encoding rounds the exact value to the nearest E4M3 value, ties to the even
@@ -181,7 +181,7 @@ def quantize_mxfp8_varlen_tokens(x, lengths, mode: str = "rceil"):
     LP-FA4 README ("MXFP8 forward and backward"): Q, K and V keep both hardware orientations
     needed across forward and backward; this is the second one, with the 32-element blocks along
     the token axis, as the PV product (K = keys) and the backward's transposed products read
-    them. Readings: the 32-token groups are aligned to the start of each sequence,
+    them. Readings taken where the pages are silent: the 32-token groups are aligned to the start of each sequence,
     4 per 128-token block; a group's amax is taken over the tokens the sequence has (a partial
     last group is not padded with data); a group with no token of the sequence holds 0x7F.
     Scale storage: the 512-byte atom of (sequence i, 128-token block b, head h) at
