@@ -40,19 +40,29 @@ FP8_OVER_BF16 = 2.0                  # nominal dense FP8 / BF16 tensor ratio
 FALLBACK_BF16_BURST = 1590.0         # used only when MEASURED_PEAKS.json is absent
 FALLBACK_HBM_GBS = 6650.0
 
-# DRAM traffic of one attention launch, from an ncu capture of the same command (see
-# profiles/attn_fwd_video_s32768_h24_fp8pv.md). Valid only for the kernel source whose
-# hash is recorded; any change to the kernel makes it null until re-captured.
+# DRAM traffic of one attention launch, from an ncu capture of the same command (the capture
+# summarised beside this kernel's profile). Valid only for the kernel source whose hash is
+# recorded; any change to the kernel makes it null until re-captured.
 TRAFFIC = {
-    # workload: (sha256 of attn_fwd.cuh [:16], dram bytes read + written per launch)
-    "video_s32768_h24_fp8pv": ("33d4954420cd5576", 309.744384e6 + 175.938560e6),
+    # workload: (sha256 of the kernel's sources [:16], dram bytes read + written per launch)
+}
+
+# The source files of the attention kernel each PV mode runs (the 8-bit P modes run over pairs
+# of query tiles), and that kernel's name.
+KERNEL_SOURCES = {
+    "fp8": (["attn_fwd_pp.cuh", "attn_fwd.cuh", "ptx.cuh"], "attn_fwd_pp_kernel"),
+    "mxfp8": (["attn_fwd_pp.cuh", "attn_fwd.cuh", "ptx.cuh"], "attn_fwd_pp_kernel"),
+    "bf16": (["attn_fwd.cuh", "ptx.cuh"], "attn_fwd_kernel"),
+    "bf16v": (["attn_fwd.cuh", "ptx.cuh"], "attn_fwd_kernel"),
 }
 
 
-def kernel_hash() -> str:
-    path = os.path.join(ROOT, "precision_attention_forward_b200", "csrc", "attn_fwd.cuh")
-    with open(path, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+def kernel_hash(pv_mode: str) -> str:
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES[pv_mode][0]:
+        with open(os.path.join(ROOT, "precision_attention_forward_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
 
 
 def load_peaks():
@@ -488,7 +498,7 @@ def main():
     fp8_peak = peaks.get("bf16_tflops", FALLBACK_BF16_BURST) * FP8_OVER_BF16
     achieved = flops / (attn_ms * 1e-3) / 1e12
     tr = TRAFFIC.get(w.name)
-    traffic = tr[1] if tr and tr[0] == kernel_hash() else None
+    traffic = tr[1] if tr and tr[0] == kernel_hash(w.pv_mode) else None
     qbytes = quantizer_bytes(Tq, H, 2 if dts["q"] == "bf16" else 4, sbq) + \
         quantizer_bytes(Tk, H, 2 if dts["k"] == "bf16" else 4, sbk) + \
         (Tk * H * 128 * 3.0 if w.pv_mode == "fp8" else
@@ -508,7 +518,7 @@ def main():
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": fp8_peak, "unit": "TFLOP/s",
                          "frac": achieved / fp8_peak, "traffic": traffic,
                          "peak_source": f"{peak_src} bf16 burst x {FP8_OVER_BF16:g} (nominal FP8/BF16 ratio)",
-                         "kernel": "attn_fwd_kernel", "flops_per_launch": flops},
+                         "kernel": KERNEL_SOURCES[w.pv_mode][1], "flops_per_launch": flops},
             "attn_kernel_ms": attn_ms,
             "attn_pct_nominal_fp8": 100.0 * achieved / NOMINAL_FP8_TFLOPS,
             "quantize": {"ms_per_step": quant_ms, "bytes_per_step": qbytes,

@@ -273,6 +273,12 @@ LPFA_API lpfa_status lpfa_attn_bwd_varlen(const uint8_t* q, const uint8_t* q_sf,
  * word of the current device, resets it to zero, and returns LPFA_OK, LPFA_ERR_TIMEOUT, or
  * LPFA_ERR_CUDA if the synchronization itself failed. *detail (may be NULL) receives the
  * recorded diagnostic (which wait gave up), 0 if none.
+ *
+ * There is one such word per device and process, shared by every kernel of this library and
+ * every stream: the first failure since the last read is kept (later ones leave it alone), and
+ * a read clears it. Calls that run concurrently on several streams therefore share one status;
+ * the stream argument only chooses what is synchronized before the read. Callers that need a
+ * status per stream must serialise the calls whose status they read.
  */
 LPFA_API lpfa_status lpfa_device_status(void* stream, int32_t* detail);
 
@@ -292,6 +298,25 @@ LPFA_API lpfa_status lpfa_attn_fwd_varlen_debug(const uint8_t* q, const uint8_t*
                                        const float* q_descale, const float* k_descale,
                                        const float* v_descale, void* out_bf16, float* lse,
                                        void* stream, int32_t debug_flags);
+
+/*
+ * Test hook for the backward's bounded-wait failure path (no counterpart on the pages). Same
+ * arguments and behaviour as lpfa_attn_bwd_varlen, plus debug_flags: with bit 0 set, the MMA
+ * issue warp of the dK/dV kernel first waits on a barrier phase that nothing completes, so its
+ * bounded wait runs out (about 2 s per wave of CTAs), the kernel records LPFA_ERR_TIMEOUT in the
+ * device status word (site 207) and every role exits after its in-flight MMAs have completed;
+ * dk, dv (and their scales) are then unspecified. The dQ kernel runs normally. The GPU context
+ * stays usable. Other bits are rejected with LPFA_ERR_INVALID_ARG; debug_flags = 0 is exactly
+ * lpfa_attn_bwd_varlen.
+ */
+LPFA_API lpfa_status lpfa_attn_bwd_varlen_debug(const uint8_t* q, const uint8_t* q_sf, const uint8_t* k,
+                                       const uint8_t* k_sf, const uint8_t* v, const uint8_t* v_sf,
+                                       const void* out_bf16, const void* dout_bf16, const float* lse,
+                                       const lpfa_varlen_meta* meta_q, const lpfa_varlen_meta* meta_k,
+                                       int32_t heads, int32_t head_dim, const lpfa_descale* q_descale,
+                                       const lpfa_descale* k_descale, const lpfa_descale* v_descale,
+                                       void* dq_bf16, void* dk, void* dv, uint8_t* dk_sf, uint8_t* dv_sf,
+                                       int32_t output_mxfp8_dkv, void* stream, int32_t debug_flags);
 
 /* Message describing the last non-OK status returned on the calling thread ("" if none). */
 LPFA_API const char* lpfa_last_error_message(void);

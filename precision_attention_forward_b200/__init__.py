@@ -39,6 +39,7 @@ EXPORTED_SYMBOLS = (
     "lpfa_scale_bytes", "lpfa_quantize_mxfp8_varlen", "lpfa_cast_e4m3", "lpfa_attn_fwd_varlen",
     "lpfa_device_status", "lpfa_last_error_message", "lpfa_version", "lpfa_attn_fwd_varlen_debug",
     "lpfa_attn_fwd_varlen_descaled", "lpfa_quantize_mxfp8_varlen_tokens", "lpfa_attn_bwd_varlen",
+    "lpfa_attn_bwd_varlen_debug",
 )
 
 
@@ -75,6 +76,8 @@ _lib.lpfa_quantize_mxfp8_varlen_tokens.restype = ctypes.c_int
 _lib.lpfa_attn_bwd_varlen.argtypes = ([_vp] * 9 + [ctypes.POINTER(_Meta), ctypes.POINTER(_Meta), _i32, _i32] +
                                       [ctypes.POINTER(_Descale)] * 3 + [_vp] * 5 + [_i32, _vp])
 _lib.lpfa_attn_bwd_varlen.restype = ctypes.c_int
+_lib.lpfa_attn_bwd_varlen_debug.argtypes = list(_lib.lpfa_attn_bwd_varlen.argtypes) + [_i32]
+_lib.lpfa_attn_bwd_varlen_debug.restype = ctypes.c_int
 _lib.lpfa_cast_e4m3.argtypes = [_vp, _i64, _i64, _i64, _i32, _i32, _vp, _vp]
 _lib.lpfa_cast_e4m3.restype = ctypes.c_int
 _lib.lpfa_attn_fwd_varlen.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, ctypes.POINTER(_Meta), ctypes.POINTER(_Meta),
@@ -284,10 +287,15 @@ def lpfa_attn_bwd_varlen(q: torch.Tensor, q_sf: torch.Tensor, k: torch.Tensor, k
                          v: torch.Tensor, v_sf: torch.Tensor, out: torch.Tensor, dout: torch.Tensor,
                          lse: torch.Tensor, meta_q: VarlenMeta, meta_k: VarlenMeta,
                          q_descale: Optional[torch.Tensor] = None, k_descale: Optional[torch.Tensor] = None,
-                         v_descale: Optional[torch.Tensor] = None, output_mxfp8_dkv: bool = False, stream=None):
+                         v_descale: Optional[torch.Tensor] = None, output_mxfp8_dkv: bool = False, stream=None,
+                         dq: Optional[torch.Tensor] = None, dk: Optional[torch.Tensor] = None,
+                         dv: Optional[torch.Tensor] = None, dk_sf: Optional[torch.Tensor] = None,
+                         dv_sf: Optional[torch.Tensor] = None, debug_flags: int = 0):
     """Attention backward (see include/lpfa.h). q/k/v with their head_dim-orientation scales, out and
     dout bf16 (Tq,H,128), lse fp32 (H,Tq). Returns (dq, dk, dv) in bf16, or with output_mxfp8_dkv
     (dq, dk_payload, dv_payload, dk_scales, dv_scales) like LP-FA4's mxfp8_flash_attn_varlen_backward.
+    Output tensors may be passed in (contiguous, of the returned shapes and dtypes); debug_flags != 0
+    calls the test hook lpfa_attn_bwd_varlen_debug.
     """
     for name, t in (("q", q), ("k", k), ("v", v)):
         if t.dtype != torch.uint8 or t.dim() != 3 or not t.is_contiguous():
@@ -306,23 +314,31 @@ def lpfa_attn_bwd_varlen(q: torch.Tensor, q_sf: torch.Tensor, k: torch.Tensor, k
         else:
             ss, hs = descale_strides(t, meta_q.num_seqs, H)
             descs.append(_Descale(t.data_ptr(), ss, hs))
-    dq = torch.empty((Tq, H, 128), dtype=torch.bfloat16, device=q.device)
+    def _out(t, shape, dtype, name):
+        if t is None:
+            return torch.empty(shape, dtype=dtype, device=q.device)
+        if t.dtype != dtype or tuple(t.shape) != tuple(shape) or not t.is_contiguous():
+            raise ValueError("%s must be a contiguous %s tensor of shape %s" % (name, dtype, tuple(shape)))
+        return t
+
+    kv_dtype = torch.uint8 if output_mxfp8_dkv else torch.bfloat16
+    dq = _out(dq, (Tq, H, 128), torch.bfloat16, "dq")
+    dk = _out(dk, (Tk, H, 128), kv_dtype, "dk")
+    dv = _out(dv, (Tk, H, 128), kv_dtype, "dv")
     if output_mxfp8_dkv:
-        dk = torch.empty((Tk, H, 128), dtype=torch.uint8, device=q.device)
-        dv = torch.empty((Tk, H, 128), dtype=torch.uint8, device=q.device)
-        dk_sf = torch.empty(meta_k.scale_bytes(H), dtype=torch.uint8, device=q.device)
-        dv_sf = torch.empty(meta_k.scale_bytes(H), dtype=torch.uint8, device=q.device)
+        dk_sf = _out(dk_sf, (meta_k.scale_bytes(H),), torch.uint8, "dk_sf")
+        dv_sf = _out(dv_sf, (meta_k.scale_bytes(H),), torch.uint8, "dv_sf")
     else:
-        dk = torch.empty((Tk, H, 128), dtype=torch.bfloat16, device=q.device)
-        dv = torch.empty((Tk, H, 128), dtype=torch.bfloat16, device=q.device)
         dk_sf = dv_sf = None
+    args = (q.data_ptr(), q_sf.data_ptr(), k.data_ptr(), k_sf.data_ptr(), v.data_ptr(), v_sf.data_ptr(),
+            out.data_ptr(), dout.data_ptr(), lse.data_ptr(), ctypes.byref(meta_q._c), ctypes.byref(meta_k._c), H, 128,
+            ctypes.byref(descs[0]), ctypes.byref(descs[1]), ctypes.byref(descs[2]), dq.data_ptr(), dk.data_ptr(),
+            dv.data_ptr(), _ptr(dk_sf), _ptr(dv_sf), 1 if output_mxfp8_dkv else 0, _stream_ptr(stream))
     with torch.cuda.device(q.device):
-        _check(_lib.lpfa_attn_bwd_varlen(q.data_ptr(), q_sf.data_ptr(), k.data_ptr(), k_sf.data_ptr(), v.data_ptr(),
-                                         v_sf.data_ptr(), out.data_ptr(), dout.data_ptr(), lse.data_ptr(),
-                                         ctypes.byref(meta_q._c), ctypes.byref(meta_k._c), H, 128,
-                                         ctypes.byref(descs[0]), ctypes.byref(descs[1]), ctypes.byref(descs[2]),
-                                         dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), _ptr(dk_sf), _ptr(dv_sf),
-                                         1 if output_mxfp8_dkv else 0, _stream_ptr(stream)))
+        if debug_flags:
+            _check(_lib.lpfa_attn_bwd_varlen_debug(*args, int(debug_flags)))
+        else:
+            _check(_lib.lpfa_attn_bwd_varlen(*args))
     if output_mxfp8_dkv:
         return dq, dk, dv, dk_sf, dv_sf
     return dq, dk, dv

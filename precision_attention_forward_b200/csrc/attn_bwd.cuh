@@ -71,6 +71,7 @@ struct BwdParams {
   int total_q_tiles;
   int total_k_tiles;
   int mxfp8_dkv;
+  int debug_stall;          // test hook: > 0 makes the dK/dV kernel's MMA warp wait on a phase that never comes
 };
 
 // Byte offset of element chunk (8 BF16) cc of row r in a 128-row BF16 tile stored as two
@@ -141,7 +142,7 @@ constexpr uint32_t kBwdOffStage = 2 * kBfTile;
 constexpr uint32_t kBwdStageBytes = 2 * kBfTile;
 constexpr uint32_t kBwdOffVec = kBwdOffStage + 2 * kBwdStageBytes;
 constexpr uint32_t kBwdOffBar = kBwdOffVec + 2 * 2 * 128 * 4;
-constexpr uint32_t kBwdNumBars = 12;
+constexpr uint32_t kBwdNumBars = 13;
 constexpr uint32_t kBwdSmem = kBwdOffBar + kBwdNumBars * 8 + 16 + 1024;
 static_assert(kBwdSmem <= 227 * 1024, "backward shared memory over the per-CTA limit");
 
@@ -153,6 +154,7 @@ constexpr int kBbEmpty = 3;      // + stage: the last MMA that reads the stage i
 constexpr int kBbSFull = 5;      // S and dP of the step in TMEM
 constexpr int kBbChunk = 6;      // + chunk (4): the chunk's P and dS in TMEM (compute threads)
 constexpr int kBbRFree = 10;     // the step's accumulating MMAs are done
+constexpr int kBbDrain = 12;     // every MMA the issue warp issued is done (before teardown)
 
 struct BwdSmem {
   uint8_t* base;
@@ -365,6 +367,15 @@ __device__ __forceinline__ void bwd_report(const BwdSmem& sm, int site) {
   if (atomicCAS(&g_lpfa_status[0], 0, 4 /* LPFA_ERR_TIMEOUT */) == 0) atomicExch(&g_lpfa_status[1], site);
 }
 
+// Issue warp, on both the normal and the abort exit: every tcgen05 operation it issued completes
+// before the CTA reaches its teardown (MMAs still reading shared memory or writing TMEM when
+// TMEM is freed would be undefined). The wait is bounded and outlasts an abort; a drain that
+// runs out is recorded as site 206.
+__device__ __forceinline__ void bwd_drain(const BwdSmem& sm, int lane) {
+  mma_commit(sm.bar(kBbDrain), lane == 0 ? 1u : 0u);
+  if (!mbar_wait_warp(sm.bar(kBbDrain), 0, nullptr) && lane == 0) bwd_report(sm, 206);
+}
+
 // ---------------------------------------------------------------------------------------------
 // The pipeline shared by both tile kernels. kDkDv: the dK/dV kernel (resident K, V are the A
 // operands of S^T and dP^T; the streamed Q, dO the B operands), else the dQ kernel (resident Q,
@@ -568,7 +579,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dkdv_kernel(const Bwd
     }
     if (!ok && lane == 0) bwd_report(sm, 202);
   } else if (warp == kBwdIssueWarp) {
-    if (!bwd_issue<true>(sm, tm, nq, lane, abort_flag) && lane == 0) bwd_report(sm, 204);
+    bool ok = true;
+    if (p.debug_stall > 0) {
+      // Test hook: wait for a phase of the drain barrier that nothing completes before the drain
+      // below, so the wait runs out and the failure path is exercised.
+      ok = mbar_wait_warp(sm.bar(kBbDrain), 0, abort_flag);
+      if (!ok && lane == 0) bwd_report(sm, 207);
+    }
+    if (ok && !bwd_issue<true>(sm, tm, nq, lane, abort_flag) && lane == 0) bwd_report(sm, 204);
+    bwd_drain(sm, lane);
   } else {
     const int r = tid;  // this thread's key row (TMEM lane)
     const uint32_t lane_addr = static_cast<uint32_t>(warp * 32) << 16;
@@ -646,6 +665,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dq_kernel(const BwdPa
     if (!ok && lane == 0) bwd_report(sm, 203);
   } else if (warp == kBwdIssueWarp) {
     if (!bwd_issue<false>(sm, tm, nk, lane, abort_flag) && lane == 0) bwd_report(sm, 205);
+    bwd_drain(sm, lane);
   } else {
     const int r = tid;  // this thread's query row (TMEM lane)
     const uint32_t lane_addr = static_cast<uint32_t>(warp * 32) << 16;

@@ -246,19 +246,21 @@ __device__ __forceinline__ float2 exp2_mufu2(float2 x) {
 }
 
 // 2^x = 2^j * q(x - j), j = round(x) by the 1.5 * 2^23 magic add; the exponent of q is
-// raised by j with one integer add on the bit pattern. x is clamped at -126 (results below
-// that are treated as zero downstream).
-__device__ __forceinline__ float2 exp2_poly2(float2 x) {
-  x.x = fmaxf(x.x, -126.0f);
-  x.y = fmaxf(x.y, -126.0f);
+// raised by j with one integer add on the bit pattern. Inputs below -126 (a masked key's -inf
+// included) give exactly 0, as the MUFU exponential does.
+__device__ __forceinline__ float2 exp2_poly2(float2 xin) {
+  float2 x;
+  x.x = fmaxf(xin.x, -126.0f);
+  x.y = fmaxf(xin.y, -126.0f);
   const float2 t = __fadd2_rn(x, make_float2(12582912.0f, 12582912.0f));
   const float2 jf = __fadd2_rn(t, make_float2(-12582912.0f, -12582912.0f));
   const float2 f = __ffma2_rn(jf, make_float2(-1.0f, -1.0f), x);
   float2 q = __ffma2_rn(make_float2(kExp2P3, kExp2P3), f, make_float2(kExp2P2, kExp2P2));
   q = __ffma2_rn(q, f, make_float2(kExp2P1, kExp2P1));
   q = __ffma2_rn(q, f, make_float2(kExp2P0, kExp2P0));
-  return make_float2(__uint_as_float(__float_as_uint(q.x) + (__float_as_uint(t.x) << 23)),
-                     __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(t.y) << 23)));
+  const float2 r = make_float2(__uint_as_float(__float_as_uint(q.x) + (__float_as_uint(t.x) << 23)),
+                               __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(t.y) << 23)));
+  return make_float2(xin.x < -126.0f ? 0.0f : r.x, xin.y < -126.0f ? 0.0f : r.y);
 }
 
 // The 128 S columns of this thread's row.

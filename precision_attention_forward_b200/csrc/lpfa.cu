@@ -16,6 +16,7 @@
 
 #include "lpfa.h"
 #include "attn_fwd.cuh"
+#include "attn_fwd_pp.cuh"
 #include "attn_bwd.cuh"
 #include "quantize.cuh"
 
@@ -349,6 +350,18 @@ static lpfa_status launch_attn(int grid, cudaStream_t s, const CUtensorMap& tq, 
   lpfa::attn_fwd_kernel<kPv, kPerUnit><<<grid, lpfa::kAttnThreads, smem, s>>>(tq, tk, tv, p);
   return LPFA_OK;
 }
+
+// The 8-bit P modes run over pairs of query tiles (attn_fwd_pp.cuh).
+template <int kPv, bool kPerUnit>
+static lpfa_status launch_attn_pp(int grid, cudaStream_t s, const CUtensorMap& tq, const CUtensorMap& tk,
+                                  const CUtensorMap& tv, const lpfa::AttnParams& p) {
+  constexpr uint32_t smem = lpfa::pp::smem_bytes<kPv == lpfa::kPvMx>();
+  const void* fn = reinterpret_cast<const void*>(lpfa::pp::attn_fwd_pp_kernel<kPv, kPerUnit>);
+  const lpfa_status st = check_attn_kernel(fn, smem);
+  if (st != LPFA_OK) return st;
+  lpfa::pp::attn_fwd_pp_kernel<kPv, kPerUnit><<<grid, lpfa::kAttnThreads, smem, s>>>(tq, tk, tv, p);
+  return LPFA_OK;
+}
 }  // extern "C++"
 
 // Internal entry shared with the test hook: debug_stall > 0 forces a bounded wait to run out.
@@ -429,14 +442,14 @@ static lpfa_status attn_fwd_impl(const uint8_t* q, const uint8_t* q_sf, const ui
   const bool per_unit = (p.q_descale.seq_stride | p.q_descale.head_stride | p.k_descale.seq_stride |
                          p.k_descale.head_stride) != 0;
   if (pv_mode == LPFA_PV_FP8) {
-    st = per_unit ? launch_attn<lpfa::kPvFp8, true>(grid, s, tq, tk, tv, p)
-                  : launch_attn<lpfa::kPvFp8, false>(grid, s, tq, tk, tv, p);
+    st = per_unit ? launch_attn_pp<lpfa::kPvFp8, true>(grid, s, tq, tk, tv, p)
+                  : launch_attn_pp<lpfa::kPvFp8, false>(grid, s, tq, tk, tv, p);
   } else if (pv_mode == LPFA_PV_BF16) {
     st = per_unit ? launch_attn<lpfa::kPvBf16Mx, true>(grid, s, tq, tk, tv, p)
                   : launch_attn<lpfa::kPvBf16Mx, false>(grid, s, tq, tk, tv, p);
   } else if (pv_mode == LPFA_PV_MXFP8) {
-    st = per_unit ? launch_attn<lpfa::kPvMx, true>(grid, s, tq, tk, tv, p)
-                  : launch_attn<lpfa::kPvMx, false>(grid, s, tq, tk, tv, p);
+    st = per_unit ? launch_attn_pp<lpfa::kPvMx, true>(grid, s, tq, tk, tv, p)
+                  : launch_attn_pp<lpfa::kPvMx, false>(grid, s, tq, tk, tv, p);
   } else {
     st = per_unit ? launch_attn<lpfa::kPvBf16In, true>(grid, s, tq, tk, tv, p)
                   : launch_attn<lpfa::kPvBf16In, false>(grid, s, tq, tk, tv, p);
@@ -468,13 +481,16 @@ lpfa_status lpfa_attn_fwd_varlen_descaled(const uint8_t* q, const uint8_t* q_sf,
                        v_descale, out_bf16, lse, stream, 0);
 }
 
-lpfa_status lpfa_attn_bwd_varlen(const uint8_t* q, const uint8_t* q_sf, const uint8_t* k, const uint8_t* k_sf,
+}  // extern "C"
+
+// Internal entry shared with the test hook: debug_stall > 0 forces a bounded wait to run out.
+static lpfa_status attn_bwd_impl(const uint8_t* q, const uint8_t* q_sf, const uint8_t* k, const uint8_t* k_sf,
                                  const uint8_t* v, const uint8_t* v_sf, const void* out_bf16, const void* dout_bf16,
                                  const float* lse, const lpfa_varlen_meta* meta_q, const lpfa_varlen_meta* meta_k,
                                  int32_t heads, int32_t head_dim, const lpfa_descale* q_descale,
                                  const lpfa_descale* k_descale, const lpfa_descale* v_descale, void* dq_bf16,
                                  void* dk, void* dv, uint8_t* dk_sf, uint8_t* dv_sf, int32_t output_mxfp8_dkv,
-                                 void* stream) {
+                                 void* stream, int debug_stall) {
   if (!q || !q_sf || !k || !k_sf || !v || !v_sf || !out_bf16 || !dout_bf16 || !lse || !dq_bf16 || !dk || !dv)
     return fail(LPFA_ERR_INVALID_ARG, "NULL tensor pointer");
   if (output_mxfp8_dkv != 0 && output_mxfp8_dkv != 1) return fail(LPFA_ERR_INVALID_ARG, "output_mxfp8_dkv must be 0 or 1");
@@ -533,6 +549,7 @@ lpfa_status lpfa_attn_bwd_varlen(const uint8_t* q, const uint8_t* q_sf, const ui
   p.total_q_tiles = meta_q->total_scale_blocks;
   p.total_k_tiles = meta_k->total_scale_blocks;
   p.mxfp8_dkv = output_mxfp8_dkv;
+  p.debug_stall = debug_stall;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   for (const void* fn : {reinterpret_cast<const void*>(lpfa::attn_bwd_dkdv_kernel),
                          reinterpret_cast<const void*>(lpfa::attn_bwd_dq_kernel)}) {
@@ -550,6 +567,33 @@ lpfa_status lpfa_attn_bwd_varlen(const uint8_t* q, const uint8_t* q_sf, const ui
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "backward launch");
   return LPFA_OK;
+}
+
+extern "C" {
+
+lpfa_status lpfa_attn_bwd_varlen(const uint8_t* q, const uint8_t* q_sf, const uint8_t* k, const uint8_t* k_sf,
+                                 const uint8_t* v, const uint8_t* v_sf, const void* out_bf16, const void* dout_bf16,
+                                 const float* lse, const lpfa_varlen_meta* meta_q, const lpfa_varlen_meta* meta_k,
+                                 int32_t heads, int32_t head_dim, const lpfa_descale* q_descale,
+                                 const lpfa_descale* k_descale, const lpfa_descale* v_descale, void* dq_bf16,
+                                 void* dk, void* dv, uint8_t* dk_sf, uint8_t* dv_sf, int32_t output_mxfp8_dkv,
+                                 void* stream) {
+  return attn_bwd_impl(q, q_sf, k, k_sf, v, v_sf, out_bf16, dout_bf16, lse, meta_q, meta_k, heads, head_dim,
+                       q_descale, k_descale, v_descale, dq_bf16, dk, dv, dk_sf, dv_sf, output_mxfp8_dkv, stream, 0);
+}
+
+lpfa_status lpfa_attn_bwd_varlen_debug(const uint8_t* q, const uint8_t* q_sf, const uint8_t* k, const uint8_t* k_sf,
+                                       const uint8_t* v, const uint8_t* v_sf, const void* out_bf16,
+                                       const void* dout_bf16, const float* lse, const lpfa_varlen_meta* meta_q,
+                                       const lpfa_varlen_meta* meta_k, int32_t heads, int32_t head_dim,
+                                       const lpfa_descale* q_descale, const lpfa_descale* k_descale,
+                                       const lpfa_descale* v_descale, void* dq_bf16, void* dk, void* dv,
+                                       uint8_t* dk_sf, uint8_t* dv_sf, int32_t output_mxfp8_dkv, void* stream,
+                                       int32_t debug_flags) {
+  if (debug_flags & ~1) return fail(LPFA_ERR_INVALID_ARG, "unknown debug flags 0x%x", debug_flags);
+  return attn_bwd_impl(q, q_sf, k, k_sf, v, v_sf, out_bf16, dout_bf16, lse, meta_q, meta_k, heads, head_dim,
+                       q_descale, k_descale, v_descale, dq_bf16, dk, dv, dk_sf, dv_sf, output_mxfp8_dkv, stream,
+                       debug_flags & 1);
 }
 
 lpfa_status lpfa_attn_fwd_varlen_debug(const uint8_t* q, const uint8_t* q_sf, const uint8_t* k, const uint8_t* k_sf,

@@ -99,6 +99,32 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
   }
 }
 
+// Bounded wait for warps that mostly wait (producers, MMA issuers): each probe may suspend the
+// thread for up to suspend_ns (woken early when the phase completes), so a long wait does not
+// take issue slots from the other warps of its SM sub-partition the way a spin loop would.
+__device__ __forceinline__ bool mbar_try_wait_suspend(uint64_t* bar, uint32_t parity, uint32_t suspend_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(suspend_ns)
+      : "memory");
+  return ok != 0;
+}
+
+__device__ __forceinline__ bool mbar_wait_suspend(uint64_t* bar, uint32_t parity, const volatile int* abort,
+                                                  uint32_t suspend_ns) {
+  if (mbar_test_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  while (true) {
+    if (mbar_try_wait_suspend(bar, parity, suspend_ns)) return true;
+    if (abort != nullptr && *abort) return false;
+    if (global_timer_ns() - t0 > kWaitTimeoutNs) return false;
+  }
+}
+
 // ---------------------------------------------------------------------------------------
 // Bulk asynchronous copies (TMA)
 // ---------------------------------------------------------------------------------------

@@ -274,3 +274,60 @@ def test_workload_sampled_check(name):
     lse_s = lse[hh, tt]
     o_scale = wl.outlier_scale(w, "v")[hs] if w.outlier_frac > 0.0 else None
     print(gu.assert_within(gu.compare_attention(o_s, lse_s, o_ref, lse_ref, o_scale), f"{name} sampled"))
+
+
+def _rising_inputs(seed, lq, lk, H):
+    """Q and K whose logits jump by about 9 binades (times a per-row slope in [0.5, 1.5]) from each
+    128-key tile to the next, through one spike key per tile; V random.
+
+    The jump exceeds the softmax reference's lag in every mode (2 binades for fp8 P, 8 otherwise)
+    for most rows, so the kernel moves the row reference and rescales O on almost every tile,
+    while the earlier tiles keep a share of the weight that a missing or wrong rescale would
+    visibly change. Logits in log2 units are a_r * level(key) + noise, with level = 9 (t - 1)
+    for the keys of tile t >= 1 and one key per tile at level + 9."""
+    g = np.random.default_rng(seed)
+    c = math.sqrt(math.log(2.0) * math.sqrt(128.0))     # (c u).(c u) / sqrt(128) = ln 2
+    u = g.standard_normal((H, 128))
+    u /= np.linalg.norm(u, axis=1, keepdims=True)
+    q_rows, k_rows = [], []
+    for n in lq:
+        a = g.uniform(0.5, 1.5, size=(n, H, 1))
+        q_rows.append(a * c * u[None] + 0.05 * g.standard_normal((n, H, 128)))
+    for n in lk:
+        tile = np.arange(n) // 128
+        level = np.where(tile >= 1, 9.0 * (tile - 1), 0.0)
+        spike = (np.arange(n) % 128 == 37) & (tile >= 1)
+        level = level + 9.0 * spike
+        k_rows.append(level[:, None, None] * c * u[None] + 0.5 * g.standard_normal((n, H, 128)))
+    q = wl.round_to_bf16(np.concatenate(q_rows).astype(np.float32))
+    k = wl.round_to_bf16(np.concatenate(k_rows).astype(np.float32))
+    v = wl.round_to_bf16(g.standard_normal((sum(lk), H, 128)).astype(np.float32))
+    return q, k, v
+
+
+@pytest.mark.parametrize("pv_mode", ["bf16", "fp8", "bf16v", "mxfp8"])
+def test_reference_moves_rescale_o(pv_mode):
+    """The online softmax's correction step: when a later key tile's logits exceed the row
+    reference by more than the lag, O and l are rescaled by an exact power of two before that
+    tile's P V is added (LP-FA4 README, "MXFP8 forward and backward": online-softmax forward).
+    Both query tiles of a pair, a single last tile, and ragged key tails are covered."""
+    lq, lk, H = [300, 256], [600, 520], 2
+    q, k, v = _rising_inputs(41, lq, lk, H)
+    if pv_mode == "fp8":
+        v = v * np.float32(2.0)
+    o, lse = gu.run_path(lp, q, k, v, lq, lk, H, pv_mode=pv_mode)
+    _status_ok()
+    o_ref, lse_ref = gu.oracle_full(q, k, v, lq, lk, H, pv_mode=pv_mode)
+    gu.assert_within(gu.compare_attention(o, lse, o_ref, lse_ref), f"rising logits {pv_mode}")
+    # The earlier tiles matter: dropping every tile but the last changes O beyond the bound, so
+    # the comparison above sees a wrong rescale of the earlier contributions.
+    qh, kh, vh = gu.oracle_inputs(q, k, v, lq, lk, H, pv_mode)
+    last = []
+    for i, (n, m) in enumerate(zip(lq, lk)):
+        k0 = sum(lk[:i])
+        t0 = (m - 1) // 128 * 128
+        oo, _ = oatt.attention_fwd(qh[sum(lq[:i]):sum(lq[:i]) + n], kh[k0 + t0:k0 + m], vh[k0 + t0:k0 + m],
+                                   [n], [m - t0], p_mode=gu.p_mode_of(pv_mode))
+        last.append(oo)
+    d = np.concatenate(last) - o_ref
+    assert np.linalg.norm(d) / np.linalg.norm(o_ref) > 5 * gu.O_REL_L2

@@ -123,3 +123,102 @@ def test_outputs_stay_inside_their_buffers(pv_mode, lens_q, lens_k, H):
         assert _guards_intact(buf, view.numel()), f"{name}: bytes outside the buffer were written"
     ro, rl = gu.oracle_full(q, k, v, lens_q, lens_k, H, pv_mode=pv_mode)
     gu.assert_within(gu.compare_attention(out, lse, ro, rl), f"guarded {pv_mode} {lens_q}/{lens_k}")
+
+
+def _backward_inputs(lq, lk, H, seed):
+    """MXFP8 Q/K/V, the forward's O and LSE, and a seeded dO on the device; the float inputs too."""
+    q, k, v = wl.small_random(seed, lq, lk, H)
+    g = np.random.default_rng(seed + 1000)
+    do = wl.round_to_bf16(g.standard_normal((sum(lq), H, 128)).astype(np.float32))
+    mq = lp.lpfa_varlen_meta_from_lengths(lq)
+    mk = lp.lpfa_varlen_meta_from_lengths(lk)
+    qp, qs = gu.gpu_quantize(lp, q, "bf16", mq)
+    kp, ks = gu.gpu_quantize(lp, k, "bf16", mk)
+    vp, vs = gu.gpu_quantize(lp, v, "bf16", mk)
+    o, lse = lp.lpfa_attn_fwd_varlen(qp, qs, kp, ks, vp, vs, mq, mk, pv_mode="bf16")
+    dev = (qp, qs, kp, ks, vp, vs, o, gu.to_device(do, "bf16"), lse, mq, mk)
+    return dev, (q, k, v, do)
+
+
+def _backward_reference(host, dev, lq, lk, H):
+    from oracle import backward as obwd
+    q, k, v, do = host
+    o, lse = dev[6], dev[8]
+    qh, kh, vh = gu.oracle_inputs(q, k, v, lq, lk, H)
+    return obwd.attention_bwd(qh, kh, vh, o.float().cpu().numpy().astype(np.float64), do.astype(np.float64),
+                              lse.cpu().numpy().astype(np.float64), lq, lk)
+
+
+def _grads_close(got, ref):
+    got = np.asarray(got, dtype=np.float64)
+    rel = np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-4 * np.sqrt(ref.size))
+    mx = np.max(np.abs(got - ref)) / max(np.max(np.abs(ref)), 1e-4)
+    return rel <= 1e-2 and mx <= 2e-2
+
+
+def test_backward_bounded_wait_runs_out_and_context_survives():
+    """The backward's waits are bounded like the forward's (LP-FA4 README, "MXFP8 forward and
+    backward": mxfp8_flash_attn_varlen_backward): the debug hook makes the dK/dV kernel's MMA warp
+    wait on a phase nothing completes; the call ends with LPFA_ERR_TIMEOUT in the status word and
+    no fault, and a normal call right after matches the oracle."""
+    lq, lk, H = [300, 77], [300, 77], 2
+    dev, host = _backward_inputs(lq, lk, H, 21)
+    torch.cuda.synchronize()
+    assert lp.lpfa_device_status() == (lp.LPFA_OK, 0)
+    t0 = time.time()
+    lp.lpfa_attn_bwd_varlen(*dev, debug_flags=1)
+    st, detail = lp.lpfa_device_status()
+    elapsed = time.time() - t0
+    assert st == lp.LPFA_ERR_TIMEOUT, (st, detail)
+    assert 200 <= detail <= 207, detail
+    assert elapsed < 30.0, elapsed
+    assert lp.lpfa_device_status() == (lp.LPFA_OK, 0)
+    dq, dk, dv = lp.lpfa_attn_bwd_varlen(*dev)
+    torch.cuda.synchronize()
+    assert lp.lpfa_device_status() == (lp.LPFA_OK, 0)
+    for got, ref in zip((dq, dk, dv), _backward_reference(host, dev, lq, lk, H)):
+        assert _grads_close(got.float().cpu().numpy(), ref)
+
+
+def test_backward_unknown_debug_flag_rejected():
+    dev, _ = _backward_inputs([5], [5], 1, 2)
+    with pytest.raises(lp.LpfaError) as e:
+        lp.lpfa_attn_bwd_varlen(*dev, debug_flags=2)
+    assert e.value.status == lp.LPFA_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("mx_dkv", [False, True])
+@pytest.mark.parametrize("lens_q,lens_k,H", [([1], [1], 1), ([300, 77, 1], [129, 700, 3], 3), ([2048], [257], 2)])
+def test_backward_outputs_stay_inside_their_buffers(mx_dkv, lens_q, lens_k, H):
+    """dQ, dK, dV and (MXFP8 output) the dK/dV scale storage, each inside pattern-filled guards."""
+    dev, host = _backward_inputs(lens_q, lens_k, H, 5)
+    Tq, Tk = sum(lens_q), sum(lens_k)
+    mk = dev[10]
+    bufs = {}
+
+    def alloc(name, nbytes):
+        bufs[name] = _guarded(nbytes)
+        return bufs[name][1]
+
+    dq = alloc("dq", Tq * H * 128 * 2).view(torch.bfloat16).view(Tq, H, 128)
+    kv_bytes = Tk * H * 128 * (1 if mx_dkv else 2)
+    kv_dtype = torch.uint8 if mx_dkv else torch.bfloat16
+    dk = alloc("dk", kv_bytes).view(kv_dtype).view(Tk, H, 128)
+    dv = alloc("dv", kv_bytes).view(kv_dtype).view(Tk, H, 128)
+    extra = {}
+    if mx_dkv:
+        extra = {"dk_sf": alloc("dk_sf", mk.scale_bytes(H)), "dv_sf": alloc("dv_sf", mk.scale_bytes(H))}
+    lp.lpfa_attn_bwd_varlen(*dev, output_mxfp8_dkv=mx_dkv, dq=dq, dk=dk, dv=dv, **extra)
+    torch.cuda.synchronize()
+    assert lp.lpfa_device_status() == (lp.LPFA_OK, 0)
+    for name, (buf, view) in bufs.items():
+        assert _guards_intact(buf, view.numel()), f"{name}: bytes outside the buffer were written"
+    rq, rk, rv = _backward_reference(host, dev, lens_q, lens_k, H)
+    assert _grads_close(dq.float().cpu().numpy(), rq)
+    if not mx_dkv:
+        assert _grads_close(dk.float().cpu().numpy(), rk) and _grads_close(dv.float().cpu().numpy(), rv)
+    else:
+        from oracle import mxfp8 as omx
+        for pl, sc, ref in ((dk, extra["dk_sf"], rk), (dv, extra["dv_sf"], rv)):
+            deq = omx.dequantize_mxfp8(pl.cpu().numpy(), sc.cpu().numpy(), lens_k, H)
+            assert np.linalg.norm(deq - ref) <= 5e-2 * max(np.linalg.norm(ref), 1e-4 * np.sqrt(ref.size))
