@@ -40,14 +40,25 @@ namespace pp {
 constexpr int kKStages = 5;
 constexpr int kVStages = 4;
 
+// P tiles rotate through kPSlots TMEM slots in the order the PV products consume them (tile j of
+// a unit: query tile 0, then 1), so a softmax warpgroup storing P waits only for the PV three P
+// tiles back, not for its own previous one.
+constexpr uint32_t kPSlots = 3;
 constexpr uint32_t kColS = 0;
 constexpr uint32_t kColO = 128;    // + 128 * i
-constexpr uint32_t kColP = 384;    // + 32 * i
-constexpr uint32_t kColSFA = 448;  // + 8 * qstage + 4 * i
-constexpr uint32_t kColSFB = 464;  // + 4 * (kc & 1)
-constexpr uint32_t kColSFP = 472;  // + 4 * i
-constexpr uint32_t kColSFV = 480;  // + 4 * (vc & 1)
-static_assert(kColSFV + 8 <= kTmemCols, "TMEM columns");
+constexpr uint32_t kColP = 384;    // + 32 * slot
+// Scale atoms. fp8 PV: the Q atoms of both tiles per unit stage and the K atoms in two slots, all
+// copied into TMEM ahead of the QK that reads them. MXFP8 PV (whose P and V atoms take the rest of
+// the columns): one Q and one K slot, copied right before each QK, once the previous QK -- the
+// slots' last reader -- is known to have completed.
+constexpr uint32_t kColSFA8 = 480;  // + 8 * qstage + 4 * i   (fp8 PV)
+constexpr uint32_t kColSFB8 = 496;  // + 4 * (kc & 1)         (fp8 PV)
+constexpr uint32_t kColSFA = 480;   // Q scale atom of the QK being issued (MXFP8 PV)
+constexpr uint32_t kColSFB = 484;   // K scale atom of the current K tile (MXFP8 PV)
+constexpr uint32_t kColSFP = 488;   // + 4 * slot: P scale atom (MXFP8 PV)
+constexpr uint32_t kColSFV = 500;   // + 4 * (vc % 3): V scale atom (MXFP8 PV)
+static_assert(kColP + 32 * kPSlots <= kColSFA && kColSFB8 + 8 <= kTmemCols && kColSFV + 4 * 3 <= kTmemCols,
+              "TMEM columns");
 
 // Shared memory (offsets from a 1024-byte aligned base).
 template <bool kMx>
@@ -58,8 +69,8 @@ struct Smem {
   static constexpr uint32_t q_sf = v + kVStages * kTileBytes;               // [kQStages][2] atoms
   static constexpr uint32_t k_sf = q_sf + kQStages * 2 * kAtomBytes;
   static constexpr uint32_t v_sf = k_sf + kKStages * kAtomBytes;            // MXFP8 PV only
-  static constexpr uint32_t p_sf = v_sf + (kMx ? kVStages * kAtomBytes : 0u);  // [2] P atoms (MXFP8 PV)
-  static constexpr uint32_t sched = p_sf + (kMx ? 2 * kAtomBytes : 0u);     // n, units, order, prefix
+  static constexpr uint32_t p_sf = v_sf + (kMx ? kVStages * kAtomBytes : 0u);  // [kPSlots] P atoms (MXFP8 PV)
+  static constexpr uint32_t sched = p_sf + (kMx ? kPSlots * kAtomBytes : 0u);  // n, units, order, prefix
   static constexpr uint32_t bars = sched + ((2 * kMaxSortSeqs + 3) * 4 + 15) / 16 * 16;
   static constexpr uint32_t num_bars = 48;
   static constexpr uint32_t misc = bars + num_bars * 8;                     // tmem base, abort flag
@@ -74,12 +85,12 @@ enum Bar : int {
   kBarVFull = 16, kBarVEmpty = 22,   // [kVStages <= 6]
   kBarSFull = 28,   // [i] S computed for warpgroup i            (MMA commit)
   kBarSFree = 30,   // S read out by the warpgroup it was for     (4 warps)
-  kBarPReady = 31,  // [i] P_i stored, O_i rescaled if needed     (4 warps)
-  kBarPVDone = 33,  // [i] PV_i complete                          (MMA commit)
-  kBarOFull = 35,   // [i] every PV_i of the unit complete        (MMA commit)
-  kBarOEmpty = 37,  // [i] O_i read out by the epilogue           (4 warps)
-  kBarDrain = 39,   // QK issuer's own tcgen05 work done
-  kBarDrainPV = 40  // PV issuer's own tcgen05 work done
+  kBarPReady = 31,  // [slot] P stored, O rescaled if needed      (4 warps)
+  kBarPVDone = 34,  // [slot] the PV reading the slot complete   (MMA commit)
+  kBarOFull = 37,   // [i] every PV_i of the unit complete        (MMA commit)
+  kBarOEmpty = 39,  // [i] O_i read out by the epilogue           (4 warps)
+  kBarDrain = 41,   // QK issuer's own tcgen05 work done
+  kBarDrainPV = 42  // PV issuer's own tcgen05 work done
 };
 static_assert(kKStages <= 6 && kVStages <= 6, "ring barriers");
 
@@ -213,22 +224,31 @@ __device__ __forceinline__ PairUnit warp_uniform(const PairUnit& u) {
 // LPFA_PP_POLY: how many of every 8 four-key groups take their exponentials from the cubic on the
 //   FMA pipe instead of the MUFU.
 #ifndef LPFA_PP_SUSPEND_NS
-#define LPFA_PP_SUSPEND_NS 0
+#define LPFA_PP_SUSPEND_NS 2000
 #endif
 #ifndef LPFA_PP_MAX2
-#define LPFA_PP_MAX2 0
+#define LPFA_PP_MAX2 1
 #endif
 #ifndef LPFA_PP_POLY
 #define LPFA_PP_POLY 0
 #endif
-
-// Barrier wait of the producer and issuer warps (warp-uniform result).
-__device__ __forceinline__ bool wait_role(uint64_t* bar, uint32_t parity, const volatile int* abort) {
-#if LPFA_PP_SUSPEND_NS > 0
-  return __all_sync(0xFFFFFFFFu, mbar_wait_suspend(bar, parity, abort, LPFA_PP_SUSPEND_NS));
-#else
-  return mbar_wait_warp(bar, parity, abort);
+// LPFA_PP_SFREE_SPIN: the QK issuer spins (no suspend) on the S buffer's release.
+#ifndef LPFA_PP_SFREE_SPIN
+#define LPFA_PP_SFREE_SPIN 0
 #endif
+
+// Bounded barrier wait by a whole warp (every lane polls; warp-uniform result), sleeping between
+// polls when `suspend` is set. (Having one lane poll and the others wait for it measured far
+// slower.)
+__device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity, const volatile int* abort, bool suspend) {
+  if (suspend && LPFA_PP_SUSPEND_NS > 0)
+    return __all_sync(0xFFFFFFFFu, mbar_wait_suspend(bar, parity, abort, LPFA_PP_SUSPEND_NS));
+  return mbar_wait_warp(bar, parity, abort);
+}
+
+// Barrier wait of the producer and issuer warps (they may sleep while waiting).
+__device__ __forceinline__ bool wait_role(uint64_t* bar, uint32_t parity, const volatile int* abort) {
+  return wait_warp(bar, parity, abort, true);
 }
 
 // Row maximum of the 128 S values of this thread's row.
@@ -300,10 +320,14 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
     mbar_init(&bars[kBarSFree], 4);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bars[kBarSFull + i], 1);
-      mbar_init(&bars[kBarPReady + i], 4);
-      mbar_init(&bars[kBarPVDone + i], 1);
       mbar_init(&bars[kBarOFull + i], 1);
       mbar_init(&bars[kBarOEmpty + i], 4);
+    }
+    for (uint32_t i = 0; i < kPSlots; ++i) {
+      // PReady counts the 4 warps of the storing warpgroup; an arrival for the slot's next P
+      // needs the PV of this one complete, so the phases of one slot cannot mix.
+      mbar_init(&bars[kBarPReady + i], 4);
+      mbar_init(&bars[kBarPVDone + i], 1);
     }
     mbar_init(&bars[kBarDrain], 1);
     mbar_init(&bars[kBarDrainPV], 1);
@@ -421,23 +445,48 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
         for (int kk = 0; kk < 4; ++kk) idq[kk] = idesc_qk(kk, negate);
         const uint32_t qs = u % kQStages;
         if (!wait_role(&bars[kBarQFull + qs], (u / kQStages) & 1, abort_flag)) { record_failure(abort_flag, kPSiteMmaQ); ok = false; break; }
-        tc_fence_after();
-        for (int i = 0; i <= ui.has_q1; ++i)
-          tmem_cp_32x128b_x4(tmem + kColSFA + qs * 8 + i * 4, dqsf0 + ((qs * 2 + i) * kAtomBytes >> 4), leader);
+        if (!kMx) {
+          // fp8 PV: both tiles' Q atoms into this unit stage's slots. Their last reader, the unit
+          // two back, completed before the first QK of the previous unit could write S.
+          tc_fence_after();
+          for (int i = 0; i <= ui.has_q1; ++i)
+            tmem_cp_32x128b_x4(tmem + kColSFA8 + qs * 8 + i * 4, dqsf0 + ((qs * 2 + i) * kAtomBytes >> 4), leader);
+        }
+        // K tile kc is waited for, and (fp8 PV) its atom copied into slot kc & 1, right after the
+        // previous tile's last QK has been issued, so that neither sits between the next SFree
+        // and the next QK. The slot's last reader, a QK of tile kc - 2, completed before the S
+        // that the last SFree released was written.
+        auto prepare_k = [&]() -> bool {
+          if (!wait_role(&bars[kBarKFull + kc % kKStages], (kc / kKStages) & 1, abort_flag)) return false;
+          if (!kMx) {
+            tc_fence_after();
+            tmem_cp_32x128b_x4(tmem + kColSFB8 + (kc & 1) * 4, dksf0 + ((kc % kKStages) * kAtomBytes >> 4), leader);
+          }
+          return true;
+        };
+        if (!prepare_k()) { record_failure(abort_flag, kPSiteMmaK); ok = false; break; }
         for (int j = 0; j < ui.nkv && ok; ++j) {
           const uint32_t s = kc % kKStages;
-          if (!wait_role(&bars[kBarKFull + s], (kc / kKStages) & 1, abort_flag)) { record_failure(abort_flag, kPSiteMmaK); ok = false; break; }
-          tc_fence_after();
-          const uint32_t sfb = tmem + kColSFB + (kc & 1) * 4;
-          tmem_cp_32x128b_x4(sfb, dksf0 + (s * kAtomBytes >> 4), leader);
           const uint64_t bdesc = dk0 + (s * kTileBytes >> 4);
+          const uint32_t sfb = tmem + (kMx ? kColSFB : kColSFB8 + (kc & 1) * 4);
           for (int i = 0; i <= ui.has_q1; ++i) {
             if (uses > 0) {
+#if LPFA_PP_SFREE_SPIN
+              if (!mbar_wait_warp(&bars[kBarSFree], (uses - 1) & 1, abort_flag)) { record_failure(abort_flag, kPSiteMmaS); ok = false; break; }
+#else
               if (!wait_role(&bars[kBarSFree], (uses - 1) & 1, abort_flag)) { record_failure(abort_flag, kPSiteMmaS); ok = false; break; }
-              tc_fence_after();
+#endif
+            }
+            tc_fence_after();
+            const uint32_t sfa = tmem + (kMx ? kColSFA : kColSFA8 + qs * 8 + i * 4);
+            if (kMx) {
+              // Scale atoms into their single TMEM slots, in order with the MMAs below. The QK that
+              // last read them wrote the previous S, which its warpgroup has read out (SFree), so
+              // it has completed.
+              tmem_cp_32x128b_x4(sfa, dqsf0 + ((qs * 2 + i) * kAtomBytes >> 4), leader);
+              if (i == 0) tmem_cp_32x128b_x4(sfb, dksf0 + (s * kAtomBytes >> 4), leader);
             }
             const uint64_t adesc = dq0 + ((qs * 2 + i) * kTileBytes >> 4);
-            const uint32_t sfa = tmem + kColSFA + qs * 8 + i * 4;
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {  // K = 32 bytes per MMA, scale byte kk
               const uint32_t byte_sel = static_cast<uint32_t>(kk) << 30;
@@ -451,6 +500,7 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
           mma_commit(&bars[kBarKEmpty + s], leader);
           if (j == ui.nkv - 1) mma_commit(&bars[kBarQEmpty + qs], leader);
           ++kc;
+          if (j + 1 < ui.nkv && !prepare_k()) { record_failure(abort_flag, kPSiteMmaK); ok = false; break; }
         }
         ++u;
       }
@@ -462,8 +512,8 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
       const uint64_t dv0 = umma_desc(sb + L::v, kTileBytes, 1024, kLayoutSw128);
       const uint64_t dpsf0 = umma_desc(sb + L::p_sf, 0, 128, kLayoutNone);
       const uint64_t dvsf0 = umma_desc(sb + L::v_sf, 0, 128, kLayoutNone);
-      uint32_t vc = 0;
-      uint32_t pc[2] = {0, 0};  // P tiles consumed per warpgroup
+      uint32_t vc = 0;          // V tiles
+      uint32_t n = 0;           // P tiles, in the order the PVs consume them
       uint32_t uc[2] = {0, 0};  // units per warpgroup
       bool ok = true;
       for (int w = blockIdx.x; w < num_units && ok; w += G) {
@@ -471,23 +521,25 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
         if (ui.nkv == 0) continue;
         for (int j = 0; j < ui.nkv && ok; ++j) {
           const uint32_t vs = vc % kVStages;
+          // V first: it is loaded well ahead, so this wait is off the path from P to PV.
+          if (!wait_role(&bars[kBarVFull + vs], (vc / kVStages) & 1, abort_flag)) { record_failure(abort_flag, kPSiteMmaV); ok = false; break; }
+          const uint64_t bdesc = dv0 + (vs * kTileBytes >> 4);
           for (int i = 0; i <= ui.has_q1; ++i) {
-            if (!wait_role(&bars[kBarPReady + i], pc[i] & 1, abort_flag)) { record_failure(abort_flag, kPSiteMmaP); ok = false; break; }
+            const uint32_t ps = n % kPSlots;
+            if (!wait_role(&bars[kBarPReady + ps], (n / kPSlots) & 1, abort_flag)) { record_failure(abort_flag, kPSiteMmaP); ok = false; break; }
             if (j == 0 && !wait_role(&bars[kBarOEmpty + i], (uc[i] & 1) ^ 1, abort_flag)) { record_failure(abort_flag, kPSiteMmaO); ok = false; break; }
-            if (i == 0 && !wait_role(&bars[kBarVFull + vs], (vc / kVStages) & 1, abort_flag)) { record_failure(abort_flag, kPSiteMmaV); ok = false; break; }
             tc_fence_after();
-            const uint32_t p_col = tmem + kColP + i * 32;
+            const uint32_t p_col = tmem + kColP + ps * 32;
             const uint32_t o_col = tmem + kColO + i * 128;
-            const uint64_t bdesc = dv0 + (vs * kTileBytes >> 4);
             if (kMx) {
-              // Scale atoms into TMEM, in order with the MMAs below: V's once per V tile (slot
-              // vc & 1: the PVs that read that slot two tiles ago completed before P_0 of this
-              // tile was stored), P_i's from the softmax's shared-memory atom (its previous
-              // reader, PV_i of the previous tile, completed before P_i was stored).
-              const uint32_t sfv = tmem + kColSFV + (vc & 1) * 4;
-              const uint32_t sfp = tmem + kColSFP + i * 4;
+              // Scale atoms into TMEM, in order with the MMAs below: V's once per V tile into slot
+              // vc % 3, P's from the softmax's shared-memory atom of this P slot into the matching
+              // TMEM slot. Before storing this P the softmax waited for the PV three P tiles
+              // back, so every PV that read either slot earlier has completed.
+              const uint32_t sfv = tmem + kColSFV + (vc % 3) * 4;
+              const uint32_t sfp = tmem + kColSFP + ps * 4;
               if (i == 0) tmem_cp_32x128b_x4(sfv, dvsf0 + (vs * kAtomBytes >> 4), leader);
-              tmem_cp_32x128b_x4(sfp, dpsf0 + (i * kAtomBytes >> 4), leader);
+              tmem_cp_32x128b_x4(sfp, dpsf0 + (ps * kAtomBytes >> 4), leader);
 #pragma unroll
               for (int kk = 0; kk < 4; ++kk) {  // keys [32kk, 32kk + 32), scale byte kk
                 const uint32_t byte_sel = static_cast<uint32_t>(kk) << 30;
@@ -499,8 +551,8 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
               for (int kk = 0; kk < 4; ++kk)  // keys [32kk, 32kk + 32): 8 columns of 4 E4M3 each
                 mma_f8f6f4_ts(o_col, p_col + kk * 8, bdesc + kk * 256, kIdescPV8, (j > 0 || kk > 0) ? 1u : 0u, leader);
             }
-            mma_commit(&bars[kBarPVDone + i], leader);
-            ++pc[i];
+            mma_commit(&bars[kBarPVDone + ps], leader);
+            ++n;
           }
           if (!ok) break;
           mma_commit(&bars[kBarVEmpty + vs], leader);
@@ -529,10 +581,14 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
     const float cscale_all = kPerUnitDescale ? 0.0f
                                              : fabsf((descale_value(p.q_descale, 0, 0) *
                                                       descale_value(p.k_descale, 0, 0)) * kLog2eRsqrtD);
-    uint32_t sc = 0, pcnt = 0, ucnt = 0;  // S tiles read, P tiles handed over, units finished
+    uint32_t sc = 0, ucnt = 0;  // S tiles read, units finished
+    uint32_t nbase = 0;         // P tiles of all earlier units, in the order the PVs consume them
     bool ok = true;
     for (int w = blockIdx.x; w < num_units && ok; w += G) {
       const PairUnit ui = pair_unit(p, sched, w);
+      const uint32_t np = 1u + static_cast<uint32_t>(ui.has_q1);  // P tiles per key tile
+      const uint32_t n0 = nbase;
+      nbase += static_cast<uint32_t>(ui.nkv) * np;
       if (grp > ui.has_q1) continue;
       const bool valid = (ui.qtile0 + grp) * kTileM + row < ui.q_len;
       const int64_t tok = ui.q_row0 + grp * kTileM + row;
@@ -552,7 +608,7 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
       float m_r = -INFINITY;  // row reference (integer, log2 units)
       float l_r = 0.0f;       // row sum of p (times 2^kBias), relative to m_r
       for (int j = 0; j < ui.nkv; ++j) {
-        if (!mbar_wait_warp(&bars[kBarSFull + grp], sc & 1, abort_flag)) { record_failure(abort_flag, kPSiteSoftS); ok = false; break; }
+        if (!wait_warp(&bars[kBarSFull + grp], sc & 1, abort_flag, false)) { record_failure(abort_flag, kPSiteSoftS); ok = false; break; }
         tc_fence_after();
         float2 sv[64];
         load_row(tmem + lane_addr + kColS, sv);
@@ -605,23 +661,27 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
         const float m_prev = m_r;
         l_r = l_r * exp2_int(m_prev - m_new) + psum;
         m_r = m_new;
-        // P_i's slot is free, and O_i holds every earlier tile, once PV_i of the previous tile
-        // has completed (at a unit's first tile that is the previous unit's last PV_i, which the
-        // epilogue already waited for).
-        if (pcnt > 0) {
-          if (!mbar_wait_warp(&bars[kBarPVDone + grp], (pcnt - 1) & 1, abort_flag)) { record_failure(abort_flag, kPSiteSoftPV); ok = false; break; }
+        // This P's slot is free once the PV three P tiles back, its previous reader, has completed.
+        const uint32_t n = n0 + static_cast<uint32_t>(j) * np + static_cast<uint32_t>(grp);
+        const uint32_t ps = n % kPSlots;
+        if (n >= kPSlots) {
+          if (!wait_warp(&bars[kBarPVDone + ps], ((n - kPSlots) / kPSlots) & 1, abort_flag, false)) { record_failure(abort_flag, kPSiteSoftPV); ok = false; break; }
           tc_fence_after();
         }
         if (kMx) {
           // The row's four scale bytes go to this warpgroup's shared-memory atom (row r at
           // (r % 32) * 16 + (r / 32) * 4), read by the PV issuer's tcgen05.cp.
-          p_sf_words[grp * (kAtomBytes / 4) + (row & 31) * 4 + (row >> 5)] = mx_sfw;
+          p_sf_words[ps * (kAtomBytes / 4) + (row & 31) * 4 + (row >> 5)] = mx_sfw;
           fence_proxy_async_smem();
         }
-        tmem_st32_sync(tmem + lane_addr + kColP + grp * 32, pk);
+        tmem_st32_sync(tmem + lane_addr + kColP + ps * 32, pk);
         // O_i holds tiles up to j - 1 relative to m_prev: rescale it when the reference moved
-        // (rare; never on a unit's first tile).
+        // (rare; never on a unit's first tile), once PV_i of tile j - 1 has completed. (That PV's
+        // slot cannot have been reused yet: its next use needs this P consumed first.)
         if (j > 0 && __any_sync(0xFFFFFFFFu, m_new != m_prev)) {
+          const uint32_t nprev = n - np;
+          if (!wait_warp(&bars[kBarPVDone + nprev % kPSlots], (nprev / kPSlots) & 1, abort_flag, false)) { record_failure(abort_flag, kPSiteSoftPV); ok = false; break; }
+          tc_fence_after();
           const float alpha = exp2_int(m_prev - m_new);
           const float2 a2 = make_float2(alpha, alpha);
           const uint32_t o_addr = tmem + lane_addr + kColO + grp * 128;
@@ -640,12 +700,11 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bars[kBarPReady + grp]);
-        ++pcnt;
+        if (lane == 0) mbar_arrive(&bars[kBarPReady + ps]);
       }
       if (!ok) break;
       // ---------------------------------------------------------------- epilogue
-      if (!mbar_wait_warp(&bars[kBarOFull + grp], ucnt & 1, abort_flag)) { record_failure(abort_flag, kPSiteSoftO); ok = false; break; }
+      if (!wait_warp(&bars[kBarOFull + grp], ucnt & 1, abort_flag, false)) { record_failure(abort_flag, kPSiteSoftO); ok = false; break; }
       tc_fence_after();
       const float oscale = descale_value(p.v_descale, ui.seq, ui.h) / l_r;
       uint4* dst = reinterpret_cast<uint4*>(p.out + (tok * p.heads + ui.h) * 128);
