@@ -351,11 +351,11 @@ static lpfa_status launch_attn(int grid, cudaStream_t s, const CUtensorMap& tq, 
   return LPFA_OK;
 }
 
-// The 8-bit P modes run over pairs of query tiles (attn_fwd_pp.cuh).
+// Every PV mode runs over pairs of query tiles (attn_fwd_pp.cuh).
 template <int kPv, bool kPerUnit>
 static lpfa_status launch_attn_pp(int grid, cudaStream_t s, const CUtensorMap& tq, const CUtensorMap& tk,
                                   const CUtensorMap& tv, const lpfa::AttnParams& p) {
-  constexpr uint32_t smem = lpfa::pp::smem_bytes<kPv == lpfa::kPvMx>();
+  constexpr uint32_t smem = lpfa::pp::smem_bytes<kPv>();
   const void* fn = reinterpret_cast<const void*>(lpfa::pp::attn_fwd_pp_kernel<kPv, kPerUnit>);
   const lpfa_status st = check_attn_kernel(fn, smem);
   if (st != LPFA_OK) return st;
@@ -445,14 +445,14 @@ static lpfa_status attn_fwd_impl(const uint8_t* q, const uint8_t* q_sf, const ui
     st = per_unit ? launch_attn_pp<lpfa::kPvFp8, true>(grid, s, tq, tk, tv, p)
                   : launch_attn_pp<lpfa::kPvFp8, false>(grid, s, tq, tk, tv, p);
   } else if (pv_mode == LPFA_PV_BF16) {
-    st = per_unit ? launch_attn<lpfa::kPvBf16Mx, true>(grid, s, tq, tk, tv, p)
-                  : launch_attn<lpfa::kPvBf16Mx, false>(grid, s, tq, tk, tv, p);
+    st = per_unit ? launch_attn_pp<lpfa::kPvBf16Mx, true>(grid, s, tq, tk, tv, p)
+                  : launch_attn_pp<lpfa::kPvBf16Mx, false>(grid, s, tq, tk, tv, p);
   } else if (pv_mode == LPFA_PV_MXFP8) {
     st = per_unit ? launch_attn_pp<lpfa::kPvMx, true>(grid, s, tq, tk, tv, p)
                   : launch_attn_pp<lpfa::kPvMx, false>(grid, s, tq, tk, tv, p);
   } else {
-    st = per_unit ? launch_attn<lpfa::kPvBf16In, true>(grid, s, tq, tk, tv, p)
-                  : launch_attn<lpfa::kPvBf16In, false>(grid, s, tq, tk, tv, p);
+    st = per_unit ? launch_attn_pp<lpfa::kPvBf16In, true>(grid, s, tq, tk, tv, p)
+                  : launch_attn_pp<lpfa::kPvBf16In, false>(grid, s, tq, tk, tv, p);
   }
   if (st != LPFA_OK) return st;
   e = cudaGetLastError();
