@@ -47,13 +47,12 @@ TRAFFIC = {
     # workload: (sha256 of the kernel's sources [:16], dram bytes read + written per launch)
 }
 
-# The source files of the attention kernel each PV mode runs (the 8-bit P modes run over pairs
-# of query tiles), and that kernel's name.
+# The source files of the attention kernel each PV mode runs, and that kernel's name.
 KERNEL_SOURCES = {
     "fp8": (["attn_fwd_pp.cuh", "attn_fwd.cuh", "ptx.cuh"], "attn_fwd_pp_kernel"),
     "mxfp8": (["attn_fwd_pp.cuh", "attn_fwd.cuh", "ptx.cuh"], "attn_fwd_pp_kernel"),
-    "bf16": (["attn_fwd.cuh", "ptx.cuh"], "attn_fwd_kernel"),
-    "bf16v": (["attn_fwd.cuh", "ptx.cuh"], "attn_fwd_kernel"),
+    "bf16": (["attn_fwd_pp.cuh", "attn_fwd.cuh", "ptx.cuh"], "attn_fwd_pp_kernel"),
+    "bf16v": (["attn_fwd_pp.cuh", "attn_fwd.cuh", "ptx.cuh"], "attn_fwd_pp_kernel"),
 }
 
 

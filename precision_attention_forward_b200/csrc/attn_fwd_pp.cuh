@@ -715,8 +715,8 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
     setmaxnreg_inc<kSoftmaxRegs>();
     // ------------------------------------------------------------------ softmax warpgroups
     // (Block-scaled and bf16 P have no E4M3 range limit to respect: they take a lag of 8 binades.)
-    constexpr float kLag = kPv == kPvFp8 ? kLagP8 : SoftmaxLag<false>::lag;
-    constexpr float kBias = kPv == kPvFp8 ? kBiasP8 : SoftmaxLag<false>::bias;
+    constexpr float kLag = kPv == kPvFp8 ? kLagP8 : kLagWide;
+    constexpr float kBias = kPv == kPvFp8 ? kBiasP8 : kBiasWide;
     uint32_t* p_sf_words = reinterpret_cast<uint32_t*>(smem + L::p_sf);
     const int grp = (warp - 4) >> 2;                 // query tile of the unit this warpgroup owns
     const int quarter = warp & 3;                    // TMEM lane quarter of this warp
@@ -778,7 +778,6 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
         float psum, prsum = 0.0f;
         uint32_t mx_sfw = 0;  // block-scaled MXFP8 P: this row's four E8M0 scale bytes
         uint32_t pk[32];      // 8-bit P as E4M3 codes, four keys per word
-        auto no_handoff = [](float) {};
         if (kMx) {
           // The reference moves only when the tile's ceiling exceeds it by more than the lag, so
           // the rescales are rare exact powers of two.
@@ -795,8 +794,8 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
             nbg[g] = nb - static_cast<float>(eg[g]);
             mx_sfw |= static_cast<uint32_t>(eg[g] + 127) << (8 * g);
           }
-          if (tail) exp_row_groups<true>(sv, cscale, nbg, key0, ui.k_len, no_handoff, gsum);
-          else exp_row_groups<false>(sv, cscale, nbg, key0, ui.k_len, no_handoff, gsum);
+          if (tail) exp_row_groups<true>(sv, cscale, nbg, key0, ui.k_len, gsum);
+          else exp_row_groups<false>(sv, cscale, nbg, key0, ui.k_len, gsum);
           psum = 0.0f;
 #pragma unroll
           for (int g = 0; g < 4; ++g)  // sum of the unscaled p: exact powers of two (2^-126 for an empty group)

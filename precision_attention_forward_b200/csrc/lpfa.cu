@@ -340,17 +340,6 @@ static lpfa_status check_attn_kernel(const void* fn, uint32_t smem_bytes) {
 }
 
 extern "C++" {
-template <int kPv, bool kPerUnit>
-static lpfa_status launch_attn(int grid, cudaStream_t s, const CUtensorMap& tq, const CUtensorMap& tk,
-                               const CUtensorMap& tv, const lpfa::AttnParams& p) {
-  constexpr uint32_t smem = lpfa::attn_smem_bytes<lpfa::pv_p8<kPv>()>();
-  const void* fn = reinterpret_cast<const void*>(lpfa::attn_fwd_kernel<kPv, kPerUnit>);
-  const lpfa_status st = check_attn_kernel(fn, smem);
-  if (st != LPFA_OK) return st;
-  lpfa::attn_fwd_kernel<kPv, kPerUnit><<<grid, lpfa::kAttnThreads, smem, s>>>(tq, tk, tv, p);
-  return LPFA_OK;
-}
-
 // Every PV mode runs over pairs of query tiles (attn_fwd_pp.cuh).
 template <int kPv, bool kPerUnit>
 static lpfa_status launch_attn_pp(int grid, cudaStream_t s, const CUtensorMap& tq, const CUtensorMap& tk,
