@@ -170,3 +170,30 @@ def attention_rows(qhat_rows, seq_of_row, head_of_row, khat, vhat, lengths_k,
         out[rows] = o
         lse[rows] = l
     return out, lse
+
+
+def attention_fwd_shared_q(qhat, khat, vhat, lengths_k, qd=1.0, kd=1.0, vd=1.0, p_mode: str = "exact"):
+    """Shared-query forward: one query set attends to each of several key/value sequences.
+
+    Reading of the LP-FA4 README's "shared-query workloads" (its opening paragraph names them
+    beside dense and packed variable-length ones but does not define them): the query sequence
+    is shared, and key/value sequence i of the packed K/V gives its own output block,
+
+        O_i = attention(Q, K_i, V_i),   LSE_i likewise,   i = 0 .. n - 1,
+
+    stacked along the tokens. qhat (Lq,H,128); khat/vhat (Tk,H,128) float64; descales are
+    indexed by (key/value sequence, head). Returns O (n*Lq, H, 128) and LSE (H, n*Lq).
+    """
+    mk = _meta.from_lengths(lengths_k)
+    Lq, H, _ = qhat.shape
+    n = mk.num_seqs
+    out = np.zeros((n * Lq, H, HEAD_DIM), dtype=np.float64)
+    lse = np.zeros((H, n * Lq), dtype=np.float64)
+    for i in range(n):
+        k0, k1 = int(mk.cu_seqlens[i]), int(mk.cu_seqlens[i + 1])
+        for h in range(H):
+            o, l = attend_block(qhat[:, h], khat[k0:k1, h], vhat[k0:k1, h],
+                                descale_at(qd, i, h), descale_at(kd, i, h), descale_at(vd, i, h), p_mode)
+            out[i * Lq:(i + 1) * Lq, h] = o
+            lse[h, i * Lq:(i + 1) * Lq] = l
+    return out, lse

@@ -325,3 +325,37 @@ def test_mxfp8_variant_differs_from_fp8_and_plain():
     err_m = abs(o_m[0, 1] - o_e[0, 1]) / o_e[0, 1]
     err_f = abs(o_f[0, 1] - o_e[0, 1]) / o_e[0, 1]
     assert err_m < 2 ** -10 and 0.07 < err_f < 0.08, (err_m, err_f)
+
+
+def test_shared_query_blocks_by_brute_force_and_closed_forms():
+    """Shared-query reading (LP-FA4 README, opening paragraph: "shared-query workloads"): block i
+    of the output is the attention of the one query set over key/value sequence i. Pinned by
+    pure-Python brute force per block (with per-(sequence, head) descales), identical key/value
+    sequences giving identical blocks, constant V giving V, and a single key giving that V row
+    with LSE equal to its logit."""
+    g = np.random.default_rng(21)
+    Lq, H, lk = 3, 2, [4, 1, 6]
+    q = g.standard_normal((Lq, H, 128))
+    k = g.standard_normal((sum(lk), H, 128))
+    v = g.standard_normal((sum(lk), H, 128))
+    qd = np.array([0.5, 2.0])
+    kd = np.array([[1.0, 0.5], [1.5, 1.0], [0.25, 3.0]])
+    vd = 1.5
+    o, lse = oatt.attention_fwd_shared_q(q, k, v, lk, qd, kd, vd)
+    assert o.shape == (len(lk) * Lq, H, 128) and lse.shape == (H, len(lk) * Lq)
+    cu = np.concatenate([[0], np.cumsum(lk)])
+    for i in range(len(lk)):
+        for h in range(H):
+            ob, lb = _brute_attention(q[:, h], k[cu[i]:cu[i + 1], h], v[cu[i]:cu[i + 1], h], qd[h], kd[i, h], vd)
+            assert np.allclose(o[i * Lq:(i + 1) * Lq, h], ob, atol=1e-12)
+            assert np.allclose(lse[h, i * Lq:(i + 1) * Lq], lb, atol=1e-12)
+    # single key (sequence 1): O = vd * v, LSE = that logit
+    s1 = (q[:, 0] @ k[cu[1], 0]) * qd[0] * kd[1, 0] * SCALE
+    assert np.allclose(o[Lq:2 * Lq, 0], vd * v[cu[1], 0][None], atol=1e-12)
+    assert np.allclose(lse[0, Lq:2 * Lq], s1, atol=1e-12)
+    # identical key/value sequences give identical blocks; constant V gives V
+    k2 = np.concatenate([k[:4], k[:4]])
+    v2 = np.concatenate([np.repeat(v[:1], 4, axis=0), np.repeat(v[:1], 4, axis=0)])
+    o2, l2 = oatt.attention_fwd_shared_q(q, k2, v2, [4, 4])
+    assert np.array_equal(o2[:Lq], o2[Lq:]) and np.array_equal(l2[:, :Lq], l2[:, Lq:])
+    assert np.allclose(o2, np.broadcast_to(v[0][None], o2.shape), atol=1e-12)
