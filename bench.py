@@ -75,6 +75,10 @@ def load_peaks():
 
 
 def attention_flops(lq, lk, heads) -> float:
+    """4 * Sq * Sk * H * 128 summed over the (query, key) sequence pairs; a single query sequence
+    with several key sequences is the shared-query workload (the query set pairs with each)."""
+    if len(lq) == 1 and len(lk) > 1:
+        return float(sum(4.0 * lq[0] * b * heads * 128 for b in lk))
     return float(sum(4.0 * a * b * heads * 128 for a, b in zip(lq, lk)))
 
 
@@ -156,7 +160,8 @@ def cpu_oracle_sample(w, seconds: float, seed: int = 0):
     units = 0
     t0 = time.perf_counter()
     while time.perf_counter() - t0 < seconds:
-        i = units % len(lq)
+        i = units % len(lk)
+        iq = 0 if w.shared_q else i   # a shared query set pairs with every K/V sequence
         h = (units // len(lq)) % w.heads
         k0, k1 = cu_k[i], cu_k[i + 1]
         kp, ke = omx.quantize_rows(k[k0:k1, h].astype(np.float64), w.scaling_mode)
@@ -171,8 +176,8 @@ def cpu_oracle_sample(w, seconds: float, seed: int = 0):
         else:
             vp, ve = omx.quantize_rows(v[k0:k1, h].astype(np.float64), w.scaling_mode)
             vh = (omx.e4m3_decode(vp).reshape(-1, 4, 32) * np.ldexp(1.0, ve)[..., None]).reshape(-1, 128)
-        r0 = cu_q[i] + (units * rows_per) % max(1, lq[i] - rows_per + 1)
-        r1 = min(cu_q[i + 1], r0 + rows_per)
+        r0 = cu_q[iq] + (units * rows_per) % max(1, lq[iq] - rows_per + 1)
+        r1 = min(cu_q[iq + 1], r0 + rows_per)
         qp, qe = omx.quantize_rows(q[r0:r1, h].astype(np.float64), w.scaling_mode)
         qh = (omx.e4m3_decode(qp).reshape(-1, 4, 32) * np.ldexp(1.0, qe)[..., None]).reshape(-1, 128)
         oatt.attend_block(qh, kh, vh, p_mode={"fp8": "fp8", "mxfp8": "mxfp8"}.get(w.pv_mode, "exact"))
@@ -187,6 +192,41 @@ def cpu_oracle_sample(w, seconds: float, seed: int = 0):
     desc = (f"{units} units of {rows_per} query rows x all keys of one (sequence, head), each with that "
             f"head's K/V quantization, fp64 numpy oracle")
     return done_flops / elapsed / 1e12, desc, cores, elapsed
+
+
+def cpu_quantizer_sample(w, x, lens, payload_dev, scales_dev, in_bytes: int, seconds: float):
+    """Time the CPU oracle's MXFP8 quantizer on a bounded sample of one input tensor: 4096-token
+    chunks (128-aligned, so each is a sequence of its own with the same scale atoms) of the packed
+    sequences in order, until `seconds` have passed. Algorithmic bytes as for the GPU quantizer
+    (in_bytes + 1 per element, 512 per (128-token block, head) atom). Every byte of the chunks it
+    quantized is compared with the GPU's payload and scales of the same tensor from this run.
+    Returns (MB/s, description, bit_exact, elapsed)."""
+    from oracle import meta as ometa
+    from oracle import mxfp8 as omx
+
+    m = ometa.from_lengths(lens)
+    H = x.shape[1]
+    chunks = []
+    for i in range(m.num_seqs):
+        n, c0 = int(m.lengths[i]), int(m.cu_seqlens[i])
+        for t0 in range(0, n, 4096):
+            chunks.append((i, c0 + t0, min(n, t0 + 4096) - t0, int(m.scale_off[i]) + t0 // 128))
+    done, exact, nbytes = 0, True, 0.0
+    t0 = time.perf_counter()
+    results = []
+    while done < len(chunks) and (done == 0 or time.perf_counter() - t0 < seconds):
+        _, row0, rows, _ = chunks[done]
+        results.append(omx.quantize_mxfp8_varlen(x[row0:row0 + rows], [rows], w.scaling_mode))
+        nbytes += rows * H * 128 * (in_bytes + 1) + ((rows + 127) // 128) * H * 512
+        done += 1
+    elapsed = time.perf_counter() - t0
+    for (_, row0, rows, b0), (ref_p, ref_s) in zip(chunks[:done], results):
+        got_p = payload_dev[row0:row0 + rows].cpu().numpy()
+        got_s = scales_dev[b0 * H * 512:b0 * H * 512 + ref_s.size].cpu().numpy()
+        exact = exact and np.array_equal(got_p, ref_p) and np.array_equal(got_s, ref_s)
+    desc = (f"{done} chunks of up to 4096 tokens x {H} heads of Q ({'fp32' if in_bytes == 4 else 'bf16'}), "
+            f"fp64 numpy oracle quantizer ({w.scaling_mode}), each compared byte for byte with the GPU's")
+    return nbytes / elapsed / 1e6, desc, exact, elapsed
 
 
 def run_reference(args, w):
@@ -266,6 +306,7 @@ def config_dict(w, lq, lk, n):
         "seq_len_q": int(max(lq)), "seq_len_k": int(max(lk)), "total_tokens_q": int(np.sum(lq)),
         "total_tokens_k": int(np.sum(lk)), "heads": w.heads, "head_dim": 128, "pv_mode": w.pv_mode,
         "in_dtype": w.in_dtype, "scaling_mode": w.scaling_mode, "global_batch": int(w.num_seqs) * n,
+        "shared_q": bool(w.shared_q),
         "parallelism": f"replicas{n}" if n > 1 else "single",
         "l2": "inputs larger than L2 (no flush)" if l2_exceeded(lk, w.heads)
               else "L2 flushed between steps (256 MB write), step time from per-step events",
@@ -383,6 +424,7 @@ def main():
     dts = {x: wl.tensor_dtype(w, x) for x in "qkv"}
     dev_in = {x: wl.to_torch(host[x], dts[x], device=dev) for x in "qkv"}
     Tq, Tk = int(np.sum(lq)), int(np.sum(lk))
+    To = Tq * len(lk) if w.shared_q else Tq   # output rows
     mq0 = lp.lpfa_varlen_meta_from_lengths(lq, device=dev)
     sbq, sbk = mq0.total_scale_blocks, lp.lpfa_varlen_meta_from_lengths(lk, device=dev).total_scale_blocks
     qp = torch.empty((Tq, H, 128), dtype=torch.uint8, device=dev)
@@ -391,8 +433,8 @@ def main():
     qs = torch.empty(sbq * H * 512, dtype=torch.uint8, device=dev)
     ks = torch.empty(sbk * H * 512, dtype=torch.uint8, device=dev)
     vs = torch.empty(sbk * H * 512, dtype=torch.uint8, device=dev) if w.pv_mode in ("bf16", "mxfp8") else None
-    out = torch.empty((Tq, H, 128), dtype=torch.bfloat16, device=dev)
-    lse = torch.empty((H, Tq), dtype=torch.float32, device=dev)
+    out = torch.empty((To, H, 128), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((H, To), dtype=torch.float32, device=dev)
 
     def step(ins, timing=None):
         mq = lp.lpfa_varlen_meta_from_lengths(lq, device=dev)
@@ -412,7 +454,8 @@ def main():
             c = torch.cuda.Event(enable_timing=True)
             c.record(stream)
         v_in = ins["v"] if w.pv_mode == "bf16v" else vp   # BF16 V goes to the kernel as is
-        lp.lpfa_attn_fwd_varlen(qp, qs, kp, ks, v_in, vs, mq, mk, pv_mode=w.pv_mode, out=out, lse=lse)
+        attn = lp.lpfa_attn_fwd_shared_q if w.shared_q else lp.lpfa_attn_fwd_varlen
+        attn(qp, qs, kp, ks, v_in, vs, mq, mk, pv_mode=w.pv_mode, out=out, lse=lse)
         if timing is not None:
             b.record(stream)
             timing.append((a, c, b))
@@ -507,8 +550,13 @@ def main():
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
             tf, desc, cores, el = cpu_oracle_sample(w, float(os.environ.get("LPFA_CPU_SECONDS", "15")))
+            qmbs, qdesc, qexact, qel = cpu_quantizer_sample(w, host["q"], lq, qp, qs,
+                                                            2 if dts["q"] == "bf16" else 4,
+                                                            float(os.environ.get("LPFA_CPU_QUANT_SECONDS", "5")))
             cpu = {"value": tf, "unit": "TFLOPS", "cores": cores, "kind": "oracle", "sample": desc,
-                   "seconds": el}
+                   "seconds": el,
+                   "quantizer": {"value": qmbs, "unit": "MB/s", "sample": qdesc, "seconds": qel,
+                                 "bit_exact_vs_gpu": bool(qexact)}}
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",

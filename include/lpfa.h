@@ -232,6 +232,33 @@ LPFA_API lpfa_status lpfa_attn_fwd_varlen_descaled(const uint8_t* q, const uint8
                                           void* stream);
 
 /*
+ * Shared-query forward (LP-FA4 README, opening paragraph: the MXFP8 API covers "dense, packed
+ * variable-length, and shared-query workloads"; the pages do not define the last). Reading taken:
+ * one query sequence is shared by n key/value sequences, and each key/value sequence i gives its
+ * own output block, O_i = attention(Q, K_i, V_i) (and LSE_i), stacked along the tokens. The kernel
+ * reads the shared Q tiles for every block instead of a copy per block, longest K/V first.
+ *
+ * q, q_sf          device, Q payload (Lq, H, 128) and its scale storage under meta_q, which must
+ *                  describe exactly one sequence of Lq tokens.
+ * k, k_sf, v, v_sf as for lpfa_attn_fwd_varlen, under meta_k (n >= 1 sequences).
+ * pv_mode          as for lpfa_attn_fwd_varlen.
+ * q/k/v_descale    as for lpfa_attn_fwd_varlen_descaled; the sequence index is that of the
+ *                  key/value sequence (0 .. n - 1).
+ * out_bf16         device, (n * Lq, H, 128) bf16: rows [i * Lq, (i + 1) * Lq) are block i.
+ * lse              device, (H, n * Lq) fp32, natural log, blocks laid out like out's rows.
+ * Alignment:       every tensor 16-byte aligned.
+ * Errors:          as for lpfa_attn_fwd_varlen, with meta_q.num_seqs != 1 (instead of a mismatch of
+ *                  sequence counts) and n * Lq above INT32_MAX returning LPFA_ERR_INVALID_ARG.
+ */
+LPFA_API lpfa_status lpfa_attn_fwd_shared_q(const uint8_t* q, const uint8_t* q_sf, const uint8_t* k,
+                                   const uint8_t* k_sf, const uint8_t* v, const uint8_t* v_sf,
+                                   const lpfa_varlen_meta* meta_q, const lpfa_varlen_meta* meta_k,
+                                   int32_t heads, int32_t head_dim, lpfa_pv_mode pv_mode,
+                                   const lpfa_descale* q_descale, const lpfa_descale* k_descale,
+                                   const lpfa_descale* v_descale, void* out_bf16, float* lse,
+                                   void* stream);
+
+/*
  * mxfp8_flash_attn_varlen_backward (LP-FA4 README, "MXFP8 forward and backward"): the gradients
  * of lpfa_attn_fwd_varlen's output with respect to the dequantized Q, K, V (quantization is not
  * differentiated), noncausal head-dim-128 MHA over packed variable-length sequences:

@@ -39,7 +39,7 @@ EXPORTED_SYMBOLS = (
     "lpfa_scale_bytes", "lpfa_quantize_mxfp8_varlen", "lpfa_cast_e4m3", "lpfa_attn_fwd_varlen",
     "lpfa_device_status", "lpfa_last_error_message", "lpfa_version", "lpfa_attn_fwd_varlen_debug",
     "lpfa_attn_fwd_varlen_descaled", "lpfa_quantize_mxfp8_varlen_tokens", "lpfa_attn_bwd_varlen",
-    "lpfa_attn_bwd_varlen_debug",
+    "lpfa_attn_bwd_varlen_debug", "lpfa_attn_fwd_shared_q",
 )
 
 
@@ -87,6 +87,8 @@ _lib.lpfa_attn_fwd_varlen_debug.argtypes = list(_lib.lpfa_attn_fwd_varlen.argtyp
 _lib.lpfa_attn_fwd_varlen_descaled.argtypes = (list(_lib.lpfa_attn_fwd_varlen.argtypes[:11]) +
                                                [ctypes.POINTER(_Descale)] * 3 + [_vp, _vp, _vp])
 _lib.lpfa_attn_fwd_varlen_descaled.restype = ctypes.c_int
+_lib.lpfa_attn_fwd_shared_q.argtypes = _lib.lpfa_attn_fwd_varlen_descaled.argtypes
+_lib.lpfa_attn_fwd_shared_q.restype = ctypes.c_int
 _lib.lpfa_attn_fwd_varlen_debug.restype = ctypes.c_int
 _lib.lpfa_device_status.argtypes = [_vp, ctypes.POINTER(_i32)]
 _lib.lpfa_device_status.restype = ctypes.c_int
@@ -280,6 +282,49 @@ def lpfa_attn_fwd_varlen(q: torch.Tensor, q_sf: torch.Tensor, k: torch.Tensor, k
         else:
             _check(_lib.lpfa_attn_fwd_varlen_descaled(*args[:11], ctypes.byref(descs[0]), ctypes.byref(descs[1]),
                                                       ctypes.byref(descs[2]), *args[14:]))
+    return out, lse
+
+
+def lpfa_attn_fwd_shared_q(q: torch.Tensor, q_sf: torch.Tensor, k: torch.Tensor, k_sf: torch.Tensor,
+                           v: torch.Tensor, v_sf: Optional[torch.Tensor], meta_q: VarlenMeta, meta_k: VarlenMeta,
+                           pv_mode: str = "bf16", q_descale: Optional[torch.Tensor] = None,
+                           k_descale: Optional[torch.Tensor] = None, v_descale: Optional[torch.Tensor] = None,
+                           out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None, stream=None):
+    """Shared-query forward (see include/lpfa.h): one query sequence (meta_q has one sequence of Lq
+    tokens) attends to each of the n key/value sequences of meta_k. Returns (out bf16 (n*Lq,H,128),
+    lse fp32 (H,n*Lq)); rows [i*Lq, (i+1)*Lq) belong to key/value sequence i. Descales as for
+    lpfa_attn_fwd_varlen, indexed by the key/value sequence."""
+    if pv_mode not in PV_MODES:
+        raise ValueError("pv_mode must be 'bf16', 'fp8', 'bf16v' or 'mxfp8'")
+    if meta_q.num_seqs != 1:
+        raise ValueError("a shared query set is one sequence")
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        want = torch.bfloat16 if (name == "v" and pv_mode == "bf16v") else torch.uint8
+        if t.dtype != want or t.dim() != 3 or not t.is_contiguous():
+            raise ValueError("%s must be a contiguous %s (tokens, heads, 128) tensor" % (name, want))
+    Lq, H = q.shape[0], q.shape[1]
+    rows = Lq * meta_k.num_seqs
+    descs = []
+    for name, t in (("q_descale", q_descale), ("k_descale", k_descale), ("v_descale", v_descale)):
+        if t is None:
+            descs.append(_Descale(None, 0, 0))
+            continue
+        ss, hs = descale_strides(t, meta_k.num_seqs, H)
+        if t.device != q.device:
+            raise ValueError("%s must be on the device of q" % name)
+        descs.append(_Descale(t.data_ptr(), ss, hs))
+    if out is None:
+        out = torch.empty((rows, H, 128), dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty((H, rows), dtype=torch.float32, device=q.device)
+    if tuple(out.shape) != (rows, H, 128) or tuple(lse.shape) != (H, rows):
+        raise ValueError("out must be (n*Lq, H, 128) and lse (H, n*Lq)")
+    with torch.cuda.device(q.device):
+        _check(_lib.lpfa_attn_fwd_shared_q(q.data_ptr(), q_sf.data_ptr(), k.data_ptr(), k_sf.data_ptr(), v.data_ptr(),
+                                           _ptr(v_sf), ctypes.byref(meta_q._c), ctypes.byref(meta_k._c), H, 128,
+                                           PV_MODES[pv_mode], ctypes.byref(descs[0]), ctypes.byref(descs[1]),
+                                           ctypes.byref(descs[2]), out.data_ptr(), lse.data_ptr(),
+                                           _stream_ptr(stream)))
     return out, lse
 
 

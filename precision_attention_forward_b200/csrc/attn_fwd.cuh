@@ -70,6 +70,8 @@ struct AttnParams {
   int total_q_tiles;        // meta_q.total_scale_blocks
   int num_units;            // heads * total_q_tiles
   int debug_stall;          // test hook: >0 makes the MMA warp wait on a phase that never comes
+  int shared_q;             // 1: one query sequence shared by num_seqs key/value sequences; output
+                            // block i (rows i * Lq ..) belongs to key/value sequence i
 };
 
 // Work order: up to this many sequences are ordered longest first (by key tiles) in shared

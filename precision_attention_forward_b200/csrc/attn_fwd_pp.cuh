@@ -133,9 +133,11 @@ enum PairSite : int {
   kPSiteConvV, kPSiteConvE
 };
 
-// A work unit: query tiles qtile0 and (has_q1) qtile0 + 1 of one (sequence, head).
+// A work unit: query tiles qtile0 and (has_q1) qtile0 + 1 of one (sequence, head). seq is the
+// key/value sequence (and the descales' sequence index); q_row0 the first query row read, o_row0
+// the first output (and LSE) row written -- they differ only for a shared query set.
 struct PairUnit {
-  int h, seq, qtile0, q_row0, q_len, k_row0, k_len, nkv, sbq, sbk, has_q1;
+  int h, seq, qtile0, q_row0, o_row0, q_len, k_row0, k_len, nkv, sbq, sbk, has_q1;
 };
 
 // Unit order in shared memory: sched[0] = n, sched[1] = number of units, then order[kMaxSortSeqs]
@@ -144,15 +146,22 @@ struct PairUnit {
 // consecutive units, pairs innermost, so that the CTAs running together share one (sequence,
 // head)'s K/V through L2 and the static round-robin over the list approximates longest-processing-
 // time scheduling. Beyond kMaxSortSeqs sequences (n = 0) every unit is a single tile in the packed
-// head-major order (the pairs' prefix would not fit in shared memory).
+// head-major order (the pairs' prefix would not fit in shared memory); with a shared query set
+// (n = -1) every key/value sequence has the same number of query tiles, so pairs stay and the
+// plain order (sequence, head, pair) needs no prefix.
+__device__ __forceinline__ int query_tiles_of(const AttnParams& p, int seq) {
+  const int qs = p.shared_q ? 0 : seq;
+  return __ldg(p.so_q + qs + 1) - __ldg(p.so_q + qs);
+}
+
 __device__ __forceinline__ void build_pair_order(const AttnParams& p, int* sched) {
   const int n = p.num_seqs;
   int* s_order = sched + 2;
   int* s_pre = sched + 2 + kMaxSortSeqs;
   if (n > kMaxSortSeqs) {
     if (threadIdx.x == 0) {
-      sched[0] = 0;
-      sched[1] = p.num_units;  // heads * total query tiles
+      sched[0] = p.shared_q ? -1 : 0;
+      sched[1] = p.shared_q ? n * p.heads * ((query_tiles_of(p, 0) + 1) >> 1) : p.num_units;
     }
     __syncthreads();
     return;
@@ -176,11 +185,7 @@ __device__ __forceinline__ void build_pair_order(const AttnParams& p, int* sched
     for (int base = 0; base < n; base += 32) {
       const int r = base + static_cast<int>(threadIdx.x);
       int v = 0;
-      if (r < n) {
-        const int sq = s_order[r];
-        const int nt = __ldg(p.so_q + sq + 1) - __ldg(p.so_q + sq);
-        v = p.heads * ((nt + 1) >> 1);
-      }
+      if (r < n) v = p.heads * ((query_tiles_of(p, s_order[r]) + 1) >> 1);
 #pragma unroll
       for (int d = 1; d < 32; d <<= 1) {
         const int o = __shfl_up_sync(0xFFFFFFFFu, v, d);
@@ -201,19 +206,26 @@ __device__ __forceinline__ void build_pair_order(const AttnParams& p, int* sched
 __device__ __forceinline__ PairUnit pair_unit(const AttnParams& p, const int* sched, int w) {
   PairUnit u;
   const int n = sched[0];
-  if (n > 0) {
-    const int* order = sched + 2;
-    const int* pre = sched + 2 + kMaxSortSeqs;
-    const int r = find_prefix_smem(pre, n, w);
-    u.seq = order[r];
-    const int sb = __ldg(p.so_q + u.seq);
-    const int nt = __ldg(p.so_q + u.seq + 1) - sb;
-    const int np = (nt + 1) >> 1;
-    const int local = w - pre[r];
+  if (n != 0) {
+    int local, np, nt;
+    if (n > 0) {
+      const int* order = sched + 2;
+      const int* pre = sched + 2 + kMaxSortSeqs;
+      const int r = find_prefix_smem(pre, n, w);
+      u.seq = order[r];
+      local = w - pre[r];
+      nt = query_tiles_of(p, u.seq);
+      np = (nt + 1) >> 1;
+    } else {  // shared query set, plain order
+      nt = query_tiles_of(p, 0);
+      np = (nt + 1) >> 1;
+      u.seq = w / (p.heads * np);
+      local = w - u.seq * (p.heads * np);
+    }
     u.h = local / np;
     const int pair = local - u.h * np;
     u.qtile0 = 2 * pair;
-    u.sbq = sb + 2 * pair;
+    u.sbq = __ldg(p.so_q + (p.shared_q ? 0 : u.seq)) + 2 * pair;
     u.has_q1 = (2 * pair + 1 < nt) ? 1 : 0;
   } else {
     u.h = w / p.total_q_tiles;
@@ -223,9 +235,11 @@ __device__ __forceinline__ PairUnit pair_unit(const AttnParams& p, const int* sc
     u.sbq = g;
     u.has_q1 = 0;
   }
-  const int cq0 = __ldg(p.cu_q + u.seq);
+  const int qseq = p.shared_q ? 0 : u.seq;
+  const int cq0 = __ldg(p.cu_q + qseq);
   u.q_row0 = cq0 + u.qtile0 * kTileM;
-  u.q_len = __ldg(p.cu_q + u.seq + 1) - cq0;
+  u.q_len = __ldg(p.cu_q + qseq + 1) - cq0;
+  u.o_row0 = p.shared_q ? u.seq * u.q_len + u.qtile0 * kTileM : u.q_row0;
   u.k_row0 = __ldg(p.cu_k + u.seq);
   u.k_len = __ldg(p.cu_k + u.seq + 1) - u.k_row0;
   u.nkv = (u.k_len + kTileN - 1) / kTileN;
@@ -239,6 +253,7 @@ __device__ __forceinline__ PairUnit warp_uniform(const PairUnit& u) {
   r.seq = lpfa::warp_uniform(u.seq);
   r.qtile0 = lpfa::warp_uniform(u.qtile0);
   r.q_row0 = lpfa::warp_uniform(u.q_row0);
+  r.o_row0 = lpfa::warp_uniform(u.o_row0);
   r.q_len = lpfa::warp_uniform(u.q_len);
   r.k_row0 = lpfa::warp_uniform(u.k_row0);
   r.k_len = lpfa::warp_uniform(u.k_len);
@@ -735,7 +750,7 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
       nbase += static_cast<uint32_t>(ui.nkv) * np;
       if (grp > ui.has_q1) continue;
       const bool valid = (ui.qtile0 + grp) * kTileM + row < ui.q_len;
-      const int64_t tok = ui.q_row0 + grp * kTileM + row;
+      const int64_t tok = ui.o_row0 + grp * kTileM + row;  // output and LSE row
       if (ui.nkv == 0) {
         // No keys: an empty sum, LSE = log 0 = -inf and O = 0.
         if (valid) {

@@ -359,7 +359,7 @@ static lpfa_status attn_fwd_impl(const uint8_t* q, const uint8_t* q_sf, const ui
                                  const lpfa_varlen_meta* meta_k, int32_t heads, int32_t head_dim,
                                  lpfa_pv_mode pv_mode, const lpfa_descale* q_descale,
                                  const lpfa_descale* k_descale, const lpfa_descale* v_descale, void* out_bf16,
-                                 float* lse, void* stream, int debug_stall) {
+                                 float* lse, void* stream, int debug_stall, int shared_q = 0) {
   if (!q || !q_sf || !k || !k_sf || !v || !out_bf16 || !lse) return fail(LPFA_ERR_INVALID_ARG, "NULL tensor pointer");
   if (pv_mode != LPFA_PV_BF16 && pv_mode != LPFA_PV_FP8 && pv_mode != LPFA_PV_BF16_V && pv_mode != LPFA_PV_MXFP8)
     return fail(LPFA_ERR_INVALID_ARG, "invalid pv_mode %d", pv_mode);
@@ -376,13 +376,22 @@ static lpfa_status attn_fwd_impl(const uint8_t* q, const uint8_t* q_sf, const ui
   lpfa_status st;
   if ((st = check_meta(meta_q, "meta_q")) != LPFA_OK) return st;
   if ((st = check_meta(meta_k, "meta_k")) != LPFA_OK) return st;
-  if (meta_q->num_seqs != meta_k->num_seqs)
+  if (shared_q) {
+    if (meta_q->num_seqs != 1)
+      return fail(LPFA_ERR_INVALID_ARG, "a shared query set is one sequence (meta_q has %d)", meta_q->num_seqs);
+  } else if (meta_q->num_seqs != meta_k->num_seqs) {
     return fail(LPFA_ERR_INVALID_ARG, "meta_q has %d sequences but meta_k has %d", meta_q->num_seqs, meta_k->num_seqs);
+  }
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(q_sf) || !aligned16(k_sf) ||
       (v_sf && !aligned16(v_sf)) || !aligned16(out_bf16) || !aligned16(lse))
     return fail(LPFA_ERR_INVALID_ARG, "all tensors must be 16-byte aligned");
-  const int64_t units = static_cast<int64_t>(heads) * meta_q->total_scale_blocks;
-  if (units > INT32_MAX) return fail(LPFA_ERR_INVALID_ARG, "too many query tiles");
+  // Output rows: the query tokens, or (shared query set) one block of them per K/V sequence.
+  const int64_t out_rows = shared_q ? static_cast<int64_t>(meta_k->num_seqs) * meta_q->total_tokens
+                                    : static_cast<int64_t>(meta_q->total_tokens);
+  const int64_t units = shared_q ? static_cast<int64_t>(meta_k->num_seqs) * heads * ((meta_q->total_scale_blocks + 1) / 2)
+                                 : static_cast<int64_t>(heads) * meta_q->total_scale_blocks;
+  if (units > INT32_MAX || out_rows * heads * 128 > INT64_MAX / 4 || out_rows > INT32_MAX)
+    return fail(LPFA_ERR_INVALID_ARG, "too many query tiles or output rows");
   DeviceInfo info;
   if ((st = require_sm100(&info)) != LPFA_OK) return st;
 
@@ -419,12 +428,13 @@ static lpfa_status attn_fwd_impl(const uint8_t* q, const uint8_t* q_sf, const ui
   p.v_descale = descale(v_descale);
   p.out = static_cast<__nv_bfloat16*>(out_bf16);
   p.lse = lse;
-  p.num_seqs = meta_q->num_seqs;
+  p.num_seqs = meta_k->num_seqs;
   p.heads = heads;
-  p.tq = meta_q->total_tokens;
+  p.tq = static_cast<int>(out_rows);
   p.total_q_tiles = meta_q->total_scale_blocks;
   p.num_units = static_cast<int>(units);
   p.debug_stall = debug_stall;
+  p.shared_q = shared_q ? 1 : 0;
 
   const int grid = static_cast<int>(units < info.sms ? units : info.sms);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -559,6 +569,15 @@ static lpfa_status attn_bwd_impl(const uint8_t* q, const uint8_t* q_sf, const ui
 }
 
 extern "C" {
+
+lpfa_status lpfa_attn_fwd_shared_q(const uint8_t* q, const uint8_t* q_sf, const uint8_t* k, const uint8_t* k_sf,
+                                   const uint8_t* v, const uint8_t* v_sf, const lpfa_varlen_meta* meta_q,
+                                   const lpfa_varlen_meta* meta_k, int32_t heads, int32_t head_dim,
+                                   lpfa_pv_mode pv_mode, const lpfa_descale* q_descale, const lpfa_descale* k_descale,
+                                   const lpfa_descale* v_descale, void* out_bf16, float* lse, void* stream) {
+  return attn_fwd_impl(q, q_sf, k, k_sf, v, v_sf, meta_q, meta_k, heads, head_dim, pv_mode, q_descale, k_descale,
+                       v_descale, out_bf16, lse, stream, 0, 1);
+}
 
 lpfa_status lpfa_attn_bwd_varlen(const uint8_t* q, const uint8_t* q_sf, const uint8_t* k, const uint8_t* k_sf,
                                  const uint8_t* v, const uint8_t* v_sf, const void* out_bf16, const void* dout_bf16,

@@ -182,3 +182,20 @@ def test_backward_argument_validation(over, needle):
     st, msg = _bwd(**over)
     assert st == lp.LPFA_ERR_INVALID_ARG
     assert needle in msg
+
+
+def test_shared_query_rejects_several_query_sequences():
+    """lpfa_attn_fwd_shared_q takes a query metadata of exactly one sequence (checked before any
+    CUDA call)."""
+    host_q = np.zeros(2 * 3, dtype=np.int32)
+    host_k = np.zeros(2 * 3, dtype=np.int32)
+    cq, ck = lp._Meta(), lp._Meta()
+    lens = np.array([5, 7], dtype=np.int32)
+    assert lp._lib.lpfa_varlen_meta_fill_host(lens.ctypes.data, 2, host_q.ctypes.data, ctypes.byref(cq)) == 0
+    assert lp._lib.lpfa_varlen_meta_fill_host(lens.ctypes.data, 2, host_k.ctypes.data, ctypes.byref(ck)) == 0
+    cq.dev = ck.dev = 16   # never dereferenced: validation fails first
+    one = lp._Descale(None, 0, 0)
+    st = lp._lib.lpfa_attn_fwd_shared_q(16, 16, 16, 16, 16, 16, ctypes.byref(cq), ctypes.byref(ck), 1, 128, 0,
+                                        ctypes.byref(one), ctypes.byref(one), ctypes.byref(one), 16, 16, None)
+    assert st == lp.LPFA_ERR_INVALID_ARG
+    assert b"one sequence" in lp._lib.lpfa_last_error_message()

@@ -52,6 +52,7 @@ class Workload:
     v_gain: float = 1.0           # V = bf16(N(0,1)) * v_gain (exact power of two)
     outlier_frac: float = 0.0     # fraction of (head, channel) pairs scaled
     outlier_gain: float = 1.0
+    shared_q: bool = False        # one query sequence (len_q) shared by num_seqs K/V sequences
     description: str = ""
 
 
@@ -100,6 +101,14 @@ _add(Workload("video_s32768_h24_mxpv", 8, heads=24, in_dtype="bf16", pv_mode="mx
               description="batch 1, 32768 tokens, 24 heads; Q/K bf16 N(0,1) MXFP8 RCEIL; V bf16 N(0,1) MXFP8 "
                           "in the token orientation, block-scaled MXFP8 PV"))
 
+# Shared-query workload (LP-FA4 README, opening paragraph: "shared-query workloads", not defined
+# there): one query sequence of 1024 tokens attending to each of 8 key/value sequences with
+# lengths U{2048..16384}.
+_add(Workload("shared_q1024_kv8_h16", 9, heads=16, in_dtype="bf16", pv_mode="bf16",
+              num_seqs=8, len_q=1024, range_k=(2048, 16384), cross=True, shared_q=True,
+              description="shared query set: 1 x 1024 queries against 8 K/V sequences, sk U{2048..16384}, "
+                          "16 heads, bf16 N(0,1), RCEIL, bf16 PV"))
+
 # The five evaluation workloads in order (the others are extra benchmark rows).
 EVAL_ORDER: List[str] = [
     "single_s256_h2",
@@ -116,7 +125,9 @@ def _rng(seed: int, w: Workload, stream: int) -> np.random.Generator:
 
 def lengths(w: Workload, seed: int = 0):
     """Return (lengths_q, lengths_k) as int32 arrays, drawn when the workload says so."""
-    if w.len_q is not None:
+    if w.shared_q:
+        lq = np.array([w.len_q], dtype=np.int32)
+    elif w.len_q is not None:
         lq = np.full(w.num_seqs, w.len_q, dtype=np.int32)
     else:
         lo, hi = w.range_q
