@@ -45,13 +45,15 @@ FALLBACK_HBM_GBS = 6650.0
 # recorded; any change to the kernel makes it null until re-captured.
 TRAFFIC = {
     # workload: (sha256 of the kernel's sources [:16], dram bytes read + written per launch)
+    "video_s32768_h24_fp8pv": ("9f57d9029e885093", 309982720 + 174723584),
 }
 
 # The source files of the attention kernel each PV mode runs, and that kernel's name.
 KERNEL_SOURCES = {
     "fp8": (["attn_fwd_pp.cuh", "attn_fwd.cuh", "ptx.cuh"], "attn_fwd_pp_kernel"),
     "mxfp8": (["attn_fwd_pp.cuh", "attn_fwd.cuh", "ptx.cuh"], "attn_fwd_pp_kernel"),
-    "bf16": (["attn_fwd_pp.cuh", "attn_fwd.cuh", "ptx.cuh"], "attn_fwd_pp_kernel"),
+    "bf16": (["attn_fwd_pp.cuh", "attn_fwd.cuh", "ptx.cuh", "dequantize.cuh"],
+             "attn_fwd_pp_kernel (+ dequantize_mxfp8_kernel for V, timed with it)"),
     "bf16v": (["attn_fwd_pp.cuh", "attn_fwd.cuh", "ptx.cuh"], "attn_fwd_pp_kernel"),
 }
 
@@ -435,6 +437,9 @@ def main():
     vs = torch.empty(sbk * H * 512, dtype=torch.uint8, device=dev) if w.pv_mode in ("bf16", "mxfp8") else None
     out = torch.empty((To, H, 128), dtype=torch.bfloat16, device=dev)
     lse = torch.empty((H, To), dtype=torch.float32, device=dev)
+    # bf16 PV: the workspace where V is dequantized to BF16 once per step.
+    ws_bytes = lp.lpfa_attn_fwd_workspace_bytes(lp.lpfa_varlen_meta_fill_host(lk), H, w.pv_mode)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev) if ws_bytes else False
 
     def step(ins, timing=None):
         mq = lp.lpfa_varlen_meta_from_lengths(lq, device=dev)
@@ -455,11 +460,11 @@ def main():
             c.record(stream)
         v_in = ins["v"] if w.pv_mode == "bf16v" else vp   # BF16 V goes to the kernel as is
         attn = lp.lpfa_attn_fwd_shared_q if w.shared_q else lp.lpfa_attn_fwd_varlen
-        attn(qp, qs, kp, ks, v_in, vs, mq, mk, pv_mode=w.pv_mode, out=out, lse=lse)
+        attn(qp, qs, kp, ks, v_in, vs, mq, mk, pv_mode=w.pv_mode, out=out, lse=lse, workspace=ws)
         if timing is not None:
             b.record(stream)
             timing.append((a, c, b))
-        return 3 if w.pv_mode == "bf16v" else 4  # kernels launched
+        return {"bf16v": 3, "bf16": 5}.get(w.pv_mode, 4)  # kernels launched
 
     ranks = Ranks(world, dev)
     barrier = ranks.barrier

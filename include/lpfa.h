@@ -160,6 +160,25 @@ LPFA_API lpfa_status lpfa_cast_e4m3(const void* v_bf16, int64_t tok_stride, int6
                            void* stream);
 
 /*
+ * MXFP8 to BF16: the exact values of a quantize_mxfp8_varlen payload (LP-FA4 README, "MXFP8
+ * forward and backward": E4M3 payload times the E8M0 power of two of its 32-element block along
+ * head_dim). Value (t, h, d) = E4M3(payload) * 2^e, computed in FP32 and rounded once to BF16:
+ * exact whenever the product is a normal BF16 number (every scale byte >= 3, i.e. e >= -124);
+ * smaller scales round the subnormal results to nearest even. These are the values that the bf16
+ * PV mode multiplies (the same bits as its in-kernel conversion).
+ *
+ * payload    device, (T, H, 128) E4M3 codes, contiguous, 16-byte aligned.
+ * scales     device, the scale storage of lpfa_quantize_mxfp8_varlen under meta.
+ * out_bf16   device, (T, H, 128) bf16, contiguous, 16-byte aligned; every token row is written.
+ * Errors:    LPFA_ERR_INVALID_ARG for NULL pointers, head_dim != 128, heads < 1, meta without a
+ *            device buffer, or misalignment; LPFA_ERR_UNSUPPORTED off sm_100; LPFA_ERR_CUDA on
+ *            launch failure.
+ */
+LPFA_API lpfa_status lpfa_dequantize_mxfp8_varlen(const uint8_t* payload, const uint8_t* scales,
+                                         const lpfa_varlen_meta* meta, int32_t heads,
+                                         int32_t head_dim, void* out_bf16, void* stream);
+
+/*
  * mxfp8_flash_attn_varlen_forward (LP-FA4 README, "MXFP8 forward and backward": noncausal,
  * head-dim-128 MHA over packed variable-length sequences, returning out and lse), with the
  * fp8 PV mode of FastVideo #1654 and the per-tensor descales of vLLM #63232.
@@ -257,6 +276,42 @@ LPFA_API lpfa_status lpfa_attn_fwd_shared_q(const uint8_t* q, const uint8_t* q_s
                                    const lpfa_descale* q_descale, const lpfa_descale* k_descale,
                                    const lpfa_descale* v_descale, void* out_bf16, float* lse,
                                    void* stream);
+
+/*
+ * The bf16 PV mode with V converted once (LP-FA4 README, "MXFP8 forward and backward": V's
+ * MXFP8 payload is dequantized exactly to BF16 for the BF16 PV product). Without a workspace the
+ * attention kernel converts each 128-key V tile in shared memory every time a pair of query
+ * tiles reads it; with one, lpfa_dequantize_mxfp8_varlen writes BF16 V there first and the
+ * kernel reads it as BF16 V input. Both give the same bits.
+ *
+ * lpfa_attn_fwd_workspace_bytes returns the workspace size a call needs: total_tokens(meta_k)
+ * * heads * 256 bytes for LPFA_PV_BF16, 0 for the other modes (and for invalid arguments).
+ *
+ * lpfa_attn_fwd_varlen_ws / lpfa_attn_fwd_shared_q_ws: arguments and behaviour of
+ * lpfa_attn_fwd_varlen_descaled / lpfa_attn_fwd_shared_q, plus
+ * workspace        device, 16-byte aligned, at least workspace_bytes bytes, owned by the caller;
+ *                  written by the call (its contents afterwards are BF16 V) and free again once
+ *                  the call's work on `stream` has finished. Ignored (may be NULL) when the mode
+ *                  needs none.
+ * Errors:          as those entry points, plus LPFA_ERR_INVALID_ARG in LPFA_PV_BF16 mode for a
+ *                  NULL or misaligned workspace or one below lpfa_attn_fwd_workspace_bytes.
+ */
+LPFA_API size_t lpfa_attn_fwd_workspace_bytes(const lpfa_varlen_meta* meta_k, int32_t heads,
+                                              lpfa_pv_mode pv_mode);
+LPFA_API lpfa_status lpfa_attn_fwd_varlen_ws(const uint8_t* q, const uint8_t* q_sf, const uint8_t* k,
+                                    const uint8_t* k_sf, const uint8_t* v, const uint8_t* v_sf,
+                                    const lpfa_varlen_meta* meta_q, const lpfa_varlen_meta* meta_k,
+                                    int32_t heads, int32_t head_dim, lpfa_pv_mode pv_mode,
+                                    const lpfa_descale* q_descale, const lpfa_descale* k_descale,
+                                    const lpfa_descale* v_descale, void* out_bf16, float* lse,
+                                    void* workspace, size_t workspace_bytes, void* stream);
+LPFA_API lpfa_status lpfa_attn_fwd_shared_q_ws(const uint8_t* q, const uint8_t* q_sf, const uint8_t* k,
+                                      const uint8_t* k_sf, const uint8_t* v, const uint8_t* v_sf,
+                                      const lpfa_varlen_meta* meta_q, const lpfa_varlen_meta* meta_k,
+                                      int32_t heads, int32_t head_dim, lpfa_pv_mode pv_mode,
+                                      const lpfa_descale* q_descale, const lpfa_descale* k_descale,
+                                      const lpfa_descale* v_descale, void* out_bf16, float* lse,
+                                      void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * mxfp8_flash_attn_varlen_backward (LP-FA4 README, "MXFP8 forward and backward"): the gradients

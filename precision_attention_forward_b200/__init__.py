@@ -39,7 +39,8 @@ EXPORTED_SYMBOLS = (
     "lpfa_scale_bytes", "lpfa_quantize_mxfp8_varlen", "lpfa_cast_e4m3", "lpfa_attn_fwd_varlen",
     "lpfa_device_status", "lpfa_last_error_message", "lpfa_version", "lpfa_attn_fwd_varlen_debug",
     "lpfa_attn_fwd_varlen_descaled", "lpfa_quantize_mxfp8_varlen_tokens", "lpfa_attn_bwd_varlen",
-    "lpfa_attn_bwd_varlen_debug", "lpfa_attn_fwd_shared_q",
+    "lpfa_attn_bwd_varlen_debug", "lpfa_attn_fwd_shared_q", "lpfa_dequantize_mxfp8_varlen",
+    "lpfa_attn_fwd_workspace_bytes", "lpfa_attn_fwd_varlen_ws", "lpfa_attn_fwd_shared_q_ws",
 )
 
 
@@ -90,6 +91,15 @@ _lib.lpfa_attn_fwd_varlen_descaled.restype = ctypes.c_int
 _lib.lpfa_attn_fwd_shared_q.argtypes = _lib.lpfa_attn_fwd_varlen_descaled.argtypes
 _lib.lpfa_attn_fwd_shared_q.restype = ctypes.c_int
 _lib.lpfa_attn_fwd_varlen_debug.restype = ctypes.c_int
+_lib.lpfa_attn_fwd_varlen_ws.argtypes = (list(_lib.lpfa_attn_fwd_varlen_descaled.argtypes[:16]) +
+                                         [_vp, ctypes.c_size_t, _vp])
+_lib.lpfa_attn_fwd_varlen_ws.restype = ctypes.c_int
+_lib.lpfa_attn_fwd_shared_q_ws.argtypes = _lib.lpfa_attn_fwd_varlen_ws.argtypes
+_lib.lpfa_attn_fwd_shared_q_ws.restype = ctypes.c_int
+_lib.lpfa_attn_fwd_workspace_bytes.argtypes = [ctypes.POINTER(_Meta), _i32, ctypes.c_int]
+_lib.lpfa_attn_fwd_workspace_bytes.restype = ctypes.c_size_t
+_lib.lpfa_dequantize_mxfp8_varlen.argtypes = [_vp, _vp, ctypes.POINTER(_Meta), _i32, _i32, _vp, _vp]
+_lib.lpfa_dequantize_mxfp8_varlen.restype = ctypes.c_int
 _lib.lpfa_device_status.argtypes = [_vp, ctypes.POINTER(_i32)]
 _lib.lpfa_device_status.restype = ctypes.c_int
 _lib.lpfa_last_error_message.argtypes = []
@@ -242,13 +252,16 @@ def lpfa_attn_fwd_varlen(q: torch.Tensor, q_sf: torch.Tensor, k: torch.Tensor, k
                          pv_mode: str = "bf16", q_descale: Optional[torch.Tensor] = None,
                          k_descale: Optional[torch.Tensor] = None, v_descale: Optional[torch.Tensor] = None,
                          out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None, stream=None,
-                         debug_flags: int = 0):
+                         debug_flags: int = 0, workspace=True):
     """Block-scaled attention forward; returns (out bf16 (Tq,H,128), lse fp32 (H,Tq)).
 
     q/k/v_descale: None (exactly 1.0), a one-element tensor (per tensor), (H,) (per head) or
     (S, H) (per sequence and head), float32 on the device; see descale_strides.
+    workspace: where the bf16 PV mode converts V to BF16 once (lpfa_attn_fwd_varlen_ws): True
+    allocates it, a uint8 device tensor of at least lpfa_attn_fwd_workspace_bytes bytes is used as
+    is, False converts V tiles inside the attention kernel instead (same bits). Other modes ignore it.
     debug_flags != 0 goes through lpfa_attn_fwd_varlen_debug (test hook, see include/lpfa.h),
-    which takes per-tensor descales only.
+    which takes per-tensor descales only and no workspace.
     """
     if pv_mode not in PV_MODES:
         raise ValueError("pv_mode must be 'bf16', 'fp8', 'bf16v' or 'mxfp8'")
@@ -276,24 +289,65 @@ def lpfa_attn_fwd_varlen(q: torch.Tensor, q_sf: torch.Tensor, k: torch.Tensor, k
             ctypes.byref(meta_q._c), ctypes.byref(meta_k._c), H, 128, PV_MODES[pv_mode],
             _ptr(q_descale), _ptr(k_descale), _ptr(v_descale), out.data_ptr(), lse.data_ptr(),
             _stream_ptr(stream))
+    ws = None if debug_flags else _workspace(workspace, meta_k, H, pv_mode, q.device)
     with torch.cuda.device(q.device):
         if debug_flags:
             _check(_lib.lpfa_attn_fwd_varlen_debug(*args, debug_flags))
+        elif ws is not None:
+            _check(_lib.lpfa_attn_fwd_varlen_ws(*args[:11], ctypes.byref(descs[0]), ctypes.byref(descs[1]),
+                                                ctypes.byref(descs[2]), out.data_ptr(), lse.data_ptr(),
+                                                ws.data_ptr(), ctypes.c_size_t(ws.numel()), _stream_ptr(stream)))
         else:
             _check(_lib.lpfa_attn_fwd_varlen_descaled(*args[:11], ctypes.byref(descs[0]), ctypes.byref(descs[1]),
                                                       ctypes.byref(descs[2]), *args[14:]))
     return out, lse
 
 
+def lpfa_attn_fwd_workspace_bytes(meta_k: VarlenMeta, heads: int, pv_mode: str) -> int:
+    """Workspace bytes the bf16 PV mode needs (Tk * H * 256); 0 for the other modes."""
+    return int(_lib.lpfa_attn_fwd_workspace_bytes(ctypes.byref(meta_k._c), heads, PV_MODES[pv_mode]))
+
+
+def _workspace(workspace, meta_k: VarlenMeta, heads: int, pv_mode: str, device):
+    """The workspace tensor for a forward call, or None (in-kernel V conversion / not needed)."""
+    need = lpfa_attn_fwd_workspace_bytes(meta_k, heads, pv_mode)
+    if need == 0 or workspace is False or workspace is None:
+        return None
+    if workspace is True:
+        return torch.empty(need, dtype=torch.uint8, device=device)
+    if not isinstance(workspace, torch.Tensor) or workspace.dtype != torch.uint8 or not workspace.is_contiguous():
+        raise ValueError("workspace must be True, False or a contiguous uint8 device tensor")
+    if workspace.numel() < need:
+        raise ValueError("workspace has %d bytes; this call needs %d" % (workspace.numel(), need))
+    return workspace
+
+
+def lpfa_dequantize_mxfp8_varlen(payload: torch.Tensor, scales: torch.Tensor, meta: VarlenMeta,
+                                 out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """MXFP8 (head_dim orientation) payload + scale storage -> BF16 (T, H, 128), exactly."""
+    if payload.dtype != torch.uint8 or payload.dim() != 3 or not payload.is_contiguous():
+        raise ValueError("payload must be a contiguous uint8 (tokens, heads, 128) tensor")
+    T, H = payload.shape[0], payload.shape[1]
+    if out is None:
+        out = torch.empty((T, H, 128), dtype=torch.bfloat16, device=payload.device)
+    if out.dtype != torch.bfloat16 or tuple(out.shape) != (T, H, 128) or not out.is_contiguous():
+        raise ValueError("out must be a contiguous bf16 (tokens, heads, 128) tensor")
+    with torch.cuda.device(payload.device):
+        _check(_lib.lpfa_dequantize_mxfp8_varlen(payload.data_ptr(), scales.data_ptr(), ctypes.byref(meta._c), H,
+                                                 128, out.data_ptr(), _stream_ptr(stream)))
+    return out
+
+
 def lpfa_attn_fwd_shared_q(q: torch.Tensor, q_sf: torch.Tensor, k: torch.Tensor, k_sf: torch.Tensor,
                            v: torch.Tensor, v_sf: Optional[torch.Tensor], meta_q: VarlenMeta, meta_k: VarlenMeta,
                            pv_mode: str = "bf16", q_descale: Optional[torch.Tensor] = None,
                            k_descale: Optional[torch.Tensor] = None, v_descale: Optional[torch.Tensor] = None,
-                           out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None, stream=None):
+                           out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None, stream=None,
+                           workspace=True):
     """Shared-query forward (see include/lpfa.h): one query sequence (meta_q has one sequence of Lq
     tokens) attends to each of the n key/value sequences of meta_k. Returns (out bf16 (n*Lq,H,128),
-    lse fp32 (H,n*Lq)); rows [i*Lq, (i+1)*Lq) belong to key/value sequence i. Descales as for
-    lpfa_attn_fwd_varlen, indexed by the key/value sequence."""
+    lse fp32 (H,n*Lq)); rows [i*Lq, (i+1)*Lq) belong to key/value sequence i. Descales and
+    workspace as for lpfa_attn_fwd_varlen; descales are indexed by the key/value sequence."""
     if pv_mode not in PV_MODES:
         raise ValueError("pv_mode must be 'bf16', 'fp8', 'bf16v' or 'mxfp8'")
     if meta_q.num_seqs != 1:
@@ -319,12 +373,16 @@ def lpfa_attn_fwd_shared_q(q: torch.Tensor, q_sf: torch.Tensor, k: torch.Tensor,
         lse = torch.empty((H, rows), dtype=torch.float32, device=q.device)
     if tuple(out.shape) != (rows, H, 128) or tuple(lse.shape) != (H, rows):
         raise ValueError("out must be (n*Lq, H, 128) and lse (H, n*Lq)")
+    ws = _workspace(workspace, meta_k, H, pv_mode, q.device)
+    args = (q.data_ptr(), q_sf.data_ptr(), k.data_ptr(), k_sf.data_ptr(), v.data_ptr(), _ptr(v_sf),
+            ctypes.byref(meta_q._c), ctypes.byref(meta_k._c), H, 128, PV_MODES[pv_mode], ctypes.byref(descs[0]),
+            ctypes.byref(descs[1]), ctypes.byref(descs[2]), out.data_ptr(), lse.data_ptr())
     with torch.cuda.device(q.device):
-        _check(_lib.lpfa_attn_fwd_shared_q(q.data_ptr(), q_sf.data_ptr(), k.data_ptr(), k_sf.data_ptr(), v.data_ptr(),
-                                           _ptr(v_sf), ctypes.byref(meta_q._c), ctypes.byref(meta_k._c), H, 128,
-                                           PV_MODES[pv_mode], ctypes.byref(descs[0]), ctypes.byref(descs[1]),
-                                           ctypes.byref(descs[2]), out.data_ptr(), lse.data_ptr(),
-                                           _stream_ptr(stream)))
+        if ws is not None:
+            _check(_lib.lpfa_attn_fwd_shared_q_ws(*args, ws.data_ptr(), ctypes.c_size_t(ws.numel()),
+                                                  _stream_ptr(stream)))
+        else:
+            _check(_lib.lpfa_attn_fwd_shared_q(*args, _stream_ptr(stream)))
     return out, lse
 
 

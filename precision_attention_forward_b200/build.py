@@ -18,7 +18,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB_PATH = os.path.join(PKG_DIR, "liblpfa.so")
 
 SOURCES = ["lpfa.cu"]
-HEADERS = ["ptx.cuh", "quantize.cuh", "attn_fwd.cuh", "attn_fwd_pp.cuh", "attn_bwd.cuh"]
+HEADERS = ["ptx.cuh", "quantize.cuh", "attn_fwd.cuh", "attn_fwd_pp.cuh", "attn_bwd.cuh", "dequantize.cuh"]
 
 
 def nvcc_path() -> str:

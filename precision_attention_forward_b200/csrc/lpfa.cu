@@ -19,6 +19,7 @@
 #include "attn_fwd_pp.cuh"
 #include "attn_bwd.cuh"
 #include "quantize.cuh"
+#include "dequantize.cuh"
 
 namespace {
 
@@ -339,6 +340,25 @@ static lpfa_status check_attn_kernel(const void* fn, uint32_t smem_bytes) {
   return LPFA_OK;
 }
 
+// MXFP8 (head_dim orientation) -> BF16 over every token of meta: one CTA per (block, head) tile.
+static lpfa_status launch_dequant(const uint8_t* payload, const uint8_t* scales, const lpfa_varlen_meta* meta,
+                                  int32_t heads, __nv_bfloat16* out, cudaStream_t s) {
+  const int64_t tiles = static_cast<int64_t>(meta->total_scale_blocks) * heads;
+  if (tiles > INT32_MAX) return fail(LPFA_ERR_INVALID_ARG, "too many (block, head) tiles");
+  lpfa::DequantParams p;
+  p.payload = payload;
+  p.scales = scales;
+  p.cu_seqlens = meta->dev;
+  p.scale_off = meta->dev + meta->num_seqs + 1;
+  p.num_seqs = meta->num_seqs;
+  p.heads = heads;
+  p.out = out;
+  lpfa::dequantize_mxfp8_kernel<<<static_cast<unsigned>(tiles), lpfa::kDequantThreads, 0, s>>>(p);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "dequantize launch");
+  return LPFA_OK;
+}
+
 extern "C++" {
 // Every PV mode runs over pairs of query tiles (attn_fwd_pp.cuh).
 template <int kPv, bool kPerUnit>
@@ -359,7 +379,8 @@ static lpfa_status attn_fwd_impl(const uint8_t* q, const uint8_t* q_sf, const ui
                                  const lpfa_varlen_meta* meta_k, int32_t heads, int32_t head_dim,
                                  lpfa_pv_mode pv_mode, const lpfa_descale* q_descale,
                                  const lpfa_descale* k_descale, const lpfa_descale* v_descale, void* out_bf16,
-                                 float* lse, void* stream, int debug_stall, int shared_q = 0) {
+                                 float* lse, void* stream, int debug_stall, int shared_q = 0,
+                                 bool with_ws = false, void* workspace = nullptr, size_t ws_bytes = 0) {
   if (!q || !q_sf || !k || !k_sf || !v || !out_bf16 || !lse) return fail(LPFA_ERR_INVALID_ARG, "NULL tensor pointer");
   if (pv_mode != LPFA_PV_BF16 && pv_mode != LPFA_PV_FP8 && pv_mode != LPFA_PV_BF16_V && pv_mode != LPFA_PV_MXFP8)
     return fail(LPFA_ERR_INVALID_ARG, "invalid pv_mode %d", pv_mode);
@@ -392,15 +413,25 @@ static lpfa_status attn_fwd_impl(const uint8_t* q, const uint8_t* q_sf, const ui
                                  : static_cast<int64_t>(heads) * meta_q->total_scale_blocks;
   if (units > INT32_MAX || out_rows * heads * 128 > INT64_MAX / 4 || out_rows > INT32_MAX)
     return fail(LPFA_ERR_INVALID_ARG, "too many query tiles or output rows");
+  // bf16 PV over a workspace: V is dequantized once into it, then read as BF16 V input.
+  const bool dequant_v = with_ws && pv_mode == LPFA_PV_BF16;
+  if (dequant_v) {
+    const size_t need = static_cast<size_t>(meta_k->total_tokens) * static_cast<size_t>(heads) * 256u;
+    if (!workspace) return fail(LPFA_ERR_INVALID_ARG, "bf16 PV mode needs a workspace of %zu bytes", need);
+    if (!aligned16(workspace)) return fail(LPFA_ERR_INVALID_ARG, "the workspace must be 16-byte aligned");
+    if (ws_bytes < need)
+      return fail(LPFA_ERR_INVALID_ARG, "workspace of %zu bytes is too small (bf16 PV mode needs %zu)", ws_bytes,
+                  need);
+  }
   DeviceInfo info;
   if ((st = require_sm100(&info)) != LPFA_OK) return st;
 
   CUtensorMap tq, tk, tv;
   if ((st = payload_tmap(&tq, q, meta_q->total_tokens, heads, lpfa::kTileM)) != LPFA_OK) return st;
   if ((st = payload_tmap(&tk, k, meta_k->total_tokens, heads, lpfa::kTileN)) != LPFA_OK) return st;
-  if (pv_mode == LPFA_PV_BF16_V) {
+  if (pv_mode == LPFA_PV_BF16_V || dequant_v) {
     // BF16 V, contiguous (Tk, H, 128): boxes of 64 elements (128 bytes) x 128 keys, 128-byte swizzle.
-    if ((st = bf16_v_tmap(&tv, v, meta_k->total_tokens, heads)) != LPFA_OK) return st;
+    if ((st = bf16_v_tmap(&tv, dequant_v ? workspace : v, meta_k->total_tokens, heads)) != LPFA_OK) return st;
   } else if ((st = payload_tmap(&tv, v, meta_k->total_tokens, heads, lpfa::kTileN)) != LPFA_OK) {
     return st;
   }
@@ -440,10 +471,15 @@ static lpfa_status attn_fwd_impl(const uint8_t* q, const uint8_t* q_sf, const ui
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const bool per_unit = (p.q_descale.seq_stride | p.q_descale.head_stride | p.k_descale.seq_stride |
                          p.k_descale.head_stride) != 0;
+  if (dequant_v) {
+    if ((st = launch_dequant(v, v_sf, meta_k, heads, static_cast<__nv_bfloat16*>(workspace), s)) != LPFA_OK)
+      return st;
+    p.v_sf = nullptr;
+  }
   if (pv_mode == LPFA_PV_FP8) {
     st = per_unit ? launch_attn_pp<lpfa::kPvFp8, true>(grid, s, tq, tk, tv, p)
                   : launch_attn_pp<lpfa::kPvFp8, false>(grid, s, tq, tk, tv, p);
-  } else if (pv_mode == LPFA_PV_BF16) {
+  } else if (pv_mode == LPFA_PV_BF16 && !dequant_v) {
     st = per_unit ? launch_attn_pp<lpfa::kPvBf16Mx, true>(grid, s, tq, tk, tv, p)
                   : launch_attn_pp<lpfa::kPvBf16Mx, false>(grid, s, tq, tk, tv, p);
   } else if (pv_mode == LPFA_PV_MXFP8) {
@@ -577,6 +613,46 @@ lpfa_status lpfa_attn_fwd_shared_q(const uint8_t* q, const uint8_t* q_sf, const 
                                    const lpfa_descale* v_descale, void* out_bf16, float* lse, void* stream) {
   return attn_fwd_impl(q, q_sf, k, k_sf, v, v_sf, meta_q, meta_k, heads, head_dim, pv_mode, q_descale, k_descale,
                        v_descale, out_bf16, lse, stream, 0, 1);
+}
+
+size_t lpfa_attn_fwd_workspace_bytes(const lpfa_varlen_meta* meta_k, int32_t heads, lpfa_pv_mode pv_mode) {
+  if (!meta_k || heads < 1 || meta_k->total_tokens < 1 || pv_mode != LPFA_PV_BF16) return 0;
+  return static_cast<size_t>(meta_k->total_tokens) * static_cast<size_t>(heads) * 256u;
+}
+
+lpfa_status lpfa_attn_fwd_varlen_ws(const uint8_t* q, const uint8_t* q_sf, const uint8_t* k, const uint8_t* k_sf,
+                                    const uint8_t* v, const uint8_t* v_sf, const lpfa_varlen_meta* meta_q,
+                                    const lpfa_varlen_meta* meta_k, int32_t heads, int32_t head_dim,
+                                    lpfa_pv_mode pv_mode, const lpfa_descale* q_descale,
+                                    const lpfa_descale* k_descale, const lpfa_descale* v_descale, void* out_bf16,
+                                    float* lse, void* workspace, size_t workspace_bytes, void* stream) {
+  return attn_fwd_impl(q, q_sf, k, k_sf, v, v_sf, meta_q, meta_k, heads, head_dim, pv_mode, q_descale, k_descale,
+                       v_descale, out_bf16, lse, stream, 0, 0, true, workspace, workspace_bytes);
+}
+
+lpfa_status lpfa_attn_fwd_shared_q_ws(const uint8_t* q, const uint8_t* q_sf, const uint8_t* k,
+                                      const uint8_t* k_sf, const uint8_t* v, const uint8_t* v_sf,
+                                      const lpfa_varlen_meta* meta_q, const lpfa_varlen_meta* meta_k, int32_t heads,
+                                      int32_t head_dim, lpfa_pv_mode pv_mode, const lpfa_descale* q_descale,
+                                      const lpfa_descale* k_descale, const lpfa_descale* v_descale, void* out_bf16,
+                                      float* lse, void* workspace, size_t workspace_bytes, void* stream) {
+  return attn_fwd_impl(q, q_sf, k, k_sf, v, v_sf, meta_q, meta_k, heads, head_dim, pv_mode, q_descale, k_descale,
+                       v_descale, out_bf16, lse, stream, 0, 1, true, workspace, workspace_bytes);
+}
+
+lpfa_status lpfa_dequantize_mxfp8_varlen(const uint8_t* payload, const uint8_t* scales, const lpfa_varlen_meta* meta,
+                                         int32_t heads, int32_t head_dim, void* out_bf16, void* stream) {
+  if (!payload || !scales || !out_bf16) return fail(LPFA_ERR_INVALID_ARG, "NULL tensor pointer");
+  if (head_dim != 128) return fail(LPFA_ERR_INVALID_ARG, "head_dim must be 128 (got %d)", head_dim);
+  if (heads < 1) return fail(LPFA_ERR_INVALID_ARG, "heads must be >= 1");
+  lpfa_status st;
+  if ((st = check_meta(meta, "meta")) != LPFA_OK) return st;
+  if (!aligned16(payload) || !aligned16(out_bf16))
+    return fail(LPFA_ERR_INVALID_ARG, "payload and out must be 16-byte aligned");
+  DeviceInfo info;
+  if ((st = require_sm100(&info)) != LPFA_OK) return st;
+  return launch_dequant(payload, scales, meta, heads, static_cast<__nv_bfloat16*>(out_bf16),
+                        static_cast<cudaStream_t>(stream));
 }
 
 lpfa_status lpfa_attn_bwd_varlen(const uint8_t* q, const uint8_t* q_sf, const uint8_t* k, const uint8_t* k_sf,

@@ -71,8 +71,9 @@ def _descale_tensor(x):
 
 
 def run_path(lp, q, k, v, lens_q, lens_k, heads, in_dtype="bf16", pv_mode="bf16", mode="rceil",
-             descales=(None, None, None)):
-    """Library path: metadata, quantize Q/K (and V in bf16 PV mode) or cast V, attention."""
+             descales=(None, None, None), workspace=True):
+    """Library path: metadata, quantize Q/K (and V in bf16 PV mode) or cast V, attention.
+    workspace=False runs the bf16 PV mode with V converted inside the attention kernel."""
     mq = lp.lpfa_varlen_meta_from_lengths(lens_q)
     mk = lp.lpfa_varlen_meta_from_lengths(lens_k)
     qp, qs = gpu_quantize(lp, q, in_dtype, mq, mode)
@@ -87,7 +88,7 @@ def run_path(lp, q, k, v, lens_q, lens_k, heads, in_dtype="bf16", pv_mode="bf16"
         vp, vs = gpu_quantize(lp, v, in_dtype, mk, mode)
     dd = [_descale_tensor(x) for x in descales]
     o, lse = lp.lpfa_attn_fwd_varlen(qp, qs, kp, ks, vp, vs, mq, mk, pv_mode=pv_mode,
-                                     q_descale=dd[0], k_descale=dd[1], v_descale=dd[2])
+                                     q_descale=dd[0], k_descale=dd[1], v_descale=dd[2], workspace=workspace)
     torch.cuda.synchronize()
     return o, lse
 

@@ -199,3 +199,35 @@ def test_shared_query_rejects_several_query_sequences():
                                         ctypes.byref(one), ctypes.byref(one), ctypes.byref(one), 16, 16, None)
     assert st == lp.LPFA_ERR_INVALID_ARG
     assert b"one sequence" in lp._lib.lpfa_last_error_message()
+
+
+def _attn_ws(ws, ws_bytes, pv=0):
+    one = lp._Descale(None, 0, 0)
+    mq, mk = _fake_meta(2, 300), _fake_meta(2, 300)
+    st = lp._lib.lpfa_attn_fwd_varlen_ws(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE if pv == 0 else None, ctypes.byref(mq),
+                                         ctypes.byref(mk), 4, 128, pv, ctypes.byref(one), ctypes.byref(one),
+                                         ctypes.byref(one), FAKE, FAKE, ws, ctypes.c_size_t(ws_bytes), None)
+    return st, lp._lib.lpfa_last_error_message().decode()
+
+
+def test_workspace_size_and_validation():
+    """bf16 PV mode over a workspace needs total_tokens(K) * heads * 256 bytes, 16-byte aligned;
+    the other modes need none (checked before any CUDA call)."""
+    mk = _fake_meta(2, 300)
+    assert lp._lib.lpfa_attn_fwd_workspace_bytes(ctypes.byref(mk), 4, 0) == 300 * 4 * 256
+    for pv in (1, 2, 3):
+        assert lp._lib.lpfa_attn_fwd_workspace_bytes(ctypes.byref(mk), 4, pv) == 0
+    assert lp._lib.lpfa_attn_fwd_workspace_bytes(None, 4, 0) == 0
+    need = 300 * 4 * 256
+    for ws, nbytes, needle in ((None, need, "workspace"), (FAKE + 8, need, "aligned"),
+                               (FAKE, need - 1, "too small")):
+        st, msg = _attn_ws(ws, nbytes)
+        assert st == lp.LPFA_ERR_INVALID_ARG and needle in msg, msg
+
+
+def test_dequantize_argument_validation():
+    m = _fake_meta(1, 10)
+    for args, needle in (((None, FAKE, 2, 128, FAKE), "NULL"), ((FAKE, FAKE, 2, 64, FAKE), "head_dim"),
+                         ((FAKE, FAKE, 0, 128, FAKE), "heads"), ((FAKE, FAKE, 2, 128, FAKE + 2), "aligned")):
+        st = lp._lib.lpfa_dequantize_mxfp8_varlen(args[0], args[1], ctypes.byref(m), args[2], args[3], args[4], None)
+        assert st == lp.LPFA_ERR_INVALID_ARG and needle in lp._lib.lpfa_last_error_message().decode()
