@@ -314,6 +314,39 @@ LPFA_API lpfa_status lpfa_attn_fwd_shared_q_ws(const uint8_t* q, const uint8_t* 
                                       void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Forward without any device allocation (the pages have no counterpart; this is a library
+ * convenience). Some callers cannot give the library device memory: code embedded in a host
+ * application or serving runtime whose own pool owns every byte of the GPU and forbids other
+ * allocations, and latency-critical paths where cudaMalloc / cudaFree (which can synchronise the
+ * whole device) are not allowed. lpfa_attn_fwd_varlen_ws needs a caller workspace in bf16 PV mode;
+ * this entry point takes the same arguments minus the workspace and uses a fixed scratch array
+ * inside the library instead (LPFA_NOALLOC_SCRATCH_BYTES = 64 MiB of device memory, reserved on
+ * every GPU where the library is loaded, until the process exits). It calls no cudaMalloc, cudaFree
+ * or other allocating routine.
+ *
+ * Arguments, results and errors: as lpfa_attn_fwd_varlen_descaled (same bits as that call and as
+ * lpfa_attn_fwd_varlen_ws). Modes other than LPFA_PV_BF16 need no scratch and take any size.
+ * Limit:   in LPFA_PV_BF16 mode, total_tokens(meta_k) * heads * 256 bytes (the BF16 copy of V) must
+ *          fit in the scratch, i.e. key tokens x heads <= 262144 (e.g. 16384 tokens at 16 heads);
+ *          larger calls return LPFA_ERR_INVALID_ARG before any work, with the sizes in the message.
+ * Set-up:  the first call on a device (with that device current) looks up the scratch array's
+ *          device address (cudaGetSymbolAddress) and keeps it; make that first call before any
+ *          stream capture on that device.
+ * Sharing: every call on a device uses the same scratch, which keeps the last call's contents (no
+ *          part of it needs to start at zero: each call writes all the scratch it reads first).
+ *          Calls whose work overlaps on the GPU (different streams, or different host threads
+ *          without ordering) race on it and give wrong results; order them on one stream.
+ */
+#define LPFA_NOALLOC_SCRATCH_BYTES (64ull << 20)
+LPFA_API lpfa_status lpfa_attn_fwd_varlen_noalloc(const uint8_t* q, const uint8_t* q_sf, const uint8_t* k,
+                                         const uint8_t* k_sf, const uint8_t* v, const uint8_t* v_sf,
+                                         const lpfa_varlen_meta* meta_q, const lpfa_varlen_meta* meta_k,
+                                         int32_t heads, int32_t head_dim, lpfa_pv_mode pv_mode,
+                                         const lpfa_descale* q_descale, const lpfa_descale* k_descale,
+                                         const lpfa_descale* v_descale, void* out_bf16, float* lse,
+                                         void* stream);
+
+/*
  * mxfp8_flash_attn_varlen_backward (LP-FA4 README, "MXFP8 forward and backward"): the gradients
  * of lpfa_attn_fwd_varlen's output with respect to the dequantized Q, K, V (quantization is not
  * differentiated), noncausal head-dim-128 MHA over packed variable-length sequences:

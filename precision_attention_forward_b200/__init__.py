@@ -41,6 +41,7 @@ EXPORTED_SYMBOLS = (
     "lpfa_attn_fwd_varlen_descaled", "lpfa_quantize_mxfp8_varlen_tokens", "lpfa_attn_bwd_varlen",
     "lpfa_attn_bwd_varlen_debug", "lpfa_attn_fwd_shared_q", "lpfa_dequantize_mxfp8_varlen",
     "lpfa_attn_fwd_workspace_bytes", "lpfa_attn_fwd_varlen_ws", "lpfa_attn_fwd_shared_q_ws",
+    "lpfa_attn_fwd_varlen_noalloc",
 )
 
 
@@ -96,6 +97,8 @@ _lib.lpfa_attn_fwd_varlen_ws.argtypes = (list(_lib.lpfa_attn_fwd_varlen_descaled
 _lib.lpfa_attn_fwd_varlen_ws.restype = ctypes.c_int
 _lib.lpfa_attn_fwd_shared_q_ws.argtypes = _lib.lpfa_attn_fwd_varlen_ws.argtypes
 _lib.lpfa_attn_fwd_shared_q_ws.restype = ctypes.c_int
+_lib.lpfa_attn_fwd_varlen_noalloc.argtypes = _lib.lpfa_attn_fwd_varlen_descaled.argtypes
+_lib.lpfa_attn_fwd_varlen_noalloc.restype = ctypes.c_int
 _lib.lpfa_attn_fwd_workspace_bytes.argtypes = [ctypes.POINTER(_Meta), _i32, ctypes.c_int]
 _lib.lpfa_attn_fwd_workspace_bytes.restype = ctypes.c_size_t
 _lib.lpfa_dequantize_mxfp8_varlen.argtypes = [_vp, _vp, ctypes.POINTER(_Meta), _i32, _i32, _vp, _vp]

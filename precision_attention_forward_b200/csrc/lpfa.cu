@@ -692,6 +692,56 @@ lpfa_status lpfa_attn_fwd_varlen_debug(const uint8_t* q, const uint8_t* q_sf, co
                        out_bf16, lse, stream, debug_flags & 1);
 }
 
+// ------------------------------------------------------------------ forward without allocation
+// bf16 PV needs a BF16 copy of V as scratch. Callers that cannot hand the library device memory get
+// it from this file-scope array instead; every GPU that loads the library holds it until exit.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[LPFA_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+void* g_noalloc_ptr[kMaxDevices] = {};
+std::mutex g_noalloc_mu;
+
+// The scratch array's device address on the current device. In host code the array's name is only
+// a host-side stand-in, so the address is looked up once per device (with it current) and kept.
+lpfa_status noalloc_scratch(void** out) {
+  DeviceInfo info;
+  int dev = 0;
+  lpfa_status st = current_device(&info, &dev);
+  if (st != LPFA_OK) return st;
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* ptr = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(no-allocation scratch)");
+    g_noalloc_ptr[dev] = ptr;
+  }
+  *out = g_noalloc_ptr[dev];
+  return LPFA_OK;
+}
+}  // namespace
+
+lpfa_status lpfa_attn_fwd_varlen_noalloc(const uint8_t* q, const uint8_t* q_sf, const uint8_t* k,
+                                         const uint8_t* k_sf, const uint8_t* v, const uint8_t* v_sf,
+                                         const lpfa_varlen_meta* meta_q, const lpfa_varlen_meta* meta_k,
+                                         int32_t heads, int32_t head_dim, lpfa_pv_mode pv_mode,
+                                         const lpfa_descale* q_descale, const lpfa_descale* k_descale,
+                                         const lpfa_descale* v_descale, void* out_bf16, float* lse, void* stream) {
+  const size_t need = lpfa_attn_fwd_workspace_bytes(meta_k, heads, pv_mode);
+  if (need > static_cast<size_t>(LPFA_NOALLOC_SCRATCH_BYTES))
+    return fail(LPFA_ERR_INVALID_ARG,
+                "lpfa_attn_fwd_varlen_noalloc: bf16 PV over %d key tokens x %d heads needs %zu bytes of scratch; "
+                "its fixed scratch holds %zu (key tokens x heads <= %zu)",
+                meta_k->total_tokens, heads, need, static_cast<size_t>(LPFA_NOALLOC_SCRATCH_BYTES),
+                static_cast<size_t>(LPFA_NOALLOC_SCRATCH_BYTES) / 256u);
+  void* scratch = nullptr;
+  if (need > 0) {
+    const lpfa_status st = noalloc_scratch(&scratch);
+    if (st != LPFA_OK) return st;
+  }
+  return attn_fwd_impl(q, q_sf, k, k_sf, v, v_sf, meta_q, meta_k, heads, head_dim, pv_mode, q_descale, k_descale,
+                       v_descale, out_bf16, lse, stream, 0, 0, true, scratch, static_cast<size_t>(LPFA_NOALLOC_SCRATCH_BYTES));
+}
+
 lpfa_status lpfa_device_status(void* stream, int32_t* detail) {
   if (detail) *detail = 0;
   cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
