@@ -15,6 +15,10 @@
 // own row sums and its own O accumulator, so nothing of the online softmax crosses warpgroups
 // (FlashAttention-4's two-tile ping-pong). Every K and V tile loaded serves both query tiles.
 //
+// At a unit boundary the softmax warps only hand their row normalisers to the epilogue warps and
+// go on; with bf16 P they also have the next unit's description decoded ahead, and the producer
+// (one Q stage) has prefetched the next unit's Q tiles into L2.
+//
 // Warp roles (512 threads):
 //   warp 0        Q/K producer: Q0, Q1 and their scale atoms once per unit, then K tiles + atoms.
 //   warp 3        V producer: V tiles (+ scale atoms for MXFP8 V; BF16 V as two swizzled boxes).
@@ -24,7 +28,10 @@
 //   warp 2        PV issuer: O_i += P V_j -- kind::f8f6f4 or kind::mxf8f6f4.block_scale with P in
 //                 TMEM (8-bit P), kind::f16 with P and BF16 V in shared memory (bf16 P).
 //   warps 4..7    softmax of Q0; warps 8..11 softmax of Q1 (one thread per query row).
-//   warps 12..15  bf16 PV with MXFP8 V: convert V tiles to BF16 in shared memory; else idle.
+//   warps 12..15  bf16 PV with MXFP8 V converted in the kernel: convert V tiles to BF16 in shared
+//                 memory (the softmax warps then write O themselves); every other mode: epilogue,
+//                 i.e. read each finished O_i from TMEM, scale, store BF16 O and the LSE, while the
+//                 softmax warps go on with the next unit.
 //
 // TMEM (512 columns): S [0, 128); O_i [128 + 128 i, 256 + 128 i); 8-bit P in three slots
 // [384 + 32 slot, +32); scale atoms after them (see the column constants). A single S buffer is what
@@ -37,6 +44,17 @@
 
 namespace lpfa {
 namespace pp {
+
+// LPFA_PP_EPI_WG: warps 12..15 write O and the LSE in the modes where they convert no V (else the
+// softmax warps do, after each unit). LPFA_PP_NEXT_UNIT: in the bf16 P modes the softmax warps read
+// the next unit's description one unit ahead (measured: +1.5-2.5 % on 16-key-tile units with bf16 P;
+// with 8-bit P the registers it holds through the unit cost 2-5 %, so those modes do not).
+#ifndef LPFA_PP_EPI_WG
+#define LPFA_PP_EPI_WG 1
+#endif
+#ifndef LPFA_PP_NEXT_UNIT
+#define LPFA_PP_NEXT_UNIT 1
+#endif
 
 // LPFA_PP_BF_P_SMEM: bf16 P in two shared-memory slots (PV as a shared-memory MMA), else in one
 // 64-column TMEM slot that the two warpgroups use in turn. Two slots decouple the warpgroups; the
@@ -101,7 +119,8 @@ struct Smem {
   static constexpr uint32_t bars = sched + ((2 * kMaxSortSeqs + 3) * 4 + 15) / 16 * 16;
   static constexpr uint32_t num_bars = 56;
   static constexpr uint32_t misc = bars + num_bars * 8;                     // tmem base, abort flag
-  static constexpr uint32_t total = misc + 64;
+  static constexpr uint32_t stats = misc + 64;                              // [2][128] (O scale, LSE)
+  static constexpr uint32_t total = stats + 2 * 128 * 8;
   static_assert(kKS <= 6 && kVS <= 6 && kVBS <= 3, "ring barriers");
 };
 template <int kPv> constexpr uint32_t smem_bytes() { return Smem<kPv>::total + 1024; }
@@ -122,7 +141,9 @@ enum Bar : int {
   kBarDrainPV = 42, // PV issuer's own tcgen05 work done
   kBarVbfFull = 43, // [3] BF16 V tile in shared memory (TMA, or the 4 converter warps)
   kBarVbfEmpty = 46, // [3] the PVs reading the BF16 V tile complete (MMA commit)
-  kBarCount = 49
+  kBarStatsFull = 49, // [i] warpgroup i's row normalisers and LSE in shared memory (4 warps)
+  kBarStatsFree = 51, // [i] the epilogue warpgroup has read them                 (4 warps)
+  kBarCount = 53
 };
 static_assert(kBarCount <= Smem<kPvFp8>::num_bars, "barrier array");
 
@@ -130,7 +151,7 @@ static_assert(kBarCount <= Smem<kPvFp8>::num_bars, "barrier array");
 enum PairSite : int {
   kPSiteProducerQ = 101, kPSiteProducerK, kPSiteProducerV, kPSiteMmaQ, kPSiteMmaK, kPSiteMmaS, kPSiteMmaP,
   kPSiteMmaO, kPSiteMmaV, kPSiteSoftS, kPSiteSoftPV, kPSiteSoftO, kPSiteDrain, kPSiteDebugStall, kPSiteTmem,
-  kPSiteConvV, kPSiteConvE
+  kPSiteConvV, kPSiteConvE, kPSiteEpiO, kPSiteEpiStats, kPSiteSoftStats
 };
 
 // A work unit: query tiles qtile0 and (has_q1) qtile0 + 1 of one (sequence, head). seq is the
@@ -399,6 +420,8 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
   constexpr bool kPSm = L::kPS_;            // bf16 P in shared memory (else in one TMEM slot)
   constexpr bool kVIn = L::kVIn;            // BF16 V input (TMA straight into the operand layout)
   constexpr bool kConv = kPv == kPvBf16Mx;  // MXFP8 V converted to BF16 by warps 12..15
+  constexpr bool kEpi = !kConv && LPFA_PP_EPI_WG;  // warps 12..15 write O and LSE (else the softmax warps do)
+  constexpr bool kNextUnit = LPFA_PP_NEXT_UNIT && kBf;  // softmax warps decode the next unit early
   constexpr int kQS = L::kQS, kKS = L::kKS;
   // Ring depths as divisors: a ring a mode does not use has depth 0 in L; its code is never reached.
   constexpr int kVS = L::kVS > 0 ? L::kVS : 1, kVBS = L::kVBS > 0 ? L::kVBS : 1;
@@ -444,6 +467,10 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
     for (uint32_t i = 0; i < kNBarsPV; ++i) mbar_init(&bars[kBarPVDone + i], 1);
     mbar_init(&bars[kBarDrain], 1);
     mbar_init(&bars[kBarDrainPV], 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bars[kBarStatsFull + i], 4);
+      mbar_init(&bars[kBarStatsFree + i], 4);
+    }
     *abort_flag = 0;
     mbar_fence_init();
   }
@@ -490,6 +517,12 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
                     &bars[kBarQFull + qs], leader);
         }
         ++qc;
+        if (kQS == 1 && w + G < num_units) {
+          // With one Q stage the next unit's tiles can only be loaded once this unit's last QK
+          // has run; bring them into L2 now so that load is an L2 hit.
+          const PairUnit un = warp_uniform(pair_unit(p, sched, w + G));
+          for (int i = 0; i <= un.has_q1; ++i) tma_prefetch_3d(&tmap_q, 0, un.h, un.q_row0 + i * kTileM, leader);
+        }
         for (int j = 0; j < ui.nkv; ++j) {
           const uint32_t s = kc % kKS, ph = (kc / kKS) & 1;
           if (!wait_role(&bars[kBarKEmpty + s], ph ^ 1, abort_flag)) { record_failure(abort_flag, kPSiteProducerK); ok = false; break; }
@@ -742,9 +775,14 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
                                                       descale_value(p.k_descale, 0, 0)) * kLog2eRsqrtD);
     uint32_t sc = 0, ucnt = 0;  // S tiles read, units finished
     uint32_t nbase = 0;         // P tiles of all earlier units, in the order the PVs consume them
+    float2* stats = reinterpret_cast<float2*>(smem + L::stats);
     bool ok = true;
+    // The next unit's description is loaded one unit ahead (its metadata reads are global loads).
+    PairUnit ui_next;
+    if (kNextUnit && static_cast<int>(blockIdx.x) < num_units) ui_next = pair_unit(p, sched, blockIdx.x);
     for (int w = blockIdx.x; w < num_units && ok; w += G) {
-      const PairUnit ui = pair_unit(p, sched, w);
+      const PairUnit ui = kNextUnit ? ui_next : pair_unit(p, sched, w);
+      if (kNextUnit && w + G < num_units) ui_next = pair_unit(p, sched, w + G);
       const uint32_t np = 1u + static_cast<uint32_t>(ui.has_q1);  // P tiles per key tile
       const uint32_t n0 = nbase;
       nbase += static_cast<uint32_t>(ui.nkv) * np;
@@ -897,6 +935,17 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
         if (lane == 0) mbar_arrive(&bars[kBarPReady + ps]);
       }
       if (!ok) break;
+      if (kEpi) {
+        // Hand the row's O scale and LSE to the epilogue warpgroup and go on to the next unit. The
+        // slot is free once the epilogue has read this warpgroup's previous unit's values.
+        if (ucnt > 0 && !wait_warp(&bars[kBarStatsFree + grp], (ucnt - 1) & 1, abort_flag, false)) { record_failure(abort_flag, kPSiteSoftStats); ok = false; break; }
+        stats[grp * kTileM + row] = make_float2(descale_value(p.v_descale, ui.seq, ui.h) / (kBf ? lr_r : l_r),
+                                                (m_r - kBias + lg2_approx(l_r)) * kLn2);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars[kBarStatsFull + grp]);
+        ++ucnt;
+        continue;
+      }
       // ---------------------------------------------------------------- epilogue
       if (!wait_warp(&bars[kBarOFull + grp], ucnt & 1, abort_flag, false)) { record_failure(abort_flag, kPSiteSoftO); ok = false; break; }
       tc_fence_after();
@@ -987,6 +1036,58 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
             mbar_arrive(&bars[kBarVEmpty + s]);
           }
           ++vc;
+        }
+      }
+    } else if (kEpi) {
+      // ---------------------------------------------------------------- epilogue (warps 12..15)
+      // Thread t owns row t of both query tiles (its warp's TMEM lane quarter). Per unit and query
+      // tile i: wait until every PV_i is complete and the softmax warpgroup has left its O scale
+      // and LSE in shared memory; read O_i from TMEM 32 columns at a time (the last read releases
+      // O_i to the next unit's PV), scale, round to BF16 and store the row; store the LSE.
+      const int quarter = warp & 3;
+      const int row = quarter * 32 + lane;
+      const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
+      const float2* stats = reinterpret_cast<const float2*>(smem + L::stats);
+      uint32_t rc[2] = {0, 0};  // units finished per query tile
+      bool ok = true;
+      for (int w = blockIdx.x; w < num_units && ok; w += G) {
+        const PairUnit ui = pair_unit(p, sched, w);
+        if (ui.nkv == 0) continue;  // the softmax warps wrote the empty-sum rows
+        for (int i = 0; i <= ui.has_q1; ++i) {
+          // Long waits (a whole unit): sleep between polls, leaving issue slots to the softmax warps.
+          if (!wait_role(&bars[kBarOFull + i], rc[i] & 1, abort_flag)) { record_failure(abort_flag, kPSiteEpiO); ok = false; break; }
+          if (!wait_role(&bars[kBarStatsFull + i], rc[i] & 1, abort_flag)) { record_failure(abort_flag, kPSiteEpiStats); ok = false; break; }
+          ++rc[i];
+          tc_fence_after();
+          const float2 st = stats[i * kTileM + row];
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bars[kBarStatsFree + i]);
+          const bool valid = (ui.qtile0 + i) * kTileM + row < ui.q_len;
+          const int64_t tok = ui.o_row0 + i * kTileM + row;
+          uint4* dst = reinterpret_cast<uint4*>(p.out + (tok * p.heads + ui.h) * 128);
+          const uint32_t o_addr = tmem + lane_addr + kColO + i * 128;
+#pragma unroll 1
+          for (int c = 0; c < 4; ++c) {
+            uint32_t r[32];
+            tmem_ld32_sync(o_addr + c * 32, r);
+            if (c == 3) {
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&bars[kBarOEmpty + i]);
+            }
+            if (valid) {
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                uint4 v;
+                v.x = cvt_bf16x2(__uint_as_float(r[8 * q + 0]) * st.x, __uint_as_float(r[8 * q + 1]) * st.x);
+                v.y = cvt_bf16x2(__uint_as_float(r[8 * q + 2]) * st.x, __uint_as_float(r[8 * q + 3]) * st.x);
+                v.z = cvt_bf16x2(__uint_as_float(r[8 * q + 4]) * st.x, __uint_as_float(r[8 * q + 5]) * st.x);
+                v.w = cvt_bf16x2(__uint_as_float(r[8 * q + 6]) * st.x, __uint_as_float(r[8 * q + 7]) * st.x);
+                dst[c * 4 + q] = v;
+              }
+            }
+          }
+          if (valid) p.lse[static_cast<int64_t>(ui.h) * p.tq + tok] = st.y;
         }
       }
     }
