@@ -46,14 +46,9 @@ namespace lpfa {
 namespace pp {
 
 // LPFA_PP_EPI_WG: warps 12..15 write O and the LSE in the modes where they convert no V (else the
-// softmax warps do, after each unit). LPFA_PP_NEXT_UNIT: in the bf16 P modes the softmax warps read
-// the next unit's description one unit ahead (measured: +1.5-2.5 % on 16-key-tile units with bf16 P;
-// with 8-bit P the registers it holds through the unit cost 2-5 %, so those modes do not).
+// softmax warps do, after each unit).
 #ifndef LPFA_PP_EPI_WG
 #define LPFA_PP_EPI_WG 1
-#endif
-#ifndef LPFA_PP_NEXT_UNIT
-#define LPFA_PP_NEXT_UNIT 1
 #endif
 
 // LPFA_PP_BF_P_SMEM: bf16 P in two shared-memory slots (PV as a shared-memory MMA), else in one
@@ -95,6 +90,10 @@ constexpr uint32_t kBfAtomBytes = 128 * 128;      // one 128-row x 128-byte swiz
 // Shared memory (offsets from a 1024-byte aligned base) and ring depths per PV mode. The bf16 P
 // modes keep BF16 V tiles (32 KB each) in shared memory, and with P there too (two 32 KB slots)
 // their Q has one stage and their V rings are shallower.
+constexpr int kSchedSplit = 2 + 2 * kMaxSortSeqs + 1;      // units before the split tail
+constexpr int kSchedMeta = kSchedSplit + 1;                // first metadata copy in sched[]
+constexpr int kSchedInts = kSchedMeta + 4 * (kMaxSortSeqs + 1);
+
 template <int kPv>
 struct Smem {
   static constexpr bool kBf = kPv == kPvBf16Mx || kPv == kPvBf16In;  // bf16 P, BF16 V
@@ -116,7 +115,7 @@ struct Smem {
   static constexpr uint32_t v_sf = k_sf + kKS * kAtomBytes;                // MXFP8 V only
   static constexpr uint32_t p_sf = v_sf + (kVsf ? kVS * kAtomBytes : 0u);  // [kPSlots] P atoms (MXFP8 PV)
   static constexpr uint32_t sched = p_sf + (kPv == kPvMx ? kPSlots * kAtomBytes : 0u);  // n, units, order, prefix
-  static constexpr uint32_t bars = sched + ((2 * kMaxSortSeqs + 3) * 4 + 15) / 16 * 16;
+  static constexpr uint32_t bars = sched + ((kSchedInts * 4) + 15) / 16 * 16;
   static constexpr uint32_t num_bars = 56;
   static constexpr uint32_t misc = bars + num_bars * 8;                     // tmem base, abort flag
   static constexpr uint32_t stats = misc + 64;                              // [2][128] (O scale, LSE)
@@ -161,8 +160,14 @@ struct PairUnit {
   int h, seq, qtile0, q_row0, o_row0, q_len, k_row0, k_len, nkv, sbq, sbk, has_q1;
 };
 
-// Unit order in shared memory: sched[0] = n, sched[1] = number of units, then order[kMaxSortSeqs]
-// and prefix[kMaxSortSeqs + 1]. For 1 <= n <= kMaxSortSeqs sequences the units are pairs of query
+// Unit order in shared memory: sched[0] = n, sched[1] = number of units, then order[kMaxSortSeqs],
+// prefix[kMaxSortSeqs + 1] and (n > 0) copies of the metadata the units are decoded from:
+// cu_q, scale_off_q, cu_k, scale_off_k, kMaxSortSeqs + 1 entries each, so that decoding a unit
+// reads only shared memory. When the pair units would leave a last partial wave of r units with
+// 2 r <= the grid size, those r pairs (the shortest, at the end of the longest-first order) are split
+// into 2 r single-tile units, one per CTA, instead of r CTAs running a whole pair while the rest
+// wait: sched[kSchedSplit] is the number of units before the split tail. A single-tile unit that
+// would be the absent second tile of a pair has nkv = -1 and is skipped by every role. For 1 <= n <= kMaxSortSeqs sequences the units are pairs of query
 // tiles: sequences by decreasing key-tile count (longest first), each taking heads * ceil(tiles / 2)
 // consecutive units, pairs innermost, so that the CTAs running together share one (sequence,
 // head)'s K/V through L2 and the static round-robin over the list approximates longest-processing-
@@ -190,6 +195,18 @@ __device__ __forceinline__ void build_pair_order(const AttnParams& p, int* sched
   int* s_cost = s_pre;  // key tiles per sequence, before s_pre holds the prefix
   for (int i = threadIdx.x; i < n; i += blockDim.x)
     s_cost[i] = (__ldg(p.cu_k + i + 1) - __ldg(p.cu_k + i) + kTileN - 1) / kTileN;
+  {
+    int* m = sched + kSchedMeta;
+    const int nq = p.shared_q ? 1 : n;
+    for (int i = threadIdx.x; i <= nq; i += blockDim.x) {
+      m[i] = __ldg(p.cu_q + i);
+      m[(kMaxSortSeqs + 1) + i] = __ldg(p.so_q + i);
+    }
+    for (int i = threadIdx.x; i <= n; i += blockDim.x) {
+      m[2 * (kMaxSortSeqs + 1) + i] = __ldg(p.cu_k + i);
+      m[3 * (kMaxSortSeqs + 1) + i] = __ldg(p.so_k + i);
+    }
+  }
   __syncthreads();
   for (int i = threadIdx.x; i < n; i += blockDim.x) {
     const int ci = s_cost[i];
@@ -218,7 +235,11 @@ __device__ __forceinline__ void build_pair_order(const AttnParams& p, int* sched
     if (threadIdx.x == 0) {
       s_pre[0] = 0;
       sched[0] = n;
-      sched[1] = carry;
+      const int grid = static_cast<int>(gridDim.x);
+      const int r = carry % grid;
+      const int split = (r > 0 && 2 * r <= grid) ? r : 0;
+      sched[kSchedSplit] = carry - split;
+      sched[1] = carry + split;
     }
   }
   __syncthreads();
@@ -227,26 +248,48 @@ __device__ __forceinline__ void build_pair_order(const AttnParams& p, int* sched
 __device__ __forceinline__ PairUnit pair_unit(const AttnParams& p, const int* sched, int w) {
   PairUnit u;
   const int n = sched[0];
-  if (n != 0) {
-    int local, np, nt;
-    if (n > 0) {
-      const int* order = sched + 2;
-      const int* pre = sched + 2 + kMaxSortSeqs;
-      const int r = find_prefix_smem(pre, n, w);
-      u.seq = order[r];
-      local = w - pre[r];
-      nt = query_tiles_of(p, u.seq);
-      np = (nt + 1) >> 1;
-    } else {  // shared query set, plain order
-      nt = query_tiles_of(p, 0);
-      np = (nt + 1) >> 1;
-      u.seq = w / (p.heads * np);
-      local = w - u.seq * (p.heads * np);
-    }
+  if (n > 0) {
+    // Everything from shared memory: the order, its prefix and the metadata copies.
+    const int* order = sched + 2;
+    const int* pre = sched + 2 + kMaxSortSeqs;
+    const int* cuq = sched + kSchedMeta;
+    const int* soq = cuq + (kMaxSortSeqs + 1);
+    const int* cuk = soq + (kMaxSortSeqs + 1);
+    const int* sok = cuk + (kMaxSortSeqs + 1);
+    // Units of the split tail: single tiles, two per pair of the order.
+    const int keep = sched[kSchedSplit];
+    const int half = w >= keep ? ((w - keep) & 1) : -1;
+    const int wp = w >= keep ? keep + ((w - keep) >> 1) : w;
+    const int r = find_prefix_smem(pre, n, wp);
+    u.seq = order[r];
+    const int local = wp - pre[r];
+    const int qseq = p.shared_q ? 0 : u.seq;
+    const int nt = soq[qseq + 1] - soq[qseq];
+    const int np = (nt + 1) >> 1;
+    u.h = local / np;
+    const int pair = local - u.h * np;
+    u.qtile0 = 2 * pair + (half > 0 ? 1 : 0);
+    u.sbq = soq[qseq] + u.qtile0;
+    u.has_q1 = (half < 0 && 2 * pair + 1 < nt) ? 1 : 0;
+    const int cq0 = cuq[qseq];
+    u.q_row0 = cq0 + u.qtile0 * kTileM;
+    u.q_len = cuq[qseq + 1] - cq0;
+    u.o_row0 = p.shared_q ? u.seq * u.q_len + u.qtile0 * kTileM : u.q_row0;
+    u.k_row0 = cuk[u.seq];
+    u.k_len = cuk[u.seq + 1] - u.k_row0;
+    u.nkv = u.qtile0 < nt ? (u.k_len + kTileN - 1) / kTileN : -1;
+    u.sbk = sok[u.seq];
+    return u;
+  }
+  if (n < 0) {  // shared query set, plain order
+    const int nt = query_tiles_of(p, 0);
+    const int np = (nt + 1) >> 1;
+    u.seq = w / (p.heads * np);
+    const int local = w - u.seq * (p.heads * np);
     u.h = local / np;
     const int pair = local - u.h * np;
     u.qtile0 = 2 * pair;
-    u.sbq = __ldg(p.so_q + (p.shared_q ? 0 : u.seq)) + 2 * pair;
+    u.sbq = __ldg(p.so_q) + 2 * pair;
     u.has_q1 = (2 * pair + 1 < nt) ? 1 : 0;
   } else {
     u.h = w / p.total_q_tiles;
@@ -421,7 +464,9 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
   constexpr bool kVIn = L::kVIn;            // BF16 V input (TMA straight into the operand layout)
   constexpr bool kConv = kPv == kPvBf16Mx;  // MXFP8 V converted to BF16 by warps 12..15
   constexpr bool kEpi = !kConv && LPFA_PP_EPI_WG;  // warps 12..15 write O and LSE (else the softmax warps do)
-  constexpr bool kNextUnit = LPFA_PP_NEXT_UNIT && kBf;  // softmax warps decode the next unit early
+  // bf16 P: the softmax warps decode the next unit one unit ahead (measured +1.5-2.5 % on
+  // 16-key-tile units; with 8-bit P the registers it holds through the unit cost 2-5 %).
+  constexpr bool kNextUnit = kBf;
   constexpr int kQS = L::kQS, kKS = L::kKS;
   // Ring depths as divisors: a ring a mode does not use has depth 0 in L; its code is never reached.
   constexpr int kVS = L::kVS > 0 ? L::kVS : 1, kVBS = L::kVBS > 0 ? L::kVBS : 1;
@@ -505,7 +550,7 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
       bool ok = true;
       for (int w = blockIdx.x; w < num_units && ok; w += G) {
         const PairUnit ui = warp_uniform(pair_unit(p, sched, w));
-        if (ui.nkv == 0) continue;  // no keys: the softmax warps write the empty-sum result
+        if (ui.nkv <= 0) continue;  // no keys (the softmax warps write the empty-sum result), or no tile
         const uint32_t qs = qc % kQS, qph = (qc / kQS) & 1;
         if (!wait_role(&bars[kBarQEmpty + qs], qph ^ 1, abort_flag)) { record_failure(abort_flag, kPSiteProducerQ); ok = false; break; }
         mbar_arrive_expect_tx(&bars[kBarQFull + qs], (ui.has_q1 ? 2u : 1u) * (kTileBytes + kAtomBytes), leader);
@@ -521,7 +566,8 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
           // With one Q stage the next unit's tiles can only be loaded once this unit's last QK
           // has run; bring them into L2 now so that load is an L2 hit.
           const PairUnit un = warp_uniform(pair_unit(p, sched, w + G));
-          for (int i = 0; i <= un.has_q1; ++i) tma_prefetch_3d(&tmap_q, 0, un.h, un.q_row0 + i * kTileM, leader);
+          if (un.nkv > 0)
+            for (int i = 0; i <= un.has_q1; ++i) tma_prefetch_3d(&tmap_q, 0, un.h, un.q_row0 + i * kTileM, leader);
         }
         for (int j = 0; j < ui.nkv; ++j) {
           const uint32_t s = kc % kKS, ph = (kc / kKS) & 1;
@@ -600,12 +646,24 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
         // drains below, so the wait runs out and the failure path is exercised.
         if (!wait_role(&bars[kBarDrain], 0, abort_flag)) { record_failure(abort_flag, kPSiteDebugStall); ok = false; }
       }
+      // The sign of the logit scale goes into the MMA (negated A); the softmax uses |scale|. The
+      // descales are global loads: each unit's are issued one unit ahead, so that their latency is
+      // not between the last QK of one unit and the first of the next.
+      float qd_next = 1.0f, kd_next = 1.0f;
+      if (static_cast<int>(blockIdx.x) < num_units) {
+        const PairUnit u0 = warp_uniform(pair_unit(p, sched, blockIdx.x));
+        qd_next = descale_value(p.q_descale, u0.seq, u0.h);
+        kd_next = descale_value(p.k_descale, u0.seq, u0.h);
+      }
       for (int w = blockIdx.x; w < num_units && ok; w += G) {
         const PairUnit ui = warp_uniform(pair_unit(p, sched, w));
-        if (ui.nkv == 0) continue;
-        // The sign of the logit scale goes into the MMA (negated A); the softmax uses |scale|.
-        const float qd = descale_value(p.q_descale, ui.seq, ui.h);
-        const float kd = descale_value(p.k_descale, ui.seq, ui.h);
+        const float qd = qd_next, kd = kd_next;
+        if (w + G < num_units) {
+          const PairUnit un = warp_uniform(pair_unit(p, sched, w + G));
+          qd_next = descale_value(p.q_descale, un.seq, un.h);
+          kd_next = descale_value(p.k_descale, un.seq, un.h);
+        }
+        if (ui.nkv <= 0) continue;
         const int negate = (qd * kd) < 0.0f ? 1 : 0;
         uint32_t idq[4];
 #pragma unroll
@@ -691,7 +749,7 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
       bool ok = true;
       for (int w = blockIdx.x; w < num_units && ok; w += G) {
         const PairUnit ui = warp_uniform(pair_unit(p, sched, w));
-        if (ui.nkv == 0) continue;
+        if (ui.nkv <= 0) continue;
         for (int j = 0; j < ui.nkv && ok; ++j) {
           const uint32_t vs = kBf ? vc % kVBS : vc % kVS;
           // V first: it is loaded well ahead, so this wait is off the path from P to PV.
@@ -777,7 +835,6 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
     uint32_t nbase = 0;         // P tiles of all earlier units, in the order the PVs consume them
     float2* stats = reinterpret_cast<float2*>(smem + L::stats);
     bool ok = true;
-    // The next unit's description is loaded one unit ahead (its metadata reads are global loads).
     PairUnit ui_next;
     if (kNextUnit && static_cast<int>(blockIdx.x) < num_units) ui_next = pair_unit(p, sched, blockIdx.x);
     for (int w = blockIdx.x; w < num_units && ok; w += G) {
@@ -785,10 +842,11 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
       if (kNextUnit && w + G < num_units) ui_next = pair_unit(p, sched, w + G);
       const uint32_t np = 1u + static_cast<uint32_t>(ui.has_q1);  // P tiles per key tile
       const uint32_t n0 = nbase;
-      nbase += static_cast<uint32_t>(ui.nkv) * np;
+      nbase += static_cast<uint32_t>(max(ui.nkv, 0)) * np;
       if (grp > ui.has_q1) continue;
       const bool valid = (ui.qtile0 + grp) * kTileM + row < ui.q_len;
       const int64_t tok = ui.o_row0 + grp * kTileM + row;  // output and LSE row
+      if (ui.nkv < 0) continue;  // the absent second tile of a split pair
       if (ui.nkv == 0) {
         // No keys: an empty sum, LSE = log 0 = -inf and O = 0.
         if (valid) {
@@ -802,6 +860,7 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
       const float cscale = kPerUnitDescale ? fabsf((descale_value(p.q_descale, ui.seq, ui.h) *
                                                     descale_value(p.k_descale, ui.seq, ui.h)) * kLog2eRsqrtD)
                                            : cscale_all;
+      const float vd = descale_value(p.v_descale, ui.seq, ui.h);  // read now, used after the last tile
       float m_r = -INFINITY;  // row reference (integer, log2 units)
       float l_r = 0.0f;       // row sum of p (times 2^kBias), relative to m_r
       float lr_r = 0.0f;      // bf16 P: the same sum over the BF16-rounded P
@@ -939,7 +998,7 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
         // Hand the row's O scale and LSE to the epilogue warpgroup and go on to the next unit. The
         // slot is free once the epilogue has read this warpgroup's previous unit's values.
         if (ucnt > 0 && !wait_warp(&bars[kBarStatsFree + grp], (ucnt - 1) & 1, abort_flag, false)) { record_failure(abort_flag, kPSiteSoftStats); ok = false; break; }
-        stats[grp * kTileM + row] = make_float2(descale_value(p.v_descale, ui.seq, ui.h) / (kBf ? lr_r : l_r),
+        stats[grp * kTileM + row] = make_float2(vd / (kBf ? lr_r : l_r),
                                                 (m_r - kBias + lg2_approx(l_r)) * kLn2);
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars[kBarStatsFull + grp]);
@@ -951,7 +1010,7 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
       tc_fence_after();
       // O is normalised by the sum of the P values the PV product used (bf16 P: the rounded ones, so
       // a row dominated by one key gets that V row exactly); the LSE keeps the unrounded sum.
-      const float oscale = descale_value(p.v_descale, ui.seq, ui.h) / (kBf ? lr_r : l_r);
+      const float oscale = vd / (kBf ? lr_r : l_r);
       uint4* dst = reinterpret_cast<uint4*>(p.out + (tok * p.heads + ui.h) * 128);
       // O_i in two halves of 64 columns; the second load releases O_i to the next unit's PV.
 #pragma unroll 1
@@ -1052,7 +1111,7 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
       bool ok = true;
       for (int w = blockIdx.x; w < num_units && ok; w += G) {
         const PairUnit ui = pair_unit(p, sched, w);
-        if (ui.nkv == 0) continue;  // the softmax warps wrote the empty-sum rows
+        if (ui.nkv <= 0) continue;  // the softmax warps wrote the empty-sum rows (or no tile)
         for (int i = 0; i <= ui.has_q1; ++i) {
           // Long waits (a whole unit): sleep between polls, leaving issue slots to the softmax warps.
           if (!wait_role(&bars[kBarOFull + i], rc[i] & 1, abort_flag)) { record_failure(abort_flag, kPSiteEpiO); ok = false; break; }
