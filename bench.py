@@ -6,7 +6,8 @@ in HBM: varlen metadata, MXFP8 quantization of Q and K (and V in bf16 PV mode), 
 unscaled E4M3 cast of V (fp8 PV mode), and the attention forward. `value` is attention
 TFLOPS (sum of 4 * Sq * Sk * H * 128 over sequences, every rank) divided by the step time;
 the `roofline` object reports the attention kernel alone against the measured dense FP8
-peak, and `e2e` repeats the step with host buffers (pinned H2D of Q/K/V, D2H of O/LSE).
+peak, and `e2e` repeats the step with host buffers (pinned H2D of Q/K/V, D2H of O/LSE every
+step, the copies of neighbouring steps overlapping this step's compute on two copy streams).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
 
@@ -443,7 +444,8 @@ def main():
     ws_bytes = lp.lpfa_attn_fwd_workspace_bytes(lp.lpfa_varlen_meta_fill_host(lk), H, w.pv_mode)
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev) if ws_bytes else False
 
-    def step(ins, timing=None):
+    def step(ins, timing=None, result=None):
+        o_dst, l_dst = result if result is not None else (out, lse)
         mq = lp.lpfa_varlen_meta_from_lengths(lq, device=dev)
         mk = lp.lpfa_varlen_meta_from_lengths(lk, device=dev)
         if timing is not None:
@@ -462,7 +464,7 @@ def main():
             c.record(stream)
         v_in = ins["v"] if w.pv_mode == "bf16v" else vp   # BF16 V goes to the kernel as is
         attn = lp.lpfa_attn_fwd_shared_q if w.shared_q else lp.lpfa_attn_fwd_varlen
-        attn(qp, qs, kp, ks, v_in, vs, mq, mk, pv_mode=w.pv_mode, out=out, lse=lse, workspace=ws)
+        attn(qp, qs, kp, ks, v_in, vs, mq, mk, pv_mode=w.pv_mode, out=o_dst, lse=l_dst, workspace=ws)
         if timing is not None:
             b.record(stream)
             timing.append((a, c, b))
@@ -510,36 +512,75 @@ def main():
     ms_per_step = total_ms / args.steps
     value = job_tflops(flops, world, ms_per_step)
 
-    # End to end through the public API with host buffers.
+    # End to end through the public API with host buffers. Each step copies its Q/K/V in from
+    # pinned host memory and its O/LSE out, pipelined the way a serving loop would run it: the
+    # next step's inputs are copied in (copy stream) and the previous step's results copied out
+    # (a second copy stream) while this step computes, into double-buffered device tensors. The
+    # timed region spans the first step's input copy to the last step's output copy.
     e2e = None
     if not args.no_e2e:
         pinned = {x: dev_in[x].cpu().pin_memory() for x in "qkv"}
-        o_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-        l_host = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
-        scratch = {x: torch.empty_like(dev_in[x]) for x in "qkv"}
+        o_host = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(2)]
+        l_host = [torch.empty(lse.shape, dtype=lse.dtype).pin_memory() for _ in range(2)]
+        ins_dev = [{x: torch.empty_like(dev_in[x]) for x in "qkv"} for _ in range(2)]
+        res_dev = [(torch.empty_like(out), torch.empty_like(lse)) for _ in range(2)]
+        h2d_s, d2h_s = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
         h2d = sum(t.numel() * t.element_size() for t in pinned.values()) + 2 * 4 * (len(lq) + 1) * 2
-        d2h = o_host.numel() * o_host.element_size() + l_host.numel() * l_host.element_size()
+        d2h = o_host[0].numel() * o_host[0].element_size() + l_host[0].numel() * l_host[0].element_size()
 
-        def e2e_step():
-            for x in "qkv":
-                scratch[x].copy_(pinned[x], non_blocking=True)
-            step(scratch)
-            o_host.copy_(out, non_blocking=True)
-            l_host.copy_(lse, non_blocking=True)
+        def run_e2e(n, start_ev=None):
+            h2d_done, comp_done, d2h_done = [None] * n, [None] * n, [None] * n
 
-        for _ in range(max(1, args.warmup // 2)):
-            e2e_step()
+            def copy_in(i):
+                if start_ev is not None:
+                    h2d_s.wait_event(start_ev)
+                if i >= 2:
+                    h2d_s.wait_event(comp_done[i - 2])   # step i - 2 has finished reading the buffer
+                with torch.cuda.stream(h2d_s):
+                    for x in "qkv":
+                        ins_dev[i % 2][x].copy_(pinned[x], non_blocking=True)
+                    ev = torch.cuda.Event()
+                    ev.record(h2d_s)
+                h2d_done[i] = ev
+
+            copy_in(0)
+            for i in range(n):
+                if i + 1 < n:
+                    copy_in(i + 1)
+                stream.wait_event(h2d_done[i])
+                if i >= 2:
+                    stream.wait_event(d2h_done[i - 2])   # step i - 2's results have been copied out
+                step(ins_dev[i % 2], result=res_dev[i % 2])
+                ce = torch.cuda.Event()
+                ce.record(stream)
+                comp_done[i] = ce
+                d2h_s.wait_event(ce)
+                with torch.cuda.stream(d2h_s):
+                    o_host[i % 2].copy_(res_dev[i % 2][0], non_blocking=True)
+                    l_host[i % 2].copy_(res_dev[i % 2][1], non_blocking=True)
+                    de = torch.cuda.Event()
+                    de.record(d2h_s)
+                d2h_done[i] = de
+            stream.wait_event(d2h_done[n - 1])
+            return (n - 1) % 2
+
+        run_e2e(max(2, args.warmup // 2))
         barrier()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         ne = max(3, args.steps // 2)
         e0.record(stream)
-        for _ in range(ne):
-            e2e_step()
+        last = run_e2e(ne, start_ev=e0)
         e1.record(stream)
         barrier()
         e_ms = max_over_ranks(e0.elapsed_time(e1)) / ne
+        # The pipelined steps must give exactly the results of the resident-input step.
+        step(dev_in)
+        torch.cuda.synchronize()
+        same = bool(torch.equal(o_host[last].view(torch.int16), out.cpu().view(torch.int16)) and
+                    torch.equal(l_host[last].view(torch.int32), lse.cpu().view(torch.int32)))
         e2e = {"value": job_tflops(flops, world, e_ms), "unit": "TFLOPS", "ms_per_step": e_ms,
-               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "pipelined": True,
+               "results_match_resident_step": same}
 
     peaks, peak_src = load_peaks()
     # The attention kernel runs at full SM clock (it is not power capped like a dense GEMM), so
