@@ -144,3 +144,22 @@ def test_workspace_is_checked_and_reusable():
         assert torch.equal(o.view(torch.int16), o3.view(torch.int16))
         assert torch.equal(l.view(torch.int32), l3.view(torch.int32))
     assert lp.lpfa_device_status() == (lp.LPFA_OK, 0)
+
+
+def test_dequantize_writes_only_its_output():
+    """The BF16 output sits inside a pattern-filled buffer; every guard byte must survive, and rows
+    of every sequence (ragged tails included) must be written."""
+    lengths, heads = [129, 1, 300], 3
+    codes, scales = _random_mx(21, lengths, heads, 100, 150)
+    meta = lp.lpfa_varlen_meta_from_lengths(lengths)
+    T = sum(lengths)
+    n = T * heads * 128 * 2
+    guard = 4096
+    buf = torch.full((n + 2 * guard,), 0xA5, dtype=torch.uint8, device="cuda")
+    out = buf[guard:guard + n].view(torch.bfloat16).view(T, heads, 128)
+    lp.lpfa_dequantize_mxfp8_varlen(torch.from_numpy(codes).cuda(), torch.from_numpy(scales).cuda(), meta, out=out)
+    torch.cuda.synchronize()
+    host = buf.cpu().numpy()
+    assert (host[:guard] == 0xA5).all() and (host[guard + n:] == 0xA5).all()
+    ref = torch.from_numpy(omx.dequantize_mxfp8(codes, scales, lengths, heads)).to(torch.float32).to(torch.bfloat16)
+    assert torch.equal(out.cpu().view(torch.int16), ref.view(torch.int16))
