@@ -263,6 +263,8 @@ def lpfa_attn_fwd_varlen(q: torch.Tensor, q_sf: torch.Tensor, k: torch.Tensor, k
     workspace: where the bf16 PV mode converts V to BF16 once (lpfa_attn_fwd_varlen_ws): True
     allocates it, a uint8 device tensor of at least lpfa_attn_fwd_workspace_bytes bytes is used as
     is, False converts V tiles inside the attention kernel instead (same bits). Other modes ignore it.
+    (An allocated workspace is recorded on `stream` when that is a torch.cuda.Stream; with a raw
+    stream handle other than the current stream, pass a workspace tensor that outlives the work.)
     debug_flags != 0 goes through lpfa_attn_fwd_varlen_debug (test hook, see include/lpfa.h),
     which takes per-tensor descales only and no workspace.
     """
@@ -292,7 +294,7 @@ def lpfa_attn_fwd_varlen(q: torch.Tensor, q_sf: torch.Tensor, k: torch.Tensor, k
             ctypes.byref(meta_q._c), ctypes.byref(meta_k._c), H, 128, PV_MODES[pv_mode],
             _ptr(q_descale), _ptr(k_descale), _ptr(v_descale), out.data_ptr(), lse.data_ptr(),
             _stream_ptr(stream))
-    ws = None if debug_flags else _workspace(workspace, meta_k, H, pv_mode, q.device)
+    ws = None if debug_flags else _workspace(workspace, meta_k, H, pv_mode, q.device, stream)
     with torch.cuda.device(q.device):
         if debug_flags:
             _check(_lib.lpfa_attn_fwd_varlen_debug(*args, debug_flags))
@@ -311,13 +313,16 @@ def lpfa_attn_fwd_workspace_bytes(meta_k: VarlenMeta, heads: int, pv_mode: str) 
     return int(_lib.lpfa_attn_fwd_workspace_bytes(ctypes.byref(meta_k._c), heads, PV_MODES[pv_mode]))
 
 
-def _workspace(workspace, meta_k: VarlenMeta, heads: int, pv_mode: str, device):
+def _workspace(workspace, meta_k: VarlenMeta, heads: int, pv_mode: str, device, stream=None):
     """The workspace tensor for a forward call, or None (in-kernel V conversion / not needed)."""
     need = lpfa_attn_fwd_workspace_bytes(meta_k, heads, pv_mode)
     if need == 0 or workspace is False or workspace is None:
         return None
     if workspace is True:
-        return torch.empty(need, dtype=torch.uint8, device=device)
+        ws = torch.empty(need, dtype=torch.uint8, device=device)
+        if isinstance(stream, torch.cuda.Stream):
+            ws.record_stream(stream)  # the kernels read it on that stream after this call returns
+        return ws
     if not isinstance(workspace, torch.Tensor) or workspace.dtype != torch.uint8 or not workspace.is_contiguous():
         raise ValueError("workspace must be True, False or a contiguous uint8 device tensor")
     if workspace.numel() < need:
@@ -376,7 +381,7 @@ def lpfa_attn_fwd_shared_q(q: torch.Tensor, q_sf: torch.Tensor, k: torch.Tensor,
         lse = torch.empty((H, rows), dtype=torch.float32, device=q.device)
     if tuple(out.shape) != (rows, H, 128) or tuple(lse.shape) != (H, rows):
         raise ValueError("out must be (n*Lq, H, 128) and lse (H, n*Lq)")
-    ws = _workspace(workspace, meta_k, H, pv_mode, q.device)
+    ws = _workspace(workspace, meta_k, H, pv_mode, q.device, stream)
     args = (q.data_ptr(), q_sf.data_ptr(), k.data_ptr(), k_sf.data_ptr(), v.data_ptr(), _ptr(v_sf),
             ctypes.byref(meta_q._c), ctypes.byref(meta_k._c), H, 128, PV_MODES[pv_mode], ctypes.byref(descs[0]),
             ctypes.byref(descs[1]), ctypes.byref(descs[2]), out.data_ptr(), lse.data_ptr())
