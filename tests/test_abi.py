@@ -231,3 +231,35 @@ def test_dequantize_argument_validation():
                          ((FAKE, FAKE, 0, 128, FAKE), "heads"), ((FAKE, FAKE, 2, 128, FAKE + 2), "aligned")):
         st = lp._lib.lpfa_dequantize_mxfp8_varlen(args[0], args[1], ctypes.byref(m), args[2], args[3], args[4], None)
         assert st == lp.LPFA_ERR_INVALID_ARG and needle in lp._lib.lpfa_last_error_message().decode()
+
+
+def test_shared_query_workspace_validation():
+    """lpfa_attn_fwd_shared_q_ws checks its bf16-PV workspace like the varlen entry point."""
+    host_q = np.zeros(2 * 2, dtype=np.int32)
+    host_k = np.zeros(2 * 3, dtype=np.int32)
+    cq, ck = lp._Meta(), lp._Meta()
+    assert lp._lib.lpfa_varlen_meta_fill_host(np.array([300], np.int32).ctypes.data, 1, host_q.ctypes.data,
+                                              ctypes.byref(cq)) == 0
+    assert lp._lib.lpfa_varlen_meta_fill_host(np.array([5, 7], np.int32).ctypes.data, 2, host_k.ctypes.data,
+                                              ctypes.byref(ck)) == 0
+    cq.dev = ck.dev = 16
+    one = lp._Descale(None, 0, 0)
+    st = lp._lib.lpfa_attn_fwd_shared_q_ws(16, 16, 16, 16, 16, 16, ctypes.byref(cq), ctypes.byref(ck), 2, 128, 0,
+                                           ctypes.byref(one), ctypes.byref(one), ctypes.byref(one), 16, 16, None,
+                                           ctypes.c_size_t(0), None)
+    assert st == lp.LPFA_ERR_INVALID_ARG
+    assert b"workspace" in lp._lib.lpfa_last_error_message()
+
+
+def test_noalloc_size_limit_is_checked_before_device_work():
+    """Beyond the scratch size, bf16 PV is rejected with the sizes before any device work (the
+    pointers here are never dereferenced)."""
+    H, tokens = 16, (64 << 20) // (256 * 16) + 1
+    ck = _fake_meta(1, tokens)
+    cq = _fake_meta(1, 128)
+    one = lp._Descale(None, 0, 0)
+    st = lp._lib.lpfa_attn_fwd_varlen_noalloc(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, ctypes.byref(cq), ctypes.byref(ck),
+                                              H, 128, 0, ctypes.byref(one), ctypes.byref(one), ctypes.byref(one),
+                                              FAKE, FAKE, None)
+    assert st == lp.LPFA_ERR_INVALID_ARG
+    assert b"scratch" in lp._lib.lpfa_last_error_message()
