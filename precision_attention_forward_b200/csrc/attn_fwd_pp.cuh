@@ -223,7 +223,11 @@ __device__ __forceinline__ void build_pair_order(const AttnParams& p, int* sched
     for (int base = 0; base < n; base += 32) {
       const int r = base + static_cast<int>(threadIdx.x);
       int v = 0;
-      if (r < n) v = p.heads * ((query_tiles_of(p, s_order[r]) + 1) >> 1);
+      if (r < n) {  // query tiles of the sequence, from the shared-memory copy of scale_off_q
+        const int* soq = sched + kSchedMeta + (kMaxSortSeqs + 1);
+        const int qs = p.shared_q ? 0 : s_order[r];
+        v = p.heads * ((soq[qs + 1] - soq[qs] + 1) >> 1);
+      }
 #pragma unroll
       for (int d = 1; d < 32; d <<= 1) {
         const int o = __shfl_up_sync(0xFFFFFFFFu, v, d);
