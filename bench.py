@@ -46,9 +46,9 @@ FALLBACK_HBM_GBS = 6650.0
 # recorded; any change to the kernel makes it null until re-captured.
 TRAFFIC = {
     # workload: (sha256 of the kernel's sources [:16], dram bytes read + written per launch)
-    "video_s32768_h24_fp8pv": ("15c78875a032c79a", 310550528 + 174260736),
-    "dense_4x2048_h16": ("950f83fdf065a3a6", 68299264 + 4990976),
-    "cross_varlen_outliers_h32": ("950f83fdf065a3a6", 3569741824 + 48004352),
+    "video_s32768_h24_fp8pv": ("388ff0548a182d31", 310078464 + 174111744),
+    "dense_4x2048_h16": ("85f4f6c42fb74a08", 68298752 + 3575808),
+    "cross_varlen_outliers_h32": ("85f4f6c42fb74a08", 3567325696 + 47040768),
 }
 
 # The source files of the attention kernel each PV mode runs, and that kernel's name.
