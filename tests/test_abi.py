@@ -263,3 +263,21 @@ def test_noalloc_size_limit_is_checked_before_device_work():
                                               FAKE, FAKE, None)
     assert st == lp.LPFA_ERR_INVALID_ARG
     assert b"scratch" in lp._lib.lpfa_last_error_message()
+
+
+def test_binding_workspace_choice():
+    """The binding's workspace argument: False/None mean in-kernel V conversion, other modes need
+    none, and a given tensor must be a large enough contiguous uint8 buffer (checked on the host)."""
+    meta = lp.lpfa_varlen_meta_fill_host([300, 5])
+    need = lp.lpfa_attn_fwd_workspace_bytes(meta, 4, "bf16")
+    assert need == 305 * 4 * 256
+    assert lp.lpfa_attn_fwd_workspace_bytes(meta, 4, "fp8") == 0
+    assert lp._workspace(False, meta, 4, "bf16", "cpu") is None
+    assert lp._workspace(None, meta, 4, "bf16", "cpu") is None
+    assert lp._workspace(True, meta, 4, "fp8", "cpu") is None
+    ok = torch.empty(need, dtype=torch.uint8)
+    assert lp._workspace(ok, meta, 4, "bf16", "cpu") is ok
+    for bad in (torch.empty(need - 1, dtype=torch.uint8), torch.empty(need, dtype=torch.int8),
+                torch.empty(2 * need, dtype=torch.uint8)[::2]):
+        with pytest.raises(ValueError):
+            lp._workspace(bad, meta, 4, "bf16", "cpu")
