@@ -91,20 +91,58 @@ def quantizer_bytes(tokens, heads, in_bytes, scale_blocks) -> float:
     return float(tokens) * heads * 128 * (in_bytes + 1) + float(scale_blocks) * heads * 512
 
 
+def smi_index_of(local_rank: int) -> int:
+    """nvidia-smi / NVML index of this rank's GPU (CUDA_VISIBLE_DEVICES maps CUDA ordinals)."""
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        ids = vis.split(",")
+        if local_rank < len(ids) and ids[local_rank].strip().isdigit():
+            return int(ids[local_rank])
+    return local_rank
+
+
 class ClockSampler:
-    """Samples nvidia-smi SM clocks and throttle reasons in the background."""
+    """SM clocks and clock-event (throttle) reasons of one GPU during the timed region.
+
+    NVML is polled every ~2 ms from a background thread, and only samples between mark("start")
+    and mark("end") (host times around the synchronised timed region) count, so even a timed
+    region of a few hundred milliseconds yields tens of samples. Without NVML it falls back to
+    `nvidia-smi -lms 100` over the whole run.
+    """
 
     QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    # NVML clock-event reason bits reported by name (the rest are idle / application settings).
+    REASON_BITS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+                   0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
 
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
         self.proc = None
         self.lines = []
         self.t = None
+        self.nvml = None
+        self.samples = []
+        self.marks = {}
+        self.halt = False
+
+    def mark(self, which: str):
+        self.marks[which] = time.perf_counter()
 
     def start(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(self.gpu)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.nvml = pynvml
+        except Exception:
+            self.nvml = None
+        if self.nvml is not None:
+            self.t = threading.Thread(target=self._poll, daemon=True)
+            self.t.start()
+            return
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
@@ -115,11 +153,43 @@ class ClockSampler:
         self.t = threading.Thread(target=self._read, daemon=True)
         self.t.start()
 
+    def _poll(self):
+        nv = self.nvml
+        while not self.halt:
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append((time.perf_counter(), float(sm), int(rs)))
+            except Exception:
+                pass
+            time.sleep(0.002)
+
     def _read(self):
         for line in self.proc.stdout:
             self.lines.append(line.strip())
 
     def stop(self):
+        if self.nvml is not None:
+            self.halt = True
+            if self.t:
+                self.t.join(timeout=2)
+            try:
+                self.nvml.nvmlShutdown()
+            except Exception:
+                pass
+            t0, t1 = self.marks.get("start"), self.marks.get("end")
+            sel = [x for x in self.samples if (t0 is None or x[0] >= t0) and (t1 is None or x[0] <= t1)]
+            inside = bool(sel)
+            if not sel:
+                sel = self.samples
+            reasons = set()
+            for _, _, rs in sel:
+                for bit, name in self.REASON_BITS.items():
+                    if rs & bit:
+                        reasons.add(name)
+            return {"sm_mhz": statistics.median(x[1] for x in sel) if sel else None,
+                    "sm_max_mhz": float(self.max_mhz), "reasons": sorted(reasons), "samples": len(sel),
+                    "source": "NVML, ~2 ms polling" + (" inside the timed region" if inside else " over the run")}
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
         self.proc.terminate()
@@ -144,7 +214,7 @@ class ClockSampler:
                 if val.lower() == "active":
                     reasons.add(n)
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": sorted(reasons), "samples": len(sm)}
+                "reasons": sorted(reasons), "samples": len(sm), "source": "nvidia-smi -lms 100 over the run"}
 
 
 def cpu_oracle_sample(w, seconds: float, seed: int = 0):
@@ -349,11 +419,12 @@ def run_backward(args, w):
     dout = wl.to_torch(wl.round_to_bf16(g.standard_normal(out.shape, dtype=np.float32)), "bf16", device=dev)
     flush = not l2_exceeded(lk, H)
     flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=dev) if flush else None
-    sampler = ClockSampler(0)
+    sampler = ClockSampler(smi_index_of(0))
     sampler.start()
     for _ in range(args.warmup):
         lp.lpfa_attn_bwd_varlen(q8, qs, k8, ks, v8, vs, out, dout, lse, mq, mk)
     torch.cuda.synchronize()
+    sampler.mark("start")
     times = []
     for _ in range(args.steps):
         if flush:
@@ -364,6 +435,7 @@ def run_backward(args, w):
         b.record(stream)
         times.append((a, b))
     torch.cuda.synchronize()
+    sampler.mark("end")
     clocks = sampler.stop()
     st, detail = lp.lpfa_device_status()
     if st != lp.LPFA_OK:
@@ -474,9 +546,7 @@ def main():
     barrier = ranks.barrier
     max_over_ranks = ranks.max
 
-    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
-    smi_index = int(vis.split(",")[local_rank]) if vis and vis.split(",")[local_rank].strip().isdigit() else local_rank
-    sampler = ClockSampler(smi_index)
+    sampler = ClockSampler(smi_index_of(local_rank))
     sampler.start()
     # Workloads whose inputs fit in L2 get it flushed before every step (a 256 MB write outside
     # the step's own events); the step time is then the sum of the per-step event intervals.
@@ -491,6 +561,7 @@ def main():
     for _ in range(args.warmup):
         timed_step()
     barrier()
+    sampler.mark("start")
     timing = []
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     launches = 0
@@ -499,6 +570,7 @@ def main():
         launches += timed_step(timing)
     end.record(stream)
     barrier()
+    sampler.mark("end")
     clocks = sampler.stop()
     total_ms = max_over_ranks(sum(a.elapsed_time(b) for a, c, b in timing) if flush else start.elapsed_time(end))
     quant_ms = sum(a.elapsed_time(c) for a, c, b in timing) / args.steps
